@@ -1,0 +1,168 @@
+"""Integer oracle of the realized chunk cost and the cost-aware LPT plan (test infrastructure only).
+
+Source: *Split-KV: Efficient Context Parallelism for Training Diffusion Drafters*,
+Abstract: the global query view lets a cost-aware longest-processing-time-first
+(LPT) strategy balance context K/V chunks by their realized attention cost, a
+requirement that is nonlinear and sample-dependent because of anchor sampling.
+Table 1 of the same page lists "Cost-aware LPT" as Split-KV's load balancing.
+
+Readings (the pages give neither the cost unit nor the LPT details):
+
+* Work item = (sample s, chunk c, kv head g, block b). Its query tile is the
+  ``block * G`` rows of block b at the G query heads of kv head g; its key tiles
+  are the ``key_tile`` (Tk = 128) slices of chunk c. Item cost = number of key
+  tiles holding at least one key the block sees; items of cost 0 are dropped.
+* Item index (chunk-major): ``base_s + (c * Hkv + g) * n_blocks_s + b`` where
+  ``base_s`` counts the items of earlier samples and ``n_chunks_s = ceil(S/C)``.
+* Chunk cost = sum of the costs of that chunk's items.
+* LPT: order items by (cost descending, item index ascending); give each in turn
+  to the worker with the least (load, worker index); loads start at 0; a
+  worker's queue lists its items in assignment order.
+* Imbalance = max(load) / mean(load) - 1.
+"""
+from __future__ import annotations
+
+import heapq
+import itertools
+from typing import Dict, List, Sequence, Tuple
+
+import numpy as np
+
+
+def item_layout(anchor_counts: Sequence[int], seq_lens: Sequence[int], chunk: int, n_kv_heads: int):
+    """Per-sample (base item index, n_chunks, n_blocks) and the total item count."""
+    out = []
+    base = 0
+    for nb, S in zip(anchor_counts, seq_lens):
+        nc = -(-int(S) // chunk)
+        out.append((base, nc, int(nb)))
+        base += nc * n_kv_heads * int(nb)
+    return out, base
+
+
+def costs_bruteforce(anchors_per_sample: Sequence[Sequence[int]], seq_lens: Sequence[int], chunk: int,
+                     key_tile: int, n_kv_heads: int, group: int, block: int = 16):
+    """Item costs by enumerating the boolean mask of every (query tile, key tile).
+
+    Returns ``(item_ids, item_costs, chunk_costs)``: visible items in ascending
+    index order, their costs, and per-(sample, chunk) costs (flattened, sample-major).
+    For small inputs only.
+    """
+    layout, _ = item_layout([len(a) for a in anchors_per_sample], seq_lens, chunk, n_kv_heads)
+    ids, costs, chunk_costs = [], [], []
+    for s, anchors in enumerate(anchors_per_sample):
+        base, nc, nb = layout[s]
+        S = int(seq_lens[s])
+        for c in range(nc):
+            lo, hi = c * chunk, min((c + 1) * chunk, S)
+            total = 0
+            for g in range(n_kv_heads):
+                for b, a in enumerate(anchors):
+                    rows = block * group
+                    keys = np.arange(lo, hi)
+                    mask = np.broadcast_to(keys < a, (rows, hi - lo))  # row sees context key iff key < anchor
+                    n_tiles = -(-(hi - lo) // key_tile)
+                    cost = 0
+                    for t in range(n_tiles):
+                        if mask[:, t * key_tile:(t + 1) * key_tile].any():
+                            cost += 1
+                    if cost:
+                        ids.append(base + (c * n_kv_heads + g) * nb + b)
+                        costs.append(cost)
+                        total += cost
+            chunk_costs.append(total)
+    return np.array(ids, np.int64), np.array(costs, np.int64), np.array(chunk_costs, np.int64)
+
+
+def costs_closed_form(anchors_per_sample, seq_lens, chunk, key_tile, n_kv_heads):
+    """Same result in closed form: ``cost = ceil(clamp(a - c*C, 0, min(C, S - c*C)) / Tk)``."""
+    layout, _ = item_layout([len(a) for a in anchors_per_sample], seq_lens, chunk, n_kv_heads)
+    ids, costs, chunk_costs = [], [], []
+    for s, anchors in enumerate(anchors_per_sample):
+        base, nc, nb = layout[s]
+        S = int(seq_lens[s])
+        a = np.asarray(anchors, np.int64)
+        for c in range(nc):
+            width = min(chunk, S - c * chunk)
+            nvis = np.clip(a - c * chunk, 0, width)
+            cost = -(-nvis // key_tile)
+            total = 0
+            for g in range(n_kv_heads):
+                for b in range(nb):
+                    if cost[b]:
+                        ids.append(base + (c * n_kv_heads + g) * nb + b)
+                        costs.append(int(cost[b]))
+                        total += int(cost[b])
+            chunk_costs.append(total)
+    return np.array(ids, np.int64), np.array(costs, np.int64), np.array(chunk_costs, np.int64)
+
+
+def lpt(costs: Sequence[int], n_workers: int):
+    """Longest-processing-time-first greedy, with a binary heap of (load, worker).
+
+    Returns ``(item_worker, queue_off, queue_items, load)``: the worker of each
+    item (items indexed by position in ``costs``), the queues in CSR form (each
+    in assignment order), and the final loads.
+    """
+    costs = [int(c) for c in costs]
+    order = sorted(range(len(costs)), key=lambda i: (-costs[i], i))
+    heap = [(0, w) for w in range(n_workers)]
+    heapq.heapify(heap)
+    item_worker = [-1] * len(costs)
+    queues: List[List[int]] = [[] for _ in range(n_workers)]
+    for i in order:
+        load, w = heapq.heappop(heap)
+        item_worker[i] = w
+        queues[w].append(i)
+        heapq.heappush(heap, (load + costs[i], w))
+    load = [0] * n_workers
+    for i, w in enumerate(item_worker):
+        load[w] += costs[i]
+    queue_off = [0]
+    for q in queues:
+        queue_off.append(queue_off[-1] + len(q))
+    queue_items = [i for q in queues for i in q]
+    return (np.array(item_worker, np.int64), np.array(queue_off, np.int64),
+            np.array(queue_items, np.int64), np.array(load, np.int64))
+
+
+def naive_split(costs: Sequence[int], n_workers: int):
+    """Cost-blind equal-count split: item list (index order) cut into contiguous pieces.
+
+    Worker ``w`` gets items ``[floor(w*n/m), floor((w+1)*n/m))``. Returns the same
+    tuple as :func:`lpt`.
+    """
+    n = len(costs)
+    bounds = [(w * n) // n_workers for w in range(n_workers + 1)]
+    item_worker = np.zeros(n, np.int64)
+    load = np.zeros(n_workers, np.int64)
+    for w in range(n_workers):
+        item_worker[bounds[w]:bounds[w + 1]] = w
+        load[w] = int(np.sum(np.asarray(costs[bounds[w]:bounds[w + 1]], np.int64)))
+    return item_worker, np.array(bounds, np.int64), np.arange(n, dtype=np.int64), load
+
+
+def makespan(load) -> int:
+    return int(np.max(load)) if len(load) else 0
+
+
+def imbalance(load) -> float:
+    """max(load) / mean(load) - 1 (0 for an empty plan)."""
+    load = np.asarray(load, np.float64)
+    if load.size == 0 or load.sum() == 0:
+        return 0.0
+    return float(load.max() / load.mean() - 1.0)
+
+
+def optimal_makespan(costs: Sequence[int], n_workers: int) -> int:
+    """Exhaustive minimum makespan over all n_workers^n assignments (tiny inputs)."""
+    costs = [int(c) for c in costs]
+    best = None
+    for assign in itertools.product(range(n_workers), repeat=len(costs)):
+        loads = [0] * n_workers
+        for c, w in zip(costs, assign):
+            loads[w] += c
+        mk = max(loads) if loads else 0
+        if best is None or mk < best:
+            best = mk
+    return 0 if best is None else best

@@ -1,0 +1,104 @@
+"""Pins of the integer cost / LPT oracle.
+
+* costs: brute-force mask enumeration equals the closed form on random small
+  cases (ragged tail chunks, anchors on tile edges), plus a hand-worked example;
+* LPT: a hand-worked plan; the textbook worst case of Graham's analysis
+  (m = 2, costs 3,3,2,2,2: LPT 7, optimum 6); exhaustive optimum for m <= 3 and
+  <= 10 items with LPT <= (4/3 - 1/(3m)) OPT; every item placed exactly once;
+  queues in assignment order.
+"""
+import numpy as np
+import pytest
+
+from oracle import schedule as Sch
+from tests._util import read_golden
+
+
+def test_cost_worked_example():
+    g = read_golden("cost_worked_example.txt")
+    for fn in (Sch.costs_bruteforce, Sch.costs_closed_form):
+        kw = dict(group=g["group"]) if fn is Sch.costs_bruteforce else {}
+        ids, costs, chunk_costs = fn([g["anchors"]], [g["seq_len"]], g["chunk"], g["key_tile"],
+                                     g["n_kv_heads"], **kw)
+        assert ids.tolist() == g["item_ids"]
+        assert costs.tolist() == g["item_costs"]
+        assert chunk_costs.tolist() == g["chunk_costs"]
+
+
+@pytest.mark.parametrize("seed", range(12))
+def test_cost_bruteforce_equals_closed_form(seed):
+    rng = np.random.default_rng(seed)
+    B = int(rng.integers(1, 4))
+    tk = int(rng.choice([8, 16, 32]))
+    chunk = tk * int(rng.integers(1, 5))
+    hkv = int(rng.integers(1, 3))
+    seq, anchors = [], []
+    for _ in range(B):
+        S = int(rng.integers(20, 300))
+        n = int(rng.integers(0, min(6, S - 16) + 1))
+        a = sorted(rng.choice(np.arange(16, S), size=n, replace=False).tolist())
+        if n and rng.random() < 0.5:  # put one anchor exactly on a tile / chunk edge
+            edge = (int(rng.integers(1, max(2, S // tk))) * tk)
+            if 16 <= edge < S and edge not in a:
+                a = sorted(a[:-1] + [edge])
+        seq.append(S)
+        anchors.append(a)
+    bf = Sch.costs_bruteforce(anchors, seq, chunk, tk, hkv, group=2, block=16)
+    cf = Sch.costs_closed_form(anchors, seq, chunk, tk, hkv)
+    for x, y in zip(bf, cf):
+        assert x.tolist() == y.tolist()
+    # every visible context pair lies in a counted tile: tiles * Tk >= visible keys per (block, head)
+    layout, total = Sch.item_layout([len(a) for a in anchors], seq, chunk, hkv)
+    assert all(i < total for i in bf[0].tolist())
+    assert int(bf[1].sum()) * tk >= hkv * sum(sum(a) for a in anchors)
+
+
+def test_lpt_worked_example():
+    g = read_golden("lpt_worked_example.txt")
+    iw, qo, qi, load = Sch.lpt(g["costs"], g["n_workers"])
+    assert iw.tolist() == g["item_worker"]
+    assert qo.tolist() == g["queue_off"]
+    assert qi.tolist() == g["queue_items"]
+    assert load.tolist() == g["load"]
+
+
+def test_lpt_graham_worst_case():
+    costs = [3, 3, 2, 2, 2]
+    _, _, _, load = Sch.lpt(costs, 2)
+    assert Sch.makespan(load) == 7
+    assert Sch.optimal_makespan(costs, 2) == 6
+    assert 7 <= (4 / 3 - 1 / 6) * 6 + 1e-12
+
+
+@pytest.mark.parametrize("seed", range(40))
+def test_lpt_within_graham_bound_of_exhaustive_optimum(seed):
+    rng = np.random.default_rng(100 + seed)
+    m = int(rng.integers(1, 4))
+    n = int(rng.integers(0, 11 if m < 3 else 10))
+    costs = rng.integers(1, 9, size=n).tolist()
+    iw, qo, qi, load = Sch.lpt(costs, m)
+    opt = Sch.optimal_makespan(costs, m)
+    assert Sch.makespan(load) <= (4 / 3 - 1 / (3 * m)) * opt + 1e-9
+    # every item exactly once; queues consistent with item_worker; loads add up
+    assert sorted(qi.tolist()) == list(range(n))
+    for w in range(m):
+        q = qi[qo[w]:qo[w + 1]].tolist()
+        assert all(iw[i] == w for i in q)
+        assert sum(costs[i] for i in q) == load[w]
+        # assignment order: non-increasing cost, ascending index among equal costs
+        keys = [(-costs[i], i) for i in q]
+        assert keys == sorted(keys)
+
+
+def test_lpt_tie_breaks_prefer_lower_worker_and_lower_index():
+    iw, qo, qi, load = Sch.lpt([1, 1, 1, 1], 3)
+    assert iw.tolist() == [0, 1, 2, 0]
+    assert load.tolist() == [2, 1, 1]
+
+
+def test_naive_split_contiguous_equal_counts():
+    costs = [5, 1, 1, 1, 1, 1, 1]
+    iw, qo, qi, load = Sch.naive_split(costs, 3)
+    assert qo.tolist() == [0, 2, 4, 7]
+    assert load.tolist() == [6, 2, 3]
+    assert Sch.imbalance(load) == pytest.approx(6 / (11 / 3) - 1)
