@@ -1,0 +1,368 @@
+"""Benchmark of the Split-KV hot path on B200: useful block-sparse attention TFLOP/s.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step = the whole hot path over one batch of synthetic input, through the C ABI:
+realized-cost pass -> LPT plan onto one queue per SM -> chunk-partial forward (tcgen05) ->
+exact LSE merge (+ backward for the training workload). Inputs are resident in HBM when timing
+starts; each timed step is bracketed by CUDA events on the launching stream and preceded (outside
+the events) by a 256 MB write that flushes the 126 MB L2.
+
+Useful FLOPs count only unmasked (query, key) pairs: each of the block rows of an anchor a sees
+a + block keys, per query head; forward 4*d per pair, backward 10*d per pair.
+
+With N > 1 (torchrun) every rank runs an independent replica of the workload on its own GPU
+(the hot path is single-GPU; there is no data-path collective); value = all ranks' useful FLOPs /
+the slowest rank's time. `--impl reference` times the float64 CPU oracle instead, on a bounded
+sample of the same workload, on the host cores (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+import workloads as W  # noqa: E402
+
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def useful_flops(inp, backward):
+    w = inp.workload
+    pairs = sum(w.block * (int(a) + w.block) for a in inp.anchors.tolist())
+    ctx_pairs = sum(w.block * int(a) for a in inp.anchors.tolist())
+    per_pair = 4 * w.head_dim * w.n_q_heads
+    fwd = per_pair * pairs
+    bwd = (10 * w.head_dim * w.n_q_heads * pairs) if backward else 0
+    return fwd + bwd, per_pair * ctx_pairs
+
+
+def peaks():
+    try:
+        with open(PEAKS_FILE) as f:
+            d = json.load(f)
+        return d, "measured"
+    except Exception:
+        return FALLBACK_PEAKS, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while the timed region runs."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-i", str(self.index), "-lms", "100"], stdout=subprocess.PIPE,
+                                         stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) != 6:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[2:]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return world, rank, local
+
+
+def max_over_ranks(x, world, device):
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def cpu_oracle_sample(inp, budget_s, backward):
+    """Time the float64 oracle on whole blocks of the workload until ~budget_s of CPU work."""
+    import numpy as np
+
+    from oracle import attention as OA
+    w = inp.workload
+
+    def f64(t):
+        return t.detach().to("cpu", torch.float64).numpy()
+
+    p = OA.Problem(inp.anchors.numpy(), inp.anchor_off.numpy(), inp.key_off.numpy(), f64(inp.q), f64(inp.k),
+                   f64(inp.v), f64(inp.kb), f64(inp.vb), block=w.block, scale=w.scale)
+    n = int(inp.anchor_off[-1])
+    order = np.random.default_rng(0).permutation(n)
+    flops = 0
+    t0 = time.perf_counter()
+    done = []
+    for j in order:
+        a = int(inp.anchors[j])
+        OA.forward(p, blocks=[j])
+        flops += 4 * w.head_dim * w.n_q_heads * w.block * (a + w.block)
+        if backward:
+            O, L = OA.forward(p, blocks=[j])
+            OA.backward(p, f64(inp.do), O=O, LSE=L, blocks=[j])
+            flops += 10 * w.head_dim * w.n_q_heads * w.block * (a + w.block)
+        done.append(int(j))
+        if time.perf_counter() - t0 > budget_s:
+            break
+    dt = time.perf_counter() - t0
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        cores = os.cpu_count()
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": int(cores), "kind": "oracle",
+            "sample": f"{len(done)} of {n} draft blocks (all {w.n_q_heads} heads{', fwd+bwd' if backward else ', fwd'}), "
+                      f"{dt:.1f} s float64 NumPy on the host"}
+
+
+def run_reference(args):
+    world, rank, _ = dist_setup(args)
+    if rank != 0:
+        return
+    w = W.get(args.workload)
+    inp = W.make_inputs(w)
+    vals = []
+    budget = args.ref_budget if args.ref_budget else max(1.0, 150.0 / (args.warmup + args.steps))
+    for i in range(args.warmup + args.steps):
+        r = cpu_oracle_sample(inp, budget, w.backward)
+        if i >= args.warmup:
+            vals.append(r["value"])
+    value = statistics.mean(vals)
+    r["value"] = value
+    line = {"impl": "reference", "metric": "useful block-sparse attention TFLOP/s (fwd+bwd)" if w.backward else
+            "useful block-sparse attention TFLOP/s (fwd)", "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name}, "cpu_baseline": r,
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line))
+
+
+def run_ours(args):
+    from split_kv_lse_splitkv_b200 import SplitKV, splitkv_attn_fwd
+
+    world, rank, local = dist_setup(args)
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    w = W.get(args.workload)
+    inp = W.make_inputs(w)
+    counts = [int(inp.anchor_off[i + 1] - inp.anchor_off[i]) for i in range(len(w.seq_lens))]
+    skv = SplitKV(w.seq_lens, counts, w.n_q_heads, w.n_kv_heads, w.head_dim, w.block, w.chunk, w.key_tile, w.scale,
+                  w.torch_dtype, n_workers=w.n_workers, device=device)
+    host = {k: getattr(inp, k) for k in ("q", "k", "v", "kb", "vb", "anchors")}
+    if w.backward:
+        host["do"] = inp.do
+    dev = {k: t.to(device) for k, t in host.items()}
+    Nq, Hq, d = inp.q.shape
+    o = torch.empty(Nq, Hq, d, dtype=w.torch_dtype, device=device)
+    lse = torch.empty(Nq, Hq, dtype=torch.float32, device=device)
+    grads = None
+    if w.backward:
+        f = dict(dtype=torch.float32, device=device)
+        grads = (torch.empty(inp.q.shape, **f), torch.empty(inp.k.shape, **f), torch.empty(inp.v.shape, **f),
+                 torch.empty(inp.kb.shape, **f), torch.empty(inp.vb.shape, **f))
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=device)
+    stream = torch.cuda.current_stream(device)
+    ev_fwd = []
+
+    def step(d, time_fwd=False):
+        skv.plan(d["anchors"], stream)
+        if time_fwd:
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+        skv.attn_fwd(d["q"], d["k"], d["v"], d["anchors"], stream=stream)
+        if time_fwd:
+            e1.record(stream)
+            ev_fwd.append((e0, e1))
+        skv.lse_merge(d["q"], d["kb"], d["vb"], d["anchors"], o, lse, stream=stream)
+        if w.backward:
+            skv.backward(d["q"], d["k"], d["v"], d["kb"], d["vb"], o, lse, d["do"], d["anchors"], grads, stream=stream)
+
+    launches_per_step = 3 + 3 + 1 + 1 + (4 if w.backward else 0)  # cost, plan, fwd, merge, bwd kernels
+    for _ in range(args.warmup):
+        step(dev)
+    torch.cuda.synchronize(device)
+    skv.check_status()
+
+    # ---- device-timed region
+    evs = []
+    barrier(world)
+    torch.cuda.synchronize(device)
+    wall0 = time.perf_counter()
+    with ClockSampler(local) as clocks:
+        for _ in range(args.steps):
+            flush.fill_(1.0)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            step(dev, time_fwd=True)
+            e1.record(stream)
+            evs.append((e0, e1))
+        torch.cuda.synchronize(device)
+    barrier(world)
+    wall = time.perf_counter() - wall0
+    ms = sum(a.elapsed_time(b) for a, b in evs) / len(evs)
+    fwd_ms = sum(a.elapsed_time(b) for a, b in ev_fwd) / len(ev_fwd)
+    ms_max = max_over_ranks(ms, world, device)
+    skv.check_status()
+
+    # ---- end to end through the public API with host buffers
+    pinned = {k: t.pin_memory() for k, t in host.items()}
+    o_host = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+    lse_host = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in pinned.values())
+    d2h = o_host.numel() * o_host.element_size() + lse_host.numel() * lse_host.element_size()
+    if w.backward:
+        d2h = sum(g.numel() * g.element_size() for g in grads)
+    dev2 = {k: torch.empty_like(t) for k, t in dev.items()}
+    grads_host = [torch.empty(g.shape, dtype=g.dtype).pin_memory() for g in grads] if w.backward else []
+
+    def e2e_step():
+        for k, t in pinned.items():
+            dev2[k].copy_(t, non_blocking=True)
+        step(dev2)
+        if w.backward:
+            for gh, g in zip(grads_host, grads):
+                gh.copy_(g, non_blocking=True)
+        else:
+            o_host.copy_(o, non_blocking=True)
+            lse_host.copy_(lse, non_blocking=True)
+
+    for _ in range(max(1, args.warmup)):
+        e2e_step()
+    torch.cuda.synchronize(device)
+    barrier(world)
+    e_evs = []
+    for _ in range(args.steps):
+        flush.fill_(1.0)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        e2e_step()
+        e1.record(stream)
+        e_evs.append((e0, e1))
+    torch.cuda.synchronize(device)
+    e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in e_evs) / len(e_evs), world, device)
+
+    flops, fwd_kernel_flops = useful_flops(inp, w.backward)
+    value = world * flops / (ms_max * 1e-3) / 1e12
+    pk, src = peaks()
+    peak = float(pk["bf16_tflops"])
+    achieved = fwd_kernel_flops / (fwd_ms * 1e-3) / 1e12
+    load = skv.load.cpu().double()
+    predicted_imb = float(load.max() / load.mean() - 1.0) if load.sum() > 0 else 0.0
+    csum = clocks.summary()
+
+    if rank == 0:
+        cpu = None
+        if world == 1 and not args.no_cpu_baseline:
+            cpu = cpu_oracle_sample(inp, args.ref_budget or 10.0, w.backward)
+        line = {
+            "metric": "useful block-sparse attention TFLOP/s (fwd+bwd)" if w.backward else
+                      "useful block-sparse attention TFLOP/s (fwd)",
+            "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms_max, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16" if w.dtype == "bf16" else "f32", "data": "synthetic",
+            "config": {"workload": w.name, "seq_lens": list(w.seq_lens), "anchors": counts,
+                       "heads": f"{w.n_q_heads}q/{w.n_kv_heads}kv", "head_dim": w.head_dim, "chunk": w.chunk,
+                       "queues": skv.n_workers, "l2": "flushed (256 MB write) before every timed step",
+                       "parallelism": f"replicas x{world}"},
+            "roofline": {"bound": "tensor", "kernel": "fwd_tc_kernel", "achieved": achieved, "peak": peak,
+                         "unit": "TFLOP/s", "frac": achieved / peak, "peak_source": f"{src} bf16 dense (burst)",
+                         "traffic": None, "kernel_ms": fwd_ms},
+            "imbalance": {"predicted_lpt": predicted_imb},
+            "clocks": csum,
+            "e2e": {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": launches_per_step * args.steps,
+            "wall_s": wall,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line))
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="drafter_s32k", choices=sorted(W.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--ref-budget", type=float, default=0.0,
+                    help="seconds of CPU work per oracle sample (default: ~150 s spread over all reference steps)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,183 @@
+/*
+ * splitkv.h — C ABI of the Split-KV hot path on one GPU (sm_100a).
+ *
+ * Operation (Split-KV: Efficient Context Parallelism for Training Diffusion Drafters, Abstract):
+ * the exact block-sparse cross-attention of a short set of anchor-sampled draft queries over a
+ * long context. Each anchor a opens a draft block of `block` queries; every query of that block
+ * attends bidirectionally to the context keys [0, a) of its sample plus the block's own `block`
+ * keys (Kb/Vb). The context K/V is cut into chunks of `chunk` keys; each chunk yields a
+ * query-sized partial output O_c plus a per-row log-sum-exp LSE_c, and the partials are merged
+ * exactly: L = log sum_c exp(LSE_c), O = sum_c exp(LSE_c - L) O_c. A cost-aware
+ * longest-processing-time-first (LPT) planner assigns the (chunk, kv head, block) work items,
+ * weighted by their realized cost (visible key tiles), to per-worker queues — here the workers
+ * are the SMs of one GPU.
+ *
+ * Conventions for every entry point
+ *   - The caller owns every buffer. The library never allocates device or host memory and never
+ *     synchronizes the host with the device. All work is enqueued on `stream` (a cudaStream_t
+ *     passed as void*; NULL = legacy default stream).
+ *   - Pointers named *_d and the tensor arguments are DEVICE pointers; `problem` and the arrays it
+ *     points to are HOST memory, read only during the call.
+ *   - Tensors are dense, row-major, innermost dimension last, 16-byte aligned.
+ *       q, o, dout          [Nq, Hq, d]      Nq = block * total anchors; rows block*j .. block*j+block-1
+ *                                            belong to global block j (the j-th anchor over all samples)
+ *       k, v, dk, dv        [sum S, Hkv, d]  samples packed one after another
+ *       kb, vb, dkb, dvb    [Nq, Hkv, d]     each block's own keys / values
+ *       lse                 [Nq, Hq]         float32, natural log
+ *     Query head h reads kv head h / (Hq/Hkv).
+ *   - Return value: SPLITKV_OK, or a negative code detected on the host BEFORE anything is
+ *     enqueued (nothing was launched), or SPLITKV_ECUDA if a launch failed. Errors that only the
+ *     device can see (bad anchors, costs out of range, an in-kernel wait that ran out) are ORed into
+ *     the device status word `status_d` (int32, caller zeroes it once); every kernel reads it first
+ *     and skips its work if it is already non-zero. Nothing traps.
+ */
+#ifndef SPLITKV_H
+#define SPLITKV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Host-side return codes. */
+#define SPLITKV_OK 0
+#define SPLITKV_EINVAL (-1)       /* null pointer, bad size, misaligned tensor, bad problem    */
+#define SPLITKV_EUNSUPPORTED (-2) /* well-formed but not supported (dtype / head_dim / shape)  */
+#define SPLITKV_ECUDA (-3)        /* a CUDA runtime or driver call failed                      */
+#define SPLITKV_ENOSPACE (-4)     /* workspace smaller than splitkv_workspace_size()           */
+
+/* Bits of the device status word. */
+#define SPLITKV_DEV_ANCHOR_ORDER 0x1 /* anchors of a sample not strictly ascending                 */
+#define SPLITKV_DEV_ANCHOR_RANGE 0x2 /* an anchor outside [block, S)                               */
+#define SPLITKV_DEV_BAD_COST 0x4     /* planner input: a cost outside [1, max_cost] or too many items */
+#define SPLITKV_DEV_BAD_PLAN 0x8     /* a queue entry or item id out of range                      */
+#define SPLITKV_DEV_TIMEOUT 0x10     /* an in-kernel wait passed its time limit; the kernel returned */
+
+/* Element types of q, k, v, kb, vb, o, dout. Accumulation is always float32. */
+#define SPLITKV_F32 0
+#define SPLITKV_BF16 1
+
+/* Largest batch (number of samples) one problem may hold. */
+#define SPLITKV_MAX_BATCH 64
+
+/* Flags of splitkv_attn_fwd. */
+#define SPLITKV_FWD_DEFAULT 0 /* bf16 with head_dim 128: tcgen05/TMEM/TMA kernel; else SIMT fp32 */
+#define SPLITKV_FWD_SIMT 1    /* force the CUDA-core kernel (any dtype): an independent GPU cross-check */
+
+/* Problem description (host memory). */
+typedef struct {
+    int32_t batch;              /* samples B, 1..SPLITKV_MAX_BATCH                                */
+    const int64_t *seq_len;     /* host [B]: context length S_s >= 1                               */
+    const int32_t *anchor_off;  /* host [B+1]: sample s owns anchors[anchor_off[s] .. anchor_off[s+1]) */
+    int32_t n_q_heads;          /* Hq                                                               */
+    int32_t n_kv_heads;         /* Hkv, divides Hq                                                  */
+    int32_t head_dim;           /* d: 128 for bf16; 8..128 (multiple of 4) for f32                  */
+    int32_t block;              /* queries per draft block (16)                                     */
+    int32_t chunk;              /* context chunk C, a multiple of key_tile, chunk/key_tile <= 64    */
+    int32_t key_tile;           /* Tk, the key tile of the cost model (128 in every workload)       */
+    float scale;                /* score scale, normally 1/sqrt(d)                                  */
+    int32_t dtype;              /* SPLITKV_F32 or SPLITKV_BF16                                      */
+} splitkv_problem;
+
+/* Derived sizes of a problem. */
+typedef struct {
+    int64_t n_items_max;    /* every (sample, chunk, kv head, block) item, visible or not           */
+    int64_t n_chunks;       /* sum_s ceil(S_s / chunk): length of chunk_cost_d                       */
+    int64_t n_queries;      /* Nq                                                                     */
+    int64_t total_keys;     /* sum_s S_s                                                              */
+    int64_t n_blocks;       /* total anchors                                                          */
+    int64_t o_part_elems;   /* float32 elements of o_part: n_items_max * block*G * d                  */
+    int64_t lse_part_elems; /* float32 elements of lse_part: n_items_max * block*G                    */
+    int32_t max_cost;       /* chunk / key_tile: the largest item cost                                */
+    int32_t rows_per_item;  /* block * G: query rows of one item (its query tile)                     */
+} splitkv_sizes;
+
+/* Fill `out` for `problem`. Returns SPLITKV_EINVAL / SPLITKV_EUNSUPPORTED for a bad problem. */
+int splitkv_query(const splitkv_problem *problem, splitkv_sizes *out);
+
+/* Bytes of scratch that splitkv_cost, splitkv_plan_lpt and splitkv_attn_bwd need for this problem
+ * with `n_workers` queues (0 on a bad problem). One buffer of this size serves every call. */
+size_t splitkv_workspace_size(const splitkv_problem *problem, int32_t n_workers);
+
+/* Human-readable text of a host return code (static storage). */
+const char *splitkv_strerror(int code);
+
+/*
+ * Realized cost pass (Split-KV paper, Abstract: chunks are weighted by the attention work they
+ * actually incur). Validates the anchors (strictly ascending per sample, each in [block, S)) and, for every
+ * item (s, c, g, b) — sample, context chunk, kv head, block — counts the key tiles of chunk c that
+ * hold at least one key the block sees: cost = ceil(clamp(a_b - c*C, 0, min(C, S - c*C)) / Tk).
+ * Items of cost 0 are dropped; the others are written in ascending item index
+ *   id = base_s + (c*Hkv + g)*n_blocks_s + b     (base_s = items of earlier samples)
+ * to item_id_d[0..n) and item_cost_d[0..n), with n stored to *n_items_d (device int32).
+ * chunk_cost_d[n_chunks] (int64, sample-major) receives the summed cost of each chunk's items.
+ * Buffers: anchors_d int32[n_blocks]; item_id_d, item_cost_d int32[n_items_max].
+ */
+int splitkv_cost(const splitkv_problem *problem, const int32_t *anchors_d, int32_t *item_id_d,
+                 int32_t *item_cost_d, int64_t *chunk_cost_d, int32_t *n_items_d, int32_t *status_d,
+                 void *workspace_d, size_t workspace_bytes, void *stream);
+
+/*
+ * Cost-aware LPT planner (Split-KV paper, Abstract, and its table of
+ * context-parallel methods, load-balancing column). Items 0..n-1 (n = *n_items_d <= max_items) with costs
+ * item_cost_d[] in [1, max_cost] are taken in order of (cost descending, index ascending) and each
+ * is given to the worker with the least (load, worker index); loads start at 0. Outputs:
+ *   item_worker_d int32[max_items]   worker of each item
+ *   queue_off_d   int32[n_workers+1] CSR offsets; queue_items_d int32[max_items] lists each
+ *                                    worker's items in assignment order
+ *   load_d        int64[n_workers]   summed cost per worker
+ * The result equals the sequential greedy bit for bit; it is computed one equal-cost run at a time.
+ */
+int splitkv_plan_lpt(const int32_t *item_cost_d, const int32_t *n_items_d, int32_t max_items,
+                     int32_t max_cost, int32_t n_workers, int32_t *item_worker_d, int32_t *queue_off_d,
+                     int32_t *queue_items_d, int64_t *load_d, int32_t *status_d, void *workspace_d,
+                     size_t workspace_bytes, void *stream);
+
+/*
+ * Chunk-partial forward (Split-KV paper, Abstract: the method is exact and
+ * exchanges only tensors the size of the query set). One persistent
+ * CTA per worker walks its queue; for each item (s, c, g, b) it computes, over the keys of chunk c
+ * that block b sees, the chunk-local softmax of s = scale * q.k for the block*G query rows
+ * (r = i*G + hl: query i of the block, query head g*G + hl) and writes
+ *   o_part  [n_items_max][d/4][block*G][4]  float32: O_c = sum softmax * v, normalised
+ *   lse_part[n_items_max][block*G]          float32: LSE_c = log sum exp(s), natural log
+ * at the item's global index. Entries of items that are not visible are not written.
+ * item_id_d, queue_off_d and queue_items_d come from splitkv_cost and splitkv_plan_lpt.
+ * flags: SPLITKV_FWD_DEFAULT or SPLITKV_FWD_SIMT.
+ */
+int splitkv_attn_fwd(const splitkv_problem *problem, const void *q, const void *k, const void *v,
+                     const int32_t *anchors_d, const int32_t *item_id_d, const int32_t *queue_off_d,
+                     const int32_t *queue_items_d, int32_t n_workers, float *o_part, float *lse_part,
+                     int32_t *status_d, int32_t flags, void *stream);
+
+/*
+ * Exact log-sum-exp merge (Split-KV paper, Abstract: exactness with query-sized exchange). For each
+ * block and query head it adds the block's own-keys partial (the `block` rows of kb/vb at the kv
+ * head) to the visible chunk partials c < ceil(a/C) and writes
+ *   L = log sum exp(LSE_c), O = sum exp(LSE_c - L) O_c
+ * to o [Nq, Hq, d] (problem dtype) and lse [Nq, Hq] (float32, natural log).
+ */
+int splitkv_lse_merge(const splitkv_problem *problem, const float *o_part, const float *lse_part,
+                      const void *q, const void *kb, const void *vb, const int32_t *anchors_d, void *o,
+                      float *lse, int32_t *status_d, void *stream);
+
+/*
+ * Backward of the same attention (Split-KV paper, title and Abstract: the method trains diffusion
+ * drafters). Recomputes P = exp(s - LSE) from the stored lse, with D = rowsum(dout * o):
+ *   dV_j += P dO,  dS = P (dO.v_j - D),  dQ += scale dS k_j,  dK_j += scale dS q
+ * for the context keys and the block's own keys. Outputs are float32 and are overwritten:
+ *   dq [Nq, Hq, d], dk, dv [sum S, Hkv, d], dkb, dvb [Nq, Hkv, d].
+ * Needs splitkv_workspace_size() bytes of workspace.
+ */
+int splitkv_attn_bwd(const splitkv_problem *problem, const void *q, const void *k, const void *v,
+                     const void *kb, const void *vb, const void *o, const float *lse, const void *dout,
+                     const int32_t *anchors_d, float *dq, float *dk, float *dv, float *dkb, float *dvb,
+                     int32_t *status_d, void *workspace_d, size_t workspace_bytes, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SPLITKV_H */

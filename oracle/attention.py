@@ -1,9 +1,10 @@
 """Float64 CPU oracle of the anchor-block cross-attention (test infrastructure only).
 
 Source: *Split-KV: Efficient Context Parallelism for Training Diffusion Drafters*,
-Abstract. Training builds compact draft queries by anchor sampling and runs
-cross-attention with a block-sparse mask over a much longer context; Split-KV is
-*exact* and keeps K/V shards local, exchanging only query-sized tensors per layer.
+Abstract. A diffusion drafter is trained on a few draft blocks, each opened at a
+sampled anchor position, whose queries cross-attend to a far longer context under
+a block-sparse mask. Split-KV computes this attention without approximation while
+K/V stay where they are; what moves between workers has the size of the queries.
 
 Readings (the pages do not spell these out):
 
@@ -200,25 +201,30 @@ def merge_partials(p: Problem, parts) -> Tuple[np.ndarray, np.ndarray]:
 # Backward: gradients of the same definition.
 # ---------------------------------------------------------------------------
 def backward(p: Problem, do: np.ndarray, O: Optional[np.ndarray] = None,
-             LSE: Optional[np.ndarray] = None):
+             LSE: Optional[np.ndarray] = None, blocks: Optional[Iterable[int]] = None):
     """Gradients of ``sum(O * dO)`` w.r.t. Q, K, V, Kb, Vb.
 
     With ``P = exp(s - LSE)`` (the softmax of each row over its visible keys),
     ``dV_j += P_j dO``, ``dP_j = dO . v_j``, ``D = sum_d dO * O``,
     ``dS_j = P_j (dP_j - D)``, ``dQ = scale sum_j dS_j k_j``,
     ``dK_j += scale dS_j q`` — the chain rule through the softmax. ``O`` and
-    ``LSE`` default to this oracle's own forward. Returns
+    ``LSE`` default to this oracle's own forward. ``blocks`` restricts the sum to
+    some global block indices (then dK/dV hold only their contributions), for
+    sampled checks at full size. Returns
     ``(dQ [Nq,Hq,d], dK [sum S,Hkv,d], dV, dKb [Nq,Hkv,d], dVb)``.
     """
     do = np.asarray(do, np.float64)
+    want = None if blocks is None else set(int(b) for b in blocks)
     if O is None or LSE is None:
-        O, LSE = forward(p)
+        O, LSE = forward(p, blocks=want)
     dQ = np.zeros_like(p.q)
     dK = np.zeros_like(p.k)
     dV = np.zeros_like(p.v)
     dKb = np.zeros_like(p.kb)
     dVb = np.zeros_like(p.vb)
     for s, j, a in p.blocks():
+        if want is not None and j not in want:
+            continue
         r = p.rows(j)
         k0 = int(p.key_off[s])
         for h in range(p.Hq):

@@ -1,10 +1,11 @@
 """Integer oracle of the realized chunk cost and the cost-aware LPT plan (test infrastructure only).
 
 Source: *Split-KV: Efficient Context Parallelism for Training Diffusion Drafters*,
-Abstract: the global query view lets a cost-aware longest-processing-time-first
-(LPT) strategy balance context K/V chunks by their realized attention cost, a
-requirement that is nonlinear and sample-dependent because of anchor sampling.
-Table 1 of the same page lists "Cost-aware LPT" as Split-KV's load balancing.
+Abstract. Since every worker knows all draft queries, the work of each context
+chunk can be counted before attention runs, and a longest-processing-time-first
+(LPT) greedy places chunks by that count; with anchor sampling the count changes
+from sample to sample and is not linear in the chunk's position.
+The page's table of context-parallel methods names cost-aware LPT as Split-KV's load balancing.
 
 Readings (the pages give neither the cost unit nor the LPT details):
 

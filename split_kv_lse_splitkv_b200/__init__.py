@@ -1,0 +1,33 @@
+"""Split-KV hot path on one B200: Python binding of the C ABI in ``include/splitkv.h``.
+
+The binding only marshals arguments (device pointers from torch tensors, the
+problem description, the current CUDA stream) into ``libsplitkv.so``; every step
+of the path runs in that library's kernels. Importing it without the built
+library raises ImportError: there is no fallback.
+
+Entry points (same names as the C ABI): :func:`splitkv_query`,
+:func:`splitkv_workspace_size`, :func:`splitkv_cost`, :func:`splitkv_plan_lpt`,
+:func:`splitkv_attn_fwd`, :func:`splitkv_lse_merge`, :func:`splitkv_attn_bwd`.
+:class:`SplitKV` strings them together with torch-allocated buffers.
+"""
+from .binding import (  # noqa: F401
+    DEV_ANCHOR_ORDER,
+    DEV_ANCHOR_RANGE,
+    DEV_BAD_COST,
+    DEV_BAD_PLAN,
+    DEV_TIMEOUT,
+    FWD_DEFAULT,
+    FWD_SIMT,
+    LIB_PATH,
+    SplitKV,
+    SplitKVError,
+    make_problem,
+    splitkv_attn_bwd,
+    splitkv_attn_fwd,
+    splitkv_cost,
+    splitkv_lse_merge,
+    splitkv_plan_lpt,
+    splitkv_query,
+    splitkv_strerror,
+    splitkv_workspace_size,
+)

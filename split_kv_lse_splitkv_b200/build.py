@@ -1,0 +1,76 @@
+"""Build libsplitkv.so (sm_100a) in-tree with nvcc.
+
+    python -m split_kv_lse_splitkv_b200.build [--verbose-ptxas]
+
+Each .cu under csrc/ is compiled to an object in parallel, then linked into
+split_kv_lse_splitkv_b200/libsplitkv.so with the CUDA runtime linked statically,
+so the library has no dependency on a particular libcudart and loads on a
+machine without a GPU (the driver is only needed when a call launches work).
+"""
+from __future__ import annotations
+
+import concurrent.futures
+import os
+import shutil
+import subprocess
+import sys
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+CSRC = os.path.join(HERE, "csrc")
+BUILD = os.path.join(HERE, "_build")
+LIB = os.path.join(HERE, "libsplitkv.so")
+ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
+SOURCES = ["abi.cu", "cost.cu", "plan.cu", "fwd_simt.cu", "fwd_tc.cu", "merge.cu", "bwd.cu"]
+
+
+def nvcc() -> str:
+    for cand in (os.environ.get("NVCC"), "/usr/local/cuda/bin/nvcc", shutil.which("nvcc")):
+        if cand and os.path.exists(cand):
+            return cand
+    raise RuntimeError("nvcc not found")
+
+
+def _newer(target: str, deps) -> bool:
+    if not os.path.exists(target):
+        return False
+    t = os.path.getmtime(target)
+    return all(os.path.getmtime(d) <= t for d in deps)
+
+
+def build(verbose_ptxas: bool = False, force: bool = False) -> str:
+    os.makedirs(BUILD, exist_ok=True)
+    headers = [os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith((".cuh", ".h"))]
+    headers.append(os.path.join(os.path.dirname(HERE), "include", "splitkv.h"))
+    flags = ARCH + ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-fvisibility=hidden",
+                    "-I" + os.path.join(os.path.dirname(HERE), "include")]
+    if verbose_ptxas:
+        flags += ["-Xptxas", "-v"]
+    nv = nvcc()
+
+    def compile_one(src):
+        path = os.path.join(CSRC, src)
+        obj = os.path.join(BUILD, src.replace(".cu", ".o"))
+        if not force and not verbose_ptxas and _newer(obj, [path] + headers):
+            return obj, ""
+        cmd = [nv, *flags, "-c", path, "-o", obj]
+        res = subprocess.run(cmd, capture_output=True, text=True)
+        if res.returncode != 0:
+            raise RuntimeError(f"nvcc failed on {src}:\n{res.stdout}\n{res.stderr}")
+        return obj, res.stderr
+
+    with concurrent.futures.ThreadPoolExecutor(max_workers=len(SOURCES)) as ex:
+        results = list(ex.map(compile_one, SOURCES))
+    if verbose_ptxas:
+        for (obj, log), src in zip(results, SOURCES):
+            print(f"== {src}\n{log}")
+    objs = [o for o, _ in results]
+    if force or verbose_ptxas or not _newer(LIB, objs):
+        cmd = [nv, *ARCH, "-shared", "-cudart", "static", "-o", LIB, *objs]
+        res = subprocess.run(cmd, capture_output=True, text=True)
+        if res.returncode != 0:
+            raise RuntimeError(f"link failed:\n{res.stdout}\n{res.stderr}")
+    return LIB
+
+
+if __name__ == "__main__":
+    print(build(verbose_ptxas="--verbose-ptxas" in sys.argv, force="--force" in sys.argv))

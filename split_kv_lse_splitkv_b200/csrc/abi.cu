@@ -1,0 +1,187 @@
+// C ABI entry points: host-side validation, problem decoding and kernel launches.
+// Every check here runs before anything is enqueued, so a rejected call launches nothing.
+#include <cstring>
+
+#include "common.cuh"
+
+#define SPLITKV_API extern "C" __attribute__((visibility("default")))
+
+namespace splitkv {
+namespace {
+
+bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+// Fill `m` from a host problem; returns SPLITKV_OK or a negative code.
+int build_meta(const splitkv_problem* p, Meta* m) {
+    if (!p || !m) return SPLITKV_EINVAL;
+    std::memset(m, 0, sizeof(Meta));
+    if (p->batch < 1 || p->batch > kMaxBatch || !p->seq_len || !p->anchor_off) return SPLITKV_EINVAL;
+    if (p->n_q_heads < 1 || p->n_kv_heads < 1 || p->n_q_heads % p->n_kv_heads) return SPLITKV_EINVAL;
+    if (p->block < 1 || p->chunk < 1 || p->key_tile < 1 || p->head_dim < 1) return SPLITKV_EINVAL;
+    if (p->chunk % p->key_tile || p->chunk / p->key_tile > kMaxCost) return SPLITKV_EUNSUPPORTED;
+    if (!(p->scale > 0.f) || p->scale != p->scale) return SPLITKV_EINVAL;
+    if (p->dtype != SPLITKV_F32 && p->dtype != SPLITKV_BF16) return SPLITKV_EUNSUPPORTED;
+    if (p->head_dim % 4 || p->head_dim > 128 || p->head_dim < 8) return SPLITKV_EUNSUPPORTED;
+    if (p->dtype == SPLITKV_BF16 && p->head_dim % 8) return SPLITKV_EUNSUPPORTED;
+    if (p->block > 32) return SPLITKV_EUNSUPPORTED;
+    m->batch = p->batch;
+    m->hq = p->n_q_heads;
+    m->hkv = p->n_kv_heads;
+    m->group = p->n_q_heads / p->n_kv_heads;
+    m->d = p->head_dim;
+    m->block = p->block;
+    m->chunk = p->chunk;
+    m->key_tile = p->key_tile;
+    m->rows = p->block * m->group;
+    if (m->rows > 256) return SPLITKV_EUNSUPPORTED;
+    m->scale = p->scale;
+    m->dtype = p->dtype;
+    if (p->anchor_off[0] != 0) return SPLITKV_EINVAL;
+    int64_t items = 0, keys = 0, chunks = 0;
+    for (int s = 0; s < p->batch; ++s) {
+        int64_t S = p->seq_len[s];
+        int32_t nb = p->anchor_off[s + 1] - p->anchor_off[s];
+        if (S < 1 || nb < 0) return SPLITKV_EINVAL;
+        int64_t nc = (S + p->chunk - 1) / p->chunk;
+        m->seq_len[s] = S;
+        m->key_off[s] = keys;
+        m->item_base[s] = items;
+        m->chunk_base[s] = chunks;
+        m->anchor_off[s] = p->anchor_off[s];
+        m->n_chunk_s[s] = (int32_t)nc;
+        if (nc > INT32_MAX) return SPLITKV_EUNSUPPORTED;
+        keys += S;
+        chunks += nc;
+        items += nc * m->hkv * nb;
+    }
+    m->key_off[p->batch] = keys;
+    m->item_base[p->batch] = items;
+    m->chunk_base[p->batch] = chunks;
+    m->anchor_off[p->batch] = p->anchor_off[p->batch];
+    m->n_items = items;
+    m->total_keys = keys;
+    m->n_chunks = chunks;
+    m->n_blocks = p->anchor_off[p->batch];
+    m->n_queries = m->n_blocks * p->block;
+    if (items >= INT32_MAX || m->n_queries * m->hq >= ((int64_t)1 << 40)) return SPLITKV_EUNSUPPORTED;
+    return SPLITKV_OK;
+}
+
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? SPLITKV_OK : SPLITKV_ECUDA; }
+
+}  // namespace
+}  // namespace splitkv
+
+using namespace splitkv;
+
+SPLITKV_API int splitkv_query(const splitkv_problem* problem, splitkv_sizes* out) {
+    Meta m;
+    int rc = build_meta(problem, &m);
+    if (rc) return rc;
+    if (!out) return SPLITKV_EINVAL;
+    out->n_items_max = m.n_items;
+    out->n_chunks = m.n_chunks;
+    out->n_queries = m.n_queries;
+    out->total_keys = m.total_keys;
+    out->n_blocks = m.n_blocks;
+    out->o_part_elems = m.n_items * m.rows * m.d;
+    out->lse_part_elems = m.n_items * m.rows;
+    out->max_cost = m.chunk / m.key_tile;
+    out->rows_per_item = m.rows;
+    return SPLITKV_OK;
+}
+
+SPLITKV_API size_t splitkv_workspace_size(const splitkv_problem* problem, int32_t n_workers) {
+    Meta m;
+    if (build_meta(problem, &m) || n_workers < 1 || n_workers > 1024) return 0;
+    size_t a = cost_workspace(m);
+    size_t b = plan_workspace((int32_t)m.n_items, m.chunk / m.key_tile, n_workers);
+    size_t c = bwd_workspace(m);
+    size_t r = a > b ? a : b;
+    return r > c ? r : c;
+}
+
+SPLITKV_API const char* splitkv_strerror(int code) {
+    switch (code) {
+        case SPLITKV_OK: return "ok";
+        case SPLITKV_EINVAL: return "invalid argument";
+        case SPLITKV_EUNSUPPORTED: return "unsupported problem";
+        case SPLITKV_ECUDA: return "CUDA call failed";
+        case SPLITKV_ENOSPACE: return "workspace too small";
+        default: return "unknown status";
+    }
+}
+
+SPLITKV_API int splitkv_cost(const splitkv_problem* problem, const int32_t* anchors_d, int32_t* item_id_d,
+                             int32_t* item_cost_d, int64_t* chunk_cost_d, int32_t* n_items_d, int32_t* status_d,
+                             void* workspace_d, size_t workspace_bytes, void* stream) {
+    Meta m;
+    int rc = build_meta(problem, &m);
+    if (rc) return rc;
+    if ((m.n_blocks && !anchors_d) || !item_id_d || !item_cost_d || !chunk_cost_d || !n_items_d || !status_d)
+        return SPLITKV_EINVAL;
+    if (!workspace_d || workspace_bytes < cost_workspace(m)) return SPLITKV_ENOSPACE;
+    return cuda_status(launch_cost(m, anchors_d, item_id_d, item_cost_d, chunk_cost_d, n_items_d, status_d,
+                                   workspace_d, (cudaStream_t)stream));
+}
+
+SPLITKV_API int splitkv_plan_lpt(const int32_t* item_cost_d, const int32_t* n_items_d, int32_t max_items,
+                                 int32_t max_cost, int32_t n_workers, int32_t* item_worker_d, int32_t* queue_off_d,
+                                 int32_t* queue_items_d, int64_t* load_d, int32_t* status_d, void* workspace_d,
+                                 size_t workspace_bytes, void* stream) {
+    if (max_items < 0 || max_cost < 1 || max_cost > kMaxCost || n_workers < 1 || n_workers > 1024)
+        return SPLITKV_EINVAL;
+    if (!item_cost_d || !n_items_d || !item_worker_d || !queue_off_d || !queue_items_d || !load_d || !status_d)
+        return SPLITKV_EINVAL;
+    if (!workspace_d || workspace_bytes < plan_workspace(max_items, max_cost, n_workers)) return SPLITKV_ENOSPACE;
+    return cuda_status(launch_plan(item_cost_d, n_items_d, max_items, max_cost, n_workers, item_worker_d,
+                                   queue_off_d, queue_items_d, load_d, status_d, workspace_d, (cudaStream_t)stream));
+}
+
+SPLITKV_API int splitkv_attn_fwd(const splitkv_problem* problem, const void* q, const void* k, const void* v,
+                                 const int32_t* anchors_d, const int32_t* item_id_d, const int32_t* queue_off_d,
+                                 const int32_t* queue_items_d, int32_t n_workers, float* o_part, float* lse_part,
+                                 int32_t* status_d, int32_t flags, void* stream) {
+    Meta m;
+    int rc = build_meta(problem, &m);
+    if (rc) return rc;
+    if (n_workers < 1 || n_workers > 65535 || (flags & ~SPLITKV_FWD_SIMT)) return SPLITKV_EINVAL;
+    if (!q || !k || !v || !item_id_d || !queue_off_d || !queue_items_d || !o_part || !lse_part || !status_d)
+        return SPLITKV_EINVAL;
+    if (m.n_blocks && !anchors_d) return SPLITKV_EINVAL;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o_part)) return SPLITKV_EINVAL;
+    cudaStream_t st = (cudaStream_t)stream;
+    if (!(flags & SPLITKV_FWD_SIMT) && fwd_tc_supported(m))
+        return cuda_status(launch_fwd_tc(m, q, k, v, anchors_d, item_id_d, queue_off_d, queue_items_d, n_workers,
+                                         o_part, lse_part, status_d, st));
+    return cuda_status(launch_fwd_simt(m, q, k, v, anchors_d, item_id_d, queue_off_d, queue_items_d, n_workers,
+                                       o_part, lse_part, status_d, st));
+}
+
+SPLITKV_API int splitkv_lse_merge(const splitkv_problem* problem, const float* o_part, const float* lse_part,
+                                  const void* q, const void* kb, const void* vb, const int32_t* anchors_d, void* o,
+                                  float* lse, int32_t* status_d, void* stream) {
+    Meta m;
+    int rc = build_meta(problem, &m);
+    if (rc) return rc;
+    if (!o_part || !lse_part || !q || !kb || !vb || !o || !lse || !status_d) return SPLITKV_EINVAL;
+    if (m.n_blocks && !anchors_d) return SPLITKV_EINVAL;
+    if (!aligned16(o_part)) return SPLITKV_EINVAL;
+    return cuda_status(launch_merge(m, o_part, lse_part, q, kb, vb, anchors_d, o, lse, status_d,
+                                    (cudaStream_t)stream));
+}
+
+SPLITKV_API int splitkv_attn_bwd(const splitkv_problem* problem, const void* q, const void* k, const void* v,
+                                 const void* kb, const void* vb, const void* o, const float* lse, const void* dout,
+                                 const int32_t* anchors_d, float* dq, float* dk, float* dv, float* dkb, float* dvb,
+                                 int32_t* status_d, void* workspace_d, size_t workspace_bytes, void* stream) {
+    Meta m;
+    int rc = build_meta(problem, &m);
+    if (rc) return rc;
+    if (!q || !k || !v || !kb || !vb || !o || !lse || !dout || !dq || !dk || !dv || !dkb || !dvb || !status_d)
+        return SPLITKV_EINVAL;
+    if (m.n_blocks && !anchors_d) return SPLITKV_EINVAL;
+    if (!workspace_d || workspace_bytes < bwd_workspace(m)) return SPLITKV_ENOSPACE;
+    return cuda_status(launch_bwd(m, q, k, v, kb, vb, o, lse, dout, anchors_d, dq, dk, dv, dkb, dvb, status_d,
+                                  workspace_d, (cudaStream_t)stream));
+}

@@ -1,0 +1,149 @@
+// Chunk-partial forward on CUDA cores (fp32 FMA), any head_dim <= 128 and any element type.
+// It serves the float32 problems and, for bfloat16 problems, an independent cross-check of the
+// tensor-core kernel. One persistent CTA per worker walks its LPT queue; per item it runs the
+// chunk-local online softmax over key tiles of 32 keys and writes the normalised partial output
+// and its natural-log LSE (Split-KV: Efficient Context Parallelism for Training Diffusion
+// Drafters, Abstract: exact attention from chunk-local, query-sized partials).
+#include "common.cuh"
+#include "scan.cuh"
+
+namespace splitkv {
+
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kBK = 32;  // keys per tile (one per lane in the softmax step)
+
+template <typename T>
+__global__ void __launch_bounds__(kThreads) fwd_simt_kernel(Meta m, const T* __restrict__ q,
+                                                            const T* __restrict__ k, const T* __restrict__ v,
+                                                            const int32_t* __restrict__ anchors,
+                                                            const int32_t* __restrict__ item_id,
+                                                            const int32_t* __restrict__ queue_off,
+                                                            const int32_t* __restrict__ queue_items,
+                                                            float* __restrict__ o_part, float* __restrict__ lse_part,
+                                                            int32_t* __restrict__ status) {
+    extern __shared__ float smem[];
+    if (status_bad(status)) return;
+    const int R = m.rows, d = m.d, G = m.group;
+    const int dp = d + 1;
+    float* Qs = smem;                 // [R][d]
+    float* Os = Qs + R * d;           // [R][d]
+    float* Ks = Os + R * d;           // [kBK][d+1]
+    float* Vs = Ks + kBK * dp;        // [kBK][d]
+    float* Ss = Vs + kBK * d;         // [R][kBK]
+    float* mS = Ss + R * kBK;         // [R]
+    float* lS = mS + R;               // [R]
+    float* aS = lS + R;               // [R]
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+
+    const int32_t q0 = queue_off[blockIdx.x], q1 = queue_off[blockIdx.x + 1];
+    for (int32_t qi = q0; qi < q1; ++qi) {
+        const int32_t kidx = queue_items[qi];
+        const int64_t id = item_id[kidx];
+        if (id < 0 || id >= m.n_items) { raise_status(status, SPLITKV_DEV_BAD_PLAN); return; }
+        const Item it = decode_item(m, id);
+        const int32_t a = anchors[it.j];
+        const int32_t nvis = visible_in_chunk(m, it.s, it.c, a);
+        const int64_t kbase = m.key_off[it.s] + (int64_t)it.c * m.chunk;
+
+        for (int e = tid; e < R * d; e += kThreads) {
+            int r = e / d, dd = e % d;
+            int i = r / G, hl = r % G;
+            int64_t row = (int64_t)m.block * it.j + i;
+            Qs[e] = to_f32(q[(row * m.hq + (int64_t)it.g * G + hl) * d + dd]);
+            Os[e] = 0.f;
+        }
+        for (int r = tid; r < R; r += kThreads) { mS[r] = -INFINITY; lS[r] = 0.f; }
+        __syncthreads();
+
+        for (int32_t t0 = 0; t0 < nvis; t0 += kBK) {
+            const int nk = min(kBK, nvis - t0);
+            for (int e = tid; e < kBK * d; e += kThreads) {
+                int jj = e / d, dd = e % d;
+                float kv = 0.f, vv = 0.f;
+                if (jj < nk) {
+                    int64_t off = ((kbase + t0 + jj) * m.hkv + it.g) * d + dd;
+                    kv = to_f32(k[off]);
+                    vv = to_f32(v[off]);
+                }
+                Ks[jj * dp + dd] = kv;
+                Vs[jj * d + dd] = vv;
+            }
+            __syncthreads();
+            for (int e = tid; e < R * kBK; e += kThreads) {
+                int r = e / kBK, jj = e % kBK;
+                float s = -INFINITY;
+                if (jj < nk) {
+                    float acc = 0.f;
+                    const float* qr = Qs + r * d;
+                    const float* kr = Ks + jj * dp;
+                    for (int dd = 0; dd < d; ++dd) acc = fmaf(qr[dd], kr[dd], acc);
+                    s = acc * m.scale;
+                }
+                Ss[e] = s;
+            }
+            __syncthreads();
+            for (int r = warp; r < R; r += kThreads / 32) {
+                float x = Ss[r * kBK + lane];
+                float mx = warp_reduce_max(x);
+                float m_old = mS[r];
+                float m_new = fmaxf(m_old, mx);
+                float p = (x == -INFINITY) ? 0.f : expf(x - m_new);
+                float sum = warp_reduce_sum(p);
+                Ss[r * kBK + lane] = p;
+                if (lane == 0) {
+                    float alpha = (m_old == -INFINITY) ? 0.f : expf(m_old - m_new);
+                    aS[r] = alpha;
+                    lS[r] = lS[r] * alpha + sum;
+                    mS[r] = m_new;
+                }
+            }
+            __syncthreads();
+            for (int e = tid; e < R * d; e += kThreads) {
+                int r = e / d, dd = e % d;
+                float acc = Os[e] * aS[r];
+                const float* pr = Ss + r * kBK;
+                for (int jj = 0; jj < nk; ++jj) acc = fmaf(pr[jj], Vs[jj * d + dd], acc);
+                Os[e] = acc;
+            }
+            __syncthreads();
+        }
+        // Normalise and store in the [d/4][R][4] tile layout, plus the natural-log LSE.
+        float* op = o_part + id * (int64_t)R * d;
+        for (int e = tid; e < R * d; e += kThreads) {
+            int d4 = e / (R * 4), rem = e % (R * 4);
+            int r = rem / 4, c4 = rem % 4;
+            op[e] = Os[r * d + d4 * 4 + c4] / lS[r];
+        }
+        for (int r = tid; r < R; r += kThreads) lse_part[id * R + r] = mS[r] + logf(lS[r]);
+        __syncthreads();
+    }
+}
+
+template <typename T>
+cudaError_t launch_t(const Meta& m, const void* q, const void* k, const void* v, const int32_t* anchors,
+                     const int32_t* item_id, const int32_t* queue_off, const int32_t* queue_items, int32_t n_workers,
+                     float* o_part, float* lse_part, int32_t* status, cudaStream_t st) {
+    const int R = m.rows, d = m.d;
+    size_t smem = sizeof(float) * ((size_t)2 * R * d + kBK * (d + 1) + kBK * d + R * kBK + 3 * R);
+    cudaError_t e = cudaFuncSetAttribute(fwd_simt_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    fwd_simt_kernel<T><<<n_workers, kThreads, smem, st>>>(m, (const T*)q, (const T*)k, (const T*)v, anchors, item_id,
+                                                          queue_off, queue_items, o_part, lse_part, status);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_fwd_simt(const Meta& m, const void* q, const void* k, const void* v, const int32_t* anchors,
+                            const int32_t* item_id, const int32_t* queue_off, const int32_t* queue_items,
+                            int32_t n_workers, float* o_part, float* lse_part, int32_t* status, cudaStream_t st) {
+    if (m.dtype == SPLITKV_F32)
+        return launch_t<float>(m, q, k, v, anchors, item_id, queue_off, queue_items, n_workers, o_part, lse_part,
+                               status, st);
+    return launch_t<__nv_bfloat16>(m, q, k, v, anchors, item_id, queue_off, queue_items, n_workers, o_part,
+                                   lse_part, status, st);
+}
+
+}  // namespace splitkv

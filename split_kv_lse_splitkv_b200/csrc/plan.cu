@@ -1,0 +1,308 @@
+// Cost-aware LPT planner on the device (Split-KV: Efficient Context Parallelism for Training
+// Diffusion Drafters, Abstract, and its table of context-parallel methods: load balancing by
+// longest-processing-time-first on the realized cost).
+//
+// Definition: items taken in order (cost desc, index asc); each goes to the worker with the
+// least (load, worker index). Computing that greedy one item at a time is a long serial chain, so
+// it is evaluated one equal-cost run at a time, exactly:
+//
+//   Within a run of n items of equal cost w, worker i can absorb items at loads L_i, L_i + w,
+//   L_i + 2w, ...; the greedy always takes the smallest (load, worker) pair still offered, so the
+//   run's picks are the n smallest elements of { (L_i + k*w, i) } in (value, worker) order.
+//   Cut the value axis into windows [V0 + r*w, V0 + (r+1)*w) with V0 = min L. Worker i offers
+//   exactly one element in every window r >= r_i = (L_i - V0) / w, at offset o_i = (L_i - V0) % w,
+//   so inside a window the order is by (o_i, i) — the same order q_i in every window. Windows
+//   below R = max r_i ("catch-up") miss the workers with r_i > r; from window R on, every window
+//   lists all m workers in q order. Hence rank(i, k) = P(r) + pos_i(r) with r = r_i + k, where
+//   P(r) counts the elements of earlier windows and pos_i(r) the workers of window r ahead of i.
+//
+// Launches: (1) per-CTA cost histograms, (2) one CTA walks the runs (cost W..1) and builds, per
+// run, the catch-up element list, the q order and each worker's pick count, then the final loads
+// and queue offsets, (3) one thread per item places it. Every quantity is an integer, so the plan
+// equals the sequential greedy bit for bit.
+#include "common.cuh"
+#include "scan.cuh"
+
+namespace splitkv {
+
+namespace {
+
+constexpr int kThreads = 1024;
+
+struct PlanWs {
+    int32_t* hist;     // [nblk][W+1]: per-CTA counts, then per-CTA start positions in sorted order
+    int32_t* run_n;    // [W+1]
+    int32_t* run_start;
+    int32_t* run_ncatch;
+    int32_t* run_rmax;
+    int32_t* run_qinv;   // [W+1][m]: worker at q position
+    int32_t* run_r;      // [W+1][m]: first window of each worker
+    int32_t* run_qbase;  // [W+1][m]: items the worker got in earlier runs
+    int2* run_catch;     // [W+1][m*W]: (worker, k) of each catch-up rank
+};
+
+__host__ __device__ inline PlanWs carve(void* ws, int32_t max_items, int32_t W, int32_t m, size_t* bytes) {
+    char* p = (char*)ws;
+    size_t off = 0;
+    auto take = [&](size_t n) { char* r = p + off; off = align_up(off + n, 256); return r; };
+    PlanWs w;
+    int32_t nblk = (max_items + kThreads - 1) / kThreads;
+    w.hist = (int32_t*)take(sizeof(int32_t) * (size_t)(nblk > 0 ? nblk : 1) * (W + 1));
+    w.run_n = (int32_t*)take(sizeof(int32_t) * (W + 1));
+    w.run_start = (int32_t*)take(sizeof(int32_t) * (W + 1));
+    w.run_ncatch = (int32_t*)take(sizeof(int32_t) * (W + 1));
+    w.run_rmax = (int32_t*)take(sizeof(int32_t) * (W + 1));
+    w.run_qinv = (int32_t*)take(sizeof(int32_t) * (size_t)(W + 1) * m);
+    w.run_r = (int32_t*)take(sizeof(int32_t) * (size_t)(W + 1) * m);
+    w.run_qbase = (int32_t*)take(sizeof(int32_t) * (size_t)(W + 1) * m);
+    w.run_catch = (int2*)take(sizeof(int2) * (size_t)(W + 1) * m * W);
+    if (bytes) *bytes = off;
+    return w;
+}
+
+__global__ void __launch_bounds__(kThreads) plan_hist_kernel(const int32_t* __restrict__ cost,
+                                                             const int32_t* __restrict__ n_items_d,
+                                                             int32_t max_items, int32_t W, PlanWs ws,
+                                                             int32_t* __restrict__ status) {
+    __shared__ int32_t h[kMaxCost + 1];
+    if (status_bad(status)) return;
+    int32_t n = *n_items_d;
+    if (n < 0 || n > max_items) {
+        if (blockIdx.x == 0 && threadIdx.x == 0) raise_status(status, SPLITKV_DEV_BAD_COST);
+        return;
+    }
+    for (int i = threadIdx.x; i <= W; i += kThreads) h[i] = 0;
+    __syncthreads();
+    int32_t k = blockIdx.x * kThreads + threadIdx.x;
+    if (k < n) {
+        int32_t w = cost[k];
+        if (w < 1 || w > W) raise_status(status, SPLITKV_DEV_BAD_COST);
+        else atomicAdd(&h[w], 1);
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i <= W; i += kThreads) ws.hist[(size_t)blockIdx.x * (W + 1) + i] = h[i];
+}
+
+__global__ void __launch_bounds__(kThreads) plan_runs_kernel(const int32_t* __restrict__ n_items_d,
+                                                             int32_t max_items, int32_t W, int32_t m, PlanWs ws,
+                                                             int32_t* __restrict__ queue_off,
+                                                             int64_t* __restrict__ load_out,
+                                                             int32_t* __restrict__ status) {
+    __shared__ int64_t L[kThreads];
+    __shared__ int32_t qcount[kThreads];
+    __shared__ int32_t rr[kThreads];
+    __shared__ int32_t oo[kThreads];
+    __shared__ int32_t qq[kThreads];
+    __shared__ int32_t total[kMaxCost + 1];
+    __shared__ int32_t start[kMaxCost + 1];
+    __shared__ int32_t cnt_r[kMaxCost + 2];
+    __shared__ int32_t P[kMaxCost + 2];
+    __shared__ int64_t red64[32];
+    __shared__ int32_t red32[33];
+    __shared__ int32_t bad;
+
+    if (status_bad(status)) return;
+    const int tid = threadIdx.x;
+    const int32_t n = *n_items_d;
+    const int32_t nblk = (n + kThreads - 1) / kThreads;
+
+    // Bucket totals, per-CTA offsets within each bucket, bucket starts (cost descending).
+    for (int w = tid; w <= W; w += kThreads) {
+        int32_t acc = 0;
+        for (int32_t b = 0; b < nblk; ++b) {
+            int32_t c = ws.hist[(size_t)b * (W + 1) + w];
+            ws.hist[(size_t)b * (W + 1) + w] = acc;
+            acc += c;
+        }
+        total[w] = acc;
+    }
+    if (tid == 0) bad = 0;
+    __syncthreads();
+    if (tid == 0) {
+        int32_t s = 0;
+        for (int w = W; w >= 1; --w) { start[w] = s; s += total[w]; }
+        start[0] = s;
+    }
+    __syncthreads();
+    for (int w = tid; w <= W; w += kThreads)
+        for (int32_t b = 0; b < nblk; ++b) ws.hist[(size_t)b * (W + 1) + w] += start[w];
+
+    if (tid < m) { L[tid] = 0; qcount[tid] = 0; }
+    __syncthreads();
+
+    int32_t h_local[kMaxCost + 1];
+    for (int w = W; w >= 1; --w) {
+        const int32_t nw = total[w];
+        if (tid == 0) { ws.run_n[w] = nw; ws.run_start[w] = start[w]; }
+        if (nw == 0) continue;  // uniform across the block
+
+        // V0 = min load.
+        int64_t li = tid < m ? L[tid] : INT64_MAX;
+        int64_t v = warp_reduce_min(li);
+        if ((tid & 31) == 0) red64[tid >> 5] = v;
+        __syncthreads();
+        if (tid < 32) {
+            int64_t x = tid < (kThreads >> 5) ? red64[tid] : INT64_MAX;
+            x = warp_reduce_min(x);
+            if (tid == 0) red64[0] = x;
+        }
+        __syncthreads();
+        const int64_t V0 = red64[0];
+        int32_t ri = 0, oi = 0;
+        if (tid < m) {
+            int64_t dlt = li - V0;
+            ri = (int32_t)(dlt / w);
+            oi = (int32_t)(dlt % w);
+            rr[tid] = ri;
+            oo[tid] = oi;
+        }
+        for (int r = tid; r <= W + 1; r += kThreads) cnt_r[r] = 0;
+        __syncthreads();
+        // q_i: position of worker i in (offset, worker) order; window histogram of r_i.
+        int32_t qi = 0;
+        if (tid < m) {
+            for (int32_t i2 = 0; i2 < m; ++i2) {
+                int32_t o2 = oo[i2];
+                qi += (o2 < oi || (o2 == oi && i2 < tid)) ? 1 : 0;
+            }
+            qq[tid] = qi;
+            if (ri > W) atomicOr(&bad, 1);
+            else atomicAdd(&cnt_r[ri], 1);
+        }
+        int32_t rmax_local = tid < m ? ri : 0;
+        int32_t rm = warp_reduce_max(rmax_local);
+        if ((tid & 31) == 0) red32[tid >> 5] = rm;
+        __syncthreads();
+        if (tid < 32) {
+            int32_t x = tid < (kThreads >> 5) ? red32[tid] : 0;
+            x = warp_reduce_max(x);
+            if (tid == 0) red32[32] = x;
+        }
+        __syncthreads();
+        if (bad) break;
+        const int32_t R = red32[32];  // <= W
+        if (tid == 0) {
+            // P[r] = sum_{r' < r} #{i : r_i <= r'}
+            int32_t le = 0, acc = 0;
+            for (int r = 0; r <= R; ++r) {
+                P[r] = acc;
+                le += cnt_r[r];
+                acc += le;
+            }
+            ws.run_ncatch[w] = P[R] < nw ? P[R] : nw;
+            ws.run_rmax[w] = R;
+        }
+        __syncthreads();
+        if (tid < m) {
+            ws.run_qinv[(size_t)w * m + qi] = tid;
+            ws.run_r[(size_t)w * m + tid] = ri;
+            // Catch-up picks: windows r_i .. R-1.
+            int32_t picks = 0;
+            if (ri < R) {
+                for (int r = 0; r <= R; ++r) h_local[r] = 0;
+                for (int32_t i2 = 0; i2 < m; ++i2)
+                    if (qq[i2] < qi) h_local[rr[i2]]++;
+                int32_t pos = 0;
+                for (int r = 0; r < ri; ++r) pos += h_local[r];
+                for (int r = ri; r < R; ++r) {
+                    pos += h_local[r];
+                    int32_t rank = P[r] + pos;
+                    if (rank >= nw) break;
+                    ws.run_catch[(size_t)w * m * W + rank] = make_int2(tid, r - ri);
+                    ++picks;
+                }
+            }
+            // Steady windows r >= R: rank = P[R] + (r - R) * m + q_i.
+            int32_t extra = nw - P[R] - qi;
+            if (extra > 0) picks += (extra + m - 1) / m;
+            ws.run_qbase[(size_t)w * m + tid] = qcount[tid];
+            qcount[tid] += picks;
+            L[tid] += (int64_t)picks * w;
+        }
+        __syncthreads();
+    }
+    if (bad) {
+        if (tid == 0) raise_status(status, SPLITKV_DEV_BAD_PLAN);
+        return;
+    }
+    __shared__ int32_t sh[33];
+    int32_t c = tid < m ? qcount[tid] : 0;
+    int32_t tot;
+    int32_t ex = block_exclusive_scan<int32_t>(c, sh, &tot);
+    if (tid < m) {
+        queue_off[tid] = ex;
+        load_out[tid] = L[tid];
+    }
+    if (tid == 0) {
+        queue_off[m] = tot;
+        if (tot != n) raise_status(status, SPLITKV_DEV_BAD_PLAN);
+    }
+}
+
+__global__ void __launch_bounds__(kThreads) plan_assign_kernel(const int32_t* __restrict__ cost,
+                                                               const int32_t* __restrict__ n_items_d,
+                                                               int32_t W, int32_t m, PlanWs ws,
+                                                               const int32_t* __restrict__ queue_off,
+                                                               int32_t* __restrict__ item_worker,
+                                                               int32_t* __restrict__ queue_items,
+                                                               int32_t* __restrict__ status) {
+    __shared__ int32_t cnt[32][kMaxCost + 1];
+    if (status_bad(status)) return;
+    const int32_t n = *n_items_d;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    for (int i = tid; i < 32 * (kMaxCost + 1); i += kThreads) (&cnt[0][0])[i] = 0;
+    __syncthreads();
+    const int32_t k = blockIdx.x * kThreads + tid;
+    const bool valid = k < n;
+    const int32_t w = valid ? cost[k] : 0;
+    const unsigned same = __match_any_sync(0xffffffffu, w);
+    const int rank_warp = __popc(same & ((1u << lane) - 1u));
+    if (valid && rank_warp == 0) cnt[warp][w] = __popc(same);
+    __syncthreads();
+    if (!valid || w < 1 || w > W) return;
+    int32_t before = 0;
+    for (int x = 0; x < warp; ++x) before += cnt[x][w];
+    const int32_t j = ws.hist[(size_t)blockIdx.x * (W + 1) + w] - ws.run_start[w] + before + rank_warp;
+    int32_t worker, kk;
+    const int32_t ncatch = ws.run_ncatch[w];
+    if (j < ncatch) {
+        int2 e = ws.run_catch[(size_t)w * m * W + j];
+        worker = e.x;
+        kk = e.y;
+    } else {
+        int32_t jj = j - ncatch;
+        int32_t window = ws.run_rmax[w] + jj / m;
+        worker = ws.run_qinv[(size_t)w * m + (jj % m)];
+        kk = window - ws.run_r[(size_t)w * m + worker];
+    }
+    const int32_t pos = queue_off[worker] + ws.run_qbase[(size_t)w * m + worker] + kk;
+    if (worker < 0 || worker >= m || kk < 0 || pos < queue_off[worker] || pos >= queue_off[worker + 1]) {
+        raise_status(status, SPLITKV_DEV_BAD_PLAN);
+        return;
+    }
+    item_worker[k] = worker;
+    queue_items[pos] = k;
+}
+
+}  // namespace
+
+size_t plan_workspace(int32_t max_items, int32_t max_cost, int32_t n_workers) {
+    size_t bytes = 0;
+    carve(nullptr, max_items, max_cost, n_workers, &bytes);
+    return bytes;
+}
+
+cudaError_t launch_plan(const int32_t* item_cost, const int32_t* n_items, int32_t max_items, int32_t max_cost,
+                        int32_t n_workers, int32_t* item_worker, int32_t* queue_off, int32_t* queue_items,
+                        int64_t* load, int32_t* status, void* ws, cudaStream_t st) {
+    PlanWs w = carve(ws, max_items, max_cost, n_workers, nullptr);
+    int32_t nblk = (max_items + kThreads - 1) / kThreads;
+    if (nblk < 1) nblk = 1;
+    plan_hist_kernel<<<nblk, kThreads, 0, st>>>(item_cost, n_items, max_items, max_cost, w, status);
+    plan_runs_kernel<<<1, kThreads, 0, st>>>(n_items, max_items, max_cost, n_workers, w, queue_off, load, status);
+    plan_assign_kernel<<<nblk, kThreads, 0, st>>>(item_cost, n_items, max_cost, n_workers, w, queue_off,
+                                                  item_worker, queue_items, status);
+    return cudaGetLastError();
+}
+
+}  // namespace splitkv

@@ -1,0 +1,103 @@
+"""Helpers shared by the GPU parity tests: run the CUDA path through the C ABI and compare it
+with the CPU oracle on the same seeded inputs."""
+import numpy as np
+import torch
+
+from oracle import attention as OA
+from oracle import schedule as OS
+from tests._util import anchors_per_sample, oracle_problem, to_np
+
+# Tolerances. The stated bar is max-abs 2e-2 for bf16 and 1e-4 relative (to max|ref|) for fp32.
+# Attention outputs over tens of thousands of keys are small (|O| ~ 1e-2), so an absolute bound
+# alone would pass an all-zero result; every float comparison therefore also bounds the error
+# relative to the tensor's largest reference value (bf16: P and O are rounded to 8-bit mantissas,
+# 2^-9 per rounding; the bound leaves ~10x headroom).
+BF16_ABS = 2e-2
+BF16_REL = 2e-2
+F32_REL = 1e-4
+
+
+def counts_of(inp):
+    off = inp.anchor_off.tolist()
+    return [off[i + 1] - off[i] for i in range(len(off) - 1)]
+
+
+def run_forward(inp, n_workers=None, flags=0, device="cuda"):
+    from split_kv_lse_splitkv_b200 import SplitKV
+    w = inp.workload
+    nw = n_workers if n_workers is not None else w.n_workers
+    skv = SplitKV(w.seq_lens, counts_of(inp), w.n_q_heads, w.n_kv_heads, w.head_dim, w.block, w.chunk, w.key_tile,
+                  w.scale, w.torch_dtype, n_workers=nw, device=device)
+    dev = {k: getattr(inp, k).to(device) for k in ("q", "k", "v", "kb", "vb")}
+    anchors = inp.anchors.to(device)
+    o, lse = skv.forward(dev["q"], dev["k"], dev["v"], dev["kb"], dev["vb"], anchors, flags=flags)
+    torch.cuda.synchronize()
+    return skv, dev, anchors, o, lse
+
+
+def assert_close(name, got, ref, dtype):
+    got = np.asarray(got, np.float64)
+    ref = np.asarray(ref, np.float64)
+    assert got.shape == ref.shape, (name, got.shape, ref.shape)
+    assert np.isfinite(got).all(), f"{name}: non-finite values"
+    err = float(np.max(np.abs(got - ref))) if got.size else 0.0
+    scale = float(np.max(np.abs(ref))) if ref.size else 0.0
+    if dtype == "f32":
+        assert err <= F32_REL * scale + 1e-30, f"{name}: max err {err:.3e} > {F32_REL} x {scale:.3e}"
+    else:
+        assert err <= BF16_ABS, f"{name}: max abs err {err:.3e} > {BF16_ABS}"
+        assert err <= BF16_REL * scale + 1e-30, f"{name}: max err {err:.3e} > {BF16_REL} x max|ref| {scale:.3e}"
+    return err, scale
+
+
+def check_cost_and_plan(skv, inp):
+    """Costs, compacted item list, chunk costs and the LPT plan must equal the oracle bit for bit."""
+    w = inp.workload
+    ids, costs, chunk_costs = OS.costs_closed_form(anchors_per_sample(inp), w.seq_lens, w.chunk, w.key_tile,
+                                                   w.n_kv_heads)
+    n = int(skv.n_items.item())
+    assert n == len(ids)
+    assert skv.item_id[:n].cpu().numpy().tolist() == ids.tolist()
+    assert skv.item_cost[:n].cpu().numpy().tolist() == costs.tolist()
+    assert skv.chunk_cost[:len(chunk_costs)].cpu().numpy().tolist() == chunk_costs.tolist()
+    iw, qo, qi, load = OS.lpt(costs.tolist(), skv.n_workers)
+    assert skv.item_worker[:n].cpu().numpy().tolist() == iw.tolist()
+    assert skv.queue_off.cpu().numpy().tolist() == qo.tolist()
+    assert skv.queue_items[:n].cpu().numpy().tolist() == qi.tolist()
+    assert skv.load.cpu().numpy().tolist() == load.tolist()
+    return ids, costs
+
+
+def check_partials(skv, inp, ids):
+    """Every visible item's partial (O_c, LSE_c) against the oracle's chunk-local softmax."""
+    w = inp.workload
+    p = oracle_problem(inp)
+    parts = OA.chunk_partials(p, w.chunk)
+    O_part, L_part = skv.o_part_view()
+    O_part = O_part.cpu().numpy()
+    L_part = L_part.cpu().numpy()
+    G, R = w.group, w.block * w.group
+    nb = counts_of(inp)
+    base, bases = 0, []
+    for s, S in enumerate(w.seq_lens):
+        bases.append(base)
+        base += (-(-S // w.chunk)) * w.n_kv_heads * nb[s]
+    got_O, ref_O, got_L, ref_L = [], [], [], []
+    off = inp.anchor_off.tolist()
+    for item in ids.tolist():
+        s = max(i for i in range(len(bases)) if bases[i] <= item)
+        local = item - bases[s]
+        b = local % nb[s]
+        c = (local // nb[s]) // w.n_kv_heads
+        g = (local // nb[s]) % w.n_kv_heads
+        j = off[s] + b
+        o_tile = O_part[item].transpose(1, 0, 2).reshape(R, -1)  # [rows, d]
+        for hl in range(G):
+            ref_o, ref_l = parts[(s, c, j, g * G + hl)]
+            rows = [i * G + hl for i in range(w.block)]
+            got_O.append(o_tile[rows])
+            ref_O.append(ref_o)
+            got_L.append(L_part[item][rows])
+            ref_L.append(ref_l)
+    assert_close("O_part", np.stack(got_O), np.stack(ref_O), w.dtype)
+    assert_close("LSE_part", np.stack(got_L), np.stack(ref_L), w.dtype)

@@ -1,0 +1,122 @@
+"""The C ABI on a machine without a GPU: the library loads, exports every entry point that
+include/splitkv.h declares, and rejects bad arguments on the host before any CUDA call."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+import torch
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "splitkv.h")
+
+skv = pytest.importorskip("split_kv_lse_splitkv_b200", reason="libsplitkv.so not built")
+from split_kv_lse_splitkv_b200 import binding as B  # noqa: E402
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(splitkv_\w+)\s*\(", src)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for n in ("splitkv_cost", "splitkv_plan_lpt", "splitkv_attn_fwd", "splitkv_lse_merge", "splitkv_attn_bwd"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported():
+    out = subprocess.run(["nm", "-D", "--defined-only", B.LIB_PATH], capture_output=True, text=True, check=True).stdout
+    exported = set(re.findall(r"\bT (splitkv_\w+)", out))
+    for n in declared_functions():
+        assert n in exported, n
+        assert hasattr(B._lib, n)
+    assert set(B.EXPORTS) == set(declared_functions())
+    # nothing else leaks out of the library's namespace
+    assert all(n.startswith("splitkv_") for n in exported)
+
+
+def prob(**kw):
+    args = dict(seq_lens=[1024], anchor_off=[0, 4], n_q_heads=1, n_kv_heads=1, head_dim=64, block=16, chunk=128,
+                key_tile=128, scale=0.125, dtype=torch.float32)
+    args.update(kw)
+    return B.make_problem(args.pop("seq_lens"), args.pop("anchor_off"), **args)
+
+
+def test_query_sizes():
+    s = B.splitkv_query(prob(seq_lens=[1000, 300], anchor_off=[0, 3, 5], n_q_heads=8, n_kv_heads=2, chunk=256))
+    # items: sample 0: ceil(1000/256)=4 chunks * 2 heads * 3 blocks; sample 1: 2 chunks * 2 * 2
+    assert s.n_items_max == 4 * 2 * 3 + 2 * 2 * 2
+    assert s.n_chunks == 6 and s.n_queries == 80 and s.total_keys == 1300 and s.n_blocks == 5
+    assert s.rows_per_item == 16 * 4 and s.max_cost == 2
+    assert s.o_part_elems == s.n_items_max * 64 * 64 and s.lse_part_elems == s.n_items_max * 64
+    assert B.splitkv_workspace_size(prob(), 4) > 0
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(n_kv_heads=3, n_q_heads=4), B.EINVAL),          # Hkv does not divide Hq
+    (dict(chunk=100), B.EUNSUPPORTED),                    # chunk not a multiple of key_tile
+    (dict(chunk=128 * 65), B.EUNSUPPORTED),               # more than 64 key tiles per chunk
+    (dict(head_dim=130), B.EUNSUPPORTED),
+    (dict(head_dim=6), B.EUNSUPPORTED),
+    (dict(scale=-1.0), B.EINVAL),
+    (dict(seq_lens=[0]), B.EINVAL),
+    (dict(anchor_off=[1, 4]), B.EINVAL),
+    (dict(block=64), B.EUNSUPPORTED),
+])
+def test_bad_problems_are_rejected(kw, code):
+    with pytest.raises(B.SplitKVError) as e:
+        B.splitkv_query(prob(**kw))
+    assert e.value.code == code
+    assert B.splitkv_workspace_size(prob(**kw), 4) == 0
+
+
+def test_bad_batch_and_workers():
+    p = prob()
+    p.struct.batch = 0
+    with pytest.raises(B.SplitKVError):
+        B.splitkv_query(p)
+    assert B.splitkv_workspace_size(prob(), 0) == 0
+    assert B.splitkv_workspace_size(prob(), 2000) == 0
+
+
+def test_null_pointers_and_small_workspace_rejected_before_launch():
+    p = prob()
+    ws = torch.empty(B.splitkv_workspace_size(p, 4), dtype=torch.uint8)
+    fake = torch.empty(64, dtype=torch.int32)  # host memory: never dereferenced, the calls fail first
+    i64 = torch.empty(64, dtype=torch.int64)
+    with pytest.raises(B.SplitKVError) as e:
+        B.splitkv_cost(p, None, fake, fake, i64, fake, fake, ws, stream=0)
+    assert e.value.code == B.EINVAL
+    with pytest.raises(B.SplitKVError) as e:
+        B.splitkv_cost(p, fake, fake, fake, i64, fake, fake, ws[:1], stream=0)
+    assert e.value.code == B.ENOSPACE
+    with pytest.raises(B.SplitKVError) as e:
+        B.splitkv_plan_lpt(fake, fake, 64, 0, 4, fake, fake, fake, i64, fake, ws, stream=0)
+    assert e.value.code == B.EINVAL
+    with pytest.raises(B.SplitKVError) as e:
+        B.splitkv_plan_lpt(fake, fake, 64, 1, 4096, fake, fake, fake, i64, fake, ws, stream=0)
+    assert e.value.code == B.EINVAL
+    with pytest.raises(B.SplitKVError) as e:
+        B.splitkv_attn_fwd(p, None, fake, fake, fake, fake, fake, fake, 4, fake, fake, fake, stream=0)
+    assert e.value.code == B.EINVAL
+    with pytest.raises(B.SplitKVError) as e:  # unknown flag
+        B.splitkv_attn_fwd(p, fake, fake, fake, fake, fake, fake, fake, 4, fake, fake, fake, flags=8, stream=0)
+    assert e.value.code == B.EINVAL
+    with pytest.raises(B.SplitKVError) as e:  # misaligned q
+        B.splitkv_attn_fwd(p, fake[1:], fake, fake, fake, fake, fake, fake, 4, fake, fake, fake, stream=0)
+    assert e.value.code == B.EINVAL
+    with pytest.raises(B.SplitKVError) as e:
+        B.splitkv_lse_merge(p, fake, fake, fake, fake, fake, fake, None, fake, fake, stream=0)
+    assert e.value.code == B.EINVAL
+    with pytest.raises(B.SplitKVError) as e:
+        B.splitkv_attn_bwd(p, *([fake] * 15), ws[:1], stream=0)
+    assert e.value.code == B.ENOSPACE
+
+
+def test_strerror():
+    assert B.splitkv_strerror(0) == "ok"
+    assert "workspace" in B.splitkv_strerror(B.ENOSPACE)
+    assert B.splitkv_strerror(12345) == "unknown status"

@@ -1,0 +1,190 @@
+"""Parity of the CUDA path (through the C ABI) with the float64 CPU oracle on seeded inputs.
+
+Costs and plans bit for bit; partials, O, LSE and gradients within the tolerances in tests/_gpu.py.
+Small cases compare every element and span several key tiles, chunks, ragged tails and queues;
+the full-size workloads compare the integer outputs completely and sampled rows of the floats.
+"""
+import numpy as np
+import pytest
+import torch
+
+import workloads as W
+from oracle import attention as OA
+from tests._gpu import (assert_close, check_cost_and_plan, check_partials, counts_of, run_forward)
+from tests._util import oracle_problem, to_np
+
+pytestmark = pytest.mark.gpu
+
+SIMT = 1
+
+
+def small(name, base, seq_lens, counts, chunk=None, seed=11, **kw):
+    return W.make_inputs(W.scaled(W.get(base), name, seq_lens, counts, chunk=chunk, seed=seed, **kw))
+
+
+def full_check(inp, n_workers, flags=0, partials=True):
+    skv, dev, anchors, o, lse = run_forward(inp, n_workers=n_workers, flags=flags)
+    skv.check_status()
+    ids, _ = check_cost_and_plan(skv, inp)
+    if partials:
+        check_partials(skv, inp, ids)
+    O, L = OA.forward(oracle_problem(inp))
+    dt = inp.workload.dtype
+    assert_close("O", to_np(o), O, dt)
+    assert_close("LSE", to_np(lse), L, dt)
+    return skv, dev, anchors, o, lse
+
+
+def test_tiny_f32_workload():
+    # 1 q / 1 kv head, d = 64, S = 1024, 4 anchors, chunk 128, 4 workers: the whole workload.
+    full_check(W.make_inputs(W.get("tiny_f32")), n_workers=4)
+
+
+@pytest.mark.parametrize("flags", [0, SIMT])
+@pytest.mark.parametrize("n_workers", [3, 148])
+def test_drafter_shape_small(flags, n_workers):
+    # GQA 8 (one 128-row query tile per item), S = 5000: ragged last chunk and ragged key tiles.
+    inp = small("drafter_small", "drafter_s32k", [5000], [7], chunk=1024)
+    full_check(inp, n_workers, flags)
+
+
+@pytest.mark.parametrize("hq,hkv", [(32, 8), (8, 4), (4, 4)])
+def test_other_group_sizes(hq, hkv):
+    # G = 4, 2, 1: 64-, 32- and 16-row query tiles in the 128-row MMA.
+    inp = small("groups", "skewed_s256k", [4096], [9], chunk=2048, n_q_heads=hq, n_kv_heads=hkv)
+    full_check(inp, n_workers=5)
+
+
+def test_anchor_edges():
+    # Anchors on key-tile and chunk boundaries, the smallest and the largest allowed anchor.
+    w = W.scaled(W.get("drafter_s32k"), "edges", [2048], [8], chunk=1024)
+    inp = W.make_inputs(w)
+    inp.anchors = torch.tensor([16, 127, 128, 129, 1023, 1024, 1025, 2047], dtype=torch.int32)
+    full_check(inp, n_workers=4)
+
+
+def test_batch_and_single_worker():
+    inp = small("batch", "train_4x64k", [3000, 2048, 4096], [2, 3, 4], chunk=1024)
+    full_check(inp, n_workers=1)
+
+
+def test_tensor_core_and_simt_kernels_agree():
+    inp = small("agree", "long_s128k", [16384], [12], chunk=2048)
+    _, _, _, o_tc, l_tc = run_forward(inp, n_workers=16, flags=0)
+    _, _, _, o_si, l_si = run_forward(inp, n_workers=16, flags=SIMT)
+    assert_close("O tc vs simt", to_np(o_tc), to_np(o_si), "bf16")
+    assert_close("LSE tc vs simt", to_np(l_tc), to_np(l_si), "bf16")
+
+
+def backward_check(inp, n_workers=4):
+    skv, dev, anchors, o, lse = run_forward(inp, n_workers=n_workers)
+    do = inp.do.to("cuda")
+    grads = skv.backward(dev["q"], dev["k"], dev["v"], dev["kb"], dev["vb"], o, lse, do, anchors)
+    torch.cuda.synchronize()
+    skv.check_status()
+    p = oracle_problem(inp)
+    ref = OA.backward(p, to_np(inp.do))
+    for name, g, r in zip(("dQ", "dK", "dV", "dKb", "dVb"), grads, ref):
+        assert_close(name, to_np(g), r, inp.workload.dtype)
+
+
+def test_backward_bf16_batch():
+    backward_check(small("bwd", "train_4x64k", [3000, 2048, 4096], [2, 3, 4], chunk=1024))
+
+
+def test_backward_f32_tiny():
+    w = W.scaled(W.get("tiny_f32"), "bwd_f32", [1024], [4], backward=True)
+    backward_check(W.make_inputs(w))
+
+
+def test_bad_anchors_raise_device_status():
+    from split_kv_lse_splitkv_b200 import DEV_ANCHOR_ORDER, DEV_ANCHOR_RANGE
+    w = W.scaled(W.get("drafter_s32k"), "bad", [2048], [4], chunk=1024)
+    for anchors, bit in (([100, 50, 300, 400], DEV_ANCHOR_ORDER), ([100, 200, 300, 4096], DEV_ANCHOR_RANGE),
+                         ([3, 200, 300, 400], DEV_ANCHOR_RANGE)):
+        inp = W.make_inputs(w)
+        inp.anchors = torch.tensor(anchors, dtype=torch.int32)
+        skv, *_ = run_forward(inp, n_workers=4)
+        assert skv.status_value() & bit
+
+
+def test_planner_rejects_out_of_range_costs():
+    from split_kv_lse_splitkv_b200 import DEV_BAD_COST, SplitKV
+    skv = SplitKV([4096], [4], 32, 4, 128, chunk=1024, n_workers=8)
+    skv.item_cost[:8] = torch.tensor([1, 2, 3, 99, 1, 1, 1, 1], dtype=torch.int32, device="cuda")
+    skv.n_items.fill_(8)
+    skv.plan_lpt()
+    torch.cuda.synchronize()
+    assert skv.status_value() & DEV_BAD_COST
+
+
+# ------------------------------------------------------------------ full-size workloads
+def sampled_blocks(inp, k=4):
+    n = int(inp.anchor_off[-1])
+    rng = np.random.default_rng(5)
+    picks = {0, n - 1, n // 2} | set(rng.integers(0, n, size=max(0, k - 3)).tolist())
+    return sorted(picks)
+
+
+@pytest.mark.parametrize("name", ["drafter_s32k", "long_s128k", "skewed_s256k"])
+def test_full_size_forward(name):
+    inp = W.make_inputs(W.get(name))
+    skv, dev, anchors, o, lse = run_forward(inp)
+    skv.check_status()
+    check_cost_and_plan(skv, inp)
+    blocks = sampled_blocks(inp)
+    w = inp.workload
+    heads = [0, w.n_q_heads // 2 + 1, w.n_q_heads - 1]
+    O, L = OA.forward(oracle_problem(inp), heads=heads, blocks=blocks)
+    rows = np.concatenate([np.arange(w.block * j, w.block * (j + 1)) for j in blocks])
+    assert_close("O sampled", to_np(o)[rows][:, heads], O[rows][:, heads], w.dtype)
+    assert_close("LSE sampled", to_np(lse)[rows][:, heads], L[rows][:, heads], w.dtype)
+
+
+def test_full_size_training_step():
+    inp = W.make_inputs(W.get("train_4x64k"))
+    w = inp.workload
+    skv, dev, anchors, o, lse = run_forward(inp)
+    do = inp.do.to("cuda")
+    dq, dk, dv, dkb, dvb = skv.backward(dev["q"], dev["k"], dev["v"], dev["kb"], dev["vb"], o, lse, do, anchors)
+    torch.cuda.synchronize()
+    skv.check_status()
+    check_cost_and_plan(skv, inp)
+    p = oracle_problem(inp)
+    off, ko = inp.anchor_off.tolist(), inp.key_off.tolist()
+    # The last block of each sample is the only one that sees keys [a_{n-2}, a_{n-1}); keys at or
+    # beyond its anchor are seen by nobody. Its oracle-only gradients pin those dK/dV rows exactly.
+    lasts = [off[s + 1] - 1 for s in range(len(off) - 1)]
+    blocks = sorted(set(lasts + [0, off[2]]))
+    O, L = OA.forward(p, blocks=blocks)
+    ref = OA.backward(p, to_np(inp.do), O=O, LSE=L, blocks=lasts)
+    rows = np.concatenate([np.arange(w.block * j, w.block * (j + 1)) for j in blocks])
+    assert_close("O sampled", to_np(o)[rows], O[rows], w.dtype)
+    assert_close("LSE sampled", to_np(lse)[rows], L[rows], w.dtype)
+    last_rows = np.concatenate([np.arange(w.block * j, w.block * (j + 1)) for j in lasts])
+    assert_close("dQ sampled", to_np(dq)[last_rows], ref[0][last_rows], w.dtype)
+    assert_close("dKb sampled", to_np(dkb)[last_rows], ref[3][last_rows], w.dtype)
+    assert_close("dVb sampled", to_np(dvb)[last_rows], ref[4][last_rows], w.dtype)
+    anchors_np = inp.anchors.numpy()
+    got_k, ref_k, got_v, ref_v = [], [], [], []
+    for s in range(len(w.seq_lens)):
+        lo = int(anchors_np[off[s + 1] - 2]) if off[s + 1] - off[s] > 1 else 0
+        hi = int(anchors_np[off[s + 1] - 1])
+        sl = slice(ko[s] + lo, ko[s] + hi)
+        got_k.append(to_np(dk)[sl]); ref_k.append(ref[1][sl])
+        got_v.append(to_np(dv)[sl]); ref_v.append(ref[2][sl])
+        # keys nobody sees
+        assert np.all(to_np(dk)[ko[s] + hi:ko[s + 1]] == 0) and np.all(to_np(dv)[ko[s] + hi:ko[s + 1]] == 0)
+    assert_close("dK sampled", np.concatenate(got_k), np.concatenate(ref_k), w.dtype)
+    assert_close("dV sampled", np.concatenate(got_v), np.concatenate(ref_v), w.dtype)
+    # Softmax invariants over every key of each (sample, kv head).
+    dkn, dvn, dkbn, dvbn, don = to_np(dk), to_np(dv), to_np(dkb), to_np(dvb), to_np(inp.do)
+    for s in range(len(w.seq_lens)):
+        r = slice(w.block * off[s], w.block * off[s + 1])
+        for g in range(w.n_kv_heads):
+            tot_k = dkn[ko[s]:ko[s + 1], g].sum(0) + dkbn[r, g].sum(0)
+            mag_k = np.abs(dkn[ko[s]:ko[s + 1], g]).sum(0) + np.abs(dkbn[r, g]).sum(0)
+            assert np.all(np.abs(tot_k) <= 1e-3 * mag_k.max() + 1e-6)
+            want_v = sum(don[r, h].sum(0) for h in range(g * w.group, (g + 1) * w.group))
+            got_v_ = dvn[ko[s]:ko[s + 1], g].sum(0) + dvbn[r, g].sum(0)
+            assert np.allclose(got_v_, want_v, rtol=1e-3, atol=1e-2)

@@ -197,3 +197,14 @@ def test_gradient_invariants():
             want = sum(do[rows, h].sum(0) for h in heads)
             got = dV[ko[s]:ko[s + 1], g].sum(0) + dVb[rows, g].sum(0)
             assert np.allclose(got, want, atol=1e-12)
+
+
+def test_restricted_backward_sums_to_full():
+    inp = tiny(counts=(3, 4))
+    p = oracle_problem(inp)
+    do = to_np(inp.do)
+    full = A.backward(p, do)
+    part_a = A.backward(p, do, blocks=[0, 2, 4, 6])
+    part_b = A.backward(p, do, blocks=[1, 3, 5])
+    for f, x, y in zip(full, part_a, part_b):
+        np.testing.assert_allclose(x + y, f, atol=1e-13)

@@ -5,9 +5,9 @@ method's arithmetic (no mask, cost, softmax or schedule). Both the CPU oracle
 (through the tests) and the CUDA path consume exactly the tensors made here.
 
 Workloads follow the shapes of *Split-KV: Efficient Context Parallelism for
-Training Diffusion Drafters* (Abstract: anchor-sampled draft blocks that
-cross-attend to a much longer context; target/drafter shape table: 32 query
-heads, 4 or 8 kv heads, head dim 128).
+Training Diffusion Drafters* (Abstract: draft blocks opened at sampled anchor
+positions attend to a context far longer than the query set; the table of
+target/drafter shapes: 32 query heads, 4 or 8 kv heads, head dim 128).
 
 Draw order for one workload, from a single CPU ``torch.Generator`` seeded with
 ``seed``: the anchors of every sample (in sample order), then Q, K, V, Kb, Vb
