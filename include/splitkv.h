@@ -104,6 +104,10 @@ size_t splitkv_workspace_size(const splitkv_problem *problem, int32_t n_workers)
 /* Human-readable text of a host return code (static storage). */
 const char *splitkv_strerror(int code);
 
+/* Detail of the most recent failure in this thread (the failing CUDA call and its error name), or ""
+ * if the last call succeeded. Valid until the next call from the same thread. */
+const char *splitkv_last_error(void);
+
 /*
  * Realized cost pass (Split-KV paper, Abstract: chunks are weighted by the attention work they
  * actually incur). Validates the anchors (strictly ascending per sample, each in [block, S)) and, for every

@@ -58,6 +58,7 @@ _SIGS = {
     "splitkv_query": (_i32, [_PP, ctypes.POINTER(Sizes)]),
     "splitkv_workspace_size": (_sz, [_PP, _i32]),
     "splitkv_strerror": (ctypes.c_char_p, [_i32]),
+    "splitkv_last_error": (ctypes.c_char_p, []),
     "splitkv_cost": (_i32, [_PP, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "splitkv_plan_lpt": (_i32, [_vp, _vp, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "splitkv_attn_fwd": (_i32, [_PP, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _vp, _i32, _vp]),
@@ -74,7 +75,12 @@ for _name, (_res, _args) in _SIGS.items():
 class SplitKVError(RuntimeError):
     def __init__(self, code: int, where: str):
         self.code = code
-        super().__init__(f"{where}: {splitkv_strerror(code)} ({code})")
+        detail = splitkv_last_error() if code == ECUDA else ""
+        super().__init__(f"{where}: {splitkv_strerror(code)} ({code})" + (f" [{detail}]" if detail else ""))
+
+
+def splitkv_last_error() -> str:
+    return _lib.splitkv_last_error().decode()
 
 
 def splitkv_strerror(code: int) -> str:

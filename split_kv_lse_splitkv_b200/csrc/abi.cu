@@ -1,5 +1,6 @@
 // C ABI entry points: host-side validation, problem decoding and kernel launches.
 // Every check here runs before anything is enqueued, so a rejected call launches nothing.
+#include <cstdio>
 #include <cstring>
 
 #include "common.cuh"
@@ -7,6 +8,18 @@
 #define SPLITKV_API extern "C" __attribute__((visibility("default")))
 
 namespace splitkv {
+
+static thread_local char g_last_error[256];
+
+cudaError_t note_error(cudaError_t e, const char* what) {
+    if (e != cudaSuccess)
+        std::snprintf(g_last_error, sizeof(g_last_error), "%s: %s (%s)", what, cudaGetErrorName(e),
+                      cudaGetErrorString(e));
+    return e;
+}
+
+void clear_error() { g_last_error[0] = 0; }
+
 namespace {
 
 bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
@@ -67,7 +80,11 @@ int build_meta(const splitkv_problem* p, Meta* m) {
     return SPLITKV_OK;
 }
 
-int cuda_status(cudaError_t e) { return e == cudaSuccess ? SPLITKV_OK : SPLITKV_ECUDA; }
+int cuda_status(cudaError_t e) {
+    if (e == cudaSuccess) return SPLITKV_OK;
+    if (!g_last_error[0]) note_error(e, "kernel launch");
+    return SPLITKV_ECUDA;
+}
 
 }  // namespace
 }  // namespace splitkv
@@ -101,6 +118,8 @@ SPLITKV_API size_t splitkv_workspace_size(const splitkv_problem* problem, int32_
     return r > c ? r : c;
 }
 
+SPLITKV_API const char* splitkv_last_error(void) { return g_last_error; }
+
 SPLITKV_API const char* splitkv_strerror(int code) {
     switch (code) {
         case SPLITKV_OK: return "ok";
@@ -115,6 +134,7 @@ SPLITKV_API const char* splitkv_strerror(int code) {
 SPLITKV_API int splitkv_cost(const splitkv_problem* problem, const int32_t* anchors_d, int32_t* item_id_d,
                              int32_t* item_cost_d, int64_t* chunk_cost_d, int32_t* n_items_d, int32_t* status_d,
                              void* workspace_d, size_t workspace_bytes, void* stream) {
+    clear_error();
     Meta m;
     int rc = build_meta(problem, &m);
     if (rc) return rc;
@@ -129,6 +149,7 @@ SPLITKV_API int splitkv_plan_lpt(const int32_t* item_cost_d, const int32_t* n_it
                                  int32_t max_cost, int32_t n_workers, int32_t* item_worker_d, int32_t* queue_off_d,
                                  int32_t* queue_items_d, int64_t* load_d, int32_t* status_d, void* workspace_d,
                                  size_t workspace_bytes, void* stream) {
+    clear_error();
     if (max_items < 0 || max_cost < 1 || max_cost > kMaxCost || n_workers < 1 || n_workers > 1024)
         return SPLITKV_EINVAL;
     if (!item_cost_d || !n_items_d || !item_worker_d || !queue_off_d || !queue_items_d || !load_d || !status_d)
@@ -142,6 +163,7 @@ SPLITKV_API int splitkv_attn_fwd(const splitkv_problem* problem, const void* q, 
                                  const int32_t* anchors_d, const int32_t* item_id_d, const int32_t* queue_off_d,
                                  const int32_t* queue_items_d, int32_t n_workers, float* o_part, float* lse_part,
                                  int32_t* status_d, int32_t flags, void* stream) {
+    clear_error();
     Meta m;
     int rc = build_meta(problem, &m);
     if (rc) return rc;
@@ -161,6 +183,7 @@ SPLITKV_API int splitkv_attn_fwd(const splitkv_problem* problem, const void* q, 
 SPLITKV_API int splitkv_lse_merge(const splitkv_problem* problem, const float* o_part, const float* lse_part,
                                   const void* q, const void* kb, const void* vb, const int32_t* anchors_d, void* o,
                                   float* lse, int32_t* status_d, void* stream) {
+    clear_error();
     Meta m;
     int rc = build_meta(problem, &m);
     if (rc) return rc;
@@ -175,6 +198,7 @@ SPLITKV_API int splitkv_attn_bwd(const splitkv_problem* problem, const void* q, 
                                  const void* kb, const void* vb, const void* o, const float* lse, const void* dout,
                                  const int32_t* anchors_d, float* dq, float* dk, float* dv, float* dkb, float* dvb,
                                  int32_t* status_d, void* workspace_d, size_t workspace_bytes, void* stream) {
+    clear_error();
     Meta m;
     int rc = build_meta(problem, &m);
     if (rc) return rc;

@@ -83,6 +83,10 @@ __device__ inline bool status_bad(const int32_t* status) {
     return status && *((volatile const int32_t*)status) != 0;
 }
 
+// Records a failure detail for splitkv_last_error() (thread-local) and passes the error through.
+cudaError_t note_error(cudaError_t e, const char* what);
+void clear_error();
+
 // ---- internal launchers (defined in the per-kernel .cu files) ----
 cudaError_t launch_cost(const Meta& m, const int32_t* anchors, int32_t* item_id, int32_t* item_cost,
                         int64_t* chunk_cost, int32_t* n_items, int32_t* status, void* ws, cudaStream_t st);

@@ -24,6 +24,8 @@
 //
 // Every wait is bounded (2 s); on expiry the CTA raises SPLITKV_DEV_TIMEOUT, drains its copies and
 // MMAs in flight, frees TMEM and returns.
+#include <cstdio>
+
 #include "common.cuh"
 #include "sm100.cuh"
 
@@ -117,7 +119,7 @@ __device__ __forceinline__ void cursor_advance(const Meta& m, const int32_t* anc
     cursor_fetch(m, anchors, item_id, queue_items, c, status);
 }
 
-__global__ void __maxnreg__(200)
+__global__ void __launch_bounds__(kThreads, 1)
     fwd_tc_kernel(const __grid_constant__ Meta m, const __grid_constant__ CUtensorMap tmQ,
                   const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                   const int32_t* __restrict__ anchors, const int32_t* __restrict__ item_id,
@@ -336,31 +338,30 @@ __global__ void __maxnreg__(200)
             for (int tt = 0; tt < t.ntiles; ++tt) {
                 if (!mbar_wait(&bars->s_full[k], tile_seq & 1u, abort_flag, kTimeoutNs)) { ok = false; break; }
                 tc_fence_after();
-                float s[128];
+                const int valid = t.nvis - tt * kKeysPerTile;  // keys of this tile the block sees (>= 1)
+                // Pass 1: row max of the visible scores, two 32-column chunks per TMEM wait.
+                float mx = -INFINITY;
+#pragma unroll 1
+                for (int cc = 0; cc < 4; cc += 2) {
+                    uint32_t ra[32], rb[32];
+                    tmem_ld32(tS[k] + lane_off + cc * 32, ra);
+                    tmem_ld32(tS[k] + lane_off + cc * 32 + 32, rb);
+                    tmem_wait_ld();
 #pragma unroll
-                for (int cc = 0; cc < 4; ++cc) {
-                    uint32_t raw[32];
-                    tmem_ld32(tS[k] + lane_off + cc * 32, raw);
-#pragma unroll
-                    for (int u = 0; u < 32; ++u) s[cc * 32 + u] = __uint_as_float(raw[u]);
+                    for (int u = 0; u < 32; ++u) {
+                        const float xa = (cc * 32 + u < valid) ? __uint_as_float(ra[u]) : -INFINITY;
+                        const float xb = (cc * 32 + 32 + u < valid) ? __uint_as_float(rb[u]) : -INFINITY;
+                        mx = fmaxf(mx, fmaxf(xa, xb));
+                    }
                 }
-                tmem_wait_ld();
-                const int valid = t.nvis - tt * kKeysPerTile;
-                if (valid < kKeysPerTile) {
-#pragma unroll
-                    for (int u = 0; u < 128; ++u)
-                        if (u >= valid) s[u] = -INFINITY;
-                }
-                float mx = s[0];
-#pragma unroll
-                for (int u = 1; u < 128; ++u) mx = fmaxf(mx, s[u]);
                 mx *= c;
                 if (tt == 0) {
                     m_used = mx;
                 } else if (mx > m_used + kRescaleLog2) {
+                    // The previous PV of this slot completed before this tile's QK^T was issued.
                     const float alpha = ex2_approx(m_used - mx);
                     l *= alpha;
-#pragma unroll
+#pragma unroll 1
                     for (int cc = 0; cc < 4; ++cc) {
                         uint32_t ov[32];
                         tmem_ld32(tO[k] + lane_off + cc * 32, ov);
@@ -372,13 +373,21 @@ __global__ void __maxnreg__(200)
                     m_used = mx;
                 }
                 const float negm = -m_used;
-#pragma unroll
+                // Pass 2: P = 2^(x - m) in bf16, written over the first 64 columns of S. Chunk cc of S
+                // (columns 32cc..32cc+31) is read before P chunk cc (columns 16cc..16cc+15) is written.
+#pragma unroll 1
                 for (int cc = 0; cc < 4; ++cc) {
+                    uint32_t raw[32];
+                    tmem_ld32(tS[k] + lane_off + cc * 32, raw);
+                    tmem_wait_ld();
                     uint32_t pk[16];
 #pragma unroll
                     for (int u = 0; u < 16; ++u) {
-                        const float p0 = ex2_approx(fmaf(s[cc * 32 + 2 * u], c, negm));
-                        const float p1 = ex2_approx(fmaf(s[cc * 32 + 2 * u + 1], c, negm));
+                        const int k0 = cc * 32 + 2 * u;
+                        const float x0 = (k0 < valid) ? __uint_as_float(raw[2 * u]) : -INFINITY;
+                        const float x1 = (k0 + 1 < valid) ? __uint_as_float(raw[2 * u + 1]) : -INFINITY;
+                        const float p0 = ex2_approx(fmaf(x0, c, negm));
+                        const float p1 = ex2_approx(fmaf(x1, c, negm));
                         l += p0 + p1;
                         __nv_bfloat162 h = __floats2bfloat162_rn(p0, p1);  // .x (low half) = even key
                         pk[u] = *reinterpret_cast<uint32_t*>(&h);
@@ -396,7 +405,7 @@ __global__ void __maxnreg__(200)
             tc_fence_after();
             const float inv_l = 1.f / l;
             float* op = o_part + t.id * (int64_t)R * 128;
-#pragma unroll
+#pragma unroll 1
             for (int cc = 0; cc < 4; ++cc) {
                 uint32_t ov[32];
                 tmem_ld32(tO[k] + lane_off + cc * 32, ov);
@@ -443,7 +452,10 @@ EncodeTiledFn encode_fn() {
 // 3-D bf16 map over [rows][heads][d] with a 128-byte swizzled box {64, box_heads, box_rows}.
 bool make_map(CUtensorMap* map, const void* base, int64_t rows, int heads, int d, int box_heads, int box_rows) {
     EncodeTiledFn fn = encode_fn();
-    if (!fn) return false;
+    if (!fn) {
+        note_error(cudaErrorNotSupported, "cudaGetDriverEntryPoint(cuTensorMapEncodeTiled)");
+        return false;
+    }
     cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)heads, (cuuint64_t)rows};
     cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)heads * d * 2};
     cuuint32_t box[3] = {64u, (cuuint32_t)box_heads, (cuuint32_t)box_rows};
@@ -451,7 +463,13 @@ bool make_map(CUtensorMap* map, const void* base, int64_t rows, int heads, int d
     CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS;
+    if (r != CUDA_SUCCESS) {
+        char what[96];
+        std::snprintf(what, sizeof(what), "cuTensorMapEncodeTiled -> CUresult %d", (int)r);
+        note_error(cudaErrorInvalidValue, what);
+        return false;
+    }
+    return true;
 }
 
 }  // namespace
@@ -471,10 +489,19 @@ cudaError_t launch_fwd_tc(const Meta& m, const void* q, const void* k, const voi
         !make_map(&tv, v, m.total_keys, m.hkv, m.d, 1, kKeysPerTile))
         return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-    if (e != cudaSuccess) return e;
+    if (e != cudaSuccess) return note_error(e, "cudaFuncSetAttribute(fwd_tc_kernel, smem)");
     fwd_tc_kernel<<<n_workers, kThreads, kSmemBytes, st>>>(m, tq, tk, tv, anchors, item_id, queue_off, queue_items,
                                                            o_part, lse_part, status);
-    return cudaGetLastError();
+    e = cudaGetLastError();
+    if (e != cudaSuccess) {
+        cudaFuncAttributes fa;
+        char what[160] = "launch fwd_tc_kernel";
+        if (cudaFuncGetAttributes(&fa, fwd_tc_kernel) == cudaSuccess)
+            std::snprintf(what, sizeof(what), "launch fwd_tc_kernel (regs %d, local %zu B, static smem %zu B, dyn smem %d B)",
+                          fa.numRegs, fa.localSizeBytes, fa.sharedSizeBytes, kSmemBytes);
+        return note_error(e, what);
+    }
+    return cudaSuccess;
 }
 
 }  // namespace splitkv
