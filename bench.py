@@ -228,20 +228,26 @@ def run_ours(args):
                  torch.empty(inp.kb.shape, **f), torch.empty(inp.vb.shape, **f))
     flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=device)
     stream = torch.cuda.current_stream(device)
-    ev_fwd = []
+    phases = {"plan": [], "fwd": [], "merge": [], "bwd": []}
 
-    def step(d, time_fwd=False):
-        skv.plan(d["anchors"], stream)
-        if time_fwd:
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-        skv.attn_fwd(d["q"], d["k"], d["v"], d["anchors"], stream=stream)
-        if time_fwd:
-            e1.record(stream)
-            ev_fwd.append((e0, e1))
-        skv.lse_merge(d["q"], d["kb"], d["vb"], d["anchors"], o, lse, stream=stream)
+    def timed(name, fn, on):
+        if not on:
+            fn()
+            return
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        fn()
+        e1.record(stream)
+        phases[name].append((e0, e1))
+
+    def step(d, time_phases=False):
+        timed("plan", lambda: skv.plan(d["anchors"], stream), time_phases)
+        timed("fwd", lambda: skv.attn_fwd(d["q"], d["k"], d["v"], d["anchors"], stream=stream), time_phases)
+        timed("merge", lambda: skv.lse_merge(d["q"], d["kb"], d["vb"], d["anchors"], o, lse, stream=stream),
+              time_phases)
         if w.backward:
-            skv.backward(d["q"], d["k"], d["v"], d["kb"], d["vb"], o, lse, d["do"], d["anchors"], grads, stream=stream)
+            timed("bwd", lambda: skv.backward(d["q"], d["k"], d["v"], d["kb"], d["vb"], o, lse, d["do"], d["anchors"],
+                                              grads, stream=stream), time_phases)
 
     launches_per_step = 3 + 3 + 1 + 1 + (4 if w.backward else 0)  # cost, plan, fwd, merge, bwd kernels
     for _ in range(args.warmup):
@@ -259,14 +265,15 @@ def run_ours(args):
             flush.fill_(1.0)
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record(stream)
-            step(dev, time_fwd=True)
+            step(dev, time_phases=True)
             e1.record(stream)
             evs.append((e0, e1))
         torch.cuda.synchronize(device)
     barrier(world)
     wall = time.perf_counter() - wall0
     ms = sum(a.elapsed_time(b) for a, b in evs) / len(evs)
-    fwd_ms = sum(a.elapsed_time(b) for a, b in ev_fwd) / len(ev_fwd)
+    phase_ms = {k: (sum(a.elapsed_time(b) for a, b in v) / len(v)) for k, v in phases.items() if v}
+    fwd_ms = phase_ms["fwd"]
     ms_max = max_over_ranks(ms, world, device)
     skv.check_status()
 
@@ -310,8 +317,15 @@ def run_ours(args):
     flops, fwd_kernel_flops = useful_flops(inp, w.backward)
     value = world * flops / (ms_max * 1e-3) / 1e12
     pk, src = peaks()
-    peak = float(pk["bf16_tflops"])
+    if w.dtype == "bf16":
+        roof = {"bound": "tensor", "kernel": "fwd_tc_kernel", "peak": float(pk["bf16_tflops"]),
+                "peak_source": f"{src} bf16 dense (burst)"}
+    else:
+        # fp32 CUDA-core kernel: 148 SMs x 128 FMA lanes x 2 FLOP x 1.965 GHz.
+        roof = {"bound": "alu", "kernel": "fwd_simt_kernel<float>", "peak": 148 * 128 * 2 * 1.965e9 / 1e12,
+                "peak_source": "derived fp32 FFMA peak at max SM clock"}
     achieved = fwd_kernel_flops / (fwd_ms * 1e-3) / 1e12
+    peak = roof["peak"]
     load = skv.load.cpu().double()
     predicted_imb = float(load.max() / load.mean() - 1.0) if load.sum() > 0 else 0.0
     csum = clocks.summary()
@@ -330,9 +344,9 @@ def run_ours(args):
                        "heads": f"{w.n_q_heads}q/{w.n_kv_heads}kv", "head_dim": w.head_dim, "chunk": w.chunk,
                        "queues": skv.n_workers, "l2": "flushed (256 MB write) before every timed step",
                        "parallelism": f"replicas x{world}"},
-            "roofline": {"bound": "tensor", "kernel": "fwd_tc_kernel", "achieved": achieved, "peak": peak,
-                         "unit": "TFLOP/s", "frac": achieved / peak, "peak_source": f"{src} bf16 dense (burst)",
-                         "traffic": None, "kernel_ms": fwd_ms},
+            "roofline": dict(roof, achieved=achieved, unit="TFLOP/s", frac=achieved / peak, traffic=None,
+                             kernel_ms=fwd_ms, algorithmic_flop=fwd_kernel_flops),
+            "phase_ms": phase_ms,
             "imbalance": {"predicted_lpt": predicted_imb},
             "clocks": csum,
             "e2e": {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",

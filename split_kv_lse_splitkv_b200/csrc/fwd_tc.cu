@@ -339,22 +339,35 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!mbar_wait(&bars->s_full[k], tile_seq & 1u, abort_flag, kTimeoutNs)) { ok = false; break; }
                 tc_fence_after();
                 const int valid = t.nvis - tt * kKeysPerTile;  // keys of this tile the block sees (>= 1)
-                // Pass 1: row max of the visible scores, two 32-column chunks per TMEM wait.
-                float mx = -INFINITY;
+                const bool full = valid >= kKeysPerTile;         // only an item's last tile can be partial
+                // Pass 1: row max, 64 columns per TMEM wait; four independent max chains.
+                float mx;
+                {
+                    float m0 = -INFINITY, m1 = -INFINITY, m2 = -INFINITY, m3 = -INFINITY;
 #pragma unroll 1
-                for (int cc = 0; cc < 4; cc += 2) {
-                    uint32_t ra[32], rb[32];
-                    tmem_ld32(tS[k] + lane_off + cc * 32, ra);
-                    tmem_ld32(tS[k] + lane_off + cc * 32 + 32, rb);
-                    tmem_wait_ld();
+                    for (int cc = 0; cc < 4; cc += 2) {
+                        uint32_t ra[32], rb[32];
+                        tmem_ld32(tS[k] + lane_off + cc * 32, ra);
+                        tmem_ld32(tS[k] + lane_off + cc * 32 + 32, rb);
+                        tmem_wait_ld();
+                        if (full) {
 #pragma unroll
-                    for (int u = 0; u < 32; ++u) {
-                        const float xa = (cc * 32 + u < valid) ? __uint_as_float(ra[u]) : -INFINITY;
-                        const float xb = (cc * 32 + 32 + u < valid) ? __uint_as_float(rb[u]) : -INFINITY;
-                        mx = fmaxf(mx, fmaxf(xa, xb));
+                            for (int u = 0; u < 32; u += 4) {
+                                m0 = max3f(m0, __uint_as_float(ra[u]), __uint_as_float(ra[u + 1]));
+                                m1 = max3f(m1, __uint_as_float(ra[u + 2]), __uint_as_float(ra[u + 3]));
+                                m2 = max3f(m2, __uint_as_float(rb[u]), __uint_as_float(rb[u + 1]));
+                                m3 = max3f(m3, __uint_as_float(rb[u + 2]), __uint_as_float(rb[u + 3]));
+                            }
+                        } else {
+#pragma unroll
+                            for (int u = 0; u < 32; ++u) {
+                                if (cc * 32 + u < valid) m0 = fmaxf(m0, __uint_as_float(ra[u]));
+                                if (cc * 32 + 32 + u < valid) m1 = fmaxf(m1, __uint_as_float(rb[u]));
+                            }
+                        }
                     }
+                    mx = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3)) * c;
                 }
-                mx *= c;
                 if (tt == 0) {
                     m_used = mx;
                 } else if (mx > m_used + kRescaleLog2) {
@@ -372,27 +385,45 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     m_used = mx;
                 }
-                const float negm = -m_used;
-                // Pass 2: P = 2^(x - m) in bf16, written over the first 64 columns of S. Chunk cc of S
-                // (columns 32cc..32cc+31) is read before P chunk cc (columns 16cc..16cc+15) is written.
+                // Pass 2: P = 2^(s*c - m) in bf16, written over the first 64 columns of S. S columns
+                // 32cc..32cc+63 are read before P columns 16cc..16cc+31 are written.
+                const uint64_t c2 = f2_pack(c, c), negm2 = f2_pack(-m_used, -m_used);
+                uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll 1
-                for (int cc = 0; cc < 4; ++cc) {
-                    uint32_t raw[32];
-                    tmem_ld32(tS[k] + lane_off + cc * 32, raw);
+                for (int cc = 0; cc < 4; cc += 2) {
+                    uint32_t ra[32], rb[32];
+                    tmem_ld32(tS[k] + lane_off + cc * 32, ra);
+                    tmem_ld32(tS[k] + lane_off + cc * 32 + 32, rb);
                     tmem_wait_ld();
-                    uint32_t pk[16];
+                    if (!full) {
 #pragma unroll
-                    for (int u = 0; u < 16; ++u) {
-                        const int k0 = cc * 32 + 2 * u;
-                        const float x0 = (k0 < valid) ? __uint_as_float(raw[2 * u]) : -INFINITY;
-                        const float x1 = (k0 + 1 < valid) ? __uint_as_float(raw[2 * u + 1]) : -INFINITY;
-                        const float p0 = ex2_approx(fmaf(x0, c, negm));
-                        const float p1 = ex2_approx(fmaf(x1, c, negm));
-                        l += p0 + p1;
+                        for (int u = 0; u < 32; ++u) {
+                            if (cc * 32 + u >= valid) ra[u] = __float_as_uint(-INFINITY);
+                            if (cc * 32 + 32 + u >= valid) rb[u] = __float_as_uint(-INFINITY);
+                        }
+                    }
+                    uint32_t pk[32];
+#pragma unroll
+                    for (int u = 0; u < 32; ++u) {
+                        const uint32_t* src = u < 16 ? ra : rb;
+                        const int v = (u & 15) * 2;
+                        float t0, t1;
+                        f2_unpack(f2_fma(f2_pack(__uint_as_float(src[v]), __uint_as_float(src[v + 1])), c2, negm2),
+                                  t0, t1);
+                        const float p0 = ex2_approx(t0), p1 = ex2_approx(t1);
+                        acc[u & 3] = f2_add(acc[u & 3], f2_pack(p0, p1));
                         __nv_bfloat162 h = __floats2bfloat162_rn(p0, p1);  // .x (low half) = even key
                         pk[u] = *reinterpret_cast<uint32_t*>(&h);
                     }
-                    tmem_st16(tS[k] + lane_off + cc * 16, pk);
+                    tmem_st32(tS[k] + lane_off + cc * 16, pk);
+                }
+                {
+                    float a0, a1, b0, b1, c0, c1, d0, d1;
+                    f2_unpack(acc[0], a0, a1);
+                    f2_unpack(acc[1], b0, b1);
+                    f2_unpack(acc[2], c0, c1);
+                    f2_unpack(acc[3], d0, d1);
+                    l += ((a0 + a1) + (b0 + b1)) + ((c0 + c1) + (d0 + d1));
                 }
                 tmem_wait_st();
                 tc_fence_before();

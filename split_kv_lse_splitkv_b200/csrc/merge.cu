@@ -6,8 +6,10 @@
 //   self partial over the block's own keys: s_t = scale q.kb_t;
 //   L = log( sum_t exp(s_t) + sum_{c < ceil(a/C)} exp(LSE_c) )          (max-shifted)
 //   O = sum_c exp(LSE_c - L) O_c + sum_t exp(s_t - L) vb_t.
-// The partial tiles are stored [d/4][rows][4], so consecutive threads (consecutive rows) read
-// consecutive 16-byte words: fully coalesced.
+// Memory-bound: every visible partial tile is read once. The per-chunk LSEs are staged in shared
+// memory with coalesced loads and turned into weights there; the partial tiles are stored
+// [d/4][rows][4], so consecutive threads (consecutive rows) read consecutive 16-byte words, and
+// each thread keeps four chunk loads in flight.
 #include "common.cuh"
 #include "scan.cuh"
 
@@ -15,10 +17,10 @@ namespace splitkv {
 
 namespace {
 
-constexpr int kThreads = 256;
+constexpr int kThreads = 512;
 
 template <typename T>
-__global__ void __launch_bounds__(kThreads) merge_kernel(Meta m, const float* __restrict__ o_part,
+__global__ void __launch_bounds__(kThreads) merge_kernel(Meta m, int32_t max_nv, const float* __restrict__ o_part,
                                                          const float* __restrict__ lse_part,
                                                          const T* __restrict__ q, const T* __restrict__ kb,
                                                          const T* __restrict__ vb,
@@ -31,8 +33,9 @@ __global__ void __launch_bounds__(kThreads) merge_kernel(Meta m, const float* __
     float* Qs = smem;             // [R][d+1]
     float* Kbs = Qs + R * dp;     // [BL][d+1]
     float* Vbs = Kbs + BL * dp;   // [BL][d]
-    float* Ps = Vbs + BL * d;     // [R][BL]
+    float* Ps = Vbs + BL * d;     // [R][BL]   self scores, then self weights
     float* Lr = Ps + R * BL;      // [R]
+    float* Wc = Lr + R;           // [max_nv][R] chunk LSEs, then chunk weights
     const int tid = threadIdx.x;
     const int32_t j = blockIdx.x / m.hkv, g = blockIdx.x % m.hkv;
     const int s = sample_of_block(m, j);
@@ -42,6 +45,9 @@ __global__ void __launch_bounds__(kThreads) merge_kernel(Meta m, const float* __
     int32_t nv = (int32_t)(((int64_t)a + m.chunk - 1) / m.chunk);
     if (nv < 0) nv = 0;
     if (nv > m.n_chunk_s[s]) nv = m.n_chunk_s[s];
+    if (nv > max_nv) nv = max_nv;
+    const int64_t item0 = m.item_base[s] + (int64_t)g * nb + b;  // chunk 0; chunk c adds c*Hkv*nb
+    const int64_t cstride = (int64_t)m.hkv * nb;
 
     for (int e = tid; e < R * d; e += kThreads) {
         int r = e / d, dd = e % d;
@@ -55,6 +61,10 @@ __global__ void __launch_bounds__(kThreads) merge_kernel(Meta m, const float* __
         Kbs[t * dp + dd] = to_f32(kb[off]);
         Vbs[t * d + dd] = to_f32(vb[off]);
     }
+    for (int e = tid; e < nv * R; e += kThreads) {
+        int c = e / R, r = e % R;
+        Wc[e] = lse_part[(item0 + c * cstride) * R + r];
+    }
     __syncthreads();
     for (int e = tid; e < R * BL; e += kThreads) {
         int r = e / BL, t = e % BL;
@@ -63,32 +73,42 @@ __global__ void __launch_bounds__(kThreads) merge_kernel(Meta m, const float* __
         Ps[e] = acc * m.scale;
     }
     __syncthreads();
-    const int64_t item0 = m.item_base[s] + (int64_t)g * nb + b;  // chunk 0; chunk c adds c*Hkv*nb
-    const int64_t cstride = (int64_t)m.hkv * nb;
     for (int r = tid; r < R; r += kThreads) {
-        float ms = -INFINITY;
-        for (int t = 0; t < BL; ++t) ms = fmaxf(ms, Ps[r * BL + t]);
-        float ls = 0.f;
-        for (int t = 0; t < BL; ++t) ls += expf(Ps[r * BL + t] - ms);
-        float lse_self = ms + logf(ls);
-        float M = lse_self;
-        for (int c = 0; c < nv; ++c) M = fmaxf(M, lse_part[(item0 + c * cstride) * R + r]);
-        float sum = expf(lse_self - M);
-        for (int c = 0; c < nv; ++c) sum += expf(lse_part[(item0 + c * cstride) * R + r] - M);
-        float L = M + logf(sum);
+        float M = -INFINITY;
+        for (int t = 0; t < BL; ++t) M = fmaxf(M, Ps[r * BL + t]);
+        for (int c = 0; c < nv; ++c) M = fmaxf(M, Wc[c * R + r]);
+        float sum = 0.f;
+        for (int t = 0; t < BL; ++t) sum += expf(Ps[r * BL + t] - M);
+        for (int c = 0; c < nv; ++c) sum += expf(Wc[c * R + r] - M);
+        const float L = M + logf(sum);
         Lr[r] = L;
         for (int t = 0; t < BL; ++t) Ps[r * BL + t] = expf(Ps[r * BL + t] - L);
+        for (int c = 0; c < nv; ++c) Wc[c * R + r] = expf(Wc[c * R + r] - L);
     }
     __syncthreads();
     const int D4 = d / 4;
+    const float4* op = reinterpret_cast<const float4*>(o_part);
     for (int e = tid; e < R * D4; e += kThreads) {
         const int r = e % R, d4 = e / R;
-        const float L = Lr[r];
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int c = 0; c < nv; ++c) {
-            const int64_t item = item0 + c * cstride;
-            const float wgt = expf(lse_part[item * R + r] - L);
-            const float4 x = *reinterpret_cast<const float4*>(o_part + item * (int64_t)R * d + ((int64_t)d4 * R + r) * 4);
+        const int64_t base = (int64_t)d4 * R + r;  // float4 index inside an item tile
+        int c = 0;
+        for (; c + 4 <= nv; c += 4) {
+            float4 x[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) x[u] = __ldcs(op + (item0 + (c + u) * cstride) * (int64_t)R * D4 + base);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const float wgt = Wc[(c + u) * R + r];
+                acc.x = fmaf(wgt, x[u].x, acc.x);
+                acc.y = fmaf(wgt, x[u].y, acc.y);
+                acc.z = fmaf(wgt, x[u].z, acc.z);
+                acc.w = fmaf(wgt, x[u].w, acc.w);
+            }
+        }
+        for (; c < nv; ++c) {
+            const float4 x = __ldcs(op + (item0 + c * cstride) * (int64_t)R * D4 + base);
+            const float wgt = Wc[c * R + r];
             acc.x = fmaf(wgt, x.x, acc.x);
             acc.y = fmaf(wgt, x.y, acc.y);
             acc.z = fmaf(wgt, x.z, acc.z);
@@ -109,7 +129,7 @@ __global__ void __launch_bounds__(kThreads) merge_kernel(Meta m, const float* __
         dst[1] = from_f32<T>(acc.y);
         dst[2] = from_f32<T>(acc.z);
         dst[3] = from_f32<T>(acc.w);
-        if (d4 == 0) lse[orow] = L;
+        if (d4 == 0) lse[orow] = Lr[r];
     }
 }
 
@@ -117,14 +137,17 @@ template <typename T>
 cudaError_t launch_t(const Meta& m, const float* o_part, const float* lse_part, const void* q, const void* kb,
                      const void* vb, const int32_t* anchors, void* o, float* lse, int32_t* status, cudaStream_t st) {
     const int R = m.rows, d = m.d, BL = m.block;
-    size_t smem = sizeof(float) * ((size_t)R * (d + 1) + BL * (d + 1) + BL * d + R * BL + R);
+    int32_t max_nv = 0;
+    for (int s = 0; s < m.batch; ++s) max_nv = m.n_chunk_s[s] > max_nv ? m.n_chunk_s[s] : max_nv;
+    size_t smem = sizeof(float) * ((size_t)R * (d + 1) + BL * (d + 1) + BL * d + R * BL + R + (size_t)max_nv * R);
+    if (smem > 227 * 1024) return note_error(cudaErrorInvalidConfiguration, "merge: too many chunks per sample");
     cudaError_t e = cudaFuncSetAttribute(merge_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
+    if (e != cudaSuccess) return note_error(e, "cudaFuncSetAttribute(merge_kernel)");
     int64_t grid = m.n_blocks * m.hkv;
     if (grid == 0) return cudaSuccess;
-    merge_kernel<T><<<(unsigned)grid, kThreads, smem, st>>>(m, o_part, lse_part, (const T*)q, (const T*)kb,
+    merge_kernel<T><<<(unsigned)grid, kThreads, smem, st>>>(m, max_nv, o_part, lse_part, (const T*)q, (const T*)kb,
                                                             (const T*)vb, anchors, (T*)o, lse, status);
-    return cudaGetLastError();
+    return note_error(cudaGetLastError(), "launch merge_kernel");
 }
 
 }  // namespace

@@ -90,19 +90,21 @@ __global__ void __launch_bounds__(kThreads) plan_runs_kernel(const int32_t* __re
                                                              int32_t* __restrict__ status) {
     __shared__ int64_t L[kThreads];
     __shared__ int32_t qcount[kThreads];
-    __shared__ int32_t rr[kThreads];
-    __shared__ int32_t oo[kThreads];
-    __shared__ int32_t qq[kThreads];
+    __shared__ int32_t rr[kThreads];       // first window of each worker
+    __shared__ int32_t by_q[kThreads];     // worker at each (offset, worker) position
+    __shared__ int32_t cnt_w[32][kMaxCost + 1];
+    __shared__ int32_t start_o[kMaxCost + 1];
     __shared__ int32_t total[kMaxCost + 1];
     __shared__ int32_t start[kMaxCost + 1];
     __shared__ int32_t cnt_r[kMaxCost + 2];
     __shared__ int32_t P[kMaxCost + 2];
     __shared__ int64_t red64[32];
     __shared__ int32_t red32[33];
+    __shared__ int32_t scan_sh[33];
     __shared__ int32_t bad;
 
     if (status_bad(status)) return;
-    const int tid = threadIdx.x;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int32_t n = *n_items_d;
     const int32_t nblk = (n + kThreads - 1) / kThreads;
 
@@ -130,57 +132,65 @@ __global__ void __launch_bounds__(kThreads) plan_runs_kernel(const int32_t* __re
     if (tid < m) { L[tid] = 0; qcount[tid] = 0; }
     __syncthreads();
 
-    int32_t h_local[kMaxCost + 1];
     for (int w = W; w >= 1; --w) {
         const int32_t nw = total[w];
         if (tid == 0) { ws.run_n[w] = nw; ws.run_start[w] = start[w]; }
         if (nw == 0) continue;  // uniform across the block
 
         // V0 = min load.
-        int64_t li = tid < m ? L[tid] : INT64_MAX;
+        const int64_t li = tid < m ? L[tid] : INT64_MAX;
         int64_t v = warp_reduce_min(li);
-        if ((tid & 31) == 0) red64[tid >> 5] = v;
+        if (lane == 0) red64[warp] = v;
+        for (int i = tid; i < 32 * (kMaxCost + 1); i += kThreads) (&cnt_w[0][0])[i] = 0;
+        for (int i = tid; i <= W + 1; i += kThreads) cnt_r[i] = 0;
         __syncthreads();
         if (tid < 32) {
-            int64_t x = tid < (kThreads >> 5) ? red64[tid] : INT64_MAX;
+            int64_t x = red64[tid];
             x = warp_reduce_min(x);
             if (tid == 0) red64[0] = x;
         }
         __syncthreads();
         const int64_t V0 = red64[0];
-        int32_t ri = 0, oi = 0;
+        int32_t ri = 0, oi = w;  // threads without a worker sort into an unused bucket
         if (tid < m) {
-            int64_t dlt = li - V0;
+            const int64_t dlt = li - V0;
             ri = (int32_t)(dlt / w);
             oi = (int32_t)(dlt % w);
             rr[tid] = ri;
-            oo[tid] = oi;
-        }
-        for (int r = tid; r <= W + 1; r += kThreads) cnt_r[r] = 0;
-        __syncthreads();
-        // q_i: position of worker i in (offset, worker) order; window histogram of r_i.
-        int32_t qi = 0;
-        if (tid < m) {
-            for (int32_t i2 = 0; i2 < m; ++i2) {
-                int32_t o2 = oo[i2];
-                qi += (o2 < oi || (o2 == oi && i2 < tid)) ? 1 : 0;
-            }
-            qq[tid] = qi;
             if (ri > W) atomicOr(&bad, 1);
             else atomicAdd(&cnt_r[ri], 1);
         }
-        int32_t rmax_local = tid < m ? ri : 0;
-        int32_t rm = warp_reduce_max(rmax_local);
-        if ((tid & 31) == 0) red32[tid >> 5] = rm;
+        // q_i: stable position of worker i in (offset, worker) order, by counting sort.
+        const unsigned same = __match_any_sync(0xffffffffu, oi);
+        const int rank_warp = __popc(same & ((1u << lane) - 1u));
+        if (tid < m && rank_warp == 0) cnt_w[warp][oi] = __popc(same);
+        int32_t rmax = warp_reduce_max(tid < m ? ri : 0);
+        if (lane == 0) red32[warp] = rmax;
         __syncthreads();
-        if (tid < 32) {
-            int32_t x = tid < (kThreads >> 5) ? red32[tid] : 0;
-            x = warp_reduce_max(x);
-            if (tid == 0) red32[32] = x;
+        if (tid <= W) {  // per-offset totals (offsets < w <= W)
+            int32_t c = 0;
+            for (int x = 0; x < 32; ++x) c += cnt_w[x][tid];
+            start_o[tid] = c;
+        }
+        if (tid == 32) {
+            int32_t x = 0;
+            for (int y = 0; y < 32; ++y) x = red32[y] > x ? red32[y] : x;
+            red32[32] = x;
+        }
+        __syncthreads();
+        if (tid == 0) {
+            int32_t acc = 0;
+            for (int o = 0; o < w; ++o) { const int32_t c = start_o[o]; start_o[o] = acc; acc += c; }
         }
         __syncthreads();
         if (bad) break;
         const int32_t R = red32[32];  // <= W
+        int32_t qi = 0;
+        if (tid < m) {
+            qi = start_o[oi] + rank_warp;
+            for (int x = 0; x < warp; ++x) qi += cnt_w[x][oi];
+            by_q[qi] = tid;
+        }
         if (tid == 0) {
             // P[r] = sum_{r' < r} #{i : r_i <= r'}
             int32_t le = 0, acc = 0;
@@ -193,27 +203,33 @@ __global__ void __launch_bounds__(kThreads) plan_runs_kernel(const int32_t* __re
             ws.run_rmax[w] = R;
         }
         __syncthreads();
+        int32_t picks = 0;  // of worker `tid`
         if (tid < m) {
             ws.run_qinv[(size_t)w * m + qi] = tid;
             ws.run_r[(size_t)w * m + tid] = ri;
-            // Catch-up picks: windows r_i .. R-1.
-            int32_t picks = 0;
-            if (ri < R) {
-                for (int r = 0; r <= R; ++r) h_local[r] = 0;
-                for (int32_t i2 = 0; i2 < m; ++i2)
-                    if (qq[i2] < qi) h_local[rr[i2]]++;
-                int32_t pos = 0;
-                for (int r = 0; r < ri; ++r) pos += h_local[r];
-                for (int r = ri; r < R; ++r) {
-                    pos += h_local[r];
-                    int32_t rank = P[r] + pos;
-                    if (rank >= nw) break;
-                    ws.run_catch[(size_t)w * m * W + rank] = make_int2(tid, r - ri);
-                    ++picks;
-                }
+        }
+        // Catch-up windows r < R: participants (r_i <= r) in q order get ranks P[r] + position.
+        // Thread x handles the worker at q position x.
+        const int32_t wx = tid < m ? by_q[tid] : -1;
+        const int32_t rx = wx >= 0 ? rr[wx] : 0;
+        int32_t picks_x = 0;
+        for (int r = 0; r < R; ++r) {
+            const int32_t part = (wx >= 0 && rx <= r) ? 1 : 0;
+            const int32_t pos = block_exclusive_scan<int32_t>(part, scan_sh, nullptr);
+            const int32_t rank = P[r] + pos;
+            if (part && rank < nw) {
+                ws.run_catch[(size_t)w * m * W + rank] = make_int2(wx, r - rx);
+                ++picks_x;
             }
+        }
+        __syncthreads();
+        // Hand the catch-up counts from position-owner to worker-owner through shared memory.
+        if (tid < m) rr[wx] = picks_x;  // rr is no longer needed: reuse it
+        __syncthreads();
+        if (tid < m) {
+            picks = rr[tid];
             // Steady windows r >= R: rank = P[R] + (r - R) * m + q_i.
-            int32_t extra = nw - P[R] - qi;
+            const int32_t extra = nw - P[R] - qi;
             if (extra > 0) picks += (extra + m - 1) / m;
             ws.run_qbase[(size_t)w * m + tid] = qcount[tid];
             qcount[tid] += picks;
@@ -225,10 +241,9 @@ __global__ void __launch_bounds__(kThreads) plan_runs_kernel(const int32_t* __re
         if (tid == 0) raise_status(status, SPLITKV_DEV_BAD_PLAN);
         return;
     }
-    __shared__ int32_t sh[33];
     int32_t c = tid < m ? qcount[tid] : 0;
     int32_t tot;
-    int32_t ex = block_exclusive_scan<int32_t>(c, sh, &tot);
+    int32_t ex = block_exclusive_scan<int32_t>(c, scan_sh, &tot);
     if (tid < m) {
         queue_off[tid] = ex;
         load_out[tid] = L[tid];
