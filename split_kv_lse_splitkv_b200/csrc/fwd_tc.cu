@@ -7,10 +7,12 @@
 // (query i, head g*G+hl) of block b at kv head g, shared by the G query heads of the GQA group —
 // against the ceil(nvis/128) key tiles of chunk c that the block sees.
 //
-// Roles (320 threads):
-//   warps 0-3 / 4-7  softmax warpgroups of slot 0 / slot 1 (one query-tile row per thread)
+// Roles (384 threads, three warpgroups):
+//   warps 0-3 / 4-7  softmax warpgroups of slot 0 / slot 1 (one query-tile row per thread); they
+//                    raise their register budget to 200 so a whole S row stays in registers
 //   warp 8           TMA producer: Q tile per item, K then V tile per key tile, 5-deep ring
 //   warp 9           MMA issuer (one thread) and TMEM owner (512 columns)
+//   warps 8-11       lower their budget to 104 registers (warps 10-11 only do that)
 // The two slots take alternate items of the queue and ping-pong on the tensor core: while one
 // slot's warpgroup runs the softmax of its tile, the tensor core runs the other slot's QK^T / PV.
 //
@@ -35,7 +37,9 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kThreads = 320;
+constexpr int kThreads = 384;
+constexpr int kSoftmaxRegs = 200;  // per SM sub-partition: 200 + 200 + 104 = 504 = 3 x 168 launched
+constexpr int kControlRegs = 104;
 constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
 constexpr int kNB = 5;               // K/V ring depth (32 KB buffers)
@@ -71,20 +75,50 @@ struct TileRef {
     int32_t nvis, ntiles, t;
 };
 
-// Items of one slot: queue positions first + 2i; tiles of each item in order.
-struct Cursor {
-    int32_t pos, end;
-    bool has;
-    TileRef cur;
+// The items of one slot (queue positions first, first+2, ...), fetched ahead: each call hands out
+// the next (item id, anchor) and issues the loads one link further for the three items after it
+// (anchor of n+1, id of n+2, queue entry of n+3), so no role waits on a dependent global load
+// chain when it moves to a new item.
+struct ItemStream {
+    int32_t pos, end, left;
+    int64_t id1;  // item n+1 (loaded)
+    int32_t a1;   // anchor of item n+1 (in flight)
+    int64_t id2;  // item n+2 (in flight)
+    int32_t k3;   // queue entry of item n+3 (in flight)
 };
 
-__device__ __forceinline__ void load_item(const Meta& m, const int32_t* __restrict__ anchors,
-                                          const int32_t* __restrict__ item_id,
-                                          const int32_t* __restrict__ queue_items, int32_t pos, TileRef& tr,
-                                          int32_t* status) {
-    const int32_t k = queue_items[pos];
-    const int64_t id = (k >= 0) ? (int64_t)item_id[k] : -1;
-    if (k < 0 || id < 0 || id >= m.n_items) {
+__device__ __forceinline__ int64_t load_id(const Meta& m, const int32_t* __restrict__ item_id, int32_t k) {
+    return k >= 0 ? (int64_t)__ldg(item_id + k) : -1;
+}
+__device__ __forceinline__ int32_t load_anchor(const Meta& m, const int32_t* __restrict__ anchors, int64_t id) {
+    return (id >= 0 && id < m.n_items) ? __ldg(anchors + decode_item(m, id).j) : 0;
+}
+
+__device__ __forceinline__ void stream_init(const Meta& m, const int32_t* anchors, const int32_t* item_id,
+                                            const int32_t* queue_items, int32_t first, int32_t end, ItemStream& st) {
+    st.end = end;
+    st.left = first < end ? (end - first + 1) / 2 : 0;
+    const int32_t k0 = st.left > 0 ? __ldg(queue_items + first) : -1;
+    const int32_t k1 = st.left > 1 ? __ldg(queue_items + first + 2) : -1;
+    st.k3 = st.left > 2 ? __ldg(queue_items + first + 4) : -1;
+    st.id1 = load_id(m, item_id, k0);
+    st.id2 = load_id(m, item_id, k1);
+    st.a1 = load_anchor(m, anchors, st.id1);
+    st.pos = first + 6;
+}
+
+// Next item as a tile reference (ntiles == 0 for an invalid entry, which raises BAD_PLAN).
+__device__ __forceinline__ void stream_next(const Meta& m, const int32_t* anchors, const int32_t* item_id,
+                                            const int32_t* queue_items, ItemStream& st, TileRef& tr, int32_t* status) {
+    const int64_t id = st.id1;
+    const int32_t a = st.a1;
+    --st.left;
+    st.a1 = load_anchor(m, anchors, st.id2);
+    st.id1 = st.id2;
+    st.id2 = load_id(m, item_id, st.k3);
+    st.k3 = st.pos < st.end ? __ldg(queue_items + st.pos) : -1;
+    st.pos += 2;
+    if (id < 0 || id >= m.n_items) {
         raise_status(status, SPLITKV_DEV_BAD_PLAN);
         tr.ntiles = 0;
         return;
@@ -95,22 +129,35 @@ __device__ __forceinline__ void load_item(const Meta& m, const int32_t* __restri
     tr.c = it.c;
     tr.g = it.g;
     tr.j = it.j;
-    tr.nvis = visible_in_chunk(m, it.s, it.c, anchors[it.j]);
+    tr.nvis = visible_in_chunk(m, it.s, it.c, a);
     tr.ntiles = (tr.nvis + kKeysPerTile - 1) / kKeysPerTile;
     tr.t = 0;
 }
 
+// Items of one slot as a sequence of key tiles.
+struct Cursor {
+    ItemStream st;
+    bool has;
+    TileRef cur;
+};
+
 __device__ __forceinline__ void cursor_fetch(const Meta& m, const int32_t* anchors, const int32_t* item_id,
                                              const int32_t* queue_items, Cursor& c, int32_t* status) {
-    while (c.pos < c.end) {
-        load_item(m, anchors, item_id, queue_items, c.pos, c.cur, status);
-        c.pos += 2;
+    while (c.st.left > 0) {
+        stream_next(m, anchors, item_id, queue_items, c.st, c.cur, status);
         if (c.cur.ntiles > 0) {
             c.has = true;
             return;
         }
     }
     c.has = false;
+}
+
+__device__ __forceinline__ void cursor_init(const Meta& m, const int32_t* anchors, const int32_t* item_id,
+                                            const int32_t* queue_items, int32_t first, int32_t end, Cursor& c,
+                                            int32_t* status) {
+    stream_init(m, anchors, item_id, queue_items, first, end, c.st);
+    cursor_fetch(m, anchors, item_id, queue_items, c, status);
 }
 
 __device__ __forceinline__ void cursor_advance(const Meta& m, const int32_t* anchors, const int32_t* item_id,
@@ -170,288 +217,271 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tS[2] = {tmem + 0u, tmem + 128u};
     const uint32_t tO[2] = {tmem + 256u, tmem + 384u};
 
-    if (!skip && warp == kProducerWarp) {
-        if (lane == 0) {
-            tma_prefetch_desc(&tmQ);
-            tma_prefetch_desc(&tmK);
-            tma_prefetch_desc(&tmV);
-            const uint32_t q_bytes = 2u * 64u * (uint32_t)G * (uint32_t)m.block * 2u;
-            Cursor cur[2];
-            TileRef pv_tile[2];
-            bool pending[2] = {false, false};
-            uint32_t kv_seq = 0, qseq[2] = {0, 0};
-            int32_t last_kv_parity[kNB];
-            bool issued[kNB];
-            for (int i = 0; i < kNB; ++i) { issued[i] = false; last_kv_parity[i] = 0; }
-            bool q_issued[2] = {false, false};
-            uint32_t q_last_parity[2] = {0, 0};
-            bool ok = true;
-            for (int k = 0; k < 2; ++k) {
-                cur[k].pos = q0 + k;
-                cur[k].end = q1;
-                cursor_fetch(m, anchors, item_id, queue_items, cur[k], status);
-            }
-            auto load_kv = [&](const CUtensorMap* map, const TileRef& t) -> bool {
-                const int buf = kv_seq % kNB;
-                const uint32_t ph = (kv_seq / kNB) & 1u;
-                if (!mbar_wait(&bars->kv_empty[buf], ph ^ 1u, abort_flag, kTimeoutNs)) return false;
-                mbar_arrive_expect_tx(&bars->kv_full[buf], kTileBytes);
-                const int32_t row = (int32_t)(m.key_off[t.s] + (int64_t)t.c * m.chunk + (int64_t)t.t * kKeysPerTile);
-                uint8_t* dst = kv_smem + buf * kTileBytes;
-                tma_load_3d(dst, map, &bars->kv_full[buf], 0, t.g, row);
-                tma_load_3d(dst + kHalfBytes, map, &bars->kv_full[buf], 64, t.g, row);
-                issued[buf] = true;
-                last_kv_parity[buf] = (int32_t)ph;
-                ++kv_seq;
-                return true;
-            };
-            auto emit_qk = [&](int k) -> bool {
-                const TileRef t = cur[k].cur;
-                if (t.t == 0) {
-                    if (!mbar_wait(&bars->q_empty[k], (qseq[k] & 1u) ^ 1u, abort_flag, kTimeoutNs)) return false;
-                    mbar_arrive_expect_tx(&bars->q_full[k], q_bytes);
-                    uint8_t* dst = q_smem + k * kTileBytes;
-                    tma_load_3d(dst, &tmQ, &bars->q_full[k], 0, t.g * G, m.block * t.j);
-                    tma_load_3d(dst + kHalfBytes, &tmQ, &bars->q_full[k], 64, t.g * G, m.block * t.j);
-                    q_issued[k] = true;
-                    q_last_parity[k] = qseq[k] & 1u;
-                    ++qseq[k];
-                }
-                if (!load_kv(&tmK, t)) return false;
-                pv_tile[k] = t;
-                pending[k] = true;
-                cursor_advance(m, anchors, item_id, queue_items, cur[k], status);
-                return true;
-            };
-            for (int k = 0; k < 2 && ok; ++k)
-                if (cur[k].has) ok = emit_qk(k);
-            while (ok && (pending[0] || pending[1])) {
-                for (int k = 0; k < 2 && ok; ++k) {
-                    if (pending[k]) {
-                        ok = load_kv(&tmV, pv_tile[k]);
-                        pending[k] = false;
+    if (warp >= 8) {
+        // Control warpgroup: give registers to the softmax warpgroups.
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(kControlRegs));
+        if (!skip && warp == kProducerWarp) {
+            if (lane == 0) {
+                tma_prefetch_desc(&tmQ);
+                tma_prefetch_desc(&tmK);
+                tma_prefetch_desc(&tmV);
+                const uint32_t q_bytes = 2u * 64u * (uint32_t)G * (uint32_t)m.block * 2u;
+                Cursor cur[2];
+                TileRef pv_tile[2];
+                bool pending[2] = {false, false};
+                uint32_t kv_seq = 0, qseq[2] = {0, 0};
+                int32_t last_kv_parity[kNB];
+                bool issued[kNB];
+                for (int i = 0; i < kNB; ++i) { issued[i] = false; last_kv_parity[i] = 0; }
+                bool q_issued[2] = {false, false};
+                uint32_t q_last_parity[2] = {0, 0};
+                bool ok = true;
+                for (int k = 0; k < 2; ++k) cursor_init(m, anchors, item_id, queue_items, q0 + k, q1, cur[k], status);
+                auto load_kv = [&](const CUtensorMap* map, const TileRef& t) -> bool {
+                    const int buf = kv_seq % kNB;
+                    const uint32_t ph = (kv_seq / kNB) & 1u;
+                    if (!mbar_wait(&bars->kv_empty[buf], ph ^ 1u, abort_flag, kTimeoutNs)) return false;
+                    mbar_arrive_expect_tx(&bars->kv_full[buf], kTileBytes);
+                    const int32_t row = (int32_t)(m.key_off[t.s] + (int64_t)t.c * m.chunk + (int64_t)t.t * kKeysPerTile);
+                    uint8_t* dst = kv_smem + buf * kTileBytes;
+                    tma_load_3d(dst, map, &bars->kv_full[buf], 0, t.g, row);
+                    tma_load_3d(dst + kHalfBytes, map, &bars->kv_full[buf], 64, t.g, row);
+                    issued[buf] = true;
+                    last_kv_parity[buf] = (int32_t)ph;
+                    ++kv_seq;
+                    return true;
+                };
+                auto emit_qk = [&](int k) -> bool {
+                    const TileRef t = cur[k].cur;
+                    if (t.t == 0) {
+                        if (!mbar_wait(&bars->q_empty[k], (qseq[k] & 1u) ^ 1u, abort_flag, kTimeoutNs)) return false;
+                        mbar_arrive_expect_tx(&bars->q_full[k], q_bytes);
+                        uint8_t* dst = q_smem + k * kTileBytes;
+                        tma_load_3d(dst, &tmQ, &bars->q_full[k], 0, t.g * G, m.block * t.j);
+                        tma_load_3d(dst + kHalfBytes, &tmQ, &bars->q_full[k], 64, t.g * G, m.block * t.j);
+                        q_issued[k] = true;
+                        q_last_parity[k] = qseq[k] & 1u;
+                        ++qseq[k];
                     }
-                    if (ok && cur[k].has) ok = emit_qk(k);
-                }
-            }
-            // Drain: every copy this warp issued must have landed before the CTA exits.
-            for (int i = 0; i < kNB; ++i)
-                if (issued[i]) {
-                    volatile int never = 0;
-                    mbar_wait(&bars->kv_full[i], (uint32_t)last_kv_parity[i], &never, kTimeoutNs);
-                }
-            for (int k = 0; k < 2; ++k)
-                if (q_issued[k]) {
-                    volatile int never = 0;
-                    mbar_wait(&bars->q_full[k], q_last_parity[k], &never, kTimeoutNs);
-                }
-        }
-        __syncwarp();
-    } else if (!skip && warp == kMmaWarp) {
-        if (lane == 0) {
-            constexpr uint32_t idesc_qk = umma_idesc_bf16_f32(128, 128, false, false);
-            constexpr uint32_t idesc_pv = umma_idesc_bf16_f32(128, 128, false, true);
-            const uint32_t q_base = smem_u32(q_smem), kv_base = smem_u32(kv_smem);
-            Cursor cur[2];
-            bool pending[2] = {false, false}, pv_first[2] = {false, false};
-            uint32_t kv_seq = 0, qseq[2] = {0, 0}, tile_seq[2] = {0, 0};
-            bool ok = true;
-            for (int k = 0; k < 2; ++k) {
-                cur[k].pos = q0 + k;
-                cur[k].end = q1;
-                cursor_fetch(m, anchors, item_id, queue_items, cur[k], status);
-            }
-            auto emit_qk = [&](int k) -> bool {
-                const TileRef t = cur[k].cur;
-                if (tile_seq[k] > 0 &&
-                    !mbar_wait(&bars->pv_done[k], (tile_seq[k] - 1) & 1u, abort_flag, kTimeoutNs))
-                    return false;
-                if (t.t == 0) {
-                    if (!mbar_wait(&bars->q_full[k], qseq[k] & 1u, abort_flag, kTimeoutNs)) return false;
-                    ++qseq[k];
-                }
-                const int buf = kv_seq % kNB;
-                if (!mbar_wait(&bars->kv_full[buf], (kv_seq / kNB) & 1u, abort_flag, kTimeoutNs)) return false;
-                tc_fence_after();
-                const uint32_t qa = q_base + k * kTileBytes, kb = kv_base + buf * kTileBytes;
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
-                    mma_ss(tS[k], umma_desc_sw128(qa + off, 16, 1024), umma_desc_sw128(kb + off, 16, 1024),
-                           idesc_qk, kk > 0 ? 1u : 0u);
-                }
-                mma_commit(&bars->s_full[k]);
-                mma_commit(&bars->kv_empty[buf]);
-                if (t.t == t.ntiles - 1) mma_commit(&bars->q_empty[k]);
-                ++kv_seq;
-                pv_first[k] = (t.t == 0);
-                pending[k] = true;
-                ++tile_seq[k];
-                cursor_advance(m, anchors, item_id, queue_items, cur[k], status);
-                return true;
-            };
-            auto emit_pv = [&](int k) -> bool {
-                if (!mbar_wait(&bars->p_full[k], (tile_seq[k] - 1) & 1u, abort_flag, kTimeoutNs)) return false;
-                const int buf = kv_seq % kNB;
-                if (!mbar_wait(&bars->kv_full[buf], (kv_seq / kNB) & 1u, abort_flag, kTimeoutNs)) return false;
-                tc_fence_after();
-                const uint32_t vb = kv_base + buf * kTileBytes;
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    // A = P[:, 16kk .. 16kk+16) packed two bf16 per column; B = V rows 16kk.., MN-major.
-                    mma_ts(tO[k], tS[k] + (uint32_t)(kk * 8), umma_desc_sw128(vb + kk * 2048, kHalfBytes, 1024),
-                           idesc_pv, (!pv_first[k] || kk > 0) ? 1u : 0u);
-                }
-                mma_commit(&bars->pv_done[k]);
-                mma_commit(&bars->kv_empty[buf]);
-                ++kv_seq;
-                pending[k] = false;
-                return true;
-            };
-            for (int k = 0; k < 2 && ok; ++k)
-                if (cur[k].has) ok = emit_qk(k);
-            while (ok && (pending[0] || pending[1])) {
-                for (int k = 0; k < 2 && ok; ++k) {
-                    if (pending[k]) ok = emit_pv(k);
-                    if (ok && cur[k].has) ok = emit_qk(k);
-                }
-            }
-            // Drain: all MMAs issued by this thread complete before TMEM is released.
-            mma_commit(&bars->drain);
-            volatile int never = 0;
-            mbar_wait(&bars->drain, 0, &never, kTimeoutNs);
-        }
-        __syncwarp();
-    } else if (!skip && warp < 8) {
-        const int k = warp >> 2;                // slot
-        const int quad = warp & 3;              // TMEM lane quadrant
-        const int r = quad * 32 + lane;         // query-tile row
-        const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
-        const float c = m.scale * 1.4426950408889634f;  // log2(e)
-        uint32_t tile_seq = 0;
-        bool ok = true;
-        for (int32_t pos = q0 + k; pos < q1 && ok; pos += 2) {
-            TileRef t;
-            load_item(m, anchors, item_id, queue_items, pos, t, status);
-            if (t.ntiles == 0) continue;
-            float m_used = -INFINITY, l = 0.f;
-            for (int tt = 0; tt < t.ntiles; ++tt) {
-                if (!mbar_wait(&bars->s_full[k], tile_seq & 1u, abort_flag, kTimeoutNs)) { ok = false; break; }
-                tc_fence_after();
-                const int valid = t.nvis - tt * kKeysPerTile;  // keys of this tile the block sees (>= 1)
-                const bool full = valid >= kKeysPerTile;         // only an item's last tile can be partial
-                // Pass 1: row max, 64 columns per TMEM wait; four independent max chains.
-                float mx;
-                {
-                    float m0 = -INFINITY, m1 = -INFINITY, m2 = -INFINITY, m3 = -INFINITY;
-#pragma unroll 1
-                    for (int cc = 0; cc < 4; cc += 2) {
-                        uint32_t ra[32], rb[32];
-                        tmem_ld32(tS[k] + lane_off + cc * 32, ra);
-                        tmem_ld32(tS[k] + lane_off + cc * 32 + 32, rb);
-                        tmem_wait_ld();
-                        if (full) {
-#pragma unroll
-                            for (int u = 0; u < 32; u += 4) {
-                                m0 = max3f(m0, __uint_as_float(ra[u]), __uint_as_float(ra[u + 1]));
-                                m1 = max3f(m1, __uint_as_float(ra[u + 2]), __uint_as_float(ra[u + 3]));
-                                m2 = max3f(m2, __uint_as_float(rb[u]), __uint_as_float(rb[u + 1]));
-                                m3 = max3f(m3, __uint_as_float(rb[u + 2]), __uint_as_float(rb[u + 3]));
-                            }
-                        } else {
-#pragma unroll
-                            for (int u = 0; u < 32; ++u) {
-                                if (cc * 32 + u < valid) m0 = fmaxf(m0, __uint_as_float(ra[u]));
-                                if (cc * 32 + 32 + u < valid) m1 = fmaxf(m1, __uint_as_float(rb[u]));
-                            }
+                    if (!load_kv(&tmK, t)) return false;
+                    pv_tile[k] = t;
+                    pending[k] = true;
+                    cursor_advance(m, anchors, item_id, queue_items, cur[k], status);
+                    return true;
+                };
+                for (int k = 0; k < 2 && ok; ++k)
+                    if (cur[k].has) ok = emit_qk(k);
+                while (ok && (pending[0] || pending[1])) {
+                    for (int k = 0; k < 2 && ok; ++k) {
+                        if (pending[k]) {
+                            ok = load_kv(&tmV, pv_tile[k]);
+                            pending[k] = false;
                         }
+                        if (ok && cur[k].has) ok = emit_qk(k);
                     }
-                    mx = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3)) * c;
                 }
-                if (tt == 0) {
-                    m_used = mx;
-                } else if (mx > m_used + kRescaleLog2) {
-                    // The previous PV of this slot completed before this tile's QK^T was issued.
-                    const float alpha = ex2_approx(m_used - mx);
-                    l *= alpha;
-#pragma unroll 1
-                    for (int cc = 0; cc < 4; ++cc) {
-                        uint32_t ov[32];
-                        tmem_ld32(tO[k] + lane_off + cc * 32, ov);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int u = 0; u < 32; ++u) ov[u] = __float_as_uint(__uint_as_float(ov[u]) * alpha);
-                        tmem_st32(tO[k] + lane_off + cc * 32, ov);
+                // Drain: every copy this warp issued must have landed before the CTA exits.
+                for (int i = 0; i < kNB; ++i)
+                    if (issued[i]) {
+                        volatile int never = 0;
+                        mbar_wait(&bars->kv_full[i], (uint32_t)last_kv_parity[i], &never, kTimeoutNs);
                     }
-                    m_used = mx;
+                for (int k = 0; k < 2; ++k)
+                    if (q_issued[k]) {
+                        volatile int never = 0;
+                        mbar_wait(&bars->q_full[k], q_last_parity[k], &never, kTimeoutNs);
+                    }
+            }
+            __syncwarp();
+        } else if (!skip && warp == kMmaWarp) {
+            if (lane == 0) {
+                constexpr uint32_t idesc_qk = umma_idesc_bf16_f32(128, 128, false, false);
+                constexpr uint32_t idesc_pv = umma_idesc_bf16_f32(128, 128, false, true);
+                const uint32_t q_base = smem_u32(q_smem), kv_base = smem_u32(kv_smem);
+                Cursor cur[2];
+                bool pending[2] = {false, false}, pv_first[2] = {false, false};
+                uint32_t kv_seq = 0, qseq[2] = {0, 0}, tile_seq[2] = {0, 0};
+                bool ok = true;
+                for (int k = 0; k < 2; ++k) cursor_init(m, anchors, item_id, queue_items, q0 + k, q1, cur[k], status);
+                auto emit_qk = [&](int k) -> bool {
+                    const TileRef t = cur[k].cur;
+                    if (tile_seq[k] > 0 &&
+                        !mbar_wait(&bars->pv_done[k], (tile_seq[k] - 1) & 1u, abort_flag, kTimeoutNs))
+                        return false;
+                    if (t.t == 0) {
+                        if (!mbar_wait(&bars->q_full[k], qseq[k] & 1u, abort_flag, kTimeoutNs)) return false;
+                        ++qseq[k];
+                    }
+                    const int buf = kv_seq % kNB;
+                    if (!mbar_wait(&bars->kv_full[buf], (kv_seq / kNB) & 1u, abort_flag, kTimeoutNs)) return false;
+                    tc_fence_after();
+                    const uint32_t qa = q_base + k * kTileBytes, kb = kv_base + buf * kTileBytes;
+    #pragma unroll
+                    for (int kk = 0; kk < 8; ++kk) {
+                        const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
+                        mma_ss(tS[k], umma_desc_sw128(qa + off, 16, 1024), umma_desc_sw128(kb + off, 16, 1024),
+                               idesc_qk, kk > 0 ? 1u : 0u);
+                    }
+                    mma_commit(&bars->s_full[k]);
+                    mma_commit(&bars->kv_empty[buf]);
+                    if (t.t == t.ntiles - 1) mma_commit(&bars->q_empty[k]);
+                    ++kv_seq;
+                    pv_first[k] = (t.t == 0);
+                    pending[k] = true;
+                    ++tile_seq[k];
+                    cursor_advance(m, anchors, item_id, queue_items, cur[k], status);
+                    return true;
+                };
+                auto emit_pv = [&](int k) -> bool {
+                    if (!mbar_wait(&bars->p_full[k], (tile_seq[k] - 1) & 1u, abort_flag, kTimeoutNs)) return false;
+                    const int buf = kv_seq % kNB;
+                    if (!mbar_wait(&bars->kv_full[buf], (kv_seq / kNB) & 1u, abort_flag, kTimeoutNs)) return false;
+                    tc_fence_after();
+                    const uint32_t vb = kv_base + buf * kTileBytes;
+    #pragma unroll
+                    for (int kk = 0; kk < 8; ++kk) {
+                        // A = P[:, 16kk .. 16kk+16) packed two bf16 per column; B = V rows 16kk.., MN-major.
+                        mma_ts(tO[k], tS[k] + (uint32_t)(kk * 8), umma_desc_sw128(vb + kk * 2048, kHalfBytes, 1024),
+                               idesc_pv, (!pv_first[k] || kk > 0) ? 1u : 0u);
+                    }
+                    mma_commit(&bars->pv_done[k]);
+                    mma_commit(&bars->kv_empty[buf]);
+                    ++kv_seq;
+                    pending[k] = false;
+                    return true;
+                };
+                for (int k = 0; k < 2 && ok; ++k)
+                    if (cur[k].has) ok = emit_qk(k);
+                while (ok && (pending[0] || pending[1])) {
+                    for (int k = 0; k < 2 && ok; ++k) {
+                        if (pending[k]) ok = emit_pv(k);
+                        if (ok && cur[k].has) ok = emit_qk(k);
+                    }
                 }
-                // Pass 2: P = 2^(s*c - m) in bf16, written over the first 64 columns of S. S columns
-                // 32cc..32cc+63 are read before P columns 16cc..16cc+31 are written.
-                const uint64_t c2 = f2_pack(c, c), negm2 = f2_pack(-m_used, -m_used);
-                uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
-#pragma unroll 1
-                for (int cc = 0; cc < 4; cc += 2) {
-                    uint32_t ra[32], rb[32];
-                    tmem_ld32(tS[k] + lane_off + cc * 32, ra);
-                    tmem_ld32(tS[k] + lane_off + cc * 32 + 32, rb);
+                // Drain: all MMAs issued by this thread complete before TMEM is released.
+                mma_commit(&bars->drain);
+                volatile int never = 0;
+                mbar_wait(&bars->drain, 0, &never, kTimeoutNs);
+            }
+            __syncwarp();
+        }
+    } else {
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(kSoftmaxRegs));
+        if (!skip) {
+            const int k = warp >> 2;                // slot
+            const int quad = warp & 3;              // TMEM lane quadrant
+            const int r = quad * 32 + lane;         // query-tile row
+            const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+            const float c = m.scale * 1.4426950408889634f;  // log2(e)
+            const uint64_t c2 = f2_pack(c, c);
+            uint32_t tile_seq = 0;
+            bool ok = true;
+            ItemStream st;
+            stream_init(m, anchors, item_id, queue_items, q0 + k, q1, st);
+            while (st.left > 0 && ok) {
+                TileRef t;
+                stream_next(m, anchors, item_id, queue_items, st, t, status);
+                if (t.ntiles == 0) continue;
+                float m_used = -INFINITY, l = 0.f;
+                for (int tt = 0; tt < t.ntiles; ++tt) {
+                    if (!mbar_wait(&bars->s_full[k], tile_seq & 1u, abort_flag, kTimeoutNs)) { ok = false; break; }
+                    tc_fence_after();
+                    // The whole S row in registers: one TMEM round trip.
+                    uint32_t sr[128];
+    #pragma unroll
+                    for (int cc = 0; cc < 4; ++cc)
+                        tmem_ld32(tS[k] + lane_off + cc * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[cc * 32]));
                     tmem_wait_ld();
-                    if (!full) {
-#pragma unroll
-                        for (int u = 0; u < 32; ++u) {
-                            if (cc * 32 + u >= valid) ra[u] = __float_as_uint(-INFINITY);
-                            if (cc * 32 + 32 + u >= valid) rb[u] = __float_as_uint(-INFINITY);
+                    const int valid = t.nvis - tt * kKeysPerTile;  // keys of this tile the block sees (>= 1)
+                    if (valid < kKeysPerTile) {                    // only an item's last tile can be partial
+    #pragma unroll
+                        for (int u = 0; u < 128; ++u)
+                            if (u >= valid) sr[u] = __float_as_uint(-INFINITY);
+                    }
+                    float mx;
+                    {
+                        float m0 = -INFINITY, m1 = -INFINITY, m2 = -INFINITY, m3 = -INFINITY;
+    #pragma unroll
+                        for (int u = 0; u < 128; u += 8) {
+                            m0 = max3f(m0, __uint_as_float(sr[u]), __uint_as_float(sr[u + 1]));
+                            m1 = max3f(m1, __uint_as_float(sr[u + 2]), __uint_as_float(sr[u + 3]));
+                            m2 = max3f(m2, __uint_as_float(sr[u + 4]), __uint_as_float(sr[u + 5]));
+                            m3 = max3f(m3, __uint_as_float(sr[u + 6]), __uint_as_float(sr[u + 7]));
+                        }
+                        mx = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3)) * c;
+                    }
+                    if (tt == 0) {
+                        m_used = mx;
+                    } else if (mx > m_used + kRescaleLog2) {
+                        // The previous PV of this slot completed before this tile's QK^T was issued.
+                        const float alpha = ex2_approx(m_used - mx);
+                        l *= alpha;
+    #pragma unroll 1
+                        for (int cc = 0; cc < 4; ++cc) {
+                            uint32_t ov[32];
+                            tmem_ld32(tO[k] + lane_off + cc * 32, ov);
+                            tmem_wait_ld();
+    #pragma unroll
+                            for (int u = 0; u < 32; ++u) ov[u] = __float_as_uint(__uint_as_float(ov[u]) * alpha);
+                            tmem_st32(tO[k] + lane_off + cc * 32, ov);
+                        }
+                        m_used = mx;
+                    }
+                    // P = 2^(s*c - m) in bf16, packed two per column over the first 64 columns of S.
+                    const uint64_t negm2 = f2_pack(-m_used, -m_used);
+                    uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
+    #pragma unroll
+                    for (int h = 0; h < 4; ++h) {
+                        uint32_t pk[16];
+    #pragma unroll
+                        for (int u = 0; u < 16; ++u) {
+                            const int v = h * 32 + 2 * u;
+                            float t0, t1;
+                            f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[v]), __uint_as_float(sr[v + 1])), c2, negm2), t0,
+                                      t1);
+                            const float p0 = ex2_approx(t0), p1 = ex2_approx(t1);
+                            acc[u & 3] = f2_add(acc[u & 3], f2_pack(p0, p1));
+                            __nv_bfloat162 hp = __floats2bfloat162_rn(p0, p1);  // .x (low half) = even key
+                            pk[u] = *reinterpret_cast<uint32_t*>(&hp);
+                        }
+                        tmem_st16(tS[k] + lane_off + h * 16, pk);
+                    }
+                    {
+                        float a0, a1, b0, b1, c0, c1, d0, d1;
+                        f2_unpack(acc[0], a0, a1);
+                        f2_unpack(acc[1], b0, b1);
+                        f2_unpack(acc[2], c0, c1);
+                        f2_unpack(acc[3], d0, d1);
+                        l += ((a0 + a1) + (b0 + b1)) + ((c0 + c1) + (d0 + d1));
+                    }
+                    tmem_wait_st();
+                    tc_fence_before();
+                    mbar_arrive(&bars->p_full[k]);
+                    ++tile_seq;
+                }
+                if (!ok) break;
+                // Epilogue: wait for the item's last PV, normalise, store partial O and LSE.
+                if (!mbar_wait(&bars->pv_done[k], (tile_seq - 1) & 1u, abort_flag, kTimeoutNs)) { ok = false; break; }
+                tc_fence_after();
+                const float inv_l = 1.f / l;
+                float* op = o_part + t.id * (int64_t)R * 128;
+    #pragma unroll 1
+                for (int cc = 0; cc < 4; ++cc) {
+                    uint32_t ov[32];
+                    tmem_ld32(tO[k] + lane_off + cc * 32, ov);
+                    tmem_wait_ld();
+                    if (r < R) {
+    #pragma unroll
+                        for (int u = 0; u < 8; ++u) {
+                            float4 x = make_float4(__uint_as_float(ov[4 * u]) * inv_l, __uint_as_float(ov[4 * u + 1]) * inv_l,
+                                                   __uint_as_float(ov[4 * u + 2]) * inv_l,
+                                                   __uint_as_float(ov[4 * u + 3]) * inv_l);
+                            *reinterpret_cast<float4*>(op + ((int64_t)(cc * 8 + u) * R + r) * 4) = x;
                         }
                     }
-                    uint32_t pk[32];
-#pragma unroll
-                    for (int u = 0; u < 32; ++u) {
-                        const uint32_t* src = u < 16 ? ra : rb;
-                        const int v = (u & 15) * 2;
-                        float t0, t1;
-                        f2_unpack(f2_fma(f2_pack(__uint_as_float(src[v]), __uint_as_float(src[v + 1])), c2, negm2),
-                                  t0, t1);
-                        const float p0 = ex2_approx(t0), p1 = ex2_approx(t1);
-                        acc[u & 3] = f2_add(acc[u & 3], f2_pack(p0, p1));
-                        __nv_bfloat162 h = __floats2bfloat162_rn(p0, p1);  // .x (low half) = even key
-                        pk[u] = *reinterpret_cast<uint32_t*>(&h);
-                    }
-                    tmem_st32(tS[k] + lane_off + cc * 16, pk);
                 }
-                {
-                    float a0, a1, b0, b1, c0, c1, d0, d1;
-                    f2_unpack(acc[0], a0, a1);
-                    f2_unpack(acc[1], b0, b1);
-                    f2_unpack(acc[2], c0, c1);
-                    f2_unpack(acc[3], d0, d1);
-                    l += ((a0 + a1) + (b0 + b1)) + ((c0 + c1) + (d0 + d1));
-                }
-                tmem_wait_st();
-                tc_fence_before();
-                mbar_arrive(&bars->p_full[k]);
-                ++tile_seq;
+                if (r < R) lse_part[t.id * R + r] = (m_used + lg2_approx(l)) * 0.6931471805599453f;
             }
-            if (!ok) break;
-            // Epilogue: wait for the item's last PV, normalise, store partial O and LSE.
-            if (!mbar_wait(&bars->pv_done[k], (tile_seq - 1) & 1u, abort_flag, kTimeoutNs)) { ok = false; break; }
-            tc_fence_after();
-            const float inv_l = 1.f / l;
-            float* op = o_part + t.id * (int64_t)R * 128;
-#pragma unroll 1
-            for (int cc = 0; cc < 4; ++cc) {
-                uint32_t ov[32];
-                tmem_ld32(tO[k] + lane_off + cc * 32, ov);
-                tmem_wait_ld();
-                if (r < R) {
-#pragma unroll
-                    for (int u = 0; u < 8; ++u) {
-                        float4 x = make_float4(__uint_as_float(ov[4 * u]) * inv_l, __uint_as_float(ov[4 * u + 1]) * inv_l,
-                                               __uint_as_float(ov[4 * u + 2]) * inv_l,
-                                               __uint_as_float(ov[4 * u + 3]) * inv_l);
-                        *reinterpret_cast<float4*>(op + ((int64_t)(cc * 8 + u) * R + r) * 4) = x;
-                    }
-                }
-            }
-            if (r < R) lse_part[t.id * R + r] = (m_used + lg2_approx(l)) * 0.6931471805599453f;
         }
     }
 
