@@ -5,24 +5,26 @@
 // log-sum-exp; the chunks are placed by the cost-aware LPT plan. Here one persistent CTA per SM
 // walks the SM's LPT queue. A work item (s, c, g, b) is one 128-row query tile — the block*G rows
 // (query i, head g*G+hl) of block b at kv head g, shared by the G query heads of the GQA group —
-// against the ceil(nvis/128) key tiles of chunk c that the block sees.
+// against the ceil(nvis/128) key tiles of chunk c that the block sees. The CTA's key tiles form
+// one sequence n = 0, 1, ... across its items i = 0, 1, ...
 //
-// Roles (384 threads, three warpgroups):
-//   warps 0-3 / 4-7  softmax warpgroups of slot 0 / slot 1 (one query-tile row per thread); they
-//                    raise their register budget to 200 so a whole S row stays in registers
-//   warp 8           TMA producer: Q tile per item, K then V tile per key tile, 5-deep ring
-//   warp 9           MMA issuer (one thread) and TMEM owner (512 columns)
-//   warps 8-11       lower their budget to 104 registers (warps 10-11 only do that)
-// The two slots take alternate items of the queue and ping-pong on the tensor core: while one
-// slot's warpgroup runs the softmax of its tile, the tensor core runs the other slot's QK^T / PV.
+// Roles (512 threads, four warpgroups; registers moved with setmaxnreg):
+//   WG0 / WG1 (warps 0-7)  softmax: row r = 32*(warp%4) + lane, key columns 0-63 / 64-127
+//   WG2 (warps 8-11)       epilogue: normalises O of a finished item and stores O_c, LSE_c
+//   warp 12                TMA producer: Q per item (2 buffers), K(n) and V(n) (2 buffers each)
+//   warp 13                MMA issuer (one thread) and TMEM owner
 //
-// TMEM: S_k = Q K^T (128 x 128 fp32) at columns 128k; P_k (bf16, 64 columns) written over the first
-// half of S_k; O_k (128 x 128 fp32) at columns 256 + 128k. The next QK^T of a slot is issued only
-// after that slot's PV has completed, because P aliases S.
+// TMEM (448 of 512 columns): S = Q K^T (128 fp32 columns), P (bf16 pairs, 64 columns) and
+// O[2] (128 fp32 columns each, one per item parity). The MMA thread issues QK^T(n) and then
+// PV(n-1): while the softmax turns S(n) into P(n), the tensor core runs PV(n-1) and, as soon as
+// the softmax holds S(n) in registers, QK^T(n+1). No MMA waits for another MMA, and an item's
+// epilogue overlaps the next item's tiles. The MMA thread only commits S-ready and PV-done; the
+// softmax warps release the K, V and Q buffers once those commits tell them the reads are over.
 //
-// Online softmax in log2 units (x = s * scale * log2 e); the running reference max is only moved
-// when a tile's max exceeds it by more than 8 (so P <= 256), which keeps O and l consistent and
-// rescales O rarely. LSE = (m + log2 l) * ln 2.
+// Online softmax in log2 units (x = s * scale * log2 e); the two halves of a row exchange their
+// maxima through shared memory. The running reference max only moves when a tile's max exceeds it
+// by more than 8 (so P <= 256), which keeps O and l consistent and rescales O rarely.
+// LSE = (m + log2 l) * ln 2.
 //
 // Every wait is bounded (2 s); on expiry the CTA raises SPLITKV_DEV_TIMEOUT, drains its copies and
 // MMAs in flight, frees TMEM and returns.
@@ -37,37 +39,47 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kThreads = 384;
-constexpr int kSoftmaxRegs = 200;  // per SM sub-partition: 200 + 200 + 104 = 504 = 3 x 168 launched
-constexpr int kControlRegs = 104;
-constexpr int kProducerWarp = 8;
-constexpr int kMmaWarp = 9;
-constexpr int kNB = 5;               // K/V ring depth (32 KB buffers)
+constexpr int kThreads = 512;
+constexpr int kEpiWarp0 = 8;
+constexpr int kProducerWarp = 12;
+constexpr int kMmaWarp = 13;
+constexpr int kSoftmaxRegs = 152;  // per SM sub-partition: 152 + 152 + 104 + 96 = 504 <= 4 x 128 launched
+constexpr int kEpilogueRegs = 104;
+constexpr int kControlRegs = 96;
 constexpr int kTileBytes = 32768;    // 128 x 128 bf16, as two 128-byte-wide halves
 constexpr int kHalfBytes = 16384;
 constexpr int kKeysPerTile = 128;
 constexpr uint64_t kTimeoutNs = 2000000000ull;
 constexpr float kRescaleLog2 = 8.0f;
+constexpr int kSoftmaxThreads = 256;
+constexpr int kEpiThreads = 128;
 
-constexpr int kOffQ = 0;                                   // 2 x 32 KB
-constexpr int kOffKV = 2 * kTileBytes;                     // kNB x 32 KB
-constexpr int kOffBar = kOffKV + kNB * kTileBytes;
-constexpr int kNumBars = 2 * kNB + 2 * 5 + 1;
-constexpr int kSmemBytes = kOffBar + kNumBars * 8 + 64 + 1024;  // + alignment slack
+constexpr uint32_t kColS = 0, kColP = 128, kColO0 = 256;  // O[b] at kColO0 + 128 b
+
+constexpr int kOffQ = 0;                                  // Q[2]
+constexpr int kOffK = 2 * kTileBytes;                     // K[2]
+constexpr int kOffV = 4 * kTileBytes;                     // V[2]
+constexpr int kOffRed = 6 * kTileBytes;                   // float [2][2][128]: row-max halves by tile parity
+constexpr int kOffStat = kOffRed + 2 * 2 * 128 * 4;       // float [2][3][128]: m, l0, l1 by item parity
+constexpr int kOffBar = kOffStat + 2 * 3 * 128 * 4;
 
 struct Bars {
-    uint64_t kv_full[kNB];
-    uint64_t kv_empty[kNB];
-    uint64_t q_full[2];
-    uint64_t q_empty[2];
-    uint64_t s_full[2];
-    uint64_t p_full[2];
-    uint64_t pv_done[2];
+    uint64_t q_full[2], q_empty[2];
+    uint64_t k_full[2], k_empty[2];
+    uint64_t v_full[2], v_empty[2];
+    uint64_t s_full, s_free;
+    uint64_t p_full, pv_done;
+    uint64_t red_bar[2];    // row-max halves of tile n written (by tile parity)
+    uint64_t stat_full[2];  // m and l of item i written (by item parity)
+    uint64_t o_ready[2];    // last PV of item i complete (by item parity)
+    uint64_t o_free[2];     // epilogue has read O[i % 2]
     uint64_t drain;
     uint32_t tmem_base;
     int32_t abort_flag;
     int32_t status0;
 };
+
+constexpr int kSmemBytes = kOffBar + (int)sizeof(Bars) + 1024;  // + alignment slack
 
 struct TileRef {
     int64_t id;
@@ -75,8 +87,8 @@ struct TileRef {
     int32_t nvis, ntiles, t;
 };
 
-// The items of one slot (queue positions first, first+2, ...), fetched ahead: each call hands out
-// the next (item id, anchor) and issues the loads one link further for the three items after it
+// The CTA's items (queue positions first, first+1, ...), fetched ahead: each call hands out the
+// next (item id, anchor) and issues the loads one link further for the three items after it
 // (anchor of n+1, id of n+2, queue entry of n+3), so no role waits on a dependent global load
 // chain when it moves to a new item.
 struct ItemStream {
@@ -87,7 +99,7 @@ struct ItemStream {
     int32_t k3;   // queue entry of item n+3 (in flight)
 };
 
-__device__ __forceinline__ int64_t load_id(const Meta& m, const int32_t* __restrict__ item_id, int32_t k) {
+__device__ __forceinline__ int64_t load_id(const int32_t* __restrict__ item_id, int32_t k) {
     return k >= 0 ? (int64_t)__ldg(item_id + k) : -1;
 }
 __device__ __forceinline__ int32_t load_anchor(const Meta& m, const int32_t* __restrict__ anchors, int64_t id) {
@@ -97,14 +109,14 @@ __device__ __forceinline__ int32_t load_anchor(const Meta& m, const int32_t* __r
 __device__ __forceinline__ void stream_init(const Meta& m, const int32_t* anchors, const int32_t* item_id,
                                             const int32_t* queue_items, int32_t first, int32_t end, ItemStream& st) {
     st.end = end;
-    st.left = first < end ? (end - first + 1) / 2 : 0;
+    st.left = first < end ? end - first : 0;
     const int32_t k0 = st.left > 0 ? __ldg(queue_items + first) : -1;
-    const int32_t k1 = st.left > 1 ? __ldg(queue_items + first + 2) : -1;
-    st.k3 = st.left > 2 ? __ldg(queue_items + first + 4) : -1;
-    st.id1 = load_id(m, item_id, k0);
-    st.id2 = load_id(m, item_id, k1);
+    const int32_t k1 = st.left > 1 ? __ldg(queue_items + first + 1) : -1;
+    st.k3 = st.left > 2 ? __ldg(queue_items + first + 2) : -1;
+    st.id1 = load_id(item_id, k0);
+    st.id2 = load_id(item_id, k1);
     st.a1 = load_anchor(m, anchors, st.id1);
-    st.pos = first + 6;
+    st.pos = first + 3;
 }
 
 // Next item as a tile reference (ntiles == 0 for an invalid entry, which raises BAD_PLAN).
@@ -115,9 +127,9 @@ __device__ __forceinline__ void stream_next(const Meta& m, const int32_t* anchor
     --st.left;
     st.a1 = load_anchor(m, anchors, st.id2);
     st.id1 = st.id2;
-    st.id2 = load_id(m, item_id, st.k3);
+    st.id2 = load_id(item_id, st.k3);
     st.k3 = st.pos < st.end ? __ldg(queue_items + st.pos) : -1;
-    st.pos += 2;
+    st.pos += 1;
     if (id < 0 || id >= m.n_items) {
         raise_status(status, SPLITKV_DEV_BAD_PLAN);
         tr.ntiles = 0;
@@ -134,7 +146,7 @@ __device__ __forceinline__ void stream_next(const Meta& m, const int32_t* anchor
     tr.t = 0;
 }
 
-// Items of one slot as a sequence of key tiles.
+// The CTA's items as one sequence of key tiles.
 struct Cursor {
     ItemStream st;
     bool has;
@@ -174,8 +186,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                   float* __restrict__ o_part, float* __restrict__ lse_part, int32_t* __restrict__ status) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t* q_smem = smem + kOffQ;
-    uint8_t* kv_smem = smem + kOffKV;
+    float* red = reinterpret_cast<float*>(smem + kOffRed);
+    float* stat = reinterpret_cast<float*>(smem + kOffStat);
     Bars* bars = reinterpret_cast<Bars*>(smem + kOffBar);
     volatile int* abort_flag = &bars->abort_flag;
 
@@ -183,17 +195,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int32_t q0 = queue_off[blockIdx.x], q1 = queue_off[blockIdx.x + 1];
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < kNB; ++i) {
-            mbar_init(&bars->kv_full[i], 1);
-            mbar_init(&bars->kv_empty[i], 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&bars->q_full[b], 1);
+            mbar_init(&bars->q_empty[b], 1);
+            mbar_init(&bars->k_full[b], 1);
+            mbar_init(&bars->k_empty[b], 1);
+            mbar_init(&bars->v_full[b], 1);
+            mbar_init(&bars->v_empty[b], 1);
+            mbar_init(&bars->red_bar[b], kSoftmaxThreads);
+            mbar_init(&bars->stat_full[b], kSoftmaxThreads);
+            mbar_init(&bars->o_ready[b], 1);
+            mbar_init(&bars->o_free[b], kEpiThreads);
         }
-        for (int k = 0; k < 2; ++k) {
-            mbar_init(&bars->q_full[k], 1);
-            mbar_init(&bars->q_empty[k], 1);
-            mbar_init(&bars->s_full[k], 1);
-            mbar_init(&bars->p_full[k], 128);
-            mbar_init(&bars->pv_done[k], 1);
-        }
+        mbar_init(&bars->s_full, 1);
+        mbar_init(&bars->s_free, kSoftmaxThreads);
+        mbar_init(&bars->p_full, kSoftmaxThreads);
+        mbar_init(&bars->pv_done, 1);
         mbar_init(&bars->drain, 1);
         bars->abort_flag = 0;
         bars->status0 = status_bad(status) ? 1 : 0;
@@ -201,7 +218,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     // Rows of the Q buffers beyond block*G are never loaded: keep them finite (zero).
     for (int i = threadIdx.x; i < 2 * kTileBytes / 16; i += kThreads)
-        reinterpret_cast<uint4*>(q_smem)[i] = make_uint4(0, 0, 0, 0);
+        reinterpret_cast<uint4*>(smem + kOffQ)[i] = make_uint4(0, 0, 0, 0);
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     if (warp == kMmaWarp) {
         tmem_alloc(&bars->tmem_base, 512);
@@ -212,239 +229,287 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     const uint32_t tmem = bars->tmem_base;
     const bool skip = bars->status0 != 0 || q0 >= q1;
-
     const int G = m.group, R = m.rows;
-    const uint32_t tS[2] = {tmem + 0u, tmem + 128u};
-    const uint32_t tO[2] = {tmem + 256u, tmem + 384u};
+    const uint32_t tS = tmem + kColS, tP = tmem + kColP;
 
-    if (warp >= 8) {
-        // Control warpgroup: give registers to the softmax warpgroups.
+    if (warp >= kProducerWarp) {
+        // ------------------------------------------------------------ control warpgroup
         asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(kControlRegs));
-        if (!skip && warp == kProducerWarp) {
-            if (lane == 0) {
-                tma_prefetch_desc(&tmQ);
-                tma_prefetch_desc(&tmK);
-                tma_prefetch_desc(&tmV);
-                const uint32_t q_bytes = 2u * 64u * (uint32_t)G * (uint32_t)m.block * 2u;
-                Cursor cur[2];
-                TileRef pv_tile[2];
-                bool pending[2] = {false, false};
-                uint32_t kv_seq = 0, qseq[2] = {0, 0};
-                int32_t last_kv_parity[kNB];
-                bool issued[kNB];
-                for (int i = 0; i < kNB; ++i) { issued[i] = false; last_kv_parity[i] = 0; }
-                bool q_issued[2] = {false, false};
-                uint32_t q_last_parity[2] = {0, 0};
-                bool ok = true;
-                for (int k = 0; k < 2; ++k) cursor_init(m, anchors, item_id, queue_items, q0 + k, q1, cur[k], status);
-                auto load_kv = [&](const CUtensorMap* map, const TileRef& t) -> bool {
-                    const int buf = kv_seq % kNB;
-                    const uint32_t ph = (kv_seq / kNB) & 1u;
-                    if (!mbar_wait(&bars->kv_empty[buf], ph ^ 1u, abort_flag, kTimeoutNs)) return false;
-                    mbar_arrive_expect_tx(&bars->kv_full[buf], kTileBytes);
-                    const int32_t row = (int32_t)(m.key_off[t.s] + (int64_t)t.c * m.chunk + (int64_t)t.t * kKeysPerTile);
-                    uint8_t* dst = kv_smem + buf * kTileBytes;
-                    tma_load_3d(dst, map, &bars->kv_full[buf], 0, t.g, row);
-                    tma_load_3d(dst + kHalfBytes, map, &bars->kv_full[buf], 64, t.g, row);
-                    issued[buf] = true;
-                    last_kv_parity[buf] = (int32_t)ph;
-                    ++kv_seq;
-                    return true;
-                };
-                auto emit_qk = [&](int k) -> bool {
-                    const TileRef t = cur[k].cur;
-                    if (t.t == 0) {
-                        if (!mbar_wait(&bars->q_empty[k], (qseq[k] & 1u) ^ 1u, abort_flag, kTimeoutNs)) return false;
-                        mbar_arrive_expect_tx(&bars->q_full[k], q_bytes);
-                        uint8_t* dst = q_smem + k * kTileBytes;
-                        tma_load_3d(dst, &tmQ, &bars->q_full[k], 0, t.g * G, m.block * t.j);
-                        tma_load_3d(dst + kHalfBytes, &tmQ, &bars->q_full[k], 64, t.g * G, m.block * t.j);
-                        q_issued[k] = true;
-                        q_last_parity[k] = qseq[k] & 1u;
-                        ++qseq[k];
+        if (!skip && warp == kProducerWarp && lane == 0) {
+            tma_prefetch_desc(&tmQ);
+            tma_prefetch_desc(&tmK);
+            tma_prefetch_desc(&tmV);
+            const uint32_t q_bytes = 2u * 64u * (uint32_t)G * (uint32_t)m.block * 2u;
+            Cursor cur;
+            TileRef prev;
+            uint32_t n = 0, item_seq = 0;
+            bool ok = true;
+            cursor_init(m, anchors, item_id, queue_items, q0, q1, cur, status);
+            auto load_tile = [&](const CUtensorMap* map, uint64_t* full, uint64_t* empty, uint32_t idx, int off,
+                                 const TileRef& t) -> bool {
+                const int b = idx & 1;
+                if (!mbar_wait(&empty[b], ((idx >> 1) & 1u) ^ 1u, abort_flag, kTimeoutNs)) return false;
+                mbar_arrive_expect_tx(&full[b], kTileBytes);
+                const int32_t row = (int32_t)(m.key_off[t.s] + (int64_t)t.c * m.chunk + (int64_t)t.t * kKeysPerTile);
+                uint8_t* dst = smem + off + b * kTileBytes;
+                tma_load_3d(dst, map, &full[b], 0, t.g, row);
+                tma_load_3d(dst + kHalfBytes, map, &full[b], 64, t.g, row);
+                return true;
+            };
+            // Order: Q (new item), K(n), V(n-1).
+            while (ok && cur.has) {
+                const TileRef t = cur.cur;
+                if (t.t == 0) {
+                    const int qb = item_seq & 1;
+                    if (!mbar_wait(&bars->q_empty[qb], ((item_seq >> 1) & 1u) ^ 1u, abort_flag, kTimeoutNs)) {
+                        ok = false;
+                        break;
                     }
-                    if (!load_kv(&tmK, t)) return false;
-                    pv_tile[k] = t;
-                    pending[k] = true;
-                    cursor_advance(m, anchors, item_id, queue_items, cur[k], status);
-                    return true;
-                };
-                for (int k = 0; k < 2 && ok; ++k)
-                    if (cur[k].has) ok = emit_qk(k);
-                while (ok && (pending[0] || pending[1])) {
-                    for (int k = 0; k < 2 && ok; ++k) {
-                        if (pending[k]) {
-                            ok = load_kv(&tmV, pv_tile[k]);
-                            pending[k] = false;
+                    mbar_arrive_expect_tx(&bars->q_full[qb], q_bytes);
+                    uint8_t* dst = smem + kOffQ + qb * kTileBytes;
+                    tma_load_3d(dst, &tmQ, &bars->q_full[qb], 0, t.g * G, m.block * t.j);
+                    tma_load_3d(dst + kHalfBytes, &tmQ, &bars->q_full[qb], 64, t.g * G, m.block * t.j);
+                    ++item_seq;
+                }
+                ok = load_tile(&tmK, bars->k_full, bars->k_empty, n, kOffK, t);
+                if (ok && n > 0) ok = load_tile(&tmV, bars->v_full, bars->v_empty, n - 1, kOffV, prev);
+                prev = t;
+                ++n;
+                cursor_advance(m, anchors, item_id, queue_items, cur, status);
+            }
+            if (ok && n > 0) ok = load_tile(&tmV, bars->v_full, bars->v_empty, n - 1, kOffV, prev);
+            // Drain: the most recent copy into every buffer has landed before the CTA exits.
+            volatile int never = 0;
+            for (uint32_t x = (n > 2 ? n - 2 : 0); x < n; ++x) {
+                mbar_wait(&bars->k_full[x & 1], (x >> 1) & 1u, &never, kTimeoutNs);
+                mbar_wait(&bars->v_full[x & 1], (x >> 1) & 1u, &never, kTimeoutNs);
+            }
+            for (uint32_t x = (item_seq > 2 ? item_seq - 2 : 0); x < item_seq; ++x)
+                mbar_wait(&bars->q_full[x & 1], (x >> 1) & 1u, &never, kTimeoutNs);
+        } else if (!skip && warp == kMmaWarp && lane == 0) {
+            constexpr uint32_t idesc_qk = umma_idesc_bf16_f32(128, 128, false, false);
+            constexpr uint32_t idesc_pv = umma_idesc_bf16_f32(128, 128, false, true);
+            // Descriptor bases; a K step only adds a constant to the (16-byte unit) start address.
+            uint64_t dq[2], dk[2], dv[2];
+            for (int b = 0; b < 2; ++b) {
+                dq[b] = umma_desc_sw128(smem_u32(smem + kOffQ + b * kTileBytes), 16, 1024);
+                dk[b] = umma_desc_sw128(smem_u32(smem + kOffK + b * kTileBytes), 16, 1024);
+                dv[b] = umma_desc_sw128(smem_u32(smem + kOffV + b * kTileBytes), kHalfBytes, 1024);
+            }
+            Cursor cur;
+            uint32_t n = 0, item_seq = 0, qb = 0, cur_item = 0;
+            bool pending = false, pv_first = false, pv_last = false;
+            uint32_t pv_n = 0, pv_item = 0;
+            bool ok = true;
+            cursor_init(m, anchors, item_id, queue_items, q0, q1, cur, status);
+            auto issue_pv = [&]() -> bool {
+                // PV(pv_n): O[item % 2] (+)= P V, A = P from TMEM (bf16 pairs), B = V, MN-major.
+                if (!mbar_wait(&bars->p_full, pv_n & 1u, abort_flag, kTimeoutNs)) return false;
+                const int ob = pv_item & 1;
+                if (pv_first && pv_item >= 2 &&
+                    !mbar_wait(&bars->o_free[ob], ((pv_item >> 1) - 1) & 1u, abort_flag, kTimeoutNs))
+                    return false;
+                const int vb = pv_n & 1;
+                if (!mbar_wait(&bars->v_full[vb], (pv_n >> 1) & 1u, abort_flag, kTimeoutNs)) return false;
+                tc_fence_after();
+                const uint32_t to = tmem + kColO0 + 128u * ob;
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_ts(to, tP + (uint32_t)(kk * 8), dv[vb] + (uint64_t)(kk * 2048 / 16), idesc_pv,
+                           (!pv_first || kk > 0) ? 1u : 0u);
+                mma_commit(&bars->pv_done);
+                if (pv_last) mma_commit(&bars->o_ready[ob]);
+                return true;
+            };
+            while (ok && cur.has) {
+                const TileRef t = cur.cur;
+                // QK^T(n) into S: the softmax must hold S(n-1) in registers already.
+                if (n >= 1 && !mbar_wait(&bars->s_free, (n - 1) & 1u, abort_flag, kTimeoutNs)) {
+                    ok = false;
+                    break;
+                }
+                if (t.t == 0) {
+                    qb = item_seq & 1;
+                    if (!mbar_wait(&bars->q_full[qb], (item_seq >> 1) & 1u, abort_flag, kTimeoutNs)) {
+                        ok = false;
+                        break;
+                    }
+                    cur_item = item_seq++;
+                }
+                const int kb = n & 1;
+                if (!mbar_wait(&bars->k_full[kb], (n >> 1) & 1u, abort_flag, kTimeoutNs)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint64_t off = (uint64_t)(((kk >> 2) * kHalfBytes + (kk & 3) * 32) / 16);
+                    mma_ss(tS, dq[qb] + off, dk[kb] + off, idesc_qk, kk > 0 ? 1u : 0u);
+                }
+                mma_commit(&bars->s_full);
+                // PV(n-1) once its P is ready.
+                if (pending && !(ok = issue_pv())) break;
+                pending = true;
+                pv_n = n;
+                pv_item = cur_item;
+                pv_first = (t.t == 0);
+                pv_last = (t.t == t.ntiles - 1);
+                ++n;
+                cursor_advance(m, anchors, item_id, queue_items, cur, status);
+            }
+            if (ok && pending) ok = issue_pv();
+            if (!ok) *abort_flag = 1;
+            // Drain: all MMAs issued by this thread complete before TMEM is released.
+            mma_commit(&bars->drain);
+            volatile int never = 0;
+            mbar_wait(&bars->drain, 0, &never, kTimeoutNs);
+        }
+        __syncwarp();
+    } else if (warp >= kEpiWarp0) {
+        // ------------------------------------------------------------ epilogue warpgroup
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(kEpilogueRegs));
+        if (!skip) {
+            const int quad = warp & 3;
+            const int r = quad * 32 + lane;
+            const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+            uint32_t i = 0;
+            ItemStream st;
+            stream_init(m, anchors, item_id, queue_items, q0, q1, st);
+            while (st.left > 0) {
+                TileRef t;
+                stream_next(m, anchors, item_id, queue_items, st, t, status);
+                if (t.ntiles == 0) continue;
+                const int ob = i & 1;
+                if (!mbar_wait(&bars->stat_full[ob], (i >> 1) & 1u, abort_flag, kTimeoutNs)) break;
+                if (!mbar_wait(&bars->o_ready[ob], (i >> 1) & 1u, abort_flag, kTimeoutNs)) break;
+                tc_fence_after();
+                const float* sp = stat + ob * 384;
+                const float m_used = sp[r];
+                const float l_row = sp[128 + r] + sp[256 + r];
+                const float inv_l = 1.f / l_row;
+                float* op = o_part + t.id * (int64_t)R * 128;
+                const uint32_t to = tmem + kColO0 + 128u * ob + lane_off;
+#pragma unroll 1
+                for (int cc = 0; cc < 4; ++cc) {
+                    uint32_t ov[32];
+                    tmem_ld32(to + cc * 32, ov);
+                    tmem_wait_ld();
+                    if (cc == 3) {  // O[ob] fully read: the MMA may start item i+2 in it
+                        tc_fence_before();
+                        mbar_arrive(&bars->o_free[ob]);
+                    }
+                    if (r < R) {
+#pragma unroll
+                        for (int u = 0; u < 8; ++u) {
+                            float4 x = make_float4(__uint_as_float(ov[4 * u]) * inv_l,
+                                                   __uint_as_float(ov[4 * u + 1]) * inv_l,
+                                                   __uint_as_float(ov[4 * u + 2]) * inv_l,
+                                                   __uint_as_float(ov[4 * u + 3]) * inv_l);
+                            *reinterpret_cast<float4*>(op + ((int64_t)(cc * 8 + u) * R + r) * 4) = x;
                         }
-                        if (ok && cur[k].has) ok = emit_qk(k);
                     }
                 }
-                // Drain: every copy this warp issued must have landed before the CTA exits.
-                for (int i = 0; i < kNB; ++i)
-                    if (issued[i]) {
-                        volatile int never = 0;
-                        mbar_wait(&bars->kv_full[i], (uint32_t)last_kv_parity[i], &never, kTimeoutNs);
-                    }
-                for (int k = 0; k < 2; ++k)
-                    if (q_issued[k]) {
-                        volatile int never = 0;
-                        mbar_wait(&bars->q_full[k], q_last_parity[k], &never, kTimeoutNs);
-                    }
+                if (r < R) lse_part[t.id * R + r] = (m_used + lg2_approx(l_row)) * 0.6931471805599453f;
+                ++i;
             }
-            __syncwarp();
-        } else if (!skip && warp == kMmaWarp) {
-            if (lane == 0) {
-                constexpr uint32_t idesc_qk = umma_idesc_bf16_f32(128, 128, false, false);
-                constexpr uint32_t idesc_pv = umma_idesc_bf16_f32(128, 128, false, true);
-                const uint32_t q_base = smem_u32(q_smem), kv_base = smem_u32(kv_smem);
-                Cursor cur[2];
-                bool pending[2] = {false, false}, pv_first[2] = {false, false};
-                uint32_t kv_seq = 0, qseq[2] = {0, 0}, tile_seq[2] = {0, 0};
-                bool ok = true;
-                for (int k = 0; k < 2; ++k) cursor_init(m, anchors, item_id, queue_items, q0 + k, q1, cur[k], status);
-                auto emit_qk = [&](int k) -> bool {
-                    const TileRef t = cur[k].cur;
-                    if (tile_seq[k] > 0 &&
-                        !mbar_wait(&bars->pv_done[k], (tile_seq[k] - 1) & 1u, abort_flag, kTimeoutNs))
-                        return false;
-                    if (t.t == 0) {
-                        if (!mbar_wait(&bars->q_full[k], qseq[k] & 1u, abort_flag, kTimeoutNs)) return false;
-                        ++qseq[k];
-                    }
-                    const int buf = kv_seq % kNB;
-                    if (!mbar_wait(&bars->kv_full[buf], (kv_seq / kNB) & 1u, abort_flag, kTimeoutNs)) return false;
-                    tc_fence_after();
-                    const uint32_t qa = q_base + k * kTileBytes, kb = kv_base + buf * kTileBytes;
-    #pragma unroll
-                    for (int kk = 0; kk < 8; ++kk) {
-                        const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
-                        mma_ss(tS[k], umma_desc_sw128(qa + off, 16, 1024), umma_desc_sw128(kb + off, 16, 1024),
-                               idesc_qk, kk > 0 ? 1u : 0u);
-                    }
-                    mma_commit(&bars->s_full[k]);
-                    mma_commit(&bars->kv_empty[buf]);
-                    if (t.t == t.ntiles - 1) mma_commit(&bars->q_empty[k]);
-                    ++kv_seq;
-                    pv_first[k] = (t.t == 0);
-                    pending[k] = true;
-                    ++tile_seq[k];
-                    cursor_advance(m, anchors, item_id, queue_items, cur[k], status);
-                    return true;
-                };
-                auto emit_pv = [&](int k) -> bool {
-                    if (!mbar_wait(&bars->p_full[k], (tile_seq[k] - 1) & 1u, abort_flag, kTimeoutNs)) return false;
-                    const int buf = kv_seq % kNB;
-                    if (!mbar_wait(&bars->kv_full[buf], (kv_seq / kNB) & 1u, abort_flag, kTimeoutNs)) return false;
-                    tc_fence_after();
-                    const uint32_t vb = kv_base + buf * kTileBytes;
-    #pragma unroll
-                    for (int kk = 0; kk < 8; ++kk) {
-                        // A = P[:, 16kk .. 16kk+16) packed two bf16 per column; B = V rows 16kk.., MN-major.
-                        mma_ts(tO[k], tS[k] + (uint32_t)(kk * 8), umma_desc_sw128(vb + kk * 2048, kHalfBytes, 1024),
-                               idesc_pv, (!pv_first[k] || kk > 0) ? 1u : 0u);
-                    }
-                    mma_commit(&bars->pv_done[k]);
-                    mma_commit(&bars->kv_empty[buf]);
-                    ++kv_seq;
-                    pending[k] = false;
-                    return true;
-                };
-                for (int k = 0; k < 2 && ok; ++k)
-                    if (cur[k].has) ok = emit_qk(k);
-                while (ok && (pending[0] || pending[1])) {
-                    for (int k = 0; k < 2 && ok; ++k) {
-                        if (pending[k]) ok = emit_pv(k);
-                        if (ok && cur[k].has) ok = emit_qk(k);
-                    }
-                }
-                // Drain: all MMAs issued by this thread complete before TMEM is released.
-                mma_commit(&bars->drain);
-                volatile int never = 0;
-                mbar_wait(&bars->drain, 0, &never, kTimeoutNs);
-            }
-            __syncwarp();
         }
     } else {
+        // ------------------------------------------------------------ softmax warpgroups
         asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(kSoftmaxRegs));
         if (!skip) {
-            const int k = warp >> 2;                // slot
+            const int wg = warp >> 2;               // key-column half
             const int quad = warp & 3;              // TMEM lane quadrant
             const int r = quad * 32 + lane;         // query-tile row
             const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
             const float c = m.scale * 1.4426950408889634f;  // log2(e)
             const uint64_t c2 = f2_pack(c, c);
-            uint32_t tile_seq = 0;
+            const bool leader = threadIdx.x == 0;
+            uint32_t n = 0, i = 0;
             bool ok = true;
             ItemStream st;
-            stream_init(m, anchors, item_id, queue_items, q0 + k, q1, st);
+            stream_init(m, anchors, item_id, queue_items, q0, q1, st);
             while (st.left > 0 && ok) {
                 TileRef t;
                 stream_next(m, anchors, item_id, queue_items, st, t, status);
                 if (t.ntiles == 0) continue;
+                const int ob = i & 1;
+                const uint32_t to = tmem + kColO0 + 128u * ob + lane_off + wg * 64;
                 float m_used = -INFINITY, l = 0.f;
-                for (int tt = 0; tt < t.ntiles; ++tt) {
-                    if (!mbar_wait(&bars->s_full[k], tile_seq & 1u, abort_flag, kTimeoutNs)) { ok = false; break; }
+                for (int tt = 0; tt < t.ntiles; ++tt, ++n) {
+                    if (!mbar_wait(&bars->s_full, n & 1u, abort_flag, kTimeoutNs)) { ok = false; break; }
                     tc_fence_after();
-                    // The whole S row in registers: one TMEM round trip.
-                    uint32_t sr[128];
-    #pragma unroll
-                    for (int cc = 0; cc < 4; ++cc)
-                        tmem_ld32(tS[k] + lane_off + cc * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[cc * 32]));
+                    uint32_t sr[64];
+                    tmem_ld32(tS + lane_off + wg * 64, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+                    tmem_ld32(tS + lane_off + wg * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
                     tmem_wait_ld();
-                    const int valid = t.nvis - tt * kKeysPerTile;  // keys of this tile the block sees (>= 1)
-                    if (valid < kKeysPerTile) {                    // only an item's last tile can be partial
-    #pragma unroll
-                        for (int u = 0; u < 128; ++u)
+                    tc_fence_before();
+                    mbar_arrive(&bars->s_free);  // S(n) is in registers: QK^T(n+1) may overwrite it
+                    if (leader) {                // QK^T(n) is complete: K(n), and Q after the item's last tile
+                        mbar_arrive(&bars->k_empty[n & 1]);
+                        if (tt == t.ntiles - 1) mbar_arrive(&bars->q_empty[i & 1]);
+                    }
+                    const int valid = t.nvis - tt * kKeysPerTile - wg * 64;  // visible keys in this half
+                    if (valid < 64) {                                        // only an item's last tile
+#pragma unroll
+                        for (int u = 0; u < 64; ++u)
                             if (u >= valid) sr[u] = __float_as_uint(-INFINITY);
                     }
                     float mx;
                     {
                         float m0 = -INFINITY, m1 = -INFINITY, m2 = -INFINITY, m3 = -INFINITY;
-    #pragma unroll
-                        for (int u = 0; u < 128; u += 8) {
+#pragma unroll
+                        for (int u = 0; u < 64; u += 8) {
                             m0 = max3f(m0, __uint_as_float(sr[u]), __uint_as_float(sr[u + 1]));
                             m1 = max3f(m1, __uint_as_float(sr[u + 2]), __uint_as_float(sr[u + 3]));
                             m2 = max3f(m2, __uint_as_float(sr[u + 4]), __uint_as_float(sr[u + 5]));
                             m3 = max3f(m3, __uint_as_float(sr[u + 6]), __uint_as_float(sr[u + 7]));
                         }
-                        mx = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3)) * c;
+                        // Exchange with the thread holding the other half of the row (bounded wait).
+                        const float mine = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
+                        float* rp = red + (n & 1) * 256;
+                        rp[wg * 128 + r] = mine;
+                        mbar_arrive(&bars->red_bar[n & 1]);
+                        if (!mbar_wait(&bars->red_bar[n & 1], (n >> 1) & 1u, abort_flag, kTimeoutNs)) {
+                            ok = false;
+                            break;
+                        }
+                        mx = fmaxf(mine, rp[(1 - wg) * 128 + r]) * c;
                     }
+                    bool pv_prev_done = (n == 0);
                     if (tt == 0) {
                         m_used = mx;
                     } else if (mx > m_used + kRescaleLog2) {
-                        // The previous PV of this slot completed before this tile's QK^T was issued.
+                        // Rescale this half of O once PV(n-1) has landed in it.
+                        if (!mbar_wait(&bars->pv_done, (n - 1) & 1u, abort_flag, kTimeoutNs)) { ok = false; break; }
+                        tc_fence_after();
+                        pv_prev_done = true;
                         const float alpha = ex2_approx(m_used - mx);
                         l *= alpha;
-    #pragma unroll 1
-                        for (int cc = 0; cc < 4; ++cc) {
+#pragma unroll 1
+                        for (int cc = 0; cc < 2; ++cc) {
                             uint32_t ov[32];
-                            tmem_ld32(tO[k] + lane_off + cc * 32, ov);
+                            tmem_ld32(to + cc * 32, ov);
                             tmem_wait_ld();
-    #pragma unroll
+#pragma unroll
                             for (int u = 0; u < 32; ++u) ov[u] = __float_as_uint(__uint_as_float(ov[u]) * alpha);
-                            tmem_st32(tO[k] + lane_off + cc * 32, ov);
+                            tmem_st32(to + cc * 32, ov);
                         }
                         m_used = mx;
                     }
-                    // P = 2^(s*c - m) in bf16, packed two per column over the first 64 columns of S.
+                    // P = 2^(s*c - m) in bf16 pairs: keys 64wg.. -> P columns 32wg..
                     const uint64_t negm2 = f2_pack(-m_used, -m_used);
                     uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
-    #pragma unroll
-                    for (int h = 0; h < 4; ++h) {
-                        uint32_t pk[16];
-    #pragma unroll
-                        for (int u = 0; u < 16; ++u) {
-                            const int v = h * 32 + 2 * u;
-                            float t0, t1;
-                            f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[v]), __uint_as_float(sr[v + 1])), c2, negm2), t0,
-                                      t1);
-                            const float p0 = ex2_approx(t0), p1 = ex2_approx(t1);
-                            acc[u & 3] = f2_add(acc[u & 3], f2_pack(p0, p1));
-                            __nv_bfloat162 hp = __floats2bfloat162_rn(p0, p1);  // .x (low half) = even key
-                            pk[u] = *reinterpret_cast<uint32_t*>(&hp);
-                        }
-                        tmem_st16(tS[k] + lane_off + h * 16, pk);
+                    uint32_t pk[32];
+#pragma unroll
+                    for (int u = 0; u < 32; ++u) {
+                        float t0, t1;
+                        f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[2 * u]), __uint_as_float(sr[2 * u + 1])), c2, negm2),
+                                  t0, t1);
+                        const float p0 = ex2_approx(t0), p1 = ex2_approx(t1);
+                        acc[u & 3] = f2_add(acc[u & 3], f2_pack(p0, p1));
+                        __nv_bfloat162 hp = __floats2bfloat162_rn(p0, p1);  // .x (low half) = even key
+                        pk[u] = *reinterpret_cast<uint32_t*>(&hp);
                     }
                     {
                         float a0, a1, b0, b1, c0, c1, d0, d1;
@@ -454,34 +519,30 @@ __global__ void __launch_bounds__(kThreads, 1)
                         f2_unpack(acc[3], d0, d1);
                         l += ((a0 + a1) + (b0 + b1)) + ((c0 + c1) + (d0 + d1));
                     }
+                    // P is single-buffered: PV(n-1), its last reader, must have completed.
+                    if (!pv_prev_done) {
+                        if (!mbar_wait(&bars->pv_done, (n - 1) & 1u, abort_flag, kTimeoutNs)) { ok = false; break; }
+                        tc_fence_after();
+                    }
+                    if (leader && n > 0) mbar_arrive(&bars->v_empty[(n - 1) & 1]);  // V(n-1) read
+                    tmem_st32(tP + lane_off + wg * 32, pk);
                     tmem_wait_st();
                     tc_fence_before();
-                    mbar_arrive(&bars->p_full[k]);
-                    ++tile_seq;
+                    mbar_arrive(&bars->p_full);
                 }
                 if (!ok) break;
-                // Epilogue: wait for the item's last PV, normalise, store partial O and LSE.
-                if (!mbar_wait(&bars->pv_done[k], (tile_seq - 1) & 1u, abort_flag, kTimeoutNs)) { ok = false; break; }
-                tc_fence_after();
-                const float inv_l = 1.f / l;
-                float* op = o_part + t.id * (int64_t)R * 128;
-    #pragma unroll 1
-                for (int cc = 0; cc < 4; ++cc) {
-                    uint32_t ov[32];
-                    tmem_ld32(tO[k] + lane_off + cc * 32, ov);
-                    tmem_wait_ld();
-                    if (r < R) {
-    #pragma unroll
-                        for (int u = 0; u < 8; ++u) {
-                            float4 x = make_float4(__uint_as_float(ov[4 * u]) * inv_l, __uint_as_float(ov[4 * u + 1]) * inv_l,
-                                                   __uint_as_float(ov[4 * u + 2]) * inv_l,
-                                                   __uint_as_float(ov[4 * u + 3]) * inv_l);
-                            *reinterpret_cast<float4*>(op + ((int64_t)(cc * 8 + u) * R + r) * 4) = x;
-                        }
-                    }
+                // Hand m and l to the epilogue; stat[i % 2] was last read by the epilogue of item i-2.
+                if (i >= 2 && !mbar_wait(&bars->o_free[ob], ((i >> 1) - 1) & 1u, abort_flag, kTimeoutNs)) {
+                    ok = false;
+                    break;
                 }
-                if (r < R) lse_part[t.id * R + r] = (m_used + lg2_approx(l)) * 0.6931471805599453f;
+                float* sp = stat + ob * 384;
+                if (wg == 0) sp[r] = m_used;
+                sp[128 + wg * 128 + r] = l;
+                mbar_arrive(&bars->stat_full[ob]);
+                ++i;
             }
+            if (!ok) *abort_flag = 1;
         }
     }
 
