@@ -9,21 +9,27 @@
 // one sequence n = 0, 1, ... across its items i = 0, 1, ...
 //
 // Roles (512 threads, four warpgroups; registers moved with setmaxnreg):
-//   WG0 / WG1 (warps 0-7)  softmax: row r = 32*(warp%4) + lane, key columns 0-63 / 64-127
+//   WG0 / WG1 (warps 0-7)  softmax of the even / odd key tiles: row r = 32*(warp%4) + lane
 //   WG2 (warps 8-11)       epilogue: normalises O of a finished item and stores O_c, LSE_c
 //   warp 12                TMA producer: Q per item (2 buffers), K(n) and V(n) (2 buffers each)
-//   warp 13                MMA issuer (one thread) and TMEM owner
+//   warp 13                QK^T issuer (one thread) and TMEM owner
+//   warp 14                PV issuer (one thread)
 //
-// TMEM (448 of 512 columns): S = Q K^T (128 fp32 columns), P (bf16 pairs, 64 columns) and
-// O[2] (128 fp32 columns each, one per item parity). The MMA thread issues QK^T(n) and then
-// PV(n-1): while the softmax turns S(n) into P(n), the tensor core runs PV(n-1) and, as soon as
-// the softmax holds S(n) in registers, QK^T(n+1). No MMA waits for another MMA, and an item's
-// epilogue overlaps the next item's tiles. The MMA thread only commits S-ready and PV-done; the
-// softmax warps release the K, V and Q buffers once those commits tell them the reads are over.
+// TMEM (all 512 columns): S[2] = Q K^T (128 fp32 columns each, tile n in S[n % 2]), P[2] (bf16
+// pairs, 64 columns each) and O (128 fp32 columns). A thread issuing tcgen05.mma waits while the
+// tensor core works through its previous instruction, and back-to-back MMAs into one accumulator
+// wait on each other; two threads issuing independent chains at the same moment keep the tensor
+// core busy. So both issuers start on the same event: when P(n) is written, one issues PV(n) and
+// the other QK^T(n+2) (S[n % 2] is free: the softmax of tile n has finished with it). The two
+// softmax warpgroups work on consecutive tiles at the same time, so one evaluates exponentials
+// while the other loads and reduces, and the epilogue warpgroup drains O while the next item's
+// scores are computed. The issuers only commit S-ready and PV-done; the softmax threads release
+// the K, V and Q buffers once those commits say the reads are over.
 //
-// Online softmax in log2 units (x = s * scale * log2 e); the two halves of a row exchange their
-// maxima through shared memory. The running reference max only moves when a tile's max exceeds it
-// by more than 8 (so P <= 256), which keeps O and l consistent and rescales O rarely.
+// Online softmax in log2 units (x = s * scale * log2 e). The running reference max m of a row only
+// moves when a tile's max exceeds it by more than 8 (so P <= 256); tile n publishes its m to tile
+// n+1 through shared memory, and a move rescales O (after PV(n-1)) and the row sums. Each
+// warpgroup sums P over its own tiles, relative to its latest m; the epilogue combines the two sums.
 // LSE = (m + log2 l) * ln 2.
 //
 // Every wait is bounded (2 s); on expiry the CTA raises SPLITKV_DEV_TIMEOUT, drains its copies and
@@ -42,7 +48,8 @@ using namespace sm100;
 constexpr int kThreads = 512;
 constexpr int kEpiWarp0 = 8;
 constexpr int kProducerWarp = 12;
-constexpr int kMmaWarp = 13;
+constexpr int kMmaWarp = 13;  // QK^T issuer, TMEM owner
+constexpr int kPvWarp = 14;
 constexpr int kSoftmaxRegs = 152;  // per SM sub-partition: 152 + 152 + 104 + 96 = 504 <= 4 x 128 launched
 constexpr int kEpilogueRegs = 104;
 constexpr int kControlRegs = 96;
@@ -51,29 +58,29 @@ constexpr int kHalfBytes = 16384;
 constexpr int kKeysPerTile = 128;
 constexpr uint64_t kTimeoutNs = 2000000000ull;
 constexpr float kRescaleLog2 = 8.0f;
-constexpr int kSoftmaxThreads = 256;
-constexpr int kEpiThreads = 128;
+constexpr int kWgThreads = 128;
 
-constexpr uint32_t kColS = 0, kColP = 128, kColO0 = 256;  // O[b] at kColO0 + 128 b
+constexpr uint32_t kColS0 = 0, kColP0 = 256, kColO = 384;  // S[b] at 128 b, P[b] at 256 + 64 b
 
 constexpr int kOffQ = 0;                                  // Q[2]
 constexpr int kOffK = 2 * kTileBytes;                     // K[2]
 constexpr int kOffV = 4 * kTileBytes;                     // V[2]
-constexpr int kOffRed = 6 * kTileBytes;                   // float [2][2][128]: row-max halves by tile parity
-constexpr int kOffStat = kOffRed + 2 * 2 * 128 * 4;       // float [2][3][128]: m, l0, l1 by item parity
-constexpr int kOffBar = kOffStat + 2 * 3 * 128 * 4;
+constexpr int kOffMdec = 6 * kTileBytes;                  // float [2][128]: reference max of tile n (n % 2)
+constexpr int kOffStat = kOffMdec + 2 * 128 * 4;          // float [2][2][2][128]: item parity, wg, (m, l)
+constexpr int kOffBar = kOffStat + 2 * 2 * 2 * 128 * 4;
 
 struct Bars {
     uint64_t q_full[2], q_empty[2];
     uint64_t k_full[2], k_empty[2];
     uint64_t v_full[2], v_empty[2];
-    uint64_t s_full, s_free;
-    uint64_t p_full, pv_done;
-    uint64_t red_bar[2];    // row-max halves of tile n written (by tile parity)
+    uint64_t s_full[2];     // QK^T(n) complete, by n % 2
+    uint64_t p_full[2];     // P(n) written, by n % 2
+    uint64_t pv_done[2];    // PV(n) complete, by n % 2
+    uint64_t mdec[2];       // reference max of tile n published, by n % 2
     uint64_t stat_full[2];  // m and l of item i written (by item parity)
     uint64_t o_ready[2];    // last PV of item i complete (by item parity)
-    uint64_t o_free[2];     // epilogue has read O[i % 2]
-    uint64_t drain;
+    uint64_t o_free[2];     // epilogue has read O for item i (by item parity)
+    uint64_t drain[2];      // all MMAs of the QK^T / PV issuer complete
     uint32_t tmem_base;
     int32_t abort_flag;
     int32_t status0;
@@ -186,7 +193,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                   float* __restrict__ o_part, float* __restrict__ lse_part, int32_t* __restrict__ status) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    float* red = reinterpret_cast<float*>(smem + kOffRed);
+    float* mdec = reinterpret_cast<float*>(smem + kOffMdec);
     float* stat = reinterpret_cast<float*>(smem + kOffStat);
     Bars* bars = reinterpret_cast<Bars*>(smem + kOffBar);
     volatile int* abort_flag = &bars->abort_flag;
@@ -202,16 +209,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&bars->k_empty[b], 1);
             mbar_init(&bars->v_full[b], 1);
             mbar_init(&bars->v_empty[b], 1);
-            mbar_init(&bars->red_bar[b], kSoftmaxThreads);
-            mbar_init(&bars->stat_full[b], kSoftmaxThreads);
+            mbar_init(&bars->s_full[b], 1);
+            mbar_init(&bars->p_full[b], kWgThreads);
+            mbar_init(&bars->pv_done[b], 1);
+            mbar_init(&bars->mdec[b], kWgThreads);
+            mbar_init(&bars->stat_full[b], 2 * kWgThreads);
             mbar_init(&bars->o_ready[b], 1);
-            mbar_init(&bars->o_free[b], kEpiThreads);
+            mbar_init(&bars->o_free[b], kWgThreads);
         }
-        mbar_init(&bars->s_full, 1);
-        mbar_init(&bars->s_free, kSoftmaxThreads);
-        mbar_init(&bars->p_full, kSoftmaxThreads);
-        mbar_init(&bars->pv_done, 1);
-        mbar_init(&bars->drain, 1);
+        mbar_init(&bars->drain[0], 1);
+        mbar_init(&bars->drain[1], 1);
         bars->abort_flag = 0;
         bars->status0 = status_bad(status) ? 1 : 0;
         fence_barrier_init();
@@ -230,7 +237,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tmem = bars->tmem_base;
     const bool skip = bars->status0 != 0 || q0 >= q1;
     const int G = m.group, R = m.rows;
-    const uint32_t tS = tmem + kColS, tP = tmem + kColP;
 
     if (warp >= kProducerWarp) {
         // ------------------------------------------------------------ control warpgroup
@@ -273,6 +279,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 ok = load_tile(&tmK, bars->k_full, bars->k_empty, n, kOffK, t);
                 if (ok && n > 0) ok = load_tile(&tmV, bars->v_full, bars->v_empty, n - 1, kOffV, prev);
+                if (!ok) break;
                 prev = t;
                 ++n;
                 cursor_advance(m, anchors, item_id, queue_items, cur, status);
@@ -287,83 +294,79 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (uint32_t x = (item_seq > 2 ? item_seq - 2 : 0); x < item_seq; ++x)
                 mbar_wait(&bars->q_full[x & 1], (x >> 1) & 1u, &never, kTimeoutNs);
         } else if (!skip && warp == kMmaWarp && lane == 0) {
+            // QK^T(0), QK^T(1) at once; QK^T(n) for n >= 2 when P(n-2) is written.
             constexpr uint32_t idesc_qk = umma_idesc_bf16_f32(128, 128, false, false);
-            constexpr uint32_t idesc_pv = umma_idesc_bf16_f32(128, 128, false, true);
             // Descriptor bases; a K step only adds a constant to the (16-byte unit) start address.
-            uint64_t dq[2], dk[2], dv[2];
+            uint64_t dq[2], dk[2];
             for (int b = 0; b < 2; ++b) {
                 dq[b] = umma_desc_sw128(smem_u32(smem + kOffQ + b * kTileBytes), 16, 1024);
                 dk[b] = umma_desc_sw128(smem_u32(smem + kOffK + b * kTileBytes), 16, 1024);
-                dv[b] = umma_desc_sw128(smem_u32(smem + kOffV + b * kTileBytes), kHalfBytes, 1024);
             }
             Cursor cur;
-            uint32_t n = 0, item_seq = 0, qb = 0, cur_item = 0;
-            bool pending = false, pv_first = false, pv_last = false;
-            uint32_t pv_n = 0, pv_item = 0;
-            bool ok = true;
+            uint32_t n = 0, item_seq = 0, qb = 0;
             cursor_init(m, anchors, item_id, queue_items, q0, q1, cur, status);
-            auto issue_pv = [&]() -> bool {
-                // PV(pv_n): O[item % 2] (+)= P V, A = P from TMEM (bf16 pairs), B = V, MN-major.
-                if (!mbar_wait(&bars->p_full, pv_n & 1u, abort_flag, kTimeoutNs)) return false;
-                const int ob = pv_item & 1;
-                if (pv_first && pv_item >= 2 &&
-                    !mbar_wait(&bars->o_free[ob], ((pv_item >> 1) - 1) & 1u, abort_flag, kTimeoutNs))
-                    return false;
-                const int vb = pv_n & 1;
-                if (!mbar_wait(&bars->v_full[vb], (pv_n >> 1) & 1u, abort_flag, kTimeoutNs)) return false;
-                tc_fence_after();
-                const uint32_t to = tmem + kColO0 + 128u * ob;
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    mma_ts(to, tP + (uint32_t)(kk * 8), dv[vb] + (uint64_t)(kk * 2048 / 16), idesc_pv,
-                           (!pv_first || kk > 0) ? 1u : 0u);
-                mma_commit(&bars->pv_done);
-                if (pv_last) mma_commit(&bars->o_ready[ob]);
-                return true;
-            };
-            while (ok && cur.has) {
+            while (cur.has) {
                 const TileRef t = cur.cur;
-                // QK^T(n) into S: the softmax must hold S(n-1) in registers already.
-                if (n >= 1 && !mbar_wait(&bars->s_free, (n - 1) & 1u, abort_flag, kTimeoutNs)) {
-                    ok = false;
-                    break;
-                }
+                const int sb = n & 1;
+                if (n >= 2 && !mbar_wait(&bars->p_full[sb], ((n >> 1) - 1) & 1u, abort_flag, kTimeoutNs)) break;
                 if (t.t == 0) {
                     qb = item_seq & 1;
-                    if (!mbar_wait(&bars->q_full[qb], (item_seq >> 1) & 1u, abort_flag, kTimeoutNs)) {
-                        ok = false;
-                        break;
-                    }
-                    cur_item = item_seq++;
+                    if (!mbar_wait(&bars->q_full[qb], (item_seq >> 1) & 1u, abort_flag, kTimeoutNs)) break;
+                    ++item_seq;
                 }
-                const int kb = n & 1;
-                if (!mbar_wait(&bars->k_full[kb], (n >> 1) & 1u, abort_flag, kTimeoutNs)) {
-                    ok = false;
-                    break;
-                }
+                if (!mbar_wait(&bars->k_full[sb], (n >> 1) & 1u, abort_flag, kTimeoutNs)) break;
                 tc_fence_after();
+                const uint32_t ts = tmem + kColS0 + 128u * sb;
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
                     const uint64_t off = (uint64_t)(((kk >> 2) * kHalfBytes + (kk & 3) * 32) / 16);
-                    mma_ss(tS, dq[qb] + off, dk[kb] + off, idesc_qk, kk > 0 ? 1u : 0u);
+                    mma_ss(ts, dq[qb] + off, dk[sb] + off, idesc_qk, kk > 0 ? 1u : 0u);
                 }
-                mma_commit(&bars->s_full);
-                // PV(n-1) once its P is ready.
-                if (pending && !(ok = issue_pv())) break;
-                pending = true;
-                pv_n = n;
-                pv_item = cur_item;
-                pv_first = (t.t == 0);
-                pv_last = (t.t == t.ntiles - 1);
+                mma_commit(&bars->s_full[sb]);
                 ++n;
                 cursor_advance(m, anchors, item_id, queue_items, cur, status);
             }
-            if (ok && pending) ok = issue_pv();
-            if (!ok) *abort_flag = 1;
             // Drain: all MMAs issued by this thread complete before TMEM is released.
-            mma_commit(&bars->drain);
+            mma_commit(&bars->drain[0]);
             volatile int never = 0;
-            mbar_wait(&bars->drain, 0, &never, kTimeoutNs);
+            mbar_wait(&bars->drain[0], 0, &never, kTimeoutNs);
+        } else if (!skip && warp == kPvWarp && lane == 0) {
+            // PV(n): O (+)= P(n) V(n), A = P[n % 2] from TMEM (bf16 pairs), B = V, MN-major. The first
+            // PV of item i overwrites O once the epilogue of item i-1 has read it.
+            constexpr uint32_t idesc_pv = umma_idesc_bf16_f32(128, 128, false, true);
+            uint64_t dv[2];
+            for (int b = 0; b < 2; ++b)
+                dv[b] = umma_desc_sw128(smem_u32(smem + kOffV + b * kTileBytes), kHalfBytes, 1024);
+            const uint32_t to = tmem + kColO;
+            Cursor cur;
+            uint32_t n = 0, item = 0;
+            cursor_init(m, anchors, item_id, queue_items, q0, q1, cur, status);
+            while (cur.has) {
+                const TileRef t = cur.cur;
+                const bool first = t.t == 0, last = t.t == t.ntiles - 1;
+                const int sb = n & 1;
+                if (!mbar_wait(&bars->p_full[sb], (n >> 1) & 1u, abort_flag, kTimeoutNs)) break;
+                if (first && item >= 1 &&
+                    !mbar_wait(&bars->o_free[(item - 1) & 1], ((item - 1) >> 1) & 1u, abort_flag, kTimeoutNs))
+                    break;
+                if (!mbar_wait(&bars->v_full[sb], (n >> 1) & 1u, abort_flag, kTimeoutNs)) break;
+                tc_fence_after();
+                const uint32_t tp = tmem + kColP0 + 64u * sb;
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_ts(to, tp + (uint32_t)(kk * 8), dv[sb] + (uint64_t)(kk * 2048 / 16), idesc_pv,
+                           (!first || kk > 0) ? 1u : 0u);
+                mma_commit(&bars->pv_done[sb]);
+                if (last) {
+                    mma_commit(&bars->o_ready[item & 1]);
+                    ++item;
+                }
+                ++n;
+                cursor_advance(m, anchors, item_id, queue_items, cur, status);
+            }
+            mma_commit(&bars->drain[1]);
+            volatile int never = 0;
+            mbar_wait(&bars->drain[1], 0, &never, kTimeoutNs);
         }
         __syncwarp();
     } else if (warp >= kEpiWarp0) {
@@ -384,18 +387,21 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!mbar_wait(&bars->stat_full[ob], (i >> 1) & 1u, abort_flag, kTimeoutNs)) break;
                 if (!mbar_wait(&bars->o_ready[ob], (i >> 1) & 1u, abort_flag, kTimeoutNs)) break;
                 tc_fence_after();
-                const float* sp = stat + ob * 384;
-                const float m_used = sp[r];
-                const float l_row = sp[128 + r] + sp[256 + r];
+                // Both warpgroups' sums, moved to the final reference max (the larger m: m only grows).
+                const float* sp = stat + ob * 512;
+                const float m0 = sp[r], l0 = sp[128 + r], m1 = sp[256 + r], l1 = sp[384 + r];
+                const float m_fin = fmaxf(m0, m1);
+                const float l_row = (l0 > 0.f ? l0 * ex2_approx(m0 - m_fin) : 0.f) +
+                                    (l1 > 0.f ? l1 * ex2_approx(m1 - m_fin) : 0.f);
                 const float inv_l = 1.f / l_row;
                 float* op = o_part + t.id * (int64_t)R * 128;
-                const uint32_t to = tmem + kColO0 + 128u * ob + lane_off;
+                const uint32_t to = tmem + kColO + lane_off;
 #pragma unroll 1
                 for (int cc = 0; cc < 4; ++cc) {
                     uint32_t ov[32];
                     tmem_ld32(to + cc * 32, ov);
                     tmem_wait_ld();
-                    if (cc == 3) {  // O[ob] fully read: the MMA may start item i+2 in it
+                    if (cc == 3) {  // O fully read: the issuer may start item i+1 in it
                         tc_fence_before();
                         mbar_arrive(&bars->o_free[ob]);
                     }
@@ -410,7 +416,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         }
                     }
                 }
-                if (r < R) lse_part[t.id * R + r] = (m_used + lg2_approx(l_row)) * 0.6931471805599453f;
+                if (r < R) lse_part[t.id * R + r] = (m_fin + lg2_approx(l_row)) * 0.6931471805599453f;
                 ++i;
             }
         }
@@ -418,13 +424,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ------------------------------------------------------------ softmax warpgroups
         asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(kSoftmaxRegs));
         if (!skip) {
-            const int wg = warp >> 2;               // key-column half
+            const int wg = warp >> 2;               // this warpgroup takes the tiles n with n % 2 == wg
             const int quad = warp & 3;              // TMEM lane quadrant
             const int r = quad * 32 + lane;         // query-tile row
             const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+            const uint32_t ts = tmem + kColS0 + 128u * wg + lane_off;  // S[wg], this row
+            const uint32_t tp = tmem + kColP0 + 64u * wg + lane_off;   // P[wg], this row
             const float c = m.scale * 1.4426950408889634f;  // log2(e)
             const uint64_t c2 = f2_pack(c, c);
-            const bool leader = threadIdx.x == 0;
+            const bool leader = (threadIdx.x & (kWgThreads - 1)) == 0;
             uint32_t n = 0, i = 0;
             bool ok = true;
             ItemStream st;
@@ -434,60 +442,68 @@ __global__ void __launch_bounds__(kThreads, 1)
                 stream_next(m, anchors, item_id, queue_items, st, t, status);
                 if (t.ntiles == 0) continue;
                 const int ob = i & 1;
-                const uint32_t to = tmem + kColO0 + 128u * ob + lane_off + wg * 64;
-                float m_used = -INFINITY, l = 0.f;
+                const uint32_t to = tmem + kColO + lane_off;
+                float m_l = -INFINITY, l = 0.f;  // this warpgroup's row sum, relative to m_l
                 for (int tt = 0; tt < t.ntiles; ++tt, ++n) {
-                    if (!mbar_wait(&bars->s_full, n & 1u, abort_flag, kTimeoutNs)) { ok = false; break; }
+                    if ((int)(n & 1) != wg) continue;
+                    if (!mbar_wait(&bars->s_full[wg], (n >> 1) & 1u, abort_flag, kTimeoutNs)) { ok = false; break; }
                     tc_fence_after();
-                    uint32_t sr[64];
-                    tmem_ld32(tS + lane_off + wg * 64, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-                    tmem_ld32(tS + lane_off + wg * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
-                    tmem_wait_ld();
-                    tc_fence_before();
-                    mbar_arrive(&bars->s_free);  // S(n) is in registers: QK^T(n+1) may overwrite it
-                    if (leader) {                // QK^T(n) is complete: K(n), and Q after the item's last tile
-                        mbar_arrive(&bars->k_empty[n & 1]);
+                    if (leader) {  // QK^T(n) complete: K(n) is free, and Q after the item's last tile
+                        mbar_arrive(&bars->k_empty[wg]);
                         if (tt == t.ntiles - 1) mbar_arrive(&bars->q_empty[i & 1]);
                     }
-                    const int valid = t.nvis - tt * kKeysPerTile - wg * 64;  // visible keys in this half
-                    if (valid < 64) {                                        // only an item's last tile
-#pragma unroll
-                        for (int u = 0; u < 64; ++u)
-                            if (u >= valid) sr[u] = __float_as_uint(-INFINITY);
-                    }
+                    const int valid = t.nvis - tt * kKeysPerTile;  // keys of this tile the block sees (>= 1)
+                    // Pass 1: row max over the visible keys, 64 columns per TMEM wait.
                     float mx;
                     {
                         float m0 = -INFINITY, m1 = -INFINITY, m2 = -INFINITY, m3 = -INFINITY;
+#pragma unroll 1
+                        for (int h = 0; h < 2; ++h) {
+                            uint32_t ra[32], rb[32];
+                            tmem_ld32(ts + h * 64, ra);
+                            tmem_ld32(ts + h * 64 + 32, rb);
+                            tmem_wait_ld();
+                            if (valid >= kKeysPerTile) {
 #pragma unroll
-                        for (int u = 0; u < 64; u += 8) {
-                            m0 = max3f(m0, __uint_as_float(sr[u]), __uint_as_float(sr[u + 1]));
-                            m1 = max3f(m1, __uint_as_float(sr[u + 2]), __uint_as_float(sr[u + 3]));
-                            m2 = max3f(m2, __uint_as_float(sr[u + 4]), __uint_as_float(sr[u + 5]));
-                            m3 = max3f(m3, __uint_as_float(sr[u + 6]), __uint_as_float(sr[u + 7]));
+                                for (int u = 0; u < 32; u += 4) {
+                                    m0 = max3f(m0, __uint_as_float(ra[u]), __uint_as_float(ra[u + 1]));
+                                    m1 = max3f(m1, __uint_as_float(ra[u + 2]), __uint_as_float(ra[u + 3]));
+                                    m2 = max3f(m2, __uint_as_float(rb[u]), __uint_as_float(rb[u + 1]));
+                                    m3 = max3f(m3, __uint_as_float(rb[u + 2]), __uint_as_float(rb[u + 3]));
+                                }
+                            } else {
+#pragma unroll
+                                for (int u = 0; u < 32; ++u) {
+                                    if (h * 64 + u < valid) m0 = fmaxf(m0, __uint_as_float(ra[u]));
+                                    if (h * 64 + 32 + u < valid) m1 = fmaxf(m1, __uint_as_float(rb[u]));
+                                }
+                            }
                         }
-                        // Exchange with the thread holding the other half of the row (bounded wait).
-                        const float mine = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
-                        float* rp = red + (n & 1) * 256;
-                        rp[wg * 128 + r] = mine;
-                        mbar_arrive(&bars->red_bar[n & 1]);
-                        if (!mbar_wait(&bars->red_bar[n & 1], (n >> 1) & 1u, abort_flag, kTimeoutNs)) {
+                        mx = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3)) * c;
+                    }
+                    // Reference max: tile n-1 publishes its m to tile n (every tile waits, which also
+                    // keeps a warpgroup from overwriting a slot its partner has not read yet).
+                    float m_prev = -INFINITY;
+                    if (n > 0) {
+                        if (!mbar_wait(&bars->mdec[(n - 1) & 1], ((n - 1) >> 1) & 1u, abort_flag, kTimeoutNs)) {
                             ok = false;
                             break;
                         }
-                        mx = fmaxf(mine, rp[(1 - wg) * 128 + r]) * c;
+                        if (tt > 0) m_prev = mdec[((n - 1) & 1) * 128 + r];
                     }
-                    bool pv_prev_done = (n == 0);
-                    if (tt == 0) {
-                        m_used = mx;
-                    } else if (mx > m_used + kRescaleLog2) {
-                        // Rescale this half of O once PV(n-1) has landed in it.
-                        if (!mbar_wait(&bars->pv_done, (n - 1) & 1u, abort_flag, kTimeoutNs)) { ok = false; break; }
+                    const float m_new = (tt == 0 || mx > m_prev + kRescaleLog2) ? mx : m_prev;
+                    mdec[(n & 1) * 128 + r] = m_new;
+                    mbar_arrive(&bars->mdec[n & 1]);
+                    if (tt > 0 && m_new != m_prev) {
+                        // The max moved: rescale this row of O once PV(n-1) has landed in it.
+                        if (!mbar_wait(&bars->pv_done[(n - 1) & 1], ((n - 1) >> 1) & 1u, abort_flag, kTimeoutNs)) {
+                            ok = false;
+                            break;
+                        }
                         tc_fence_after();
-                        pv_prev_done = true;
-                        const float alpha = ex2_approx(m_used - mx);
-                        l *= alpha;
+                        const float alpha = ex2_approx(m_prev - m_new);
 #pragma unroll 1
-                        for (int cc = 0; cc < 2; ++cc) {
+                        for (int cc = 0; cc < 4; ++cc) {
                             uint32_t ov[32];
                             tmem_ld32(to + cc * 32, ov);
                             tmem_wait_ld();
@@ -495,21 +511,50 @@ __global__ void __launch_bounds__(kThreads, 1)
                             for (int u = 0; u < 32; ++u) ov[u] = __float_as_uint(__uint_as_float(ov[u]) * alpha);
                             tmem_st32(to + cc * 32, ov);
                         }
-                        m_used = mx;
                     }
-                    // P = 2^(s*c - m) in bf16 pairs: keys 64wg.. -> P columns 32wg..
-                    const uint64_t negm2 = f2_pack(-m_used, -m_used);
+                    if (m_l != m_new) {
+                        l = (m_l == -INFINITY) ? 0.f : l * ex2_approx(m_l - m_new);
+                        m_l = m_new;
+                    }
+                    // P[wg] was last read by PV(n-2); once that completed, V(n-2) is free as well.
+                    if (n >= 2) {
+                        if (!mbar_wait(&bars->pv_done[wg], ((n >> 1) - 1) & 1u, abort_flag, kTimeoutNs)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        if (leader) mbar_arrive(&bars->v_empty[wg]);
+                    }
+                    // Pass 2: P = 2^(s*c - m) in bf16 pairs into P[wg] (keys 64h.. -> columns 32h..).
+                    const uint64_t negm2 = f2_pack(-m_new, -m_new);
                     uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
-                    uint32_t pk[32];
+#pragma unroll 1
+                    for (int h = 0; h < 2; ++h) {
+                        uint32_t ra[32], rb[32];
+                        tmem_ld32(ts + h * 64, ra);
+                        tmem_ld32(ts + h * 64 + 32, rb);
+                        tmem_wait_ld();
+                        if (valid < kKeysPerTile) {
 #pragma unroll
-                    for (int u = 0; u < 32; ++u) {
-                        float t0, t1;
-                        f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[2 * u]), __uint_as_float(sr[2 * u + 1])), c2, negm2),
-                                  t0, t1);
-                        const float p0 = ex2_approx(t0), p1 = ex2_approx(t1);
-                        acc[u & 3] = f2_add(acc[u & 3], f2_pack(p0, p1));
-                        __nv_bfloat162 hp = __floats2bfloat162_rn(p0, p1);  // .x (low half) = even key
-                        pk[u] = *reinterpret_cast<uint32_t*>(&hp);
+                            for (int u = 0; u < 32; ++u) {
+                                if (h * 64 + u >= valid) ra[u] = __float_as_uint(-INFINITY);
+                                if (h * 64 + 32 + u >= valid) rb[u] = __float_as_uint(-INFINITY);
+                            }
+                        }
+                        uint32_t pk[32];
+#pragma unroll
+                        for (int u = 0; u < 32; ++u) {
+                            const uint32_t* src = u < 16 ? ra : rb;
+                            const int v = (u & 15) * 2;
+                            float t0, t1;
+                            f2_unpack(f2_fma(f2_pack(__uint_as_float(src[v]), __uint_as_float(src[v + 1])), c2, negm2),
+                                      t0, t1);
+                            const float p0 = ex2_approx(t0), p1 = ex2_approx(t1);
+                            acc[u & 3] = f2_add(acc[u & 3], f2_pack(p0, p1));
+                            __nv_bfloat162 hp = __floats2bfloat162_rn(p0, p1);  // .x (low half) = even key
+                            pk[u] = *reinterpret_cast<uint32_t*>(&hp);
+                        }
+                        tmem_st32(tp + h * 32, pk);
                     }
                     {
                         float a0, a1, b0, b1, c0, c1, d0, d1;
@@ -519,26 +564,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                         f2_unpack(acc[3], d0, d1);
                         l += ((a0 + a1) + (b0 + b1)) + ((c0 + c1) + (d0 + d1));
                     }
-                    // P is single-buffered: PV(n-1), its last reader, must have completed.
-                    if (!pv_prev_done) {
-                        if (!mbar_wait(&bars->pv_done, (n - 1) & 1u, abort_flag, kTimeoutNs)) { ok = false; break; }
-                        tc_fence_after();
-                    }
-                    if (leader && n > 0) mbar_arrive(&bars->v_empty[(n - 1) & 1]);  // V(n-1) read
-                    tmem_st32(tP + lane_off + wg * 32, pk);
                     tmem_wait_st();
                     tc_fence_before();
-                    mbar_arrive(&bars->p_full);
+                    mbar_arrive(&bars->p_full[wg]);
                 }
                 if (!ok) break;
-                // Hand m and l to the epilogue; stat[i % 2] was last read by the epilogue of item i-2.
+                // Hand this warpgroup's (m, l) to the epilogue; stat[i % 2] was last read by the
+                // epilogue of item i-2.
                 if (i >= 2 && !mbar_wait(&bars->o_free[ob], ((i >> 1) - 1) & 1u, abort_flag, kTimeoutNs)) {
                     ok = false;
                     break;
                 }
-                float* sp = stat + ob * 384;
-                if (wg == 0) sp[r] = m_used;
-                sp[128 + wg * 128 + r] = l;
+                float* sp = stat + ob * 512 + wg * 256;
+                sp[r] = m_l;
+                sp[128 + r] = l;
                 mbar_arrive(&bars->stat_full[ob]);
                 ++i;
             }
@@ -554,7 +593,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_dealloc(tmem, 512);
     }
 }
-
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);

@@ -216,6 +216,17 @@ __device__ __forceinline__ float max3f(float a, float b, float c) {
     return d;
 }
 
+// 2^x for two bf16 values in one MUFU operation (argument and result rounded to bf16).
+__device__ __forceinline__ uint32_t ex2_bf16x2(uint32_t x) {
+    uint32_t y;
+    asm("ex2.approx.ftz.bf16x2 %0, %1;" : "=r"(y) : "r"(x));
+    return y;
+}
+// The two bf16 halves of a 32-bit word as one packed fp32 pair (exact: bf16 is the top of fp32).
+__device__ __forceinline__ uint64_t bf16x2_to_f2(uint32_t v) {
+    return f2_pack(__uint_as_float(v << 16), __uint_as_float(v & 0xFFFF0000u));
+}
+
 __device__ __forceinline__ float ex2_approx(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
