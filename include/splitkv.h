@@ -140,6 +140,28 @@ int splitkv_plan_lpt(const int32_t *item_cost_d, const int32_t *n_items_d, int32
                      size_t workspace_bytes, void *stream);
 
 /*
+ * Allocation-free variant of splitkv_plan_lpt (the Split-KV paper has no counterpart: this is a
+ * deployment convenience). Same arguments, same result, no workspace argument: its scratch is a
+ * fixed 4 MiB array inside the library's own device memory, which every GPU that loads the library
+ * holds until the process exits. It is meant for callers that cannot call cudaMalloc: code running
+ * while a CUDA graph is being captured, or inside a framework whose caching allocator owns all
+ * device memory and forbids side allocations, or a latency-critical path that cannot afford the
+ * synchronisation an allocation may imply.
+ *   - The first call on a device looks up the array's device address (cudaGetSymbolAddress) with
+ *     that device current and caches it; make that first call before any stream capture.
+ *   - Returns SPLITKV_ENOSPACE (with splitkv_last_error() stating both sizes) when the plan would
+ *     need more scratch than the array holds, i.e. splitkv_workspace_size() grows with max_items,
+ *     max_cost and n_workers.
+ *   - It allocates nothing and frees nothing. Every call shares the one array and leaves its
+ *     contents behind (the planner rewrites all it reads before reading it), so calls whose GPU
+ *     work overlaps — on two streams, or from two host threads — race and corrupt each other's
+ *     plans; order them on one stream.
+ */
+int splitkv_plan_lpt_noalloc(const int32_t *item_cost_d, const int32_t *n_items_d, int32_t max_items,
+                             int32_t max_cost, int32_t n_workers, int32_t *item_worker_d, int32_t *queue_off_d,
+                             int32_t *queue_items_d, int64_t *load_d, int32_t *status_d, void *stream);
+
+/*
  * Chunk-partial forward (Split-KV paper, Abstract: the method is exact and
  * exchanges only tensors the size of the query set). One persistent
  * CTA per worker walks its queue; for each item (s, c, g, b) it computes, over the keys of chunk c

@@ -61,6 +61,7 @@ _SIGS = {
     "splitkv_last_error": (ctypes.c_char_p, []),
     "splitkv_cost": (_i32, [_PP, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "splitkv_plan_lpt": (_i32, [_vp, _vp, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "splitkv_plan_lpt_noalloc": (_i32, [_vp, _vp, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _vp]),
     "splitkv_attn_fwd": (_i32, [_PP, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _vp, _i32, _vp]),
     "splitkv_lse_merge": (_i32, [_PP, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
     "splitkv_attn_bwd": (_i32, [_PP] + [_vp] * 15 + [_vp, _sz, _vp]),
@@ -75,7 +76,7 @@ for _name, (_res, _args) in _SIGS.items():
 class SplitKVError(RuntimeError):
     def __init__(self, code: int, where: str):
         self.code = code
-        detail = splitkv_last_error() if code == ECUDA else ""
+        detail = splitkv_last_error() if code in (ECUDA, ENOSPACE) else ""
         super().__init__(f"{where}: {splitkv_strerror(code)} ({code})" + (f" [{detail}]" if detail else ""))
 
 
@@ -149,6 +150,15 @@ def splitkv_plan_lpt(item_cost, n_items, max_items, max_cost, n_workers, item_wo
                                  _p(item_worker), _p(queue_off), _p(queue_items), _p(load), _p(status),
                                  _p(workspace), workspace.numel() * workspace.element_size(), _stream(stream)),
            "splitkv_plan_lpt")
+
+
+def splitkv_plan_lpt_noalloc(item_cost, n_items, max_items, max_cost, n_workers, item_worker, queue_off, queue_items,
+                             load, status, stream=None):
+    """splitkv_plan_lpt without a workspace: scratch comes from a static array inside the library
+    (for callers that cannot allocate device memory, e.g. during CUDA graph capture)."""
+    _check(_lib.splitkv_plan_lpt_noalloc(_p(item_cost), _p(n_items), int(max_items), int(max_cost), int(n_workers),
+                                         _p(item_worker), _p(queue_off), _p(queue_items), _p(load), _p(status),
+                                         _stream(stream)), "splitkv_plan_lpt_noalloc")
 
 
 def splitkv_attn_fwd(problem, q, k, v, anchors, item_id, queue_off, queue_items, n_workers, o_part, lse_part,

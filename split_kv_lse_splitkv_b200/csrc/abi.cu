@@ -159,6 +159,28 @@ SPLITKV_API int splitkv_plan_lpt(const int32_t* item_cost_d, const int32_t* n_it
                                    queue_off_d, queue_items_d, load_d, status_d, workspace_d, (cudaStream_t)stream));
 }
 
+SPLITKV_API int splitkv_plan_lpt_noalloc(const int32_t* item_cost_d, const int32_t* n_items_d, int32_t max_items,
+                                         int32_t max_cost, int32_t n_workers, int32_t* item_worker_d,
+                                         int32_t* queue_off_d, int32_t* queue_items_d, int64_t* load_d,
+                                         int32_t* status_d, void* stream) {
+    clear_error();
+    if (max_items < 0 || max_cost < 1 || max_cost > kMaxCost || n_workers < 1 || n_workers > 1024)
+        return SPLITKV_EINVAL;
+    if (!item_cost_d || !n_items_d || !item_worker_d || !queue_off_d || !queue_items_d || !load_d || !status_d)
+        return SPLITKV_EINVAL;
+    const size_t need = plan_workspace(max_items, max_cost, n_workers);
+    if (need > kStaticPlanScratchBytes) {
+        std::snprintf(g_last_error, sizeof(g_last_error),
+                      "splitkv_plan_lpt_noalloc: needs %zu bytes of scratch, the static array holds %zu", need,
+                      kStaticPlanScratchBytes);
+        return SPLITKV_ENOSPACE;
+    }
+    void* ws = nullptr;
+    if (static_plan_scratch(&ws) != cudaSuccess) return SPLITKV_ECUDA;
+    return cuda_status(launch_plan(item_cost_d, n_items_d, max_items, max_cost, n_workers, item_worker_d,
+                                   queue_off_d, queue_items_d, load_d, status_d, ws, (cudaStream_t)stream));
+}
+
 SPLITKV_API int splitkv_attn_fwd(const splitkv_problem* problem, const void* q, const void* k, const void* v,
                                  const int32_t* anchors_d, const int32_t* item_id_d, const int32_t* queue_off_d,
                                  const int32_t* queue_items_d, int32_t n_workers, float* o_part, float* lse_part,

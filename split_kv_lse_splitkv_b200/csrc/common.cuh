@@ -96,6 +96,10 @@ cudaError_t launch_plan(const int32_t* item_cost, const int32_t* n_items, int32_
                         int32_t n_workers, int32_t* item_worker, int32_t* queue_off, int32_t* queue_items,
                         int64_t* load, int32_t* status, void* ws, cudaStream_t st);
 size_t plan_workspace(int32_t max_items, int32_t max_cost, int32_t n_workers);
+// Device address of the planner's static scratch array on the current device (looked up once per device).
+constexpr size_t kStaticPlanScratchBytes = (size_t)4 << 20;
+constexpr int kMaxDevices = 64;
+cudaError_t static_plan_scratch(void** out);
 
 cudaError_t launch_fwd_simt(const Meta& m, const void* q, const void* k, const void* v, const int32_t* anchors,
                             const int32_t* item_id, const int32_t* queue_off, const int32_t* queue_items,

@@ -20,10 +20,17 @@
 // run, the catch-up element list, the q order and each worker's pick count, then the final loads
 // and queue offsets, (3) one thread per item places it. Every quantity is an integer, so the plan
 // equals the sequential greedy bit for bit.
+#include <mutex>
+
 #include "common.cuh"
 #include "scan.cuh"
 
 namespace splitkv {
+
+// Scratch for splitkv_plan_lpt_noalloc: a fixed array in the library's own device memory, so that
+// entry point needs no allocation. Every device that loads the library holds it until exit, and
+// all calls share it.
+static __device__ __align__(256) unsigned char g_plan_scratch[kStaticPlanScratchBytes];
 
 namespace {
 
@@ -300,6 +307,26 @@ __global__ void __launch_bounds__(kThreads) plan_assign_kernel(const int32_t* __
 }
 
 }  // namespace
+
+cudaError_t static_plan_scratch(void** out) {
+    // The array's device address differs per device; look it up once per device, with that device
+    // current (cudaGetSymbolAddress), and keep it. Host code must not use the symbol itself.
+    static std::mutex mu;
+    static void* addr[kMaxDevices] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return note_error(e, "cudaGetDevice");
+    if (dev < 0 || dev >= kMaxDevices) return note_error(cudaErrorInvalidDevice, "plan scratch: device index");
+    std::lock_guard<std::mutex> lock(mu);
+    if (!addr[dev]) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_plan_scratch);
+        if (e != cudaSuccess) return note_error(e, "cudaGetSymbolAddress(plan scratch)");
+        addr[dev] = p;
+    }
+    *out = addr[dev];
+    return cudaSuccess;
+}
 
 size_t plan_workspace(int32_t max_items, int32_t max_cost, int32_t n_workers) {
     size_t bytes = 0;
