@@ -48,6 +48,30 @@ def useful_flops(inp, backward):
     return fwd + bwd, per_pair * ctx_pairs
 
 
+def profiled_traffic(kernel, workload):
+    """DRAM bytes per launch from the committed ncu summary of `kernel` on `workload`, or None when
+    the summary is missing or the kernel's sources changed since it was captured."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", f"{kernel}.{workload}.txt")
+    try:
+        lines = open(path).read().splitlines()
+    except OSError:
+        return None
+    traffic = None
+    for ln in lines:
+        if ln.startswith("traffic_bytes_per_launch:"):
+            traffic = int(ln.split(":")[1])
+        elif ln.startswith("source_sha256 "):
+            rel, digest = ln[len("source_sha256 "):].split(": ")
+            try:
+                cur = hashlib.sha256(open(os.path.join(ROOT, rel), "rb").read()).hexdigest()
+            except OSError:
+                return None
+            if cur != digest.strip():
+                return None
+    return traffic
+
+
 def peaks():
     try:
         with open(PEAKS_FILE) as f:
@@ -344,7 +368,8 @@ def run_ours(args):
                        "heads": f"{w.n_q_heads}q/{w.n_kv_heads}kv", "head_dim": w.head_dim, "chunk": w.chunk,
                        "queues": skv.n_workers, "l2": "flushed (256 MB write) before every timed step",
                        "parallelism": f"replicas x{world}"},
-            "roofline": dict(roof, achieved=achieved, unit="TFLOP/s", frac=achieved / peak, traffic=None,
+            "roofline": dict(roof, achieved=achieved, unit="TFLOP/s", frac=achieved / peak,
+                             traffic=profiled_traffic("fwd_tc_kernel", w.name) if w.dtype == "bf16" else None,
                              kernel_ms=fwd_ms, algorithmic_flop=fwd_kernel_flops),
             "phase_ms": phase_ms,
             "imbalance": {"predicted_lpt": predicted_imb},
