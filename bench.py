@@ -40,12 +40,13 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 def useful_flops(inp, backward):
     w = inp.workload
+    # (query, key) pairs: each query of a block sees the a context keys and the block's own keys;
+    # the forward kernel computes both (context items and self items).
     pairs = sum(w.block * (int(a) + w.block) for a in inp.anchors.tolist())
-    ctx_pairs = sum(w.block * int(a) for a in inp.anchors.tolist())
     per_pair = 4 * w.head_dim * w.n_q_heads
     fwd = per_pair * pairs
     bwd = (10 * w.head_dim * w.n_q_heads * pairs) if backward else 0
-    return fwd + bwd, per_pair * ctx_pairs
+    return fwd + bwd, fwd
 
 
 def profiled_traffic(kernel, workload):
@@ -228,7 +229,7 @@ def run_reference(args):
 
 
 def run_ours(args):
-    from split_kv_lse_splitkv_b200 import SplitKV, splitkv_attn_fwd
+    from split_kv_lse_splitkv_b200 import SplitKV
 
     world, rank, local = dist_setup(args)
     device = torch.device("cuda", local)
@@ -266,9 +267,9 @@ def run_ours(args):
 
     def step(d, time_phases=False):
         timed("plan", lambda: skv.plan(d["anchors"], stream), time_phases)
-        timed("fwd", lambda: skv.attn_fwd(d["q"], d["k"], d["v"], d["anchors"], stream=stream), time_phases)
-        timed("merge", lambda: skv.lse_merge(d["q"], d["kb"], d["vb"], d["anchors"], o, lse, stream=stream),
+        timed("fwd", lambda: skv.attn_fwd(d["q"], d["k"], d["v"], d["kb"], d["vb"], d["anchors"], stream=stream),
               time_phases)
+        timed("merge", lambda: skv.lse_merge(d["anchors"], o, lse, stream=stream), time_phases)
         if w.backward:
             timed("bwd", lambda: skv.backward(d["q"], d["k"], d["v"], d["kb"], d["vb"], o, lse, d["do"], d["anchors"],
                                               grads, stream=stream), time_phases)

@@ -88,8 +88,8 @@ typedef struct {
     int64_t n_queries;      /* Nq                                                                     */
     int64_t total_keys;     /* sum_s S_s                                                              */
     int64_t n_blocks;       /* total anchors                                                          */
-    int64_t o_part_elems;   /* float32 elements of o_part: n_items_max * block*G * d                  */
-    int64_t lse_part_elems; /* float32 elements of lse_part: n_items_max * block*G                    */
+    int64_t o_part_elems;   /* float32 elements of o_part: (n_items_max + n_blocks*Hkv) * block*G * d */
+    int64_t lse_part_elems; /* float32 elements of lse_part: (n_items_max + n_blocks*Hkv) * block*G   */
     int32_t max_cost;       /* chunk / key_tile: the largest item cost                                */
     int32_t rows_per_item;  /* block * G: query rows of one item (its query tile)                     */
 } splitkv_sizes;
@@ -162,32 +162,35 @@ int splitkv_plan_lpt_noalloc(const int32_t *item_cost_d, const int32_t *n_items_
                              int32_t *queue_items_d, int64_t *load_d, int32_t *status_d, void *stream);
 
 /*
- * Chunk-partial forward (Split-KV paper, Abstract: the method is exact and
- * exchanges only tensors the size of the query set). One persistent
- * CTA per worker walks its queue; for each item (s, c, g, b) it computes, over the keys of chunk c
- * that block b sees, the chunk-local softmax of s = scale * q.k for the block*G query rows
- * (r = i*G + hl: query i of the block, query head g*G + hl) and writes
- *   o_part  [n_items_max][d/4][block*G][4]  float32: O_c = sum softmax * v, normalised
- *   lse_part[n_items_max][block*G]          float32: LSE_c = log sum exp(s), natural log
- * at the item's global index. Entries of items that are not visible are not written.
+ * Partial forward (Split-KV paper, Abstract: the method is exact and exchanges only tensors the
+ * size of the query set). One persistent CTA per worker walks its queue; for each item
+ * (s, c, g, b) it computes, over the keys of chunk c that block b sees, the chunk-local softmax of
+ * s = scale * q.k for the block*G query rows (r = i*G + hl: query i of the block, query head
+ * g*G + hl). After the queues the same CTAs compute the self partials: for global block j and kv
+ * head g, the softmax over the block's own `block` keys, kb/vb rows block*j .. block*j + block - 1
+ * ([Nq, Hkv, d], problem dtype), stored at slot n_items_max + j*Hkv + g. Both kinds write
+ *   o_part  [slot][d/4][block*G][4]  float32: O_p = sum softmax * v, normalised
+ *   lse_part[slot][block*G]          float32: LSE_p = log sum exp(s), natural log
+ * Entries of items that are not visible are not written.
  * item_id_d, queue_off_d and queue_items_d come from splitkv_cost and splitkv_plan_lpt.
- * flags: SPLITKV_FWD_DEFAULT or SPLITKV_FWD_SIMT.
+ * q, k, v, kb, vb and o_part must be 16-byte aligned. flags: SPLITKV_FWD_DEFAULT or
+ * SPLITKV_FWD_SIMT.
  */
 int splitkv_attn_fwd(const splitkv_problem *problem, const void *q, const void *k, const void *v,
-                     const int32_t *anchors_d, const int32_t *item_id_d, const int32_t *queue_off_d,
-                     const int32_t *queue_items_d, int32_t n_workers, float *o_part, float *lse_part,
-                     int32_t *status_d, int32_t flags, void *stream);
+                     const void *kb, const void *vb, const int32_t *anchors_d, const int32_t *item_id_d,
+                     const int32_t *queue_off_d, const int32_t *queue_items_d, int32_t n_workers,
+                     float *o_part, float *lse_part, int32_t *status_d, int32_t flags, void *stream);
 
 /*
  * Exact log-sum-exp merge (Split-KV paper, Abstract: exactness with query-sized exchange). For each
- * block and query head it adds the block's own-keys partial (the `block` rows of kb/vb at the kv
- * head) to the visible chunk partials c < ceil(a/C) and writes
- *   L = log sum exp(LSE_c), O = sum exp(LSE_c - L) O_c
- * to o [Nq, Hq, d] (problem dtype) and lse [Nq, Hq] (float32, natural log).
+ * block j, kv head g and row r it combines the self partial (slot n_items_max + j*Hkv + g) with the
+ * visible chunk partials c < ceil(a_j / C):
+ *   L = log sum_p exp(LSE_p),  O = sum_p exp(LSE_p - L) O_p
+ * and writes o [Nq, Hq, d] (problem dtype) and lse [Nq, Hq] (float32, natural log). o_part,
+ * lse_part and o must be 16-byte aligned. Reads only what splitkv_attn_fwd wrote.
  */
 int splitkv_lse_merge(const splitkv_problem *problem, const float *o_part, const float *lse_part,
-                      const void *q, const void *kb, const void *vb, const int32_t *anchors_d, void *o,
-                      float *lse, int32_t *status_d, void *stream);
+                      const int32_t *anchors_d, void *o, float *lse, int32_t *status_d, void *stream);
 
 /*
  * Backward of the same attention (Split-KV paper, title and Abstract: the method trains diffusion

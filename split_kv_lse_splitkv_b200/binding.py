@@ -62,8 +62,8 @@ _SIGS = {
     "splitkv_cost": (_i32, [_PP, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "splitkv_plan_lpt": (_i32, [_vp, _vp, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "splitkv_plan_lpt_noalloc": (_i32, [_vp, _vp, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _vp]),
-    "splitkv_attn_fwd": (_i32, [_PP, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _vp, _i32, _vp]),
-    "splitkv_lse_merge": (_i32, [_PP, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "splitkv_attn_fwd": (_i32, [_PP, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _vp, _i32, _vp]),
+    "splitkv_lse_merge": (_i32, [_PP, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
     "splitkv_attn_bwd": (_i32, [_PP] + [_vp] * 15 + [_vp, _sz, _vp]),
 }
 EXPORTS = tuple(_SIGS)
@@ -161,16 +161,16 @@ def splitkv_plan_lpt_noalloc(item_cost, n_items, max_items, max_cost, n_workers,
                                          _stream(stream)), "splitkv_plan_lpt_noalloc")
 
 
-def splitkv_attn_fwd(problem, q, k, v, anchors, item_id, queue_off, queue_items, n_workers, o_part, lse_part,
-                     status, flags=FWD_DEFAULT, stream=None):
-    _check(_lib.splitkv_attn_fwd(problem.ptr, _p(q), _p(k), _p(v), _p(anchors), _p(item_id), _p(queue_off),
-                                 _p(queue_items), int(n_workers), _p(o_part), _p(lse_part), _p(status), int(flags),
-                                 _stream(stream)), "splitkv_attn_fwd")
+def splitkv_attn_fwd(problem, q, k, v, kb, vb, anchors, item_id, queue_off, queue_items, n_workers, o_part,
+                     lse_part, status, flags=FWD_DEFAULT, stream=None):
+    _check(_lib.splitkv_attn_fwd(problem.ptr, _p(q), _p(k), _p(v), _p(kb), _p(vb), _p(anchors), _p(item_id),
+                                 _p(queue_off), _p(queue_items), int(n_workers), _p(o_part), _p(lse_part), _p(status),
+                                 int(flags), _stream(stream)), "splitkv_attn_fwd")
 
 
-def splitkv_lse_merge(problem, o_part, lse_part, q, kb, vb, anchors, o, lse, status, stream=None):
-    _check(_lib.splitkv_lse_merge(problem.ptr, _p(o_part), _p(lse_part), _p(q), _p(kb), _p(vb), _p(anchors), _p(o),
-                                  _p(lse), _p(status), _stream(stream)), "splitkv_lse_merge")
+def splitkv_lse_merge(problem, o_part, lse_part, anchors, o, lse, status, stream=None):
+    _check(_lib.splitkv_lse_merge(problem.ptr, _p(o_part), _p(lse_part), _p(anchors), _p(o), _p(lse), _p(status),
+                                  _stream(stream)), "splitkv_lse_merge")
 
 
 def splitkv_attn_bwd(problem, q, k, v, kb, vb, o, lse, dout, anchors, dq, dk, dv, dkb, dvb, status, workspace,
@@ -196,6 +196,7 @@ class SplitKV:
             off.append(off[-1] + int(c))
         self.device = torch.device(device)
         self.dtype = dtype
+        self.n_q_heads, self.n_kv_heads, self.head_dim = int(n_q_heads), int(n_kv_heads), int(head_dim)
         self.problem = make_problem(seq_lens, off, n_q_heads, n_kv_heads, head_dim, block, chunk, key_tile, scale,
                                     dtype)
         self.sizes = splitkv_query(self.problem)
@@ -236,24 +237,24 @@ class SplitKV:
         self.cost(anchors, stream)
         self.plan_lpt(stream)
 
-    def attn_fwd(self, q, k, v, anchors, flags=FWD_DEFAULT, stream=None):
-        splitkv_attn_fwd(self.problem, q, k, v, anchors, self.item_id, self.queue_off, self.queue_items,
+    def attn_fwd(self, q, k, v, kb, vb, anchors, flags=FWD_DEFAULT, stream=None):
+        splitkv_attn_fwd(self.problem, q, k, v, kb, vb, anchors, self.item_id, self.queue_off, self.queue_items,
                          self.n_workers, self.o_part, self.lse_part, self.status, flags, stream)
 
-    def lse_merge(self, q, kb, vb, anchors, o=None, lse=None, stream=None):
-        Nq, Hq = int(self.sizes.n_queries), q.shape[1]
+    def lse_merge(self, anchors, o=None, lse=None, stream=None):
+        Nq, Hq, d = int(self.sizes.n_queries), self.n_q_heads, self.head_dim
         if o is None:
-            o = torch.empty(Nq, Hq, q.shape[2], dtype=self.dtype, device=self.device)
+            o = torch.empty(Nq, Hq, d, dtype=self.dtype, device=self.device)
         if lse is None:
             lse = torch.empty(Nq, Hq, dtype=torch.float32, device=self.device)
-        splitkv_lse_merge(self.problem, self.o_part, self.lse_part, q, kb, vb, anchors, o, lse, self.status, stream)
+        splitkv_lse_merge(self.problem, self.o_part, self.lse_part, anchors, o, lse, self.status, stream)
         return o, lse
 
     def forward(self, q, k, v, kb, vb, anchors, flags=FWD_DEFAULT, plan=True, o=None, lse=None, stream=None):
         if plan:
             self.plan(anchors, stream)
-        self.attn_fwd(q, k, v, anchors, flags, stream)
-        return self.lse_merge(q, kb, vb, anchors, o, lse, stream)
+        self.attn_fwd(q, k, v, kb, vb, anchors, flags, stream)
+        return self.lse_merge(anchors, o, lse, stream)
 
     def backward(self, q, k, v, kb, vb, o, lse, dout, anchors, grads=None, stream=None):
         if grads is None:
@@ -275,9 +276,8 @@ class SplitKV:
             raise RuntimeError(f"device status word 0x{st:x}")
 
     def o_part_view(self):
-        """O_part as [n_items_max, d/4, rows, 4] and LSE_part as [n_items_max, rows]."""
-        s = self.sizes
-        R = int(s.rows_per_item)
-        n = int(s.n_items_max)
-        d = int(s.o_part_elems // max(1, n * R)) if n else 0
+        """Partials as [slots, d/4, rows, 4] and their LSEs as [slots, rows]: chunk items first
+        (n_items_max slots), then the self partials, slot n_items_max + j*Hkv + g."""
+        R, d = int(self.sizes.rows_per_item), self.head_dim
+        n = int(self.sizes.lse_part_elems) // R
         return self.o_part[: n * R * d].view(n, d // 4, R, 4), self.lse_part[: n * R].view(n, R)

@@ -101,8 +101,8 @@ SPLITKV_API int splitkv_query(const splitkv_problem* problem, splitkv_sizes* out
     out->n_queries = m.n_queries;
     out->total_keys = m.total_keys;
     out->n_blocks = m.n_blocks;
-    out->o_part_elems = m.n_items * m.rows * m.d;
-    out->lse_part_elems = m.n_items * m.rows;
+    out->o_part_elems = (m.n_items + m.n_blocks * m.hkv) * m.rows * m.d;
+    out->lse_part_elems = (m.n_items + m.n_blocks * m.hkv) * m.rows;
     out->max_cost = m.chunk / m.key_tile;
     out->rows_per_item = m.rows;
     return SPLITKV_OK;
@@ -182,7 +182,8 @@ SPLITKV_API int splitkv_plan_lpt_noalloc(const int32_t* item_cost_d, const int32
 }
 
 SPLITKV_API int splitkv_attn_fwd(const splitkv_problem* problem, const void* q, const void* k, const void* v,
-                                 const int32_t* anchors_d, const int32_t* item_id_d, const int32_t* queue_off_d,
+                                 const void* kb, const void* vb, const int32_t* anchors_d, const int32_t* item_id_d,
+                                 const int32_t* queue_off_d,
                                  const int32_t* queue_items_d, int32_t n_workers, float* o_part, float* lse_part,
                                  int32_t* status_d, int32_t flags, void* stream) {
     clear_error();
@@ -190,30 +191,30 @@ SPLITKV_API int splitkv_attn_fwd(const splitkv_problem* problem, const void* q, 
     int rc = build_meta(problem, &m);
     if (rc) return rc;
     if (n_workers < 1 || n_workers > 65535 || (flags & ~SPLITKV_FWD_SIMT)) return SPLITKV_EINVAL;
-    if (!q || !k || !v || !item_id_d || !queue_off_d || !queue_items_d || !o_part || !lse_part || !status_d)
+    if (!q || !k || !v || !kb || !vb || !item_id_d || !queue_off_d || !queue_items_d || !o_part || !lse_part ||
+        !status_d)
         return SPLITKV_EINVAL;
     if (m.n_blocks && !anchors_d) return SPLITKV_EINVAL;
-    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o_part)) return SPLITKV_EINVAL;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(kb) || !aligned16(vb) || !aligned16(o_part))
+        return SPLITKV_EINVAL;
     cudaStream_t st = (cudaStream_t)stream;
     if (!(flags & SPLITKV_FWD_SIMT) && fwd_tc_supported(m))
-        return cuda_status(launch_fwd_tc(m, q, k, v, anchors_d, item_id_d, queue_off_d, queue_items_d, n_workers,
-                                         o_part, lse_part, status_d, st));
-    return cuda_status(launch_fwd_simt(m, q, k, v, anchors_d, item_id_d, queue_off_d, queue_items_d, n_workers,
-                                       o_part, lse_part, status_d, st));
+        return cuda_status(launch_fwd_tc(m, q, k, v, kb, vb, anchors_d, item_id_d, queue_off_d, queue_items_d,
+                                         n_workers, o_part, lse_part, status_d, st));
+    return cuda_status(launch_fwd_simt(m, q, k, v, kb, vb, anchors_d, item_id_d, queue_off_d, queue_items_d,
+                                       n_workers, o_part, lse_part, status_d, st));
 }
 
 SPLITKV_API int splitkv_lse_merge(const splitkv_problem* problem, const float* o_part, const float* lse_part,
-                                  const void* q, const void* kb, const void* vb, const int32_t* anchors_d, void* o,
-                                  float* lse, int32_t* status_d, void* stream) {
+                                  const int32_t* anchors_d, void* o, float* lse, int32_t* status_d, void* stream) {
     clear_error();
     Meta m;
     int rc = build_meta(problem, &m);
     if (rc) return rc;
-    if (!o_part || !lse_part || !q || !kb || !vb || !o || !lse || !status_d) return SPLITKV_EINVAL;
+    if (!o_part || !lse_part || !o || !lse || !status_d) return SPLITKV_EINVAL;
     if (m.n_blocks && !anchors_d) return SPLITKV_EINVAL;
-    if (!aligned16(o_part)) return SPLITKV_EINVAL;
-    return cuda_status(launch_merge(m, o_part, lse_part, q, kb, vb, anchors_d, o, lse, status_d,
-                                    (cudaStream_t)stream));
+    if (!aligned16(o_part) || !aligned16(lse_part) || !aligned16(o)) return SPLITKV_EINVAL;
+    return cuda_status(launch_merge(m, o_part, lse_part, anchors_d, o, lse, status_d, (cudaStream_t)stream));
 }
 
 SPLITKV_API int splitkv_attn_bwd(const splitkv_problem* problem, const void* q, const void* k, const void* v,

@@ -101,18 +101,19 @@ constexpr size_t kStaticPlanScratchBytes = (size_t)4 << 20;
 constexpr int kMaxDevices = 64;
 cudaError_t static_plan_scratch(void** out);
 
-cudaError_t launch_fwd_simt(const Meta& m, const void* q, const void* k, const void* v, const int32_t* anchors,
-                            const int32_t* item_id, const int32_t* queue_off, const int32_t* queue_items,
-                            int32_t n_workers, float* o_part, float* lse_part, int32_t* status, cudaStream_t st);
+cudaError_t launch_fwd_simt(const Meta& m, const void* q, const void* k, const void* v, const void* kb,
+                            const void* vb, const int32_t* anchors, const int32_t* item_id, const int32_t* queue_off,
+                            const int32_t* queue_items, int32_t n_workers, float* o_part, float* lse_part,
+                            int32_t* status, cudaStream_t st);
 
-cudaError_t launch_fwd_tc(const Meta& m, const void* q, const void* k, const void* v, const int32_t* anchors,
-                          const int32_t* item_id, const int32_t* queue_off, const int32_t* queue_items,
-                          int32_t n_workers, float* o_part, float* lse_part, int32_t* status, cudaStream_t st);
+cudaError_t launch_fwd_tc(const Meta& m, const void* q, const void* k, const void* v, const void* kb, const void* vb,
+                          const int32_t* anchors, const int32_t* item_id, const int32_t* queue_off,
+                          const int32_t* queue_items, int32_t n_workers, float* o_part, float* lse_part,
+                          int32_t* status, cudaStream_t st);
 bool fwd_tc_supported(const Meta& m);
 
-cudaError_t launch_merge(const Meta& m, const float* o_part, const float* lse_part, const void* q, const void* kb,
-                         const void* vb, const int32_t* anchors, void* o, float* lse, int32_t* status,
-                         cudaStream_t st);
+cudaError_t launch_merge(const Meta& m, const float* o_part, const float* lse_part, const int32_t* anchors, void* o,
+                         float* lse, int32_t* status, cudaStream_t st);
 
 cudaError_t launch_bwd(const Meta& m, const void* q, const void* k, const void* v, const void* kb, const void* vb,
                        const void* o, const float* lse, const void* dout, const int32_t* anchors, float* dq,

@@ -3,7 +3,9 @@
 // tensor-core kernel. One persistent CTA per worker walks its LPT queue; per item it runs the
 // chunk-local online softmax over key tiles of 32 keys and writes the normalised partial output
 // and its natural-log LSE (Split-KV: Efficient Context Parallelism for Training Diffusion
-// Drafters, Abstract: exact attention from chunk-local, query-sized partials).
+// Drafters, Abstract: exact attention from chunk-local, query-sized partials). After its queue each
+// CTA also computes a share of the self partials (block j, kv head g) over the block's own keys,
+// stored at slot n_items + j*Hkv + g.
 #include "common.cuh"
 #include "scan.cuh"
 
@@ -17,6 +19,7 @@ constexpr int kBK = 32;  // keys per tile (one per lane in the softmax step)
 template <typename T>
 __global__ void __launch_bounds__(kThreads) fwd_simt_kernel(Meta m, const T* __restrict__ q,
                                                             const T* __restrict__ k, const T* __restrict__ v,
+                                                            const T* __restrict__ kb, const T* __restrict__ vb,
                                                             const int32_t* __restrict__ anchors,
                                                             const int32_t* __restrict__ item_id,
                                                             const int32_t* __restrict__ queue_off,
@@ -38,14 +41,31 @@ __global__ void __launch_bounds__(kThreads) fwd_simt_kernel(Meta m, const T* __r
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
     const int32_t q0 = queue_off[blockIdx.x], q1 = queue_off[blockIdx.x + 1];
-    for (int32_t qi = q0; qi < q1; ++qi) {
-        const int32_t kidx = queue_items[qi];
-        const int64_t id = item_id[kidx];
-        if (id < 0 || id >= m.n_items) { raise_status(status, SPLITKV_DEV_BAD_PLAN); return; }
-        const Item it = decode_item(m, id);
-        const int32_t a = anchors[it.j];
-        const int32_t nvis = visible_in_chunk(m, it.s, it.c, a);
-        const int64_t kbase = m.key_off[it.s] + (int64_t)it.c * m.chunk;
+    const int64_t n_self = m.n_blocks * m.hkv;
+    // Entries: the queue's items, then self items blockIdx.x, blockIdx.x + gridDim.x, ...
+    for (int64_t e_idx = q0;; ++e_idx) {
+        int64_t id, kbase;
+        int32_t nvis;
+        Item it;
+        const T *kp = k, *vp = v;
+        if (e_idx < q1) {
+            const int32_t kidx = queue_items[e_idx];
+            id = item_id[kidx];
+            if (id < 0 || id >= m.n_items) { raise_status(status, SPLITKV_DEV_BAD_PLAN); return; }
+            it = decode_item(m, id);
+            nvis = visible_in_chunk(m, it.s, it.c, anchors[it.j]);
+            kbase = m.key_off[it.s] + (int64_t)it.c * m.chunk;
+        } else {
+            const int64_t sid = blockIdx.x + (e_idx - q1) * (int64_t)gridDim.x;
+            if (sid >= n_self) break;
+            id = m.n_items + sid;
+            it.j = (int32_t)(sid / m.hkv);
+            it.g = (int32_t)(sid % m.hkv);
+            nvis = m.block;
+            kbase = (int64_t)m.block * it.j;
+            kp = kb;
+            vp = vb;
+        }
 
         for (int e = tid; e < R * d; e += kThreads) {
             int r = e / d, dd = e % d;
@@ -64,8 +84,8 @@ __global__ void __launch_bounds__(kThreads) fwd_simt_kernel(Meta m, const T* __r
                 float kv = 0.f, vv = 0.f;
                 if (jj < nk) {
                     int64_t off = ((kbase + t0 + jj) * m.hkv + it.g) * d + dd;
-                    kv = to_f32(k[off]);
-                    vv = to_f32(v[off]);
+                    kv = to_f32(kp[off]);
+                    vv = to_f32(vp[off]);
                 }
                 Ks[jj * dp + dd] = kv;
                 Vs[jj * d + dd] = vv;
@@ -122,27 +142,30 @@ __global__ void __launch_bounds__(kThreads) fwd_simt_kernel(Meta m, const T* __r
 }
 
 template <typename T>
-cudaError_t launch_t(const Meta& m, const void* q, const void* k, const void* v, const int32_t* anchors,
-                     const int32_t* item_id, const int32_t* queue_off, const int32_t* queue_items, int32_t n_workers,
-                     float* o_part, float* lse_part, int32_t* status, cudaStream_t st) {
+cudaError_t launch_t(const Meta& m, const void* q, const void* k, const void* v, const void* kb, const void* vb,
+                     const int32_t* anchors, const int32_t* item_id, const int32_t* queue_off,
+                     const int32_t* queue_items, int32_t n_workers, float* o_part, float* lse_part, int32_t* status,
+                     cudaStream_t st) {
     const int R = m.rows, d = m.d;
     size_t smem = sizeof(float) * ((size_t)2 * R * d + kBK * (d + 1) + kBK * d + R * kBK + 3 * R);
     cudaError_t e = cudaFuncSetAttribute(fwd_simt_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    fwd_simt_kernel<T><<<n_workers, kThreads, smem, st>>>(m, (const T*)q, (const T*)k, (const T*)v, anchors, item_id,
-                                                          queue_off, queue_items, o_part, lse_part, status);
+    fwd_simt_kernel<T><<<n_workers, kThreads, smem, st>>>(m, (const T*)q, (const T*)k, (const T*)v, (const T*)kb,
+                                                          (const T*)vb, anchors, item_id, queue_off, queue_items,
+                                                          o_part, lse_part, status);
     return cudaGetLastError();
 }
 
 }  // namespace
 
-cudaError_t launch_fwd_simt(const Meta& m, const void* q, const void* k, const void* v, const int32_t* anchors,
-                            const int32_t* item_id, const int32_t* queue_off, const int32_t* queue_items,
-                            int32_t n_workers, float* o_part, float* lse_part, int32_t* status, cudaStream_t st) {
+cudaError_t launch_fwd_simt(const Meta& m, const void* q, const void* k, const void* v, const void* kb,
+                            const void* vb, const int32_t* anchors, const int32_t* item_id, const int32_t* queue_off,
+                            const int32_t* queue_items, int32_t n_workers, float* o_part, float* lse_part,
+                            int32_t* status, cudaStream_t st) {
     if (m.dtype == SPLITKV_F32)
-        return launch_t<float>(m, q, k, v, anchors, item_id, queue_off, queue_items, n_workers, o_part, lse_part,
-                               status, st);
-    return launch_t<__nv_bfloat16>(m, q, k, v, anchors, item_id, queue_off, queue_items, n_workers, o_part,
+        return launch_t<float>(m, q, k, v, kb, vb, anchors, item_id, queue_off, queue_items, n_workers, o_part,
+                               lse_part, status, st);
+    return launch_t<__nv_bfloat16>(m, q, k, v, kb, vb, anchors, item_id, queue_off, queue_items, n_workers, o_part,
                                    lse_part, status, st);
 }
 

@@ -5,8 +5,11 @@
 // log-sum-exp; the chunks are placed by the cost-aware LPT plan. Here one persistent CTA per SM
 // walks the SM's LPT queue. A work item (s, c, g, b) is one 128-row query tile — the block*G rows
 // (query i, head g*G+hl) of block b at kv head g, shared by the G query heads of the GQA group —
-// against the ceil(nvis/128) key tiles of chunk c that the block sees. The CTA's key tiles form
-// one sequence n = 0, 1, ... across its items i = 0, 1, ...
+// against the ceil(nvis/128) key tiles of chunk c that the block sees. After its queue, every CTA
+// also takes a share of the self items (block j, kv head g): the same query tile against the
+// block's own 16 keys (Kb, Vb), one tile with 16 visible keys, whose partial goes to slot
+// n_items + j*Hkv + g. The CTA's key tiles form one sequence n = 0, 1, ... across its items
+// i = 0, 1, ...
 //
 // Roles (512 threads, four warpgroups; registers moved with setmaxnreg):
 //   WG0 / WG1 (warps 0-7)  softmax of the even / odd key tiles: row r = 32*(warp%4) + lane
@@ -89,9 +92,10 @@ struct Bars {
 constexpr int kSmemBytes = kOffBar + (int)sizeof(Bars) + 1024;  // + alignment slack
 
 struct TileRef {
-    int64_t id;
+    int64_t id;                // partial slot: item id, or n_items + j*Hkv + g for a self item
     int32_t s, c, g, j;
     int32_t nvis, ntiles, t;
+    int32_t self_item;         // 1: keys are the block's own (Kb/Vb rows block*j ..)
 };
 
 // The CTA's items (queue positions first, first+1, ...), fetched ahead: each call hands out the
@@ -104,6 +108,7 @@ struct ItemStream {
     int32_t a1;   // anchor of item n+1 (in flight)
     int64_t id2;  // item n+2 (in flight)
     int32_t k3;   // queue entry of item n+3 (in flight)
+    int32_t self_pos, self_n;  // self items blockIdx.x, blockIdx.x + gridDim.x, ... < self_n
 };
 
 __device__ __forceinline__ int64_t load_id(const int32_t* __restrict__ item_id, int32_t k) {
@@ -124,11 +129,30 @@ __device__ __forceinline__ void stream_init(const Meta& m, const int32_t* anchor
     st.id2 = load_id(item_id, k1);
     st.a1 = load_anchor(m, anchors, st.id1);
     st.pos = first + 3;
+    st.self_pos = blockIdx.x;
+    st.self_n = (int32_t)(m.n_blocks * m.hkv);
 }
+
+__device__ __forceinline__ bool stream_more(const ItemStream& st) { return st.left > 0 || st.self_pos < st.self_n; }
 
 // Next item as a tile reference (ntiles == 0 for an invalid entry, which raises BAD_PLAN).
 __device__ __forceinline__ void stream_next(const Meta& m, const int32_t* anchors, const int32_t* item_id,
                                             const int32_t* queue_items, ItemStream& st, TileRef& tr, int32_t* status) {
+    tr.t = 0;
+    if (st.left <= 0) {  // self item
+        const int32_t sid = st.self_pos;
+        st.self_pos += gridDim.x;
+        tr.self_item = 1;
+        tr.id = m.n_items + sid;
+        tr.j = sid / m.hkv;
+        tr.g = sid % m.hkv;
+        tr.s = sample_of_block(m, tr.j);
+        tr.c = 0;
+        tr.nvis = m.block;
+        tr.ntiles = 1;
+        return;
+    }
+    tr.self_item = 0;
     const int64_t id = st.id1;
     const int32_t a = st.a1;
     --st.left;
@@ -162,7 +186,7 @@ struct Cursor {
 
 __device__ __forceinline__ void cursor_fetch(const Meta& m, const int32_t* anchors, const int32_t* item_id,
                                              const int32_t* queue_items, Cursor& c, int32_t* status) {
-    while (c.st.left > 0) {
+    while (stream_more(c.st)) {
         stream_next(m, anchors, item_id, queue_items, c.st, c.cur, status);
         if (c.cur.ntiles > 0) {
             c.has = true;
@@ -188,6 +212,7 @@ __device__ __forceinline__ void cursor_advance(const Meta& m, const int32_t* anc
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_tc_kernel(const __grid_constant__ Meta m, const __grid_constant__ CUtensorMap tmQ,
                   const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                  const __grid_constant__ CUtensorMap tmKb, const __grid_constant__ CUtensorMap tmVb,
                   const int32_t* __restrict__ anchors, const int32_t* __restrict__ item_id,
                   const int32_t* __restrict__ queue_off, const int32_t* __restrict__ queue_items,
                   float* __restrict__ o_part, float* __restrict__ lse_part, int32_t* __restrict__ status) {
@@ -235,7 +260,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = bars->tmem_base;
-    const bool skip = bars->status0 != 0 || q0 >= q1;
+    const bool skip = bars->status0 != 0 || (q0 >= q1 && (int64_t)blockIdx.x >= m.n_blocks * m.hkv);
     const int G = m.group, R = m.rows;
 
     if (warp >= kProducerWarp) {
@@ -245,6 +270,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             tma_prefetch_desc(&tmQ);
             tma_prefetch_desc(&tmK);
             tma_prefetch_desc(&tmV);
+            tma_prefetch_desc(&tmKb);
+            tma_prefetch_desc(&tmVb);
             const uint32_t q_bytes = 2u * 64u * (uint32_t)G * (uint32_t)m.block * 2u;
             Cursor cur;
             TileRef prev;
@@ -256,7 +283,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int b = idx & 1;
                 if (!mbar_wait(&empty[b], ((idx >> 1) & 1u) ^ 1u, abort_flag, kTimeoutNs)) return false;
                 mbar_arrive_expect_tx(&full[b], kTileBytes);
-                const int32_t row = (int32_t)(m.key_off[t.s] + (int64_t)t.c * m.chunk + (int64_t)t.t * kKeysPerTile);
+                const int32_t row = t.self_item ? m.block * t.j
+                                                : (int32_t)(m.key_off[t.s] + (int64_t)t.c * m.chunk +
+                                                            (int64_t)t.t * kKeysPerTile);
                 uint8_t* dst = smem + off + b * kTileBytes;
                 tma_load_3d(dst, map, &full[b], 0, t.g, row);
                 tma_load_3d(dst + kHalfBytes, map, &full[b], 64, t.g, row);
@@ -277,14 +306,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tma_load_3d(dst + kHalfBytes, &tmQ, &bars->q_full[qb], 64, t.g * G, m.block * t.j);
                     ++item_seq;
                 }
-                ok = load_tile(&tmK, bars->k_full, bars->k_empty, n, kOffK, t);
-                if (ok && n > 0) ok = load_tile(&tmV, bars->v_full, bars->v_empty, n - 1, kOffV, prev);
+                ok = load_tile(t.self_item ? &tmKb : &tmK, bars->k_full, bars->k_empty, n, kOffK, t);
+                if (ok && n > 0)
+                    ok = load_tile(prev.self_item ? &tmVb : &tmV, bars->v_full, bars->v_empty, n - 1, kOffV, prev);
                 if (!ok) break;
                 prev = t;
                 ++n;
                 cursor_advance(m, anchors, item_id, queue_items, cur, status);
             }
-            if (ok && n > 0) ok = load_tile(&tmV, bars->v_full, bars->v_empty, n - 1, kOffV, prev);
+            if (ok && n > 0)
+                ok = load_tile(prev.self_item ? &tmVb : &tmV, bars->v_full, bars->v_empty, n - 1, kOffV, prev);
             // Drain: the most recent copy into every buffer has landed before the CTA exits.
             volatile int never = 0;
             for (uint32_t x = (n > 2 ? n - 2 : 0); x < n; ++x) {
@@ -379,7 +410,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t i = 0;
             ItemStream st;
             stream_init(m, anchors, item_id, queue_items, q0, q1, st);
-            while (st.left > 0) {
+            while (stream_more(st)) {
                 TileRef t;
                 stream_next(m, anchors, item_id, queue_items, st, t, status);
                 if (t.ntiles == 0) continue;
@@ -437,7 +468,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             bool ok = true;
             ItemStream st;
             stream_init(m, anchors, item_id, queue_items, q0, q1, st);
-            while (st.left > 0 && ok) {
+            while (stream_more(st) && ok) {
                 TileRef t;
                 stream_next(m, anchors, item_id, queue_items, st, t, status);
                 if (t.ntiles == 0) continue;
@@ -639,19 +670,22 @@ bool fwd_tc_supported(const Meta& m) {
            m.total_keys < INT32_MAX && m.n_queries < INT32_MAX;
 }
 
-cudaError_t launch_fwd_tc(const Meta& m, const void* q, const void* k, const void* v, const int32_t* anchors,
-                          const int32_t* item_id, const int32_t* queue_off, const int32_t* queue_items,
-                          int32_t n_workers, float* o_part, float* lse_part, int32_t* status, cudaStream_t st) {
-    CUtensorMap tq, tk, tv;
+cudaError_t launch_fwd_tc(const Meta& m, const void* q, const void* k, const void* v, const void* kb, const void* vb,
+                          const int32_t* anchors, const int32_t* item_id, const int32_t* queue_off,
+                          const int32_t* queue_items, int32_t n_workers, float* o_part, float* lse_part,
+                          int32_t* status, cudaStream_t st) {
+    CUtensorMap tq, tk, tv, tkb, tvb;
     if (m.n_queries == 0 || m.total_keys == 0) return cudaSuccess;
     if (!make_map(&tq, q, m.n_queries, m.hq, m.d, m.group, m.block) ||
         !make_map(&tk, k, m.total_keys, m.hkv, m.d, 1, kKeysPerTile) ||
-        !make_map(&tv, v, m.total_keys, m.hkv, m.d, 1, kKeysPerTile))
+        !make_map(&tv, v, m.total_keys, m.hkv, m.d, 1, kKeysPerTile) ||
+        !make_map(&tkb, kb, m.n_queries, m.hkv, m.d, 1, kKeysPerTile) ||
+        !make_map(&tvb, vb, m.n_queries, m.hkv, m.d, 1, kKeysPerTile))
         return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return note_error(e, "cudaFuncSetAttribute(fwd_tc_kernel, smem)");
-    fwd_tc_kernel<<<n_workers, kThreads, kSmemBytes, st>>>(m, tq, tk, tv, anchors, item_id, queue_off, queue_items,
-                                                           o_part, lse_part, status);
+    fwd_tc_kernel<<<n_workers, kThreads, kSmemBytes, st>>>(m, tq, tk, tv, tkb, tvb, anchors, item_id, queue_off,
+                                                           queue_items, o_part, lse_part, status);
     e = cudaGetLastError();
     if (e != cudaSuccess) {
         cudaFuncAttributes fa;

@@ -1,43 +1,70 @@
-// Exact log-sum-exp merge of the chunk partials, fused with the block's own-keys partial
-// (Split-KV: Efficient Context Parallelism for Training Diffusion Drafters, Abstract: exact
-// attention assembled from chunk-local, query-sized partial results).
+// Exact log-sum-exp merge of the partials of one query block (Split-KV: Efficient Context
+// Parallelism for Training Diffusion Drafters, Abstract: exact attention assembled from
+// chunk-local, query-sized partial results).
 //
-// One CTA per (global block j, kv head g): its block*G query rows r = i*G + hl. For every row:
-//   self partial over the block's own keys: s_t = scale q.kb_t;
-//   L = log( sum_t exp(s_t) + sum_{c < ceil(a/C)} exp(LSE_c) )          (max-shifted)
-//   O = sum_c exp(LSE_c - L) O_c + sum_t exp(s_t - L) vb_t.
-// Memory-bound: every visible partial tile is read once. The per-chunk LSEs are staged in shared
-// memory with coalesced loads and turned into weights there; the partial tiles are stored
-// [d/4][rows][4], so consecutive threads (consecutive rows) read consecutive 16-byte words, and
-// each thread keeps four chunk loads in flight.
+// Block j, kv head g has the self partial (its own keys, slot n_items + j*Hkv + g) and one chunk
+// partial per visible chunk c < ceil(a/C) (item base_s + (c*Hkv + g)*nb_s + b). For each of its
+// block*G query rows r:
+//   L = log( sum_p exp(LSE_p) ),     O = sum_p exp(LSE_p - L) O_p
+// over those partials p, accumulated online (running maximum, rescaled sum) so that the partial
+// tiles are read exactly once, in one pass.
+//
+// Memory-bound. A thread owns one row r and a group of four 16-byte columns (16 floats); a CTA
+// owns kThreads consecutive (row, group) units of one (j, g). The partial tiles are stored
+// [d/4][rows][4], so a warp's 32 consecutive rows read 512 contiguous bytes per column, and each
+// thread keeps four partials' loads in flight. The output row receives 16 contiguous values.
 #include "common.cuh"
-#include "scan.cuh"
 
 namespace splitkv {
 
 namespace {
 
-constexpr int kThreads = 512;
+constexpr int kThreads = 256;
+constexpr int kCols = 4;    // float4 columns per thread
+constexpr int kUnroll = 4;  // partials loaded ahead
+
+struct Online {
+    float m, l;
+    float4 acc[kCols];
+};
+
+__device__ __forceinline__ void online_add(Online& st, float lse_p, const float4 (&x)[kCols]) {
+    if (lse_p == -INFINITY) return;  // an empty partial contributes nothing
+    const float m_new = fmaxf(st.m, lse_p);
+    const float a = __expf(st.m - m_new), w = __expf(lse_p - m_new);
+    st.l = fmaf(st.l, a, w);
+    st.m = m_new;
+#pragma unroll
+    for (int u = 0; u < kCols; ++u) {
+        st.acc[u].x = fmaf(w, x[u].x, st.acc[u].x * a);
+        st.acc[u].y = fmaf(w, x[u].y, st.acc[u].y * a);
+        st.acc[u].z = fmaf(w, x[u].z, st.acc[u].z * a);
+        st.acc[u].w = fmaf(w, x[u].w, st.acc[u].w * a);
+    }
+}
+
+__device__ __forceinline__ void load_cols(const float4* __restrict__ tile, int R, int r, int d40, int D4,
+                                          float4 (&x)[kCols]) {
+#pragma unroll
+    for (int u = 0; u < kCols; ++u)
+        x[u] = (d40 + u < D4) ? __ldcs(tile + (int64_t)(d40 + u) * R + r) : make_float4(0.f, 0.f, 0.f, 0.f);
+}
 
 template <typename T>
-__global__ void __launch_bounds__(kThreads) merge_kernel(Meta m, int32_t max_nv, const float* __restrict__ o_part,
+__global__ void __launch_bounds__(kThreads) merge_kernel(Meta m, int32_t ctas_per_head,
+                                                         const float* __restrict__ o_part,
                                                          const float* __restrict__ lse_part,
-                                                         const T* __restrict__ q, const T* __restrict__ kb,
-                                                         const T* __restrict__ vb,
                                                          const int32_t* __restrict__ anchors, T* __restrict__ o,
                                                          float* __restrict__ lse, const int32_t* __restrict__ status) {
-    extern __shared__ float smem[];
     if (status_bad(status)) return;
-    const int R = m.rows, d = m.d, G = m.group, BL = m.block;
-    const int dp = d + 1;
-    float* Qs = smem;             // [R][d+1]
-    float* Kbs = Qs + R * dp;     // [BL][d+1]
-    float* Vbs = Kbs + BL * dp;   // [BL][d]
-    float* Ps = Vbs + BL * d;     // [R][BL]   self scores, then self weights
-    float* Lr = Ps + R * BL;      // [R]
-    float* Wc = Lr + R;           // [max_nv][R] chunk LSEs, then chunk weights
-    const int tid = threadIdx.x;
-    const int32_t j = blockIdx.x / m.hkv, g = blockIdx.x % m.hkv;
+    const int R = m.rows, d = m.d, G = m.group, BL = m.block, D4 = d / 4;
+    const int64_t jg = blockIdx.x / ctas_per_head;
+    const int32_t j = (int32_t)(jg / m.hkv), g = (int32_t)(jg % m.hkv);
+    const int unit = (blockIdx.x % ctas_per_head) * kThreads + threadIdx.x;
+    const int groups = (D4 + kCols - 1) / kCols;
+    if (unit >= R * groups) return;
+    const int r = unit % R, d40 = (unit / R) * kCols;
+
     const int s = sample_of_block(m, j);
     const int32_t b = j - m.anchor_off[s];
     const int32_t nb = m.anchor_off[s + 1] - m.anchor_off[s];
@@ -45,119 +72,77 @@ __global__ void __launch_bounds__(kThreads) merge_kernel(Meta m, int32_t max_nv,
     int32_t nv = (int32_t)(((int64_t)a + m.chunk - 1) / m.chunk);
     if (nv < 0) nv = 0;
     if (nv > m.n_chunk_s[s]) nv = m.n_chunk_s[s];
-    if (nv > max_nv) nv = max_nv;
     const int64_t item0 = m.item_base[s] + (int64_t)g * nb + b;  // chunk 0; chunk c adds c*Hkv*nb
     const int64_t cstride = (int64_t)m.hkv * nb;
-
-    for (int e = tid; e < R * d; e += kThreads) {
-        int r = e / d, dd = e % d;
-        int i = r / G, hl = r % G;
-        int64_t row = (int64_t)BL * j + i;
-        Qs[r * dp + dd] = to_f32(q[(row * m.hq + (int64_t)g * G + hl) * d + dd]);
-    }
-    for (int e = tid; e < BL * d; e += kThreads) {
-        int t = e / d, dd = e % d;
-        int64_t off = (((int64_t)BL * j + t) * m.hkv + g) * d + dd;
-        Kbs[t * dp + dd] = to_f32(kb[off]);
-        Vbs[t * d + dd] = to_f32(vb[off]);
-    }
-    for (int e = tid; e < nv * R; e += kThreads) {
-        int c = e / R, r = e % R;
-        Wc[e] = lse_part[(item0 + c * cstride) * R + r];
-    }
-    __syncthreads();
-    for (int e = tid; e < R * BL; e += kThreads) {
-        int r = e / BL, t = e % BL;
-        float acc = 0.f;
-        for (int dd = 0; dd < d; ++dd) acc = fmaf(Qs[r * dp + dd], Kbs[t * dp + dd], acc);
-        Ps[e] = acc * m.scale;
-    }
-    __syncthreads();
-    for (int r = tid; r < R; r += kThreads) {
-        float M = -INFINITY;
-        for (int t = 0; t < BL; ++t) M = fmaxf(M, Ps[r * BL + t]);
-        for (int c = 0; c < nv; ++c) M = fmaxf(M, Wc[c * R + r]);
-        float sum = 0.f;
-        for (int t = 0; t < BL; ++t) sum += expf(Ps[r * BL + t] - M);
-        for (int c = 0; c < nv; ++c) sum += expf(Wc[c * R + r] - M);
-        const float L = M + logf(sum);
-        Lr[r] = L;
-        for (int t = 0; t < BL; ++t) Ps[r * BL + t] = expf(Ps[r * BL + t] - L);
-        for (int c = 0; c < nv; ++c) Wc[c * R + r] = expf(Wc[c * R + r] - L);
-    }
-    __syncthreads();
-    const int D4 = d / 4;
+    const int64_t tile4 = (int64_t)R * D4;  // float4s per partial tile
     const float4* op = reinterpret_cast<const float4*>(o_part);
-    for (int e = tid; e < R * D4; e += kThreads) {
-        const int r = e % R, d4 = e / R;
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        const int64_t base = (int64_t)d4 * R + r;  // float4 index inside an item tile
-        int c = 0;
-        for (; c + 4 <= nv; c += 4) {
-            float4 x[4];
+
+    Online st;
+    st.m = -INFINITY;
+    st.l = 0.f;
 #pragma unroll
-            for (int u = 0; u < 4; ++u) x[u] = __ldcs(op + (item0 + (c + u) * cstride) * (int64_t)R * D4 + base);
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const float wgt = Wc[(c + u) * R + r];
-                acc.x = fmaf(wgt, x[u].x, acc.x);
-                acc.y = fmaf(wgt, x[u].y, acc.y);
-                acc.z = fmaf(wgt, x[u].z, acc.z);
-                acc.w = fmaf(wgt, x[u].w, acc.w);
-            }
-        }
-        for (; c < nv; ++c) {
-            const float4 x = __ldcs(op + (item0 + c * cstride) * (int64_t)R * D4 + base);
-            const float wgt = Wc[c * R + r];
-            acc.x = fmaf(wgt, x.x, acc.x);
-            acc.y = fmaf(wgt, x.y, acc.y);
-            acc.z = fmaf(wgt, x.z, acc.z);
-            acc.w = fmaf(wgt, x.w, acc.w);
-        }
-        for (int t = 0; t < BL; ++t) {
-            const float p = Ps[r * BL + t];
-            const float* vr = Vbs + t * d + d4 * 4;
-            acc.x = fmaf(p, vr[0], acc.x);
-            acc.y = fmaf(p, vr[1], acc.y);
-            acc.z = fmaf(p, vr[2], acc.z);
-            acc.w = fmaf(p, vr[3], acc.w);
-        }
-        const int i = r / G, hl = r % G;
-        const int64_t orow = ((int64_t)BL * j + i) * m.hq + (int64_t)g * G + hl;
-        T* dst = o + orow * d + d4 * 4;
-        dst[0] = from_f32<T>(acc.x);
-        dst[1] = from_f32<T>(acc.y);
-        dst[2] = from_f32<T>(acc.z);
-        dst[3] = from_f32<T>(acc.w);
-        if (d4 == 0) lse[orow] = Lr[r];
+    for (int u = 0; u < kCols; ++u) st.acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+    {
+        const int64_t self = m.n_items + jg;
+        float4 x[kCols];
+        load_cols(op + self * tile4, R, r, d40, D4, x);
+        online_add(st, __ldcs(lse_part + self * R + r), x);
     }
+    int32_t c = 0;
+    for (; c + kUnroll <= nv; c += kUnroll) {
+        float4 x[kUnroll][kCols];
+        float lp[kUnroll];
+#pragma unroll
+        for (int k = 0; k < kUnroll; ++k) {
+            const int64_t item = item0 + (int64_t)(c + k) * cstride;
+            lp[k] = __ldcs(lse_part + item * R + r);
+            load_cols(op + item * tile4, R, r, d40, D4, x[k]);
+        }
+#pragma unroll
+        for (int k = 0; k < kUnroll; ++k) online_add(st, lp[k], x[k]);
+    }
+    for (; c < nv; ++c) {
+        const int64_t item = item0 + (int64_t)c * cstride;
+        float4 x[kCols];
+        load_cols(op + item * tile4, R, r, d40, D4, x);
+        online_add(st, __ldcs(lse_part + item * R + r), x);
+    }
+
+    const float inv = 1.f / st.l;
+    const int i = r / G, hl = r % G;
+    const int64_t orow = ((int64_t)BL * j + i) * m.hq + (int64_t)g * G + hl;
+    T* dst = o + orow * d + d40 * 4;
+#pragma unroll
+    for (int u = 0; u < kCols; ++u) {
+        if (d40 + u < D4) {
+            dst[4 * u + 0] = from_f32<T>(st.acc[u].x * inv);
+            dst[4 * u + 1] = from_f32<T>(st.acc[u].y * inv);
+            dst[4 * u + 2] = from_f32<T>(st.acc[u].z * inv);
+            dst[4 * u + 3] = from_f32<T>(st.acc[u].w * inv);
+        }
+    }
+    if (d40 == 0) lse[orow] = st.m + logf(st.l);
 }
 
 template <typename T>
-cudaError_t launch_t(const Meta& m, const float* o_part, const float* lse_part, const void* q, const void* kb,
-                     const void* vb, const int32_t* anchors, void* o, float* lse, int32_t* status, cudaStream_t st) {
-    const int R = m.rows, d = m.d, BL = m.block;
-    int32_t max_nv = 0;
-    for (int s = 0; s < m.batch; ++s) max_nv = m.n_chunk_s[s] > max_nv ? m.n_chunk_s[s] : max_nv;
-    size_t smem = sizeof(float) * ((size_t)R * (d + 1) + BL * (d + 1) + BL * d + R * BL + R + (size_t)max_nv * R);
-    if (smem > 227 * 1024) return note_error(cudaErrorInvalidConfiguration, "merge: too many chunks per sample");
-    cudaError_t e = cudaFuncSetAttribute(merge_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return note_error(e, "cudaFuncSetAttribute(merge_kernel)");
-    int64_t grid = m.n_blocks * m.hkv;
+cudaError_t launch_t(const Meta& m, const float* o_part, const float* lse_part, const int32_t* anchors, void* o,
+                     float* lse, int32_t* status, cudaStream_t st) {
+    const int groups = (m.d / 4 + kCols - 1) / kCols;
+    const int32_t ctas_per_head = (m.rows * groups + kThreads - 1) / kThreads;
+    const int64_t grid = m.n_blocks * m.hkv * ctas_per_head;
     if (grid == 0) return cudaSuccess;
-    merge_kernel<T><<<(unsigned)grid, kThreads, smem, st>>>(m, max_nv, o_part, lse_part, (const T*)q, (const T*)kb,
-                                                            (const T*)vb, anchors, (T*)o, lse, status);
+    if (grid > 0x7fffffff) return note_error(cudaErrorInvalidConfiguration, "merge: grid too large");
+    merge_kernel<T><<<(unsigned)grid, kThreads, 0, st>>>(m, ctas_per_head, o_part, lse_part, anchors, (T*)o, lse,
+                                                         status);
     return note_error(cudaGetLastError(), "launch merge_kernel");
 }
 
 }  // namespace
 
-cudaError_t launch_merge(const Meta& m, const float* o_part, const float* lse_part, const void* q, const void* kb,
-                         const void* vb, const int32_t* anchors, void* o, float* lse, int32_t* status,
-                         cudaStream_t st) {
-    if (m.dtype == SPLITKV_F32)
-        return launch_t<float>(m, o_part, lse_part, q, kb, vb, anchors, o, lse, status, st);
-    return launch_t<__nv_bfloat16>(m, o_part, lse_part, q, kb, vb, anchors, o, lse, status, st);
+cudaError_t launch_merge(const Meta& m, const float* o_part, const float* lse_part, const int32_t* anchors, void* o,
+                         float* lse, int32_t* status, cudaStream_t st) {
+    if (m.dtype == SPLITKV_F32) return launch_t<float>(m, o_part, lse_part, anchors, o, lse, status, st);
+    return launch_t<__nv_bfloat16>(m, o_part, lse_part, anchors, o, lse, status, st);
 }
 
 }  // namespace splitkv

@@ -69,7 +69,8 @@ def check_cost_and_plan(skv, inp):
 
 
 def check_partials(skv, inp, ids):
-    """Every visible item's partial (O_c, LSE_c) against the oracle's chunk-local softmax."""
+    """Every visible item's partial (O_c, LSE_c), and every block's self partial over its own keys,
+    against the oracle's chunk-local softmax."""
     w = inp.workload
     p = oracle_problem(inp)
     parts = OA.chunk_partials(p, w.chunk)
@@ -101,3 +102,20 @@ def check_partials(skv, inp, ids):
             ref_L.append(ref_l)
     assert_close("O_part", np.stack(got_O), np.stack(ref_O), w.dtype)
     assert_close("LSE_part", np.stack(got_L), np.stack(ref_L), w.dtype)
+    n_max = int(skv.sizes.n_items_max)
+    got_O, ref_O, got_L, ref_L = [], [], [], []
+    for s in range(len(w.seq_lens)):
+        for j in range(off[s], off[s + 1]):
+            for g in range(w.n_kv_heads):
+                slot = n_max + j * w.n_kv_heads + g
+                o_tile = O_part[slot].transpose(1, 0, 2).reshape(R, -1)
+                for hl in range(G):
+                    ref_o, ref_l = parts[(s, -1, j, g * G + hl)]
+                    rows = [i * G + hl for i in range(w.block)]
+                    got_O.append(o_tile[rows])
+                    ref_O.append(ref_o)
+                    got_L.append(L_part[slot][rows])
+                    ref_L.append(ref_l)
+    if got_O:
+        assert_close("O_self", np.stack(got_O), np.stack(ref_O), w.dtype)
+        assert_close("LSE_self", np.stack(got_L), np.stack(ref_L), w.dtype)

@@ -51,7 +51,8 @@ def test_query_sizes():
     assert s.n_items_max == 4 * 2 * 3 + 2 * 2 * 2
     assert s.n_chunks == 6 and s.n_queries == 80 and s.total_keys == 1300 and s.n_blocks == 5
     assert s.rows_per_item == 16 * 4 and s.max_cost == 2
-    assert s.o_part_elems == s.n_items_max * 64 * 64 and s.lse_part_elems == s.n_items_max * 64
+    # partial slots: every item, then one self partial per (block, kv head)
+    assert s.o_part_elems == (s.n_items_max + 5 * 2) * 64 * 64 and s.lse_part_elems == (s.n_items_max + 5 * 2) * 64
     assert B.splitkv_workspace_size(prob(), 4) > 0
 
 
@@ -100,16 +101,26 @@ def test_null_pointers_and_small_workspace_rejected_before_launch():
         B.splitkv_plan_lpt(fake, fake, 64, 1, 4096, fake, fake, fake, i64, fake, ws, stream=0)
     assert e.value.code == B.EINVAL
     with pytest.raises(B.SplitKVError) as e:
-        B.splitkv_attn_fwd(p, None, fake, fake, fake, fake, fake, fake, 4, fake, fake, fake, stream=0)
+        B.splitkv_attn_fwd(p, None, fake, fake, fake, fake, fake, fake, fake, fake, 4, fake, fake, fake, stream=0)
+    assert e.value.code == B.EINVAL
+    with pytest.raises(B.SplitKVError) as e:  # missing kb
+        B.splitkv_attn_fwd(p, fake, fake, fake, None, fake, fake, fake, fake, fake, 4, fake, fake, fake, stream=0)
     assert e.value.code == B.EINVAL
     with pytest.raises(B.SplitKVError) as e:  # unknown flag
-        B.splitkv_attn_fwd(p, fake, fake, fake, fake, fake, fake, fake, 4, fake, fake, fake, flags=8, stream=0)
+        B.splitkv_attn_fwd(p, fake, fake, fake, fake, fake, fake, fake, fake, fake, 4, fake, fake, fake, flags=8,
+                           stream=0)
     assert e.value.code == B.EINVAL
     with pytest.raises(B.SplitKVError) as e:  # misaligned q
-        B.splitkv_attn_fwd(p, fake[1:], fake, fake, fake, fake, fake, fake, 4, fake, fake, fake, stream=0)
+        B.splitkv_attn_fwd(p, fake[1:], fake, fake, fake, fake, fake, fake, fake, fake, 4, fake, fake, fake, stream=0)
+    assert e.value.code == B.EINVAL
+    with pytest.raises(B.SplitKVError) as e:  # misaligned vb
+        B.splitkv_attn_fwd(p, fake, fake, fake, fake, fake[1:], fake, fake, fake, fake, 4, fake, fake, fake, stream=0)
     assert e.value.code == B.EINVAL
     with pytest.raises(B.SplitKVError) as e:
-        B.splitkv_lse_merge(p, fake, fake, fake, fake, fake, fake, None, fake, fake, stream=0)
+        B.splitkv_lse_merge(p, fake, fake, fake, None, fake, fake, stream=0)
+    assert e.value.code == B.EINVAL
+    with pytest.raises(B.SplitKVError) as e:  # misaligned o
+        B.splitkv_lse_merge(p, fake, fake, fake, fake[1:], fake, fake, stream=0)
     assert e.value.code == B.EINVAL
     with pytest.raises(B.SplitKVError) as e:
         B.splitkv_attn_bwd(p, *([fake] * 15), ws[:1], stream=0)
