@@ -22,7 +22,6 @@ import argparse
 import json
 import os
 import statistics
-import subprocess
 import sys
 import threading
 import time
@@ -83,58 +82,80 @@ def peaks():
 
 
 class ClockSampler:
-    """nvidia-smi samples of SM clock and throttle reasons while the timed region runs."""
+    """SM clock and clock-event (throttle) reasons sampled through NVML every millisecond while the
+    timed region runs, plus one sample as it ends; falls back to nvidia-smi when NVML is missing."""
 
-    FIELDS = ("clocks.sm,clocks.max.sm,clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = (("hw_slowdown", 0x8), ("hw_thermal_slowdown", 0x40), ("sw_thermal_slowdown", 0x20),
+               ("sw_power_cap", 0x4))
 
-    def __init__(self, index):
-        self.index = index
-        self.proc = None
-        self.lines = []
+    def __init__(self, device_index):
+        self.device_index = device_index
+        self.samples = []  # (sm_mhz, max_mhz, reason bits)
+        self.stop = threading.Event()
+        self.nvml = None
+        self.handle = None
+
+    def _open(self):
+        import pynvml
+        pynvml.nvmlInit()
+        self.nvml = pynvml
+        props = torch.cuda.get_device_properties(self.device_index)
+        uuid = getattr(props, "uuid", None)
+        if uuid is not None:
+            try:
+                self.handle = pynvml.nvmlDeviceGetHandleByUUID("GPU-" + str(uuid))
+                return
+            except Exception:
+                pass
+        bus = getattr(props, "pci_bus_id", None)
+        if bus is not None:
+            dom, dev = getattr(props, "pci_domain_id", 0), getattr(props, "pci_device_id", 0)
+            self.handle = pynvml.nvmlDeviceGetHandleByPciBusId_v2(f"{dom:08x}:{bus:02x}:{dev:02x}.0")
+            return
+        self.handle = pynvml.nvmlDeviceGetHandleByIndex(self.device_index)
+
+    def _sample(self):
+        n = self.nvml
+        sm = n.nvmlDeviceGetClockInfo(self.handle, n.NVML_CLOCK_SM)
+        mx = n.nvmlDeviceGetMaxClockInfo(self.handle, n.NVML_CLOCK_SM)
+        try:
+            bits = n.nvmlDeviceGetCurrentClocksEventReasons(self.handle)
+        except AttributeError:
+            bits = n.nvmlDeviceGetCurrentClocksThrottleReasons(self.handle)
+        self.samples.append((float(sm), float(mx), int(bits)))
+
+    def _loop(self):
+        while not self.stop.wait(0.001):
+            try:
+                self._sample()
+            except Exception:
+                return
 
     def __enter__(self):
         try:
-            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                                          "-i", str(self.index), "-lms", "100"], stdout=subprocess.PIPE,
-                                         stderr=subprocess.DEVNULL, text=True)
-            self.thread = threading.Thread(target=self._read, daemon=True)
+            self._open()
+            self.thread = threading.Thread(target=self._loop, daemon=True)
             self.thread.start()
         except Exception:
-            self.proc = None
+            self.handle = None
         return self
 
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append(line.strip())
-
     def __exit__(self, *a):
-        if self.proc:
-            self.proc.terminate()
+        if self.handle is not None:
+            self.stop.set()
+            self.thread.join(timeout=5)
             try:
-                self.proc.wait(timeout=5)
+                self._sample()
             except Exception:
-                self.proc.kill()
+                pass
 
     def summary(self):
-        sm, mx, reasons = [], [], set()
-        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
-        for ln in self.lines:
-            parts = [p.strip() for p in ln.split(",")]
-            if len(parts) != 6:
-                continue
-            try:
-                sm.append(float(parts[0]))
-                mx.append(float(parts[1]))
-            except ValueError:
-                continue
-            for n, v in zip(names, parts[2:]):
-                if v.lower() == "active":
-                    reasons.add(n)
-        if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
-                "samples": len(sm)}
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0, "source": "none"}
+        reasons = sorted({name for _, _, bits in self.samples for name, bit in self.REASONS if bits & bit})
+        return {"sm_mhz": statistics.median(s[0] for s in self.samples),
+                "sm_max_mhz": max(s[1] for s in self.samples), "reasons": reasons, "samples": len(self.samples),
+                "source": "nvml"}
 
 
 def dist_setup(args):

@@ -11,28 +11,28 @@
 // n_items + j*Hkv + g. The CTA's key tiles form one sequence n = 0, 1, ... across its items
 // i = 0, 1, ...
 //
+// Two lanes. The CTA's items are dealt to two independent pipelines (lanes), each item to the
+// lane with fewer key tiles so far (ties to lane 0); every role derives the same split from the
+// item list. A lane owns its Q, K and V buffers, its S and O in TMEM, a softmax warpgroup, an MMA
+// issuer and a TMA producer; the lanes share only the tensor core and the epilogue, so one lane's
+// exponentials overlap the other's matrix products.
+//
 // Roles (512 threads, four warpgroups; registers moved with setmaxnreg):
-//   WG0 / WG1 (warps 0-7)  softmax of the even / odd key tiles: row r = 32*(warp%4) + lane
-//   WG2 (warps 8-11)       epilogue: normalises O of a finished item and stores O_c, LSE_c
-//   warp 12                TMA producer: Q per item (2 buffers), K(n) and V(n) (2 buffers each)
-//   warp 13                QK^T issuer (one thread) and TMEM owner
-//   warp 14                PV issuer (one thread)
+//   WG0 / WG1 (warps 0-7)  softmax of lane 0 / 1: row r = 32*(warp%4) + lane
+//   WG2 (warps 8-11)       epilogue: stores O_c, LSE_c of whichever lane finished an item
+//   warp 12 / 15           TMA producer of lane 0 / 1: Q per item, K(n) and V(n) per key tile
+//   warp 13 / 14           tcgen05.mma issuer of lane 0 / 1 (warp 13 owns TMEM)
 //
-// TMEM (all 512 columns): S[2] = Q K^T (128 fp32 columns each, tile n in S[n % 2]), P[2] (bf16
-// pairs, 64 columns each) and O (128 fp32 columns). A thread issuing tcgen05.mma waits while the
-// tensor core works through its previous instruction, and back-to-back MMAs into one accumulator
-// wait on each other; two threads issuing independent chains at the same moment keep the tensor
-// core busy. So both issuers start on the same event: when P(n) is written, one issues PV(n) and
-// the other QK^T(n+2) (S[n % 2] is free: the softmax of tile n has finished with it). The two
-// softmax warpgroups work on consecutive tiles at the same time, so one evaluates exponentials
-// while the other loads and reduces, and the epilogue warpgroup drains O while the next item's
-// scores are computed. The issuers only commit S-ready and PV-done; the softmax threads release
-// the K, V and Q buffers once those commits say the reads are over.
+// TMEM (512 columns): S_L = Q K^T of lane L's current key tile (128 fp32 columns at 128 L), with
+// P_L = softmax numerators written over its first 64 columns as bf16 pairs, and O_L (128 fp32
+// columns at 256 + 128 L). Issuer L runs QK(n) -> [P(n) ready] -> PV(n) -> QK(n+1) -> ...: the
+// tensor core executes one thread's MMAs in issue order, so QK(n+1) overwrites S_L only after
+// PV(n) has read P_L from it, and S_L(n+1) ready implies PV(n) complete (so O_L is current when
+// the softmax rescales it). A thread issuing tcgen05.mma waits while the tensor core works through
+// its previous instruction; two issuers with independent chains keep it busy.
 //
-// Online softmax in log2 units (x = s * scale * log2 e). The running reference max m of a row only
-// moves when a tile's max exceeds it by more than 8 (so P <= 256); tile n publishes its m to tile
-// n+1 through shared memory, and a move rescales O (after PV(n-1)) and the row sums. Each
-// warpgroup sums P over its own tiles, relative to its latest m; the epilogue combines the two sums.
+// Online softmax in log2 units (x = s * scale * log2 e). The reference max m of a row only moves
+// when a tile's max exceeds it by more than 8 (so P <= 256); a move rescales O_L and the row sum l.
 // LSE = (m + log2 l) * ln 2.
 //
 // Every wait is bounded (2 s); on expiry the CTA raises SPLITKV_DEV_TIMEOUT, drains its copies and
@@ -50,40 +50,40 @@ using namespace sm100;
 
 constexpr int kThreads = 512;
 constexpr int kEpiWarp0 = 8;
-constexpr int kProducerWarp = 12;
-constexpr int kMmaWarp = 13;  // QK^T issuer, TMEM owner
-constexpr int kPvWarp = 14;
-constexpr int kSoftmaxRegs = 152;  // per SM sub-partition: 152 + 152 + 104 + 96 = 504 <= 4 x 128 launched
-constexpr int kEpilogueRegs = 104;
-constexpr int kControlRegs = 96;
-constexpr int kTileBytes = 32768;    // 128 x 128 bf16, as two 128-byte-wide halves
+constexpr int kLoadWarp0 = 12;  // TMA producer of lane 0 (lane 1: warp 15)
+constexpr int kLoadWarp1 = 15;
+constexpr int kMmaWarp0 = 13;  // issuer of lane 0, TMEM owner (lane 1: warp 14)
+constexpr int kMmaWarp1 = 14;
+constexpr int kSoftmaxRegs = 152;  // per SM sub-partition: 152 + 152 + 88 + 120 = 512 = 4 x 128 launched
+constexpr int kEpilogueRegs = 88;
+constexpr int kControlRegs = 120;
+constexpr int kTileBytes = 32768;  // 128 x 128 bf16, as two 128-byte-wide halves
 constexpr int kHalfBytes = 16384;
 constexpr int kKeysPerTile = 128;
 constexpr uint64_t kTimeoutNs = 2000000000ull;
 constexpr float kRescaleLog2 = 8.0f;
 constexpr int kWgThreads = 128;
 
-constexpr uint32_t kColS0 = 0, kColP0 = 256, kColO = 384;  // S[b] at 128 b, P[b] at 256 + 64 b
+constexpr uint32_t kColS = 0, kColO = 256;  // S_L at 128 L, O_L at 256 + 128 L
 
-constexpr int kOffQ = 0;                                  // Q[2]
-constexpr int kOffK = 2 * kTileBytes;                     // K[2]
-constexpr int kOffV = 4 * kTileBytes;                     // V[2]
-constexpr int kOffMdec = 6 * kTileBytes;                  // float [2][128]: reference max of tile n (n % 2)
-constexpr int kOffStat = kOffMdec + 2 * 128 * 4;          // float [2][2][2][128]: item parity, wg, (m, l)
+constexpr int kOffQ = 0;                  // Q[lane]
+constexpr int kOffK = 2 * kTileBytes;     // K[lane]
+constexpr int kOffV = 4 * kTileBytes;     // V[lane]
+constexpr int kOffStat = 6 * kTileBytes;  // float [lane][item parity][m, l][128]
 constexpr int kOffBar = kOffStat + 2 * 2 * 2 * 128 * 4;
 
+// Per lane L (one buffer each; phases count the lane's items k or key tiles n).
 struct Bars {
-    uint64_t q_full[2], q_empty[2];
-    uint64_t k_full[2], k_empty[2];
-    uint64_t v_full[2], v_empty[2];
-    uint64_t s_full[2];     // QK^T(n) complete, by n % 2
-    uint64_t p_full[2];     // P(n) written, by n % 2
-    uint64_t pv_done[2];    // PV(n) complete, by n % 2
-    uint64_t mdec[2];       // reference max of tile n published, by n % 2
-    uint64_t stat_full[2];  // m and l of item i written (by item parity)
-    uint64_t o_ready[2];    // last PV of item i complete (by item parity)
-    uint64_t o_free[2];     // epilogue has read O for item i (by item parity)
-    uint64_t drain[2];      // all MMAs of the QK^T / PV issuer complete
+    uint64_t q_full[2], q_empty[2];  // Q of item k landed / every QK^T of item k complete
+    uint64_t k_full[2], k_empty[2];  // K(n) landed / QK^T(n) complete
+    uint64_t v_full[2], v_empty[2];  // V(n) landed / PV(n) complete
+    uint64_t s_full[2];              // QK^T(n) complete
+    uint64_t p_full[2];              // P(n) written
+    uint64_t o_ready[2];             // last PV of item k complete
+    uint64_t o_free[2][2];           // [lane][k % 2]: epilogue has read O_L of item k
+    uint64_t stat_full[2][2];        // [lane][k % 2]: (m, l) of item k written
+    uint64_t drain[2];               // all MMAs of issuer L complete
+    int32_t exp_slot[4];             // per SM sub-partition: 1 while a softmax warp is in its exponential pass
     uint32_t tmem_base;
     int32_t abort_flag;
     int32_t status0;
@@ -94,14 +94,14 @@ constexpr int kSmemBytes = kOffBar + (int)sizeof(Bars) + 1024;  // + alignment s
 struct TileRef {
     int64_t id;                // partial slot: item id, or n_items + j*Hkv + g for a self item
     int32_t s, c, g, j;
-    int32_t nvis, ntiles, t;
+    int32_t nvis, ntiles;
     int32_t self_item;         // 1: keys are the block's own (Kb/Vb rows block*j ..)
 };
 
 // The CTA's items (queue positions first, first+1, ...), fetched ahead: each call hands out the
 // next (item id, anchor) and issues the loads one link further for the three items after it
 // (anchor of n+1, id of n+2, queue entry of n+3), so no role waits on a dependent global load
-// chain when it moves to a new item.
+// chain when it moves to a new item. The self items follow the queue.
 struct ItemStream {
     int32_t pos, end, left;
     int64_t id1;  // item n+1 (loaded)
@@ -138,7 +138,6 @@ __device__ __forceinline__ bool stream_more(const ItemStream& st) { return st.le
 // Next item as a tile reference (ntiles == 0 for an invalid entry, which raises BAD_PLAN).
 __device__ __forceinline__ void stream_next(const Meta& m, const int32_t* anchors, const int32_t* item_id,
                                             const int32_t* queue_items, ItemStream& st, TileRef& tr, int32_t* status) {
-    tr.t = 0;
     if (st.left <= 0) {  // self item
         const int32_t sid = st.self_pos;
         st.self_pos += gridDim.x;
@@ -174,39 +173,121 @@ __device__ __forceinline__ void stream_next(const Meta& m, const int32_t* anchor
     tr.j = it.j;
     tr.nvis = visible_in_chunk(m, it.s, it.c, a);
     tr.ntiles = (tr.nvis + kKeysPerTile - 1) / kKeysPerTile;
-    tr.t = 0;
 }
 
-// The CTA's items as one sequence of key tiles.
-struct Cursor {
-    ItemStream st;
-    bool has;
-    TileRef cur;
-};
+// Next valid item (ntiles > 0); false at the end of the CTA's work.
+__device__ __forceinline__ bool next_item(const Meta& m, const int32_t* anchors, const int32_t* item_id,
+                                          const int32_t* queue_items, ItemStream& st, TileRef& tr, int32_t* status) {
+    while (stream_more(st)) {
+        stream_next(m, anchors, item_id, queue_items, st, tr, status);
+        if (tr.ntiles > 0) return true;
+    }
+    return false;
+}
 
-__device__ __forceinline__ void cursor_fetch(const Meta& m, const int32_t* anchors, const int32_t* item_id,
-                                             const int32_t* queue_items, Cursor& c, int32_t* status) {
-    while (stream_more(c.st)) {
-        stream_next(m, anchors, item_id, queue_items, c.st, c.cur, status);
-        if (c.cur.ntiles > 0) {
-            c.has = true;
-            return;
+// The two softmax warps of one SM sub-partition (warp q of each lane) take turns in the
+// exponential pass: the MUFU unit is the sub-partition's bottleneck, and when the passes alternate,
+// each lane's exponentials overlap the other lane's matrix products. Lane 0 of the warp takes the
+// slot; false on abort or after the time limit.
+__device__ __forceinline__ bool exp_slot_take(int32_t* slot, volatile int* abort_flag, uint64_t limit_ns) {
+    bool got = false;
+    if ((threadIdx.x & 31) == 0) {
+        const uint64_t t0 = globaltimer();
+        for (uint32_t n = 0;; ++n) {
+            if (atomicCAS(slot, 0, 1) == 0) {
+                got = true;
+                break;
+            }
+            __nanosleep(32);
+            if ((n & 63u) == 63u && (*abort_flag || globaltimer() - t0 > limit_ns)) break;
         }
     }
-    c.has = false;
+    return __shfl_sync(0xffffffffu, got ? 1 : 0, 0) != 0;
 }
 
-__device__ __forceinline__ void cursor_init(const Meta& m, const int32_t* anchors, const int32_t* item_id,
-                                            const int32_t* queue_items, int32_t first, int32_t end, Cursor& c,
-                                            int32_t* status) {
-    stream_init(m, anchors, item_id, queue_items, first, end, c.st);
-    cursor_fetch(m, anchors, item_id, queue_items, c, status);
+__device__ __forceinline__ void exp_slot_give(int32_t* slot) {
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) atomicExch(slot, 0);
 }
 
-__device__ __forceinline__ void cursor_advance(const Meta& m, const int32_t* anchors, const int32_t* item_id,
-                                               const int32_t* queue_items, Cursor& c, int32_t* status) {
-    if (++c.cur.t < c.cur.ntiles) return;
-    cursor_fetch(m, anchors, item_id, queue_items, c, status);
+// S columns 64h .. 64h+63 of this thread's row; keys at or beyond `valid` read as -inf.
+__device__ __forceinline__ void load_half(uint32_t ts, int h, int valid, uint32_t (&ra)[32], uint32_t (&rb)[32]) {
+    tmem_ld32(ts + h * 64, ra);
+    tmem_ld32(ts + h * 64 + 32, rb);
+    tmem_wait_ld();
+    if (valid < h * 64 + 64) {
+#pragma unroll
+        for (int u = 0; u < 32; ++u) {
+            if (h * 64 + u >= valid) ra[u] = __float_as_uint(-INFINITY);
+            if (h * 64 + 32 + u >= valid) rb[u] = __float_as_uint(-INFINITY);
+        }
+    }
+}
+
+__device__ __forceinline__ float max_half(const uint32_t (&ra)[32], const uint32_t (&rb)[32]) {
+    float m0 = -INFINITY, m1 = -INFINITY, m2 = -INFINITY, m3 = -INFINITY;
+#pragma unroll
+    for (int u = 0; u < 32; u += 4) {
+        m0 = max3f(m0, __uint_as_float(ra[u]), __uint_as_float(ra[u + 1]));
+        m1 = max3f(m1, __uint_as_float(ra[u + 2]), __uint_as_float(ra[u + 3]));
+        m2 = max3f(m2, __uint_as_float(rb[u]), __uint_as_float(rb[u + 1]));
+        m3 = max3f(m3, __uint_as_float(rb[u + 2]), __uint_as_float(rb[u + 3]));
+    }
+    return fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
+}
+
+// P = 2^(s*c - m) for 64 keys as 32 bf16 pairs (low half = even key), summed into acc.
+__device__ __forceinline__ void exp_half(const uint32_t (&ra)[32], const uint32_t (&rb)[32], uint64_t c2,
+                                         uint64_t negm2, uint64_t (&acc)[4], uint32_t (&pk)[32]) {
+#pragma unroll
+    for (int u = 0; u < 32; ++u) {
+        const uint32_t* src = u < 16 ? ra : rb;
+        const int v = (u & 15) * 2;
+        float t0, t1;
+        f2_unpack(f2_fma(f2_pack(__uint_as_float(src[v]), __uint_as_float(src[v + 1])), c2, negm2), t0, t1);
+        const float p0 = ex2_approx(t0), p1 = ex2_approx(t1);
+        acc[u & 3] = f2_add(acc[u & 3], f2_pack(p0, p1));
+        __nv_bfloat162 hp = __floats2bfloat162_rn(p0, p1);
+        pk[u] = *reinterpret_cast<uint32_t*>(&hp);
+    }
+}
+
+// O_L *= alpha for this thread's row (128 columns).
+__device__ __forceinline__ void rescale_o(uint32_t to, float alpha) {
+#pragma unroll 1
+    for (int cc = 0; cc < 8; ++cc) {
+        uint32_t ov[16];
+        tmem_ld16(to + cc * 16, ov);
+        tmem_wait_ld();
+#pragma unroll
+        for (int u = 0; u < 16; ++u) ov[u] = __float_as_uint(__uint_as_float(ov[u]) * alpha);
+        tmem_st16(to + cc * 16, ov);
+    }
+}
+
+// Items dealt to lane L: every role walks the CTA's items in order and gives each to the lane with
+// fewer key tiles so far (ties to lane 0), keeping those of lane L.
+struct LaneWalk {
+    ItemStream st;
+    int32_t tiles0, tiles1;
+};
+
+__device__ __forceinline__ void lane_init(const Meta& m, const int32_t* anchors, const int32_t* item_id,
+                                          const int32_t* queue_items, int32_t first, int32_t end, LaneWalk& w) {
+    stream_init(m, anchors, item_id, queue_items, first, end, w.st);
+    w.tiles0 = w.tiles1 = 0;
+}
+
+__device__ __forceinline__ bool lane_next(const Meta& m, const int32_t* anchors, const int32_t* item_id,
+                                          const int32_t* queue_items, LaneWalk& w, int L, TileRef& t,
+                                          int32_t* status) {
+    while (next_item(m, anchors, item_id, queue_items, w.st, t, status)) {
+        const int lane = w.tiles0 <= w.tiles1 ? 0 : 1;
+        if (lane == 0) w.tiles0 += t.ntiles;
+        else w.tiles1 += t.ntiles;
+        if (lane == L) return true;
+    }
+    return false;
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -218,7 +299,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                   float* __restrict__ o_part, float* __restrict__ lse_part, int32_t* __restrict__ status) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    float* mdec = reinterpret_cast<float*>(smem + kOffMdec);
     float* stat = reinterpret_cast<float*>(smem + kOffStat);
     Bars* bars = reinterpret_cast<Bars*>(smem + kOffBar);
     volatile int* abort_flag = &bars->abort_flag;
@@ -236,14 +316,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&bars->v_empty[b], 1);
             mbar_init(&bars->s_full[b], 1);
             mbar_init(&bars->p_full[b], kWgThreads);
-            mbar_init(&bars->pv_done[b], 1);
-            mbar_init(&bars->mdec[b], kWgThreads);
-            mbar_init(&bars->stat_full[b], 2 * kWgThreads);
             mbar_init(&bars->o_ready[b], 1);
-            mbar_init(&bars->o_free[b], kWgThreads);
+            mbar_init(&bars->o_free[b][0], kWgThreads);
+            mbar_init(&bars->o_free[b][1], kWgThreads);
+            mbar_init(&bars->stat_full[b][0], kWgThreads);
+            mbar_init(&bars->stat_full[b][1], kWgThreads);
+            mbar_init(&bars->drain[b], 1);
         }
-        mbar_init(&bars->drain[0], 1);
-        mbar_init(&bars->drain[1], 1);
+        for (int q = 0; q < 4; ++q) bars->exp_slot[q] = 0;
         bars->abort_flag = 0;
         bars->status0 = status_bad(status) ? 1 : 0;
         fence_barrier_init();
@@ -252,7 +332,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = threadIdx.x; i < 2 * kTileBytes / 16; i += kThreads)
         reinterpret_cast<uint4*>(smem + kOffQ)[i] = make_uint4(0, 0, 0, 0);
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-    if (warp == kMmaWarp) {
+    if (warp == kMmaWarp0) {
         tmem_alloc(&bars->tmem_base, 512);
         tmem_relinquish();
     }
@@ -263,330 +343,267 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool skip = bars->status0 != 0 || (q0 >= q1 && (int64_t)blockIdx.x >= m.n_blocks * m.hkv);
     const int G = m.group, R = m.rows;
 
-    if (warp >= kProducerWarp) {
+    if (warp >= kLoadWarp0) {
         // ------------------------------------------------------------ control warpgroup
         asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(kControlRegs));
-        if (!skip && warp == kProducerWarp && lane == 0) {
-            tma_prefetch_desc(&tmQ);
-            tma_prefetch_desc(&tmK);
-            tma_prefetch_desc(&tmV);
-            tma_prefetch_desc(&tmKb);
-            tma_prefetch_desc(&tmVb);
+        if (!skip && (warp == kLoadWarp0 || warp == kLoadWarp1) && lane == 0) {
+            // Lane L: Q of item k, then K(n) and V(n) for each of its key tiles.
+            const int L = warp == kLoadWarp0 ? 0 : 1;
+            tma_prefetch_desc(L ? &tmK : &tmQ);
+            tma_prefetch_desc(L ? &tmKb : &tmV);
             const uint32_t q_bytes = 2u * 64u * (uint32_t)G * (uint32_t)m.block * 2u;
-            Cursor cur;
-            TileRef prev;
-            uint32_t n = 0, item_seq = 0;
+            uint8_t* qdst = smem + kOffQ + L * kTileBytes;
+            uint8_t* kdst = smem + kOffK + L * kTileBytes;
+            uint8_t* vdst = smem + kOffV + L * kTileBytes;
+            LaneWalk w;
+            lane_init(m, anchors, item_id, queue_items, q0, q1, w);
+            TileRef t;
+            uint32_t k = 0, n = 0;
+            uint32_t inflight = 0;  // 1: Q(k-1), 2: K(n-1), 4: V(n-1) may still be landing
             bool ok = true;
-            cursor_init(m, anchors, item_id, queue_items, q0, q1, cur, status);
-            auto load_tile = [&](const CUtensorMap* map, uint64_t* full, uint64_t* empty, uint32_t idx, int off,
-                                 const TileRef& t) -> bool {
-                const int b = idx & 1;
-                if (!mbar_wait(&empty[b], ((idx >> 1) & 1u) ^ 1u, abort_flag, kTimeoutNs)) return false;
-                mbar_arrive_expect_tx(&full[b], kTileBytes);
-                const int32_t row = t.self_item ? m.block * t.j
-                                                : (int32_t)(m.key_off[t.s] + (int64_t)t.c * m.chunk +
-                                                            (int64_t)t.t * kKeysPerTile);
-                uint8_t* dst = smem + off + b * kTileBytes;
-                tma_load_3d(dst, map, &full[b], 0, t.g, row);
-                tma_load_3d(dst + kHalfBytes, map, &full[b], 64, t.g, row);
-                return true;
-            };
-            // Order: Q (new item), K(n), V(n-1).
-            while (ok && cur.has) {
-                const TileRef t = cur.cur;
-                if (t.t == 0) {
-                    const int qb = item_seq & 1;
-                    if (!mbar_wait(&bars->q_empty[qb], ((item_seq >> 1) & 1u) ^ 1u, abort_flag, kTimeoutNs)) {
+            while (ok && lane_next(m, anchors, item_id, queue_items, w, L, t, status)) {
+                if (k >= 1 && !mbar_wait(&bars->q_empty[L], (k - 1) & 1u, abort_flag, kTimeoutNs)) {
+                    ok = false;
+                    break;
+                }
+                mbar_arrive_expect_tx(&bars->q_full[L], q_bytes);
+                tma_load_3d(qdst, &tmQ, &bars->q_full[L], 0, t.g * G, m.block * t.j);
+                tma_load_3d(qdst + kHalfBytes, &tmQ, &bars->q_full[L], 64, t.g * G, m.block * t.j);
+                ++k;
+                inflight = 1;
+                const CUtensorMap* mk = t.self_item ? &tmKb : &tmK;
+                const CUtensorMap* mv = t.self_item ? &tmVb : &tmV;
+                for (int32_t tt = 0; tt < t.ntiles; ++tt, ++n) {
+                    const uint32_t ph = (n & 1u) ^ 1u;
+                    const int32_t row = t.self_item ? m.block * t.j
+                                                    : (int32_t)(m.key_off[t.s] + (int64_t)t.c * m.chunk +
+                                                                (int64_t)tt * kKeysPerTile);
+                    if (!mbar_wait(&bars->k_empty[L], ph, abort_flag, kTimeoutNs)) {
                         ok = false;
                         break;
                     }
-                    mbar_arrive_expect_tx(&bars->q_full[qb], q_bytes);
-                    uint8_t* dst = smem + kOffQ + qb * kTileBytes;
-                    tma_load_3d(dst, &tmQ, &bars->q_full[qb], 0, t.g * G, m.block * t.j);
-                    tma_load_3d(dst + kHalfBytes, &tmQ, &bars->q_full[qb], 64, t.g * G, m.block * t.j);
-                    ++item_seq;
+                    mbar_arrive_expect_tx(&bars->k_full[L], kTileBytes);
+                    tma_load_3d(kdst, mk, &bars->k_full[L], 0, t.g, row);
+                    tma_load_3d(kdst + kHalfBytes, mk, &bars->k_full[L], 64, t.g, row);
+                    inflight = 3;
+                    if (!mbar_wait(&bars->v_empty[L], ph, abort_flag, kTimeoutNs)) {
+                        ++n;
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&bars->v_full[L], kTileBytes);
+                    tma_load_3d(vdst, mv, &bars->v_full[L], 0, t.g, row);
+                    tma_load_3d(vdst + kHalfBytes, mv, &bars->v_full[L], 64, t.g, row);
+                    inflight = 7;
                 }
-                ok = load_tile(t.self_item ? &tmKb : &tmK, bars->k_full, bars->k_empty, n, kOffK, t);
-                if (ok && n > 0)
-                    ok = load_tile(prev.self_item ? &tmVb : &tmV, bars->v_full, bars->v_empty, n - 1, kOffV, prev);
-                if (!ok) break;
-                prev = t;
-                ++n;
-                cursor_advance(m, anchors, item_id, queue_items, cur, status);
             }
-            if (ok && n > 0)
-                ok = load_tile(prev.self_item ? &tmVb : &tmV, bars->v_full, bars->v_empty, n - 1, kOffV, prev);
-            // Drain: the most recent copy into every buffer has landed before the CTA exits.
+            if (!ok) *abort_flag = 1;
+            // Drain: the most recent copy into each buffer has landed before the CTA exits.
             volatile int never = 0;
-            for (uint32_t x = (n > 2 ? n - 2 : 0); x < n; ++x) {
-                mbar_wait(&bars->k_full[x & 1], (x >> 1) & 1u, &never, kTimeoutNs);
-                mbar_wait(&bars->v_full[x & 1], (x >> 1) & 1u, &never, kTimeoutNs);
-            }
-            for (uint32_t x = (item_seq > 2 ? item_seq - 2 : 0); x < item_seq; ++x)
-                mbar_wait(&bars->q_full[x & 1], (x >> 1) & 1u, &never, kTimeoutNs);
-        } else if (!skip && warp == kMmaWarp && lane == 0) {
-            // QK^T(0), QK^T(1) at once; QK^T(n) for n >= 2 when P(n-2) is written.
+            if (k > 0) mbar_wait(&bars->q_full[L], (k - 1) & 1u, &never, kTimeoutNs);
+            if (n > 0 && (inflight & 2)) mbar_wait(&bars->k_full[L], (n - 1) & 1u, &never, kTimeoutNs);
+            if (n > 0 && (inflight & 4)) mbar_wait(&bars->v_full[L], (n - 1) & 1u, &never, kTimeoutNs);
+        } else if (!skip && (warp == kMmaWarp0 || warp == kMmaWarp1) && lane == 0) {
+            // Issuer L: QK(n) -> wait P(n) -> PV(n) -> QK(n+1) -> ...
+            const int L = warp == kMmaWarp0 ? 0 : 1;
             constexpr uint32_t idesc_qk = umma_idesc_bf16_f32(128, 128, false, false);
-            // Descriptor bases; a K step only adds a constant to the (16-byte unit) start address.
-            uint64_t dq[2], dk[2];
-            for (int b = 0; b < 2; ++b) {
-                dq[b] = umma_desc_sw128(smem_u32(smem + kOffQ + b * kTileBytes), 16, 1024);
-                dk[b] = umma_desc_sw128(smem_u32(smem + kOffK + b * kTileBytes), 16, 1024);
-            }
-            Cursor cur;
-            uint32_t n = 0, item_seq = 0, qb = 0;
-            cursor_init(m, anchors, item_id, queue_items, q0, q1, cur, status);
-            while (cur.has) {
-                const TileRef t = cur.cur;
-                const int sb = n & 1;
-                if (n >= 2 && !mbar_wait(&bars->p_full[sb], ((n >> 1) - 1) & 1u, abort_flag, kTimeoutNs)) break;
-                if (t.t == 0) {
-                    qb = item_seq & 1;
-                    if (!mbar_wait(&bars->q_full[qb], (item_seq >> 1) & 1u, abort_flag, kTimeoutNs)) break;
-                    ++item_seq;
-                }
-                if (!mbar_wait(&bars->k_full[sb], (n >> 1) & 1u, abort_flag, kTimeoutNs)) break;
-                tc_fence_after();
-                const uint32_t ts = tmem + kColS0 + 128u * sb;
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    const uint64_t off = (uint64_t)(((kk >> 2) * kHalfBytes + (kk & 3) * 32) / 16);
-                    mma_ss(ts, dq[qb] + off, dk[sb] + off, idesc_qk, kk > 0 ? 1u : 0u);
-                }
-                mma_commit(&bars->s_full[sb]);
-                ++n;
-                cursor_advance(m, anchors, item_id, queue_items, cur, status);
-            }
-            // Drain: all MMAs issued by this thread complete before TMEM is released.
-            mma_commit(&bars->drain[0]);
-            volatile int never = 0;
-            mbar_wait(&bars->drain[0], 0, &never, kTimeoutNs);
-        } else if (!skip && warp == kPvWarp && lane == 0) {
-            // PV(n): O (+)= P(n) V(n), A = P[n % 2] from TMEM (bf16 pairs), B = V, MN-major. The first
-            // PV of item i overwrites O once the epilogue of item i-1 has read it.
             constexpr uint32_t idesc_pv = umma_idesc_bf16_f32(128, 128, false, true);
-            uint64_t dv[2];
-            for (int b = 0; b < 2; ++b)
-                dv[b] = umma_desc_sw128(smem_u32(smem + kOffV + b * kTileBytes), kHalfBytes, 1024);
-            const uint32_t to = tmem + kColO;
-            Cursor cur;
-            uint32_t n = 0, item = 0;
-            cursor_init(m, anchors, item_id, queue_items, q0, q1, cur, status);
-            while (cur.has) {
-                const TileRef t = cur.cur;
-                const bool first = t.t == 0, last = t.t == t.ntiles - 1;
-                const int sb = n & 1;
-                if (!mbar_wait(&bars->p_full[sb], (n >> 1) & 1u, abort_flag, kTimeoutNs)) break;
-                if (first && item >= 1 &&
-                    !mbar_wait(&bars->o_free[(item - 1) & 1], ((item - 1) >> 1) & 1u, abort_flag, kTimeoutNs))
+            // Descriptor bases; a K step only adds a constant to the (16-byte unit) start address.
+            const uint64_t dq = umma_desc_sw128(smem_u32(smem + kOffQ + L * kTileBytes), 16, 1024);
+            const uint64_t dk = umma_desc_sw128(smem_u32(smem + kOffK + L * kTileBytes), 16, 1024);
+            const uint64_t dv = umma_desc_sw128(smem_u32(smem + kOffV + L * kTileBytes), kHalfBytes, 1024);
+            const uint32_t ts = tmem + kColS + 128u * L, to = tmem + kColO + 128u * L;
+            LaneWalk w;
+            lane_init(m, anchors, item_id, queue_items, q0, q1, w);
+            TileRef t;
+            uint32_t k = 0, n = 0;
+            bool ok = true;
+            while (ok && lane_next(m, anchors, item_id, queue_items, w, L, t, status)) {
+                if (!mbar_wait(&bars->q_full[L], k & 1u, abort_flag, kTimeoutNs)) {
+                    ok = false;
                     break;
-                if (!mbar_wait(&bars->v_full[sb], (n >> 1) & 1u, abort_flag, kTimeoutNs)) break;
-                tc_fence_after();
-                const uint32_t tp = tmem + kColP0 + 64u * sb;
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    mma_ts(to, tp + (uint32_t)(kk * 8), dv[sb] + (uint64_t)(kk * 2048 / 16), idesc_pv,
-                           (!first || kk > 0) ? 1u : 0u);
-                mma_commit(&bars->pv_done[sb]);
-                if (last) {
-                    mma_commit(&bars->o_ready[item & 1]);
-                    ++item;
                 }
-                ++n;
-                cursor_advance(m, anchors, item_id, queue_items, cur, status);
+                for (int32_t tt = 0; tt < t.ntiles; ++tt, ++n) {
+                    const uint32_t ph = n & 1u;
+                    if (!mbar_wait(&bars->k_full[L], ph, abort_flag, kTimeoutNs)) { ok = false; break; }
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk) {
+                        const uint64_t off = (uint64_t)(((kk >> 2) * kHalfBytes + (kk & 3) * 32) / 16);
+                        mma_ss(ts, dq + off, dk + off, idesc_qk, kk > 0 ? 1u : 0u);
+                    }
+                    mma_commit(&bars->s_full[L]);
+                    mma_commit(&bars->k_empty[L]);
+                    if (tt == t.ntiles - 1) mma_commit(&bars->q_empty[L]);
+                    if (!mbar_wait(&bars->p_full[L], ph, abort_flag, kTimeoutNs)) { ok = false; break; }
+                    // The first PV of item k overwrites O_L once the epilogue has read item k-1.
+                    if (tt == 0 && k >= 1 &&
+                        !mbar_wait(&bars->o_free[L][(k - 1) & 1], ((k - 1) >> 1) & 1u, abort_flag, kTimeoutNs)) {
+                        ok = false;
+                        break;
+                    }
+                    if (!mbar_wait(&bars->v_full[L], ph, abort_flag, kTimeoutNs)) { ok = false; break; }
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)
+                        mma_ts(to, ts + (uint32_t)(kk * 8), dv + (uint64_t)(kk * 2048 / 16), idesc_pv,
+                               (tt > 0 || kk > 0) ? 1u : 0u);
+                    mma_commit(&bars->v_empty[L]);
+                    if (tt == t.ntiles - 1) mma_commit(&bars->o_ready[L]);
+                }
+                ++k;
             }
-            mma_commit(&bars->drain[1]);
+            if (!ok) *abort_flag = 1;
+            // Drain: all MMAs issued by this thread complete before TMEM is released.
+            mma_commit(&bars->drain[L]);
             volatile int never = 0;
-            mbar_wait(&bars->drain[1], 0, &never, kTimeoutNs);
+            mbar_wait(&bars->drain[L], 0, &never, kTimeoutNs);
         }
         __syncwarp();
     } else if (warp >= kEpiWarp0) {
         // ------------------------------------------------------------ epilogue warpgroup
         asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(kEpilogueRegs));
         if (!skip) {
+            // Each warp serves its 32 rows of both lanes, taking whichever lane has an item ready.
             const int quad = warp & 3;
             const int r = quad * 32 + lane;
             const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
-            uint32_t i = 0;
-            ItemStream st;
-            stream_init(m, anchors, item_id, queue_items, q0, q1, st);
-            while (stream_more(st)) {
-                TileRef t;
-                stream_next(m, anchors, item_id, queue_items, st, t, status);
-                if (t.ntiles == 0) continue;
-                const int ob = i & 1;
-                if (!mbar_wait(&bars->stat_full[ob], (i >> 1) & 1u, abort_flag, kTimeoutNs)) break;
-                if (!mbar_wait(&bars->o_ready[ob], (i >> 1) & 1u, abort_flag, kTimeoutNs)) break;
+            LaneWalk w0, w1;
+            lane_init(m, anchors, item_id, queue_items, q0, q1, w0);
+            lane_init(m, anchors, item_id, queue_items, q0, q1, w1);
+            TileRef t0, t1;
+            bool has0 = lane_next(m, anchors, item_id, queue_items, w0, 0, t0, status);
+            bool has1 = lane_next(m, anchors, item_id, queue_items, w1, 1, t1, status);
+            uint32_t k0 = 0, k1 = 0;
+            uint64_t deadline = globaltimer() + kTimeoutNs;
+            bool ok = true;
+            while (has0 || has1) {
+                int pick = -1;
+                if (has0 && mbar_try_wait(&bars->stat_full[0][k0 & 1], (k0 >> 1) & 1u) &&
+                    mbar_try_wait(&bars->o_ready[0], k0 & 1u))
+                    pick = 0;
+                else if (has1 && mbar_try_wait(&bars->stat_full[1][k1 & 1], (k1 >> 1) & 1u) &&
+                         mbar_try_wait(&bars->o_ready[1], k1 & 1u))
+                    pick = 1;
+                pick = __shfl_sync(0xffffffffu, pick, 0);
+                if (pick < 0) {
+                    if (*abort_flag || globaltimer() > deadline) {
+                        ok = false;
+                        break;
+                    }
+                    continue;
+                }
+                const uint32_t k = pick ? k1 : k0;
+                // Lane 0 saw both phases complete; every thread observes them too (acquire), at once.
+                mbar_wait(&bars->stat_full[pick][k & 1], (k >> 1) & 1u, abort_flag, kTimeoutNs);
+                mbar_wait(&bars->o_ready[pick], k & 1u, abort_flag, kTimeoutNs);
                 tc_fence_after();
-                // Both warpgroups' sums, moved to the final reference max (the larger m: m only grows).
-                const float* sp = stat + ob * 512;
-                const float m0 = sp[r], l0 = sp[128 + r], m1 = sp[256 + r], l1 = sp[384 + r];
-                const float m_fin = fmaxf(m0, m1);
-                const float l_row = (l0 > 0.f ? l0 * ex2_approx(m0 - m_fin) : 0.f) +
-                                    (l1 > 0.f ? l1 * ex2_approx(m1 - m_fin) : 0.f);
-                const float inv_l = 1.f / l_row;
+                const TileRef& t = pick ? t1 : t0;
+                const float* sp = stat + (pick * 2 + (int)(k & 1)) * 256;
+                const float m_l = sp[r], l = sp[128 + r];
+                const float inv = 1.f / l;
                 float* op = o_part + t.id * (int64_t)R * 128;
-                const uint32_t to = tmem + kColO + lane_off;
+                const uint32_t to = tmem + kColO + 128u * pick + lane_off;
 #pragma unroll 1
-                for (int cc = 0; cc < 4; ++cc) {
-                    uint32_t ov[32];
-                    tmem_ld32(to + cc * 32, ov);
+                for (int cc = 0; cc < 8; ++cc) {
+                    uint32_t ov[16];
+                    tmem_ld16(to + cc * 16, ov);
                     tmem_wait_ld();
-                    if (cc == 3) {  // O fully read: the issuer may start item i+1 in it
+                    if (cc == 7) {  // O_L fully read: issuer L may start the lane's next item in it
                         tc_fence_before();
-                        mbar_arrive(&bars->o_free[ob]);
+                        mbar_arrive(&bars->o_free[pick][k & 1]);
                     }
                     if (r < R) {
 #pragma unroll
-                        for (int u = 0; u < 8; ++u) {
-                            float4 x = make_float4(__uint_as_float(ov[4 * u]) * inv_l,
-                                                   __uint_as_float(ov[4 * u + 1]) * inv_l,
-                                                   __uint_as_float(ov[4 * u + 2]) * inv_l,
-                                                   __uint_as_float(ov[4 * u + 3]) * inv_l);
-                            *reinterpret_cast<float4*>(op + ((int64_t)(cc * 8 + u) * R + r) * 4) = x;
+                        for (int u = 0; u < 4; ++u) {
+                            const float4 x = make_float4(__uint_as_float(ov[4 * u]) * inv,
+                                                         __uint_as_float(ov[4 * u + 1]) * inv,
+                                                         __uint_as_float(ov[4 * u + 2]) * inv,
+                                                         __uint_as_float(ov[4 * u + 3]) * inv);
+                            *reinterpret_cast<float4*>(op + ((int64_t)(cc * 4 + u) * R + r) * 4) = x;
                         }
                     }
                 }
-                if (r < R) lse_part[t.id * R + r] = (m_fin + lg2_approx(l_row)) * 0.6931471805599453f;
-                ++i;
+                if (r < R) lse_part[t.id * R + r] = (m_l + lg2_approx(l)) * 0.6931471805599453f;
+                if (pick) {
+                    ++k1;
+                    has1 = lane_next(m, anchors, item_id, queue_items, w1, 1, t1, status);
+                } else {
+                    ++k0;
+                    has0 = lane_next(m, anchors, item_id, queue_items, w0, 0, t0, status);
+                }
+                deadline = globaltimer() + kTimeoutNs;
             }
+            if (!ok) *abort_flag = 1;
         }
     } else {
         // ------------------------------------------------------------ softmax warpgroups
         asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(kSoftmaxRegs));
         if (!skip) {
-            const int wg = warp >> 2;               // this warpgroup takes the tiles n with n % 2 == wg
+            const int L = warp >> 2;                // lane
             const int quad = warp & 3;              // TMEM lane quadrant
             const int r = quad * 32 + lane;         // query-tile row
             const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
-            const uint32_t ts = tmem + kColS0 + 128u * wg + lane_off;  // S[wg], this row
-            const uint32_t tp = tmem + kColP0 + 64u * wg + lane_off;   // P[wg], this row
+            const uint32_t ts = tmem + kColS + 128u * L + lane_off;  // S_L / P_L, this row
+            const uint32_t to = tmem + kColO + 128u * L + lane_off;  // O_L, this row
             const float c = m.scale * 1.4426950408889634f;  // log2(e)
             const uint64_t c2 = f2_pack(c, c);
-            const bool leader = (threadIdx.x & (kWgThreads - 1)) == 0;
-            uint32_t n = 0, i = 0;
+            uint32_t k = 0, n = 0;
             bool ok = true;
-            ItemStream st;
-            stream_init(m, anchors, item_id, queue_items, q0, q1, st);
-            while (stream_more(st) && ok) {
-                TileRef t;
-                stream_next(m, anchors, item_id, queue_items, st, t, status);
-                if (t.ntiles == 0) continue;
-                const int ob = i & 1;
-                const uint32_t to = tmem + kColO + lane_off;
-                float m_l = -INFINITY, l = 0.f;  // this warpgroup's row sum, relative to m_l
-                for (int tt = 0; tt < t.ntiles; ++tt, ++n) {
-                    if ((int)(n & 1) != wg) continue;
-                    if (!mbar_wait(&bars->s_full[wg], (n >> 1) & 1u, abort_flag, kTimeoutNs)) { ok = false; break; }
+            LaneWalk w;
+            lane_init(m, anchors, item_id, queue_items, q0, q1, w);
+            TileRef t;
+            while (ok && lane_next(m, anchors, item_id, queue_items, w, L, t, status)) {
+                float m_l = -INFINITY, l = 0.f;  // reference max and row sum (relative to m_l)
+                for (int32_t tt = 0; tt < t.ntiles; ++tt, ++n) {
+                    // The whole warp leaves together on a timeout: the TMEM accesses below are collective.
+                    if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_full[L], n & 1u, abort_flag, kTimeoutNs))) {
+                        ok = false;
+                        break;
+                    }
                     tc_fence_after();
-                    if (leader) {  // QK^T(n) complete: K(n) is free, and Q after the item's last tile
-                        mbar_arrive(&bars->k_empty[wg]);
-                        if (tt == t.ntiles - 1) mbar_arrive(&bars->q_empty[i & 1]);
-                    }
-                    const int valid = t.nvis - tt * kKeysPerTile;  // keys of this tile the block sees (>= 1)
-                    // Pass 1: row max over the visible keys, 64 columns per TMEM wait.
-                    float mx;
-                    {
-                        float m0 = -INFINITY, m1 = -INFINITY, m2 = -INFINITY, m3 = -INFINITY;
+                    const int valid = t.nvis - tt * kKeysPerTile;  // keys of the tile the block sees (>= 1)
+                    // Pass 1: row max over the visible keys, 64 columns per TMEM wait. tcgen05.ld/st are
+                    // warp-collective, so the rescale below is decided by a warp vote (rows that do not
+                    // move scale by 1).
+                    uint32_t ra[32], rb[32];
+                    float mx = -INFINITY;
 #pragma unroll 1
-                        for (int h = 0; h < 2; ++h) {
-                            uint32_t ra[32], rb[32];
-                            tmem_ld32(ts + h * 64, ra);
-                            tmem_ld32(ts + h * 64 + 32, rb);
-                            tmem_wait_ld();
-                            if (valid >= kKeysPerTile) {
-#pragma unroll
-                                for (int u = 0; u < 32; u += 4) {
-                                    m0 = max3f(m0, __uint_as_float(ra[u]), __uint_as_float(ra[u + 1]));
-                                    m1 = max3f(m1, __uint_as_float(ra[u + 2]), __uint_as_float(ra[u + 3]));
-                                    m2 = max3f(m2, __uint_as_float(rb[u]), __uint_as_float(rb[u + 1]));
-                                    m3 = max3f(m3, __uint_as_float(rb[u + 2]), __uint_as_float(rb[u + 3]));
-                                }
-                            } else {
-#pragma unroll
-                                for (int u = 0; u < 32; ++u) {
-                                    if (h * 64 + u < valid) m0 = fmaxf(m0, __uint_as_float(ra[u]));
-                                    if (h * 64 + 32 + u < valid) m1 = fmaxf(m1, __uint_as_float(rb[u]));
-                                }
-                            }
-                        }
-                        mx = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3)) * c;
+                    for (int h = 0; h < 2; ++h) {
+                        load_half(ts, h, valid, ra, rb);
+                        mx = fmaxf(mx, max_half(ra, rb));
                     }
-                    // Reference max: tile n-1 publishes its m to tile n (every tile waits, which also
-                    // keeps a warpgroup from overwriting a slot its partner has not read yet).
-                    float m_prev = -INFINITY;
-                    if (n > 0) {
-                        if (!mbar_wait(&bars->mdec[(n - 1) & 1], ((n - 1) >> 1) & 1u, abort_flag, kTimeoutNs)) {
-                            ok = false;
-                            break;
-                        }
-                        if (tt > 0) m_prev = mdec[((n - 1) & 1) * 128 + r];
-                    }
-                    const float m_new = (tt == 0 || mx > m_prev + kRescaleLog2) ? mx : m_prev;
-                    mdec[(n & 1) * 128 + r] = m_new;
-                    mbar_arrive(&bars->mdec[n & 1]);
-                    if (tt > 0 && m_new != m_prev) {
-                        // The max moved: rescale this row of O once PV(n-1) has landed in it.
-                        if (!mbar_wait(&bars->pv_done[(n - 1) & 1], ((n - 1) >> 1) & 1u, abort_flag, kTimeoutNs)) {
-                            ok = false;
-                            break;
-                        }
-                        tc_fence_after();
-                        const float alpha = ex2_approx(m_prev - m_new);
-#pragma unroll 1
-                        for (int cc = 0; cc < 4; ++cc) {
-                            uint32_t ov[32];
-                            tmem_ld32(to + cc * 32, ov);
-                            tmem_wait_ld();
-#pragma unroll
-                            for (int u = 0; u < 32; ++u) ov[u] = __float_as_uint(__uint_as_float(ov[u]) * alpha);
-                            tmem_st32(to + cc * 32, ov);
+                    mx *= c;
+                    if (tt == 0) {
+                        m_l = mx;
+                    } else {
+                        const bool move = mx > m_l + kRescaleLog2;
+                        if (__any_sync(0xffffffffu, move)) {
+                            // The max moved: rescale O_L (PV of the previous tile is complete) and the sum.
+                            const float alpha = move ? ex2_approx(m_l - mx) : 1.f;
+                            rescale_o(to, alpha);
+                            l *= alpha;
+                            if (move) m_l = mx;
                         }
                     }
-                    if (m_l != m_new) {
-                        l = (m_l == -INFINITY) ? 0.f : l * ex2_approx(m_l - m_new);
-                        m_l = m_new;
+                    // Pass 2: P = 2^(s*c - m) as bf16 pairs over the first 64 columns of S_L (keys 2u, 2u+1
+                    // -> column u). Half h reads S columns 64h.. and writes P columns 32h.., which it has
+                    // already read.
+                    if (!exp_slot_take(&bars->exp_slot[quad], abort_flag, kTimeoutNs)) {
+                        *abort_flag = 1;
+                        ok = false;
+                        break;
                     }
-                    // P[wg] was last read by PV(n-2); once that completed, V(n-2) is free as well.
-                    if (n >= 2) {
-                        if (!mbar_wait(&bars->pv_done[wg], ((n >> 1) - 1) & 1u, abort_flag, kTimeoutNs)) {
-                            ok = false;
-                            break;
-                        }
-                        tc_fence_after();
-                        if (leader) mbar_arrive(&bars->v_empty[wg]);
-                    }
-                    // Pass 2: P = 2^(s*c - m) in bf16 pairs into P[wg] (keys 64h.. -> columns 32h..).
-                    const uint64_t negm2 = f2_pack(-m_new, -m_new);
+                    const uint64_t negm2 = f2_pack(-m_l, -m_l);
                     uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll 1
                     for (int h = 0; h < 2; ++h) {
-                        uint32_t ra[32], rb[32];
-                        tmem_ld32(ts + h * 64, ra);
-                        tmem_ld32(ts + h * 64 + 32, rb);
-                        tmem_wait_ld();
-                        if (valid < kKeysPerTile) {
-#pragma unroll
-                            for (int u = 0; u < 32; ++u) {
-                                if (h * 64 + u >= valid) ra[u] = __float_as_uint(-INFINITY);
-                                if (h * 64 + 32 + u >= valid) rb[u] = __float_as_uint(-INFINITY);
-                            }
-                        }
+                        load_half(ts, h, valid, ra, rb);
                         uint32_t pk[32];
-#pragma unroll
-                        for (int u = 0; u < 32; ++u) {
-                            const uint32_t* src = u < 16 ? ra : rb;
-                            const int v = (u & 15) * 2;
-                            float t0, t1;
-                            f2_unpack(f2_fma(f2_pack(__uint_as_float(src[v]), __uint_as_float(src[v + 1])), c2, negm2),
-                                      t0, t1);
-                            const float p0 = ex2_approx(t0), p1 = ex2_approx(t1);
-                            acc[u & 3] = f2_add(acc[u & 3], f2_pack(p0, p1));
-                            __nv_bfloat162 hp = __floats2bfloat162_rn(p0, p1);  // .x (low half) = even key
-                            pk[u] = *reinterpret_cast<uint32_t*>(&hp);
-                        }
-                        tmem_st32(tp + h * 32, pk);
+                        exp_half(ra, rb, c2, negm2, acc, pk);
+                        tmem_st32(ts + h * 32, pk);
                     }
+                    exp_slot_give(&bars->exp_slot[quad]);
                     {
                         float a0, a1, b0, b1, c0, c1, d0, d1;
                         f2_unpack(acc[0], a0, a1);
@@ -597,20 +614,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     tmem_wait_st();
                     tc_fence_before();
-                    mbar_arrive(&bars->p_full[wg]);
+                    mbar_arrive(&bars->p_full[L]);
                 }
                 if (!ok) break;
-                // Hand this warpgroup's (m, l) to the epilogue; stat[i % 2] was last read by the
-                // epilogue of item i-2.
-                if (i >= 2 && !mbar_wait(&bars->o_free[ob], ((i >> 1) - 1) & 1u, abort_flag, kTimeoutNs)) {
+                // Hand (m, l) of item k to the epilogue; stat[L][k % 2] was last read for item k-2.
+                if (k >= 2 && !mbar_wait(&bars->o_free[L][k & 1], ((k >> 1) - 1) & 1u, abort_flag, kTimeoutNs)) {
                     ok = false;
                     break;
                 }
-                float* sp = stat + ob * 512 + wg * 256;
+                float* sp = stat + (L * 2 + (int)(k & 1)) * 256;
                 sp[r] = m_l;
                 sp[128 + r] = l;
-                mbar_arrive(&bars->stat_full[ob]);
-                ++i;
+                mbar_arrive(&bars->stat_full[L][k & 1]);
+                ++k;
             }
             if (!ok) *abort_flag = 1;
         }
@@ -619,7 +635,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_before();
     __syncthreads();
     if (threadIdx.x == 0 && bars->abort_flag) raise_status(status, SPLITKV_DEV_TIMEOUT);
-    if (warp == kMmaWarp) {
+    if (warp == kMmaWarp0) {
         tc_fence_after();
         tmem_dealloc(tmem, 512);
     }

@@ -48,6 +48,17 @@ def test_drafter_shape_small(flags, n_workers):
     full_check(inp, n_workers, flags)
 
 
+@pytest.mark.parametrize("flags", [0, SIMT])
+def test_score_jumps_inside_items(flags):
+    # Keys with 12x the norm make a row's running max jump far past the lazy-rescale threshold: in
+    # an item's first tile, in the first and in the second half of later tiles. The softmax must
+    # move its reference max there (rescaling O, the row sum and the part of P already written).
+    inp = small("jumps", "drafter_s32k", [3000], [6], chunk=1024, seed=13)
+    for pos in (5, 2 * 128 + 10, 3 * 128 + 100, 1024 + 5 * 128 + 70, 2048 + 4 * 128 + 88):
+        inp.k[pos] *= 12
+    full_check(inp, n_workers=7, flags=flags)
+
+
 @pytest.mark.parametrize("hq,hkv", [(32, 8), (8, 4), (4, 4)])
 def test_other_group_sizes(hq, hkv):
     # G = 4, 2, 1: 64-, 32- and 16-row query tiles in the 128-row MMA.
