@@ -64,7 +64,7 @@ _SIGS = {
     "splitkv_plan_lpt_noalloc": (_i32, [_vp, _vp, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _vp]),
     "splitkv_attn_fwd": (_i32, [_PP, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _vp, _i32, _vp]),
     "splitkv_lse_merge": (_i32, [_PP, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
-    "splitkv_attn_bwd": (_i32, [_PP] + [_vp] * 15 + [_vp, _sz, _vp]),
+    "splitkv_attn_bwd": (_i32, [_PP] + [_vp] * 12 + [_i32] + [_vp] * 6 + [_vp, _sz, _vp]),
 }
 EXPORTS = tuple(_SIGS)
 for _name, (_res, _args) in _SIGS.items():
@@ -173,10 +173,11 @@ def splitkv_lse_merge(problem, o_part, lse_part, anchors, o, lse, status, stream
                                   _stream(stream)), "splitkv_lse_merge")
 
 
-def splitkv_attn_bwd(problem, q, k, v, kb, vb, o, lse, dout, anchors, dq, dk, dv, dkb, dvb, status, workspace,
-                     stream=None):
+def splitkv_attn_bwd(problem, q, k, v, kb, vb, o, lse, dout, anchors, item_id, queue_off, queue_items, n_workers,
+                     dq, dk, dv, dkb, dvb, status, workspace, stream=None):
     _check(_lib.splitkv_attn_bwd(problem.ptr, _p(q), _p(k), _p(v), _p(kb), _p(vb), _p(o), _p(lse), _p(dout),
-                                 _p(anchors), _p(dq), _p(dk), _p(dv), _p(dkb), _p(dvb), _p(status), _p(workspace),
+                                 _p(anchors), _p(item_id), _p(queue_off), _p(queue_items), int(n_workers), _p(dq),
+                                 _p(dk), _p(dv), _p(dkb), _p(dvb), _p(status), _p(workspace),
                                  workspace.numel() * workspace.element_size(), _stream(stream)), "splitkv_attn_bwd")
 
 
@@ -257,13 +258,15 @@ class SplitKV:
         return self.lse_merge(anchors, o, lse, stream)
 
     def backward(self, q, k, v, kb, vb, o, lse, dout, anchors, grads=None, stream=None):
+        """dQ, dK, dV, dKb, dVb (float32). The bf16 tensor-core path walks the items of the plan made by
+        the last :meth:`plan` call, which must be for these anchors (the forward's plan)."""
         if grads is None:
             f = dict(dtype=torch.float32, device=self.device)
             grads = (torch.empty(q.shape, **f), torch.empty(k.shape, **f), torch.empty(v.shape, **f),
                      torch.empty(kb.shape, **f), torch.empty(vb.shape, **f))
         dq, dk, dv, dkb, dvb = grads
-        splitkv_attn_bwd(self.problem, q, k, v, kb, vb, o, lse, dout, anchors, dq, dk, dv, dkb, dvb, self.status,
-                         self.workspace, stream)
+        splitkv_attn_bwd(self.problem, q, k, v, kb, vb, o, lse, dout, anchors, self.item_id, self.queue_off,
+                         self.queue_items, self.n_workers, dq, dk, dv, dkb, dvb, self.status, self.workspace, stream)
         return grads
 
     # -- host-side reads (synchronizing; for tests and reports)

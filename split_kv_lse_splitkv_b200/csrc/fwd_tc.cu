@@ -41,6 +41,7 @@
 
 #include "common.cuh"
 #include "sm100.cuh"
+#include "tma_map.cuh"
 
 namespace splitkv {
 
@@ -640,6 +641,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_dealloc(tmem, 512);
     }
 }
+}  // namespace
+
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
@@ -656,8 +659,8 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// 3-D bf16 map over [rows][heads][d] with a 128-byte swizzled box {64, box_heads, box_rows}.
-bool make_map(CUtensorMap* map, const void* base, int64_t rows, int heads, int d, int box_heads, int box_rows) {
+// 3-D bf16 map (declared in tma_map.cuh) over [rows][heads][d] with a 128-byte swizzled box {64, box_heads, box_rows}.
+bool make_bf16_map(CUtensorMap* map, const void* base, int64_t rows, int heads, int d, int box_heads, int box_rows) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) {
         note_error(cudaErrorNotSupported, "cudaGetDriverEntryPoint(cuTensorMapEncodeTiled)");
@@ -679,7 +682,6 @@ bool make_map(CUtensorMap* map, const void* base, int64_t rows, int heads, int d
     return true;
 }
 
-}  // namespace
 
 bool fwd_tc_supported(const Meta& m) {
     return m.dtype == SPLITKV_BF16 && m.d == 128 && m.rows <= 128 && m.block <= 256 && m.group <= 256 &&
@@ -692,11 +694,11 @@ cudaError_t launch_fwd_tc(const Meta& m, const void* q, const void* k, const voi
                           int32_t* status, cudaStream_t st) {
     CUtensorMap tq, tk, tv, tkb, tvb;
     if (m.n_queries == 0 || m.total_keys == 0) return cudaSuccess;
-    if (!make_map(&tq, q, m.n_queries, m.hq, m.d, m.group, m.block) ||
-        !make_map(&tk, k, m.total_keys, m.hkv, m.d, 1, kKeysPerTile) ||
-        !make_map(&tv, v, m.total_keys, m.hkv, m.d, 1, kKeysPerTile) ||
-        !make_map(&tkb, kb, m.n_queries, m.hkv, m.d, 1, kKeysPerTile) ||
-        !make_map(&tvb, vb, m.n_queries, m.hkv, m.d, 1, kKeysPerTile))
+    if (!make_bf16_map(&tq, q, m.n_queries, m.hq, m.d, m.group, m.block) ||
+        !make_bf16_map(&tk, k, m.total_keys, m.hkv, m.d, 1, kKeysPerTile) ||
+        !make_bf16_map(&tv, v, m.total_keys, m.hkv, m.d, 1, kKeysPerTile) ||
+        !make_bf16_map(&tkb, kb, m.n_queries, m.hkv, m.d, 1, kKeysPerTile) ||
+        !make_bf16_map(&tvb, vb, m.n_queries, m.hkv, m.d, 1, kKeysPerTile))
         return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return note_error(e, "cudaFuncSetAttribute(fwd_tc_kernel, smem)");

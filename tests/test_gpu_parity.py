@@ -103,6 +103,13 @@ def test_backward_bf16_batch():
     backward_check(small("bwd", "train_4x64k", [3000, 2048, 4096], [2, 3, 4], chunk=1024))
 
 
+@pytest.mark.parametrize("hq,hkv", [(32, 8), (8, 4), (4, 4)])
+def test_backward_other_group_sizes(hq, hkv):
+    # G = 4, 2, 1: 64-, 32- and 16-row query tiles; ragged key tiles at both sample ends.
+    inp = small("bwd_groups", "train_4x64k", [2500, 1300], [3, 2], chunk=1024, n_q_heads=hq, n_kv_heads=hkv)
+    backward_check(inp, n_workers=5)
+
+
 def test_backward_f32_tiny():
     w = W.scaled(W.get("tiny_f32"), "bwd_f32", [1024], [4], backward=True)
     backward_check(W.make_inputs(w))
