@@ -295,7 +295,7 @@ def run_ours(args):
             timed("bwd", lambda: skv.backward(d["q"], d["k"], d["v"], d["kb"], d["vb"], o, lse, d["do"], d["anchors"],
                                               grads, stream=stream), time_phases)
 
-    launches_per_step = 3 + 3 + 1 + 1 + (4 if w.backward else 0)  # cost, plan, fwd, merge, bwd kernels
+    launches_per_step = 3 + 3 + 1 + 1 + (3 if w.backward else 0)  # cost, plan, fwd, merge; bwd: rows, kv, q
     for _ in range(args.warmup):
         step(dev)
     torch.cuda.synchronize(device)
@@ -395,6 +395,12 @@ def run_ours(args):
                              kernel_ms=fwd_ms, algorithmic_flop=fwd_kernel_flops),
             "phase_ms": phase_ms,
             "imbalance": {"predicted_lpt": predicted_imb},
+            **({"backward_roofline": {"kernels": "rows_kernel + bwd_kv_kernel + bwd_q_kernel",
+                                      "algorithmic_flop": flops - fwd_kernel_flops,
+                                      "achieved": (flops - fwd_kernel_flops) / (phase_ms["bwd"] * 1e-3) / 1e12,
+                                      "peak": peak, "unit": "TFLOP/s",
+                                      "frac": (flops - fwd_kernel_flops) / (phase_ms["bwd"] * 1e-3) / 1e12 / peak}}
+               if w.backward and "bwd" in phase_ms and w.dtype == "bf16" else {}),
             "clocks": csum,
             "e2e": {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
