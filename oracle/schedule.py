@@ -16,6 +16,11 @@ Readings (the pages give neither the cost unit nor the LPT details):
 * Item index (chunk-major): ``base_s + (c * Hkv + g) * n_blocks_s + b`` where
   ``base_s`` counts the items of earlier samples and ``n_chunks_s = ceil(S/C)``.
 * Chunk cost = sum of the costs of that chunk's items.
+* Query tiles of several blocks (``pack`` = P >= 1, default 1). With P > 1 an item
+  is (s, c, g, t): the query tile holds blocks ``tP .. min(tP+P, n_blocks_s) - 1``
+  of sample s (their rows stacked, each row masked by its own block's anchor), and
+  its cost counts the key tiles that any of those rows sees. P = 1 is the item of
+  the lines above. Index: ``base_s + (c * Hkv + g) * ceil(n_blocks_s / P) + t``.
 * LPT: order items by (cost descending, item index ascending); give each in turn
   to the worker with the least (load, worker index); loads start at 0; a
   worker's queue lists its items in assignment order.
@@ -30,70 +35,75 @@ from typing import Dict, List, Sequence, Tuple
 import numpy as np
 
 
-def item_layout(anchor_counts: Sequence[int], seq_lens: Sequence[int], chunk: int, n_kv_heads: int):
-    """Per-sample (base item index, n_chunks, n_blocks) and the total item count."""
+def item_layout(anchor_counts: Sequence[int], seq_lens: Sequence[int], chunk: int, n_kv_heads: int,
+                pack: int = 1):
+    """Per-sample (base item index, n_chunks, n_query_tiles) and the total item count."""
     out = []
     base = 0
     for nb, S in zip(anchor_counts, seq_lens):
         nc = -(-int(S) // chunk)
-        out.append((base, nc, int(nb)))
-        base += nc * n_kv_heads * int(nb)
+        nt = -(-int(nb) // pack)
+        out.append((base, nc, nt))
+        base += nc * n_kv_heads * nt
     return out, base
 
 
 def costs_bruteforce(anchors_per_sample: Sequence[Sequence[int]], seq_lens: Sequence[int], chunk: int,
-                     key_tile: int, n_kv_heads: int, group: int, block: int = 16):
+                     key_tile: int, n_kv_heads: int, group: int, block: int = 16, pack: int = 1):
     """Item costs by enumerating the boolean mask of every (query tile, key tile).
 
     Returns ``(item_ids, item_costs, chunk_costs)``: visible items in ascending
     index order, their costs, and per-(sample, chunk) costs (flattened, sample-major).
     For small inputs only.
     """
-    layout, _ = item_layout([len(a) for a in anchors_per_sample], seq_lens, chunk, n_kv_heads)
+    layout, _ = item_layout([len(a) for a in anchors_per_sample], seq_lens, chunk, n_kv_heads, pack)
     ids, costs, chunk_costs = [], [], []
     for s, anchors in enumerate(anchors_per_sample):
-        base, nc, nb = layout[s]
+        base, nc, nt = layout[s]
         S = int(seq_lens[s])
         for c in range(nc):
             lo, hi = c * chunk, min((c + 1) * chunk, S)
+            keys = np.arange(lo, hi)
             total = 0
             for g in range(n_kv_heads):
-                for b, a in enumerate(anchors):
-                    rows = block * group
-                    keys = np.arange(lo, hi)
-                    mask = np.broadcast_to(keys < a, (rows, hi - lo))  # row sees context key iff key < anchor
+                for t in range(nt):
+                    # rows of every block of the tile; a row sees context key k iff k < its block's anchor
+                    members = anchors[t * pack:(t + 1) * pack]
+                    mask = np.concatenate([np.broadcast_to(keys < a, (block * group, hi - lo)) for a in members])
                     n_tiles = -(-(hi - lo) // key_tile)
                     cost = 0
-                    for t in range(n_tiles):
-                        if mask[:, t * key_tile:(t + 1) * key_tile].any():
+                    for kt in range(n_tiles):
+                        if mask[:, kt * key_tile:(kt + 1) * key_tile].any():
                             cost += 1
                     if cost:
-                        ids.append(base + (c * n_kv_heads + g) * nb + b)
+                        ids.append(base + (c * n_kv_heads + g) * nt + t)
                         costs.append(cost)
                         total += cost
             chunk_costs.append(total)
     return np.array(ids, np.int64), np.array(costs, np.int64), np.array(chunk_costs, np.int64)
 
 
-def costs_closed_form(anchors_per_sample, seq_lens, chunk, key_tile, n_kv_heads):
-    """Same result in closed form: ``cost = ceil(clamp(a - c*C, 0, min(C, S - c*C)) / Tk)``."""
-    layout, _ = item_layout([len(a) for a in anchors_per_sample], seq_lens, chunk, n_kv_heads)
+def costs_closed_form(anchors_per_sample, seq_lens, chunk, key_tile, n_kv_heads, pack: int = 1):
+    """Same result in closed form: ``cost = ceil(clamp(a - c*C, 0, min(C, S - c*C)) / Tk)`` with ``a``
+    the largest anchor of the item's blocks (the last one: anchors ascend)."""
+    layout, _ = item_layout([len(a) for a in anchors_per_sample], seq_lens, chunk, n_kv_heads, pack)
     ids, costs, chunk_costs = [], [], []
     for s, anchors in enumerate(anchors_per_sample):
-        base, nc, nb = layout[s]
+        base, nc, nt = layout[s]
         S = int(seq_lens[s])
         a = np.asarray(anchors, np.int64)
+        a_last = np.array([a[min((t + 1) * pack, len(a)) - 1] for t in range(nt)], np.int64)
         for c in range(nc):
             width = min(chunk, S - c * chunk)
-            nvis = np.clip(a - c * chunk, 0, width)
+            nvis = np.clip(a_last - c * chunk, 0, width)
             cost = -(-nvis // key_tile)
             total = 0
             for g in range(n_kv_heads):
-                for b in range(nb):
-                    if cost[b]:
-                        ids.append(base + (c * n_kv_heads + g) * nb + b)
-                        costs.append(int(cost[b]))
-                        total += int(cost[b])
+                for t in range(nt):
+                    if cost[t]:
+                        ids.append(base + (c * n_kv_heads + g) * nt + t)
+                        costs.append(int(cost[t]))
+                        total += int(cost[t])
             chunk_costs.append(total)
     return np.array(ids, np.int64), np.array(costs, np.int64), np.array(chunk_costs, np.int64)
 

@@ -53,6 +53,42 @@ def test_cost_bruteforce_equals_closed_form(seed):
     assert int(bf[1].sum()) * tk >= hkv * sum(sum(a) for a in anchors)
 
 
+@pytest.mark.parametrize("seed", range(12))
+@pytest.mark.parametrize("pack", [2, 3, 4])
+def test_multi_block_tile_costs(seed, pack):
+    # Query tiles of `pack` blocks: brute-force mask enumeration equals the closed form, and a tile's
+    # cost is the largest of its blocks' one-block costs (their visible key ranges are nested prefixes).
+    rng = np.random.default_rng(1000 + seed)
+    tk = int(rng.choice([8, 16, 32]))
+    chunk = tk * int(rng.integers(1, 5))
+    hkv = int(rng.integers(1, 3))
+    seq, anchors = [], []
+    for _ in range(int(rng.integers(1, 4))):
+        S = int(rng.integers(20, 300))
+        n = int(rng.integers(0, min(7, S - 16) + 1))
+        seq.append(S)
+        anchors.append(sorted(rng.choice(np.arange(16, S), size=n, replace=False).tolist()))
+    bf = Sch.costs_bruteforce(anchors, seq, chunk, tk, hkv, group=2, block=16, pack=pack)
+    cf = Sch.costs_closed_form(anchors, seq, chunk, tk, hkv, pack=pack)
+    for x, y in zip(bf, cf):
+        assert x.tolist() == y.tolist()
+    one = Sch.costs_closed_form(anchors, seq, chunk, tk, hkv)
+    one_cost = dict(zip(one[0].tolist(), one[1].tolist()))
+    lay1, _ = Sch.item_layout([len(a) for a in anchors], seq, chunk, hkv)
+    layp, _ = Sch.item_layout([len(a) for a in anchors], seq, chunk, hkv, pack)
+    got = dict(zip(cf[0].tolist(), cf[1].tolist()))
+    for s, a in enumerate(anchors):
+        (b1, nc, nb), (bp, _, nt) = lay1[s], layp[s]
+        assert nt == -(-len(a) // pack)
+        for c in range(nc):
+            for g in range(hkv):
+                for t in range(nt):
+                    members = range(t * pack, min((t + 1) * pack, nb))
+                    want = max(one_cost.get(b1 + (c * hkv + g) * nb + b, 0) for b in members)
+                    assert got.get(bp + (c * hkv + g) * nt + t, 0) == want
+    assert cf[2].tolist() != [] or not seq  # chunk costs present for every chunk
+
+
 def test_lpt_worked_example():
     g = read_golden("lpt_worked_example.txt")
     iw, qo, qi, load = Sch.lpt(g["costs"], g["n_workers"])
