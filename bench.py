@@ -259,7 +259,7 @@ def run_ours(args):
     inp = W.make_inputs(w)
     counts = [int(inp.anchor_off[i + 1] - inp.anchor_off[i]) for i in range(len(w.seq_lens))]
     skv = SplitKV(w.seq_lens, counts, w.n_q_heads, w.n_kv_heads, w.head_dim, w.block, w.chunk, w.key_tile, w.scale,
-                  w.torch_dtype, n_workers=w.n_workers, device=device)
+                  w.torch_dtype, n_workers=w.n_workers, device=device, blocks_per_item=w.blocks_per_item)
     host = {k: getattr(inp, k) for k in ("q", "k", "v", "kb", "vb", "anchors")}
     if w.backward:
         host["do"] = inp.do

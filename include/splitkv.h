@@ -79,19 +79,22 @@ typedef struct {
     int32_t key_tile;           /* Tk, the key tile of the cost model (128 in every workload)       */
     float scale;                /* score scale, normally 1/sqrt(d)                                  */
     int32_t dtype;              /* SPLITKV_F32 or SPLITKV_BF16                                      */
+    int32_t blocks_per_item;    /* P: consecutive blocks of a sample sharing one query tile (0 = 1);
+                                   an item is then (sample, chunk, kv head, tile of P blocks) and
+                                   P * block * G <= 128 on the tensor-core path                     */
 } splitkv_problem;
 
 /* Derived sizes of a problem. */
 typedef struct {
-    int64_t n_items_max;    /* every (sample, chunk, kv head, block) item, visible or not           */
+    int64_t n_items_max;    /* every (sample, chunk, kv head, query tile) item, visible or not      */
     int64_t n_chunks;       /* sum_s ceil(S_s / chunk): length of chunk_cost_d                       */
     int64_t n_queries;      /* Nq                                                                     */
     int64_t total_keys;     /* sum_s S_s                                                              */
     int64_t n_blocks;       /* total anchors                                                          */
-    int64_t o_part_elems;   /* float32 elements of o_part: (n_items_max + n_blocks*Hkv) * block*G * d */
-    int64_t lse_part_elems; /* float32 elements of lse_part: (n_items_max + n_blocks*Hkv) * block*G   */
+    int64_t o_part_elems;   /* float32 elements of o_part: (n_items_max + n_blocks*Hkv) * rows * d   */
+    int64_t lse_part_elems; /* float32 elements of lse_part: (n_items_max + n_blocks*Hkv) * rows       */
     int32_t max_cost;       /* chunk / key_tile: the largest item cost                                */
-    int32_t rows_per_item;  /* block * G: query rows of one item (its query tile)                     */
+    int32_t rows_per_item;  /* rows = P * block * G: query rows of one item (its query tile)          */
 } splitkv_sizes;
 
 /* Fill `out` for `problem`. Returns SPLITKV_EINVAL / SPLITKV_EUNSUPPORTED for a bad problem. */

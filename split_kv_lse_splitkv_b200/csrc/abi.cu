@@ -46,7 +46,10 @@ int build_meta(const splitkv_problem* p, Meta* m) {
     m->chunk = p->chunk;
     m->key_tile = p->key_tile;
     m->rows = p->block * m->group;
-    if (m->rows > 256) return SPLITKV_EUNSUPPORTED;
+    m->pack = p->blocks_per_item == 0 ? 1 : p->blocks_per_item;
+    if (m->pack < 1 || m->pack > 64) return SPLITKV_EINVAL;
+    m->rows_item = m->pack * m->rows;
+    if (m->rows_item > 256) return SPLITKV_EUNSUPPORTED;
     m->scale = p->scale;
     m->dtype = p->dtype;
     if (p->anchor_off[0] != 0) return SPLITKV_EINVAL;
@@ -65,7 +68,7 @@ int build_meta(const splitkv_problem* p, Meta* m) {
         if (nc > INT32_MAX) return SPLITKV_EUNSUPPORTED;
         keys += S;
         chunks += nc;
-        items += nc * m->hkv * nb;
+        items += nc * m->hkv * ((nb + m->pack - 1) / m->pack);
     }
     m->key_off[p->batch] = keys;
     m->item_base[p->batch] = items;
@@ -101,10 +104,10 @@ SPLITKV_API int splitkv_query(const splitkv_problem* problem, splitkv_sizes* out
     out->n_queries = m.n_queries;
     out->total_keys = m.total_keys;
     out->n_blocks = m.n_blocks;
-    out->o_part_elems = (m.n_items + m.n_blocks * m.hkv) * m.rows * m.d;
-    out->lse_part_elems = (m.n_items + m.n_blocks * m.hkv) * m.rows;
+    out->o_part_elems = (m.n_items + m.n_blocks * m.hkv) * m.rows_item * m.d;
+    out->lse_part_elems = (m.n_items + m.n_blocks * m.hkv) * m.rows_item;
     out->max_cost = m.chunk / m.key_tile;
-    out->rows_per_item = m.rows;
+    out->rows_per_item = m.rows_item;
     return SPLITKV_OK;
 }
 

@@ -364,8 +364,9 @@ constexpr int kQSmemBytes = kQOffBar + (int)sizeof(QBars) + 1024;
 
 struct QItem {
     int64_t id;
-    int32_t s, c, g, j;
-    int32_t nvis, ntiles, self_item;
+    int32_t s, c, g, j;       // j: first block of the query tile
+    int32_t nbt;              // blocks in the tile
+    int32_t nvis, ntiles, self_item;  // nvis: keys the tile's last (largest-anchor) block sees
 };
 
 // The CTA's items: its queue (positions pos .. end-1), then self items blockIdx.x, blockIdx.x +
@@ -387,7 +388,8 @@ __device__ __forceinline__ bool q_next(const Meta& m, const int32_t* __restrict_
         t.c = it.c;
         t.g = it.g;
         t.j = it.j;
-        t.nvis = visible_in_chunk(m, it.s, it.c, __ldg(anchors + it.j));
+        t.nbt = it.nbt;
+        t.nvis = visible_in_chunk(m, it.s, it.c, __ldg(anchors + it.j + it.nbt - 1));
         t.ntiles = (t.nvis + kKeys - 1) / kKeys;
         t.self_item = 0;
         if (t.ntiles > 0) return true;
@@ -400,6 +402,7 @@ __device__ __forceinline__ bool q_next(const Meta& m, const int32_t* __restrict_
         t.g = (int32_t)(sid % m.hkv);
         t.s = sample_of_block(m, t.j);
         t.c = 0;
+        t.nbt = 1;
         t.nvis = m.block;
         t.ntiles = 1;
         t.self_item = 1;
@@ -421,7 +424,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
     QBars* bars = reinterpret_cast<QBars*>(smem + kQOffBar);
     volatile int* abort_flag = &bars->abort_flag;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int G = m.group, R = m.rows;
+    const int G = m.group, R = m.rows_item, RB = m.rows;  // rows of a query tile / of one block
     const int32_t q0 = queue_off[blockIdx.x], q1 = queue_off[blockIdx.x + 1];
 
     if (threadIdx.x == 0) {
@@ -457,7 +460,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
 
     if (warp == 4) {
         if (!skip && lane == 0) {
-            const uint32_t q_bytes = 2u * 64u * (uint32_t)G * (uint32_t)m.block * 2u;
+            const uint32_t q_bytes = 2u * 64u * (uint32_t)G * (uint32_t)(m.block * m.pack) * 2u;
             int32_t pos = q0;
             int64_t self_pos = blockIdx.x;
             QItem t;
@@ -563,15 +566,21 @@ __global__ void __launch_bounds__(kQThreads, 1)
         uint32_t i = 0, n = 0;
         bool ok = true;
         while (ok && q_next(m, anchors, item_id, queue_items, pos, q1, self_pos, t, status)) {
-            const int64_t rb = ((int64_t)t.j * m.hkv + t.g) * R + r;
-            const float L2 = r < R ? l2[rb] : 0.f, Dr = r < R ? dvec[rb] : 0.f;
+            // Row r belongs to block t.j + x of the tile; it sees that block's prefix of the chunk (a
+            // self item: its own keys, rows of its block only).
+            const int32_t x = r / RB;
+            const bool live = x < t.nbt && (!t.self_item || x == 0);
+            const int32_t row_nvis =
+                !live ? 0 : t.self_item ? m.block : visible_in_chunk(m, t.s, t.c, __ldg(anchors + t.j + x));
+            const int64_t rb = ((int64_t)(t.j + x) * m.hkv + t.g) * RB + r % RB;
+            const float L2 = live ? l2[rb] : 0.f, Dr = live ? dvec[rb] : 0.f;
             for (int32_t tt = 0; tt < t.ntiles; ++tt, ++n) {
                 if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_full, n & 1u, abort_flag, kTimeoutNs))) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                const int valid = r < R ? t.nvis - tt * kKeys : 0;  // keys of the tile this row sees
+                const int valid = row_nvis - tt * kKeys;  // keys of the tile this row sees
 #pragma unroll 1
                 for (int cc = 0; cc < 4; ++cc) {
                     uint32_t sv[32], pv[32];
@@ -615,7 +624,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
                     tc_fence_before();
                     mbar_arrive(&bars->dq_free);
                 }
-                if (r < R) {
+                if (live) {
 #pragma unroll
                     for (int e = 0; e < 32; e += 4)
                         atomicAdd(reinterpret_cast<float4*>(dst + cc * 32 + e),
@@ -641,7 +650,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
 }  // namespace
 
 bool bwd_tc_supported(const Meta& m) {
-    return m.dtype == SPLITKV_BF16 && m.d == 128 && m.rows <= 128 && m.group >= 1 && m.total_keys < INT32_MAX &&
+    return m.dtype == SPLITKV_BF16 && m.d == 128 && m.rows_item <= 128 && m.group >= 1 && m.total_keys < INT32_MAX &&
            m.n_queries < INT32_MAX;
 }
 
@@ -667,9 +676,12 @@ cudaError_t launch_bwd_tc(const Meta& m, const void* q, const void* k, const voi
         m, (const __nv_bfloat16*)o, (const __nv_bfloat16*)dout, lse, l2, dvec);
     e = cudaGetLastError();
     if (e != cudaSuccess) return note_error(e, "launch rows_kernel");
-    CUtensorMap tq, tdo, tk, tv, tkb, tvb;
+    // Per-block Q/dO boxes for the key-stationary kernel, per-item (P blocks) boxes for the dQ kernel.
+    CUtensorMap tq, tdo, tqi, tdoi, tk, tv, tkb, tvb;
     if (!make_bf16_map(&tq, q, m.n_queries, m.hq, m.d, m.group, m.block) ||
         !make_bf16_map(&tdo, dout, m.n_queries, m.hq, m.d, m.group, m.block) ||
+        !make_bf16_map(&tqi, q, m.n_queries, m.hq, m.d, m.group, m.block * m.pack) ||
+        !make_bf16_map(&tdoi, dout, m.n_queries, m.hq, m.d, m.group, m.block * m.pack) ||
         !make_bf16_map(&tk, k, m.total_keys, m.hkv, m.d, 1, kKeys) ||
         !make_bf16_map(&tv, v, m.total_keys, m.hkv, m.d, 1, kKeys) ||
         !make_bf16_map(&tkb, kb, m.n_queries, m.hkv, m.d, 1, kKeys) ||
@@ -690,7 +702,7 @@ cudaError_t launch_bwd_tc(const Meta& m, const void* q, const void* k, const voi
                                                                        l2, dvec, dk, dv, dkb, dvb, status);
     e = cudaGetLastError();
     if (e != cudaSuccess) return note_error(e, "launch bwd_kv_kernel");
-    bwd_q_kernel<<<(unsigned)n_workers, kQThreads, kQSmemBytes, st>>>(m, tq, tdo, tk, tv, tkb, tvb, anchors, item_id,
+    bwd_q_kernel<<<(unsigned)n_workers, kQThreads, kQSmemBytes, st>>>(m, tqi, tdoi, tk, tv, tkb, tvb, anchors, item_id,
                                                                       queue_off, queue_items, l2, dvec, dq, status);
     return note_error(cudaGetLastError(), "launch bwd_q_kernel");
 }

@@ -17,7 +17,8 @@ constexpr int kMaxCost = 64;  // chunk / key_tile upper bound (planner bucket co
 // Everything a kernel needs to decode an item or a query row, by value (no device copy).
 struct Meta {
     int32_t batch;
-    int32_t hq, hkv, group, d, block, chunk, key_tile, rows;  // rows = block * group
+    int32_t hq, hkv, group, d, block, chunk, key_tile, rows;  // rows = block * group (one block)
+    int32_t pack, rows_item;              // blocks per query tile; rows_item = pack * rows
     float scale;
     int32_t dtype;
     int64_t n_items;                      // all items, visible or not
@@ -33,10 +34,12 @@ struct Meta {
     int32_t n_chunk_s[kMaxBatch];         // ceil(S_s / chunk)
 };
 
-// Decoded work item.
+// Decoded work item: query tile t of sample s (blocks b .. b + nbt - 1 of the sample) against chunk c
+// at kv head g.
 struct Item {
-    int32_t s, c, g, b;   // sample, chunk, kv head, block within sample
-    int32_t j;            // global block index = anchor_off[s] + b
+    int32_t s, c, g, b;   // sample, chunk, kv head, first block of the tile within its sample
+    int32_t j;            // its global block index = anchor_off[s] + b
+    int32_t nbt;          // blocks in the tile: min(pack, blocks of the sample - b)
 };
 
 __host__ __device__ inline int sample_of_item(const Meta& m, int64_t id) {
@@ -50,11 +53,14 @@ __host__ __device__ inline Item decode_item(const Meta& m, int64_t id) {
     it.s = sample_of_item(m, id);
     int64_t local = id - m.item_base[it.s];
     int32_t nb = m.anchor_off[it.s + 1] - m.anchor_off[it.s];
-    it.b = (int32_t)(local % nb);
-    int64_t t = local / nb;
+    int32_t nt = (nb + m.pack - 1) / m.pack;
+    int32_t tile = (int32_t)(local % nt);
+    int64_t t = local / nt;
     it.g = (int32_t)(t % m.hkv);
     it.c = (int32_t)(t / m.hkv);
+    it.b = tile * m.pack;
     it.j = m.anchor_off[it.s] + it.b;
+    it.nbt = nb - it.b < m.pack ? nb - it.b : m.pack;
     return it;
 }
 

@@ -1,9 +1,10 @@
 // Realized cost pass (Split-KV: Efficient Context Parallelism for Training Diffusion Drafters,
 // Abstract: chunks are weighted by the attention work they actually incur).
 //
-// One thread per item (s, c, g, b) of the chunk-major index space. The cost of an item is the
-// number of key tiles of chunk c holding a key the block sees:
-//     nvis = clamp(a_b - c*C, 0, min(C, S - c*C)),  cost = ceil(nvis / Tk).
+// One thread per item (s, c, g, t) of the chunk-major index space: query tile t holds blocks
+// tP .. tP+P-1 of sample s (P = 1: one block). The cost of an item is the number of key tiles of
+// chunk c holding a key one of its rows sees; with a the tile's largest (last) anchor:
+//     nvis = clamp(a - c*C, 0, min(C, S - c*C)),  cost = ceil(nvis / Tk).
 // Three launches: count visible items per CTA (and validate anchors, add chunk costs), scan the
 // CTA counts, then write the compacted (item id, cost) list in ascending id order.
 #include "common.cuh"
@@ -17,7 +18,7 @@ constexpr int kThreads = 1024;
 
 __device__ inline int32_t item_cost_of(const Meta& m, const int32_t* anchors, int64_t id, Item* out) {
     Item it = decode_item(m, id);
-    int32_t a = anchors[it.j];
+    int32_t a = anchors[it.j + it.nbt - 1];
     int32_t nvis = visible_in_chunk(m, it.s, it.c, a);
     if (out) *out = it;
     return (nvis + m.key_tile - 1) / m.key_tile;
@@ -33,11 +34,13 @@ __global__ void __launch_bounds__(kThreads) cost_count_kernel(Meta m, const int3
     if (id < m.n_items) {
         Item it;
         int32_t cost = item_cost_of(m, anchors, id, &it);
-        // Anchor validation, once per block: at its chunk-0 / head-0 item.
+        // Anchor validation, once per block: at its tile's chunk-0 / head-0 item.
         if (it.c == 0 && it.g == 0) {
-            int32_t a = anchors[it.j];
-            if (a < m.block || (int64_t)a >= m.seq_len[it.s]) raise_status(status, SPLITKV_DEV_ANCHOR_RANGE);
-            if (it.b > 0 && anchors[it.j - 1] >= a) raise_status(status, SPLITKV_DEV_ANCHOR_ORDER);
+            for (int32_t x = 0; x < it.nbt; ++x) {
+                int32_t a = anchors[it.j + x];
+                if (a < m.block || (int64_t)a >= m.seq_len[it.s]) raise_status(status, SPLITKV_DEV_ANCHOR_RANGE);
+                if (it.b + x > 0 && anchors[it.j + x - 1] >= a) raise_status(status, SPLITKV_DEV_ANCHOR_ORDER);
+            }
         }
         if (cost > 0) {
             vis = 1;

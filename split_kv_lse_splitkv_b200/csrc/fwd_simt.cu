@@ -28,7 +28,7 @@ __global__ void __launch_bounds__(kThreads) fwd_simt_kernel(Meta m, const T* __r
                                                             int32_t* __restrict__ status) {
     extern __shared__ float smem[];
     if (status_bad(status)) return;
-    const int R = m.rows, d = m.d, G = m.group;
+    const int R = m.rows_item, d = m.d, G = m.group;
     const int dp = d + 1;
     float* Qs = smem;                 // [R][d]
     float* Os = Qs + R * d;           // [R][d]
@@ -38,6 +38,7 @@ __global__ void __launch_bounds__(kThreads) fwd_simt_kernel(Meta m, const T* __r
     float* mS = Ss + R * kBK;         // [R]
     float* lS = mS + R;               // [R]
     float* aS = lS + R;               // [R]
+    int* vS = reinterpret_cast<int*>(aS + R);  // [R] keys of the chunk each row sees
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
     const int32_t q0 = queue_off[blockIdx.x], q1 = queue_off[blockIdx.x + 1];
@@ -45,7 +46,7 @@ __global__ void __launch_bounds__(kThreads) fwd_simt_kernel(Meta m, const T* __r
     // Entries: the queue's items, then self items blockIdx.x, blockIdx.x + gridDim.x, ...
     for (int64_t e_idx = q0;; ++e_idx) {
         int64_t id, kbase;
-        int32_t nvis;
+        int32_t nvis;  // keys the tile's last (largest-anchor) block sees: the most of any row
         Item it;
         const T *kp = k, *vp = v;
         if (e_idx < q1) {
@@ -53,7 +54,7 @@ __global__ void __launch_bounds__(kThreads) fwd_simt_kernel(Meta m, const T* __r
             id = item_id[kidx];
             if (id < 0 || id >= m.n_items) { raise_status(status, SPLITKV_DEV_BAD_PLAN); return; }
             it = decode_item(m, id);
-            nvis = visible_in_chunk(m, it.s, it.c, anchors[it.j]);
+            nvis = visible_in_chunk(m, it.s, it.c, anchors[it.j + it.nbt - 1]);
             kbase = m.key_off[it.s] + (int64_t)it.c * m.chunk;
         } else {
             const int64_t sid = blockIdx.x + (e_idx - q1) * (int64_t)gridDim.x;
@@ -61,6 +62,7 @@ __global__ void __launch_bounds__(kThreads) fwd_simt_kernel(Meta m, const T* __r
             id = m.n_items + sid;
             it.j = (int32_t)(sid / m.hkv);
             it.g = (int32_t)(sid % m.hkv);
+            it.nbt = 1;
             nvis = m.block;
             kbase = (int64_t)m.block * it.j;
             kp = kb;
@@ -70,11 +72,19 @@ __global__ void __launch_bounds__(kThreads) fwd_simt_kernel(Meta m, const T* __r
         for (int e = tid; e < R * d; e += kThreads) {
             int r = e / d, dd = e % d;
             int i = r / G, hl = r % G;
-            int64_t row = (int64_t)m.block * it.j + i;
-            Qs[e] = to_f32(q[(row * m.hq + (int64_t)it.g * G + hl) * d + dd]);
+            int64_t row = (int64_t)m.block * it.j + i;  // rows past the tile's blocks are masked below
+            Qs[e] = row < m.n_queries ? to_f32(q[(row * m.hq + (int64_t)it.g * G + hl) * d + dd]) : 0.f;
             Os[e] = 0.f;
         }
-        for (int r = tid; r < R; r += kThreads) { mS[r] = -INFINITY; lS[r] = 0.f; }
+        for (int r = tid; r < R; r += kThreads) {
+            mS[r] = -INFINITY;
+            lS[r] = 0.f;
+            const int x = r / m.rows;  // block of the tile this row belongs to
+            int v = 0;
+            if (e_idx >= q1) v = x == 0 ? m.block : 0;  // self item: the block's own keys, its rows only
+            else if (x < it.nbt) v = visible_in_chunk(m, it.s, it.c, anchors[it.j + x]);
+            vS[r] = v;
+        }
         __syncthreads();
 
         for (int32_t t0 = 0; t0 < nvis; t0 += kBK) {
@@ -94,7 +104,7 @@ __global__ void __launch_bounds__(kThreads) fwd_simt_kernel(Meta m, const T* __r
             for (int e = tid; e < R * kBK; e += kThreads) {
                 int r = e / kBK, jj = e % kBK;
                 float s = -INFINITY;
-                if (jj < nk) {
+                if (jj < nk && t0 + jj < vS[r]) {
                     float acc = 0.f;
                     const float* qr = Qs + r * d;
                     const float* kr = Ks + jj * dp;
@@ -109,7 +119,7 @@ __global__ void __launch_bounds__(kThreads) fwd_simt_kernel(Meta m, const T* __r
                 float mx = warp_reduce_max(x);
                 float m_old = mS[r];
                 float m_new = fmaxf(m_old, mx);
-                float p = (x == -INFINITY) ? 0.f : expf(x - m_new);
+                float p = (x == -INFINITY) ? 0.f : expf(x - m_new);  // (m_new = -inf only if x is too)
                 float sum = warp_reduce_sum(p);
                 Ss[r * kBK + lane] = p;
                 if (lane == 0) {
@@ -134,9 +144,9 @@ __global__ void __launch_bounds__(kThreads) fwd_simt_kernel(Meta m, const T* __r
         for (int e = tid; e < R * d; e += kThreads) {
             int d4 = e / (R * 4), rem = e % (R * 4);
             int r = rem / 4, c4 = rem % 4;
-            op[e] = Os[r * d + d4 * 4 + c4] / lS[r];
+            op[e] = lS[r] > 0.f ? Os[r * d + d4 * 4 + c4] / lS[r] : 0.f;  // a row that sees no key: O = 0
         }
-        for (int r = tid; r < R; r += kThreads) lse_part[id * R + r] = mS[r] + logf(lS[r]);
+        for (int r = tid; r < R; r += kThreads) lse_part[id * R + r] = lS[r] > 0.f ? mS[r] + logf(lS[r]) : -INFINITY;
         __syncthreads();
     }
 }
@@ -146,8 +156,8 @@ cudaError_t launch_t(const Meta& m, const void* q, const void* k, const void* v,
                      const int32_t* anchors, const int32_t* item_id, const int32_t* queue_off,
                      const int32_t* queue_items, int32_t n_workers, float* o_part, float* lse_part, int32_t* status,
                      cudaStream_t st) {
-    const int R = m.rows, d = m.d;
-    size_t smem = sizeof(float) * ((size_t)2 * R * d + kBK * (d + 1) + kBK * d + R * kBK + 3 * R);
+    const int R = m.rows_item, d = m.d;
+    size_t smem = sizeof(float) * ((size_t)2 * R * d + kBK * (d + 1) + kBK * d + R * kBK + 4 * R);
     cudaError_t e = cudaFuncSetAttribute(fwd_simt_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     fwd_simt_kernel<T><<<n_workers, kThreads, smem, st>>>(m, (const T*)q, (const T*)k, (const T*)v, (const T*)kb,

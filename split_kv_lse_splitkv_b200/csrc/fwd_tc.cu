@@ -95,7 +95,8 @@ constexpr int kSmemBytes = kOffBar + (int)sizeof(Bars) + 1024;  // + alignment s
 struct TileRef {
     int64_t id;                // partial slot: item id, or n_items + j*Hkv + g for a self item
     int32_t s, c, g, j;
-    int32_t nvis, ntiles;
+    int32_t nvis, ntiles;      // keys its last block sees (the most), key tiles
+    int32_t nbt;               // blocks in the query tile (rows of block x: x*block*G ..)
     int32_t self_item;         // 1: keys are the block's own (Kb/Vb rows block*j ..)
 };
 
@@ -116,7 +117,9 @@ __device__ __forceinline__ int64_t load_id(const int32_t* __restrict__ item_id, 
     return k >= 0 ? (int64_t)__ldg(item_id + k) : -1;
 }
 __device__ __forceinline__ int32_t load_anchor(const Meta& m, const int32_t* __restrict__ anchors, int64_t id) {
-    return (id >= 0 && id < m.n_items) ? __ldg(anchors + decode_item(m, id).j) : 0;
+    if (id < 0 || id >= m.n_items) return 0;
+    const Item it = decode_item(m, id);
+    return __ldg(anchors + it.j + it.nbt - 1);  // the tile's largest anchor
 }
 
 __device__ __forceinline__ void stream_init(const Meta& m, const int32_t* anchors, const int32_t* item_id,
@@ -150,6 +153,7 @@ __device__ __forceinline__ void stream_next(const Meta& m, const int32_t* anchor
         tr.c = 0;
         tr.nvis = m.block;
         tr.ntiles = 1;
+        tr.nbt = 1;
         return;
     }
     tr.self_item = 0;
@@ -172,6 +176,7 @@ __device__ __forceinline__ void stream_next(const Meta& m, const int32_t* anchor
     tr.c = it.c;
     tr.g = it.g;
     tr.j = it.j;
+    tr.nbt = it.nbt;
     tr.nvis = visible_in_chunk(m, it.s, it.c, a);
     tr.ntiles = (tr.nvis + kKeysPerTile - 1) / kKeysPerTile;
 }
@@ -342,7 +347,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     const uint32_t tmem = bars->tmem_base;
     const bool skip = bars->status0 != 0 || (q0 >= q1 && (int64_t)blockIdx.x >= m.n_blocks * m.hkv);
-    const int G = m.group, R = m.rows;
+    const int G = m.group, R = m.rows_item;
 
     if (warp >= kLoadWarp0) {
         // ------------------------------------------------------------ control warpgroup
@@ -352,7 +357,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int L = warp == kLoadWarp0 ? 0 : 1;
             tma_prefetch_desc(L ? &tmK : &tmQ);
             tma_prefetch_desc(L ? &tmKb : &tmV);
-            const uint32_t q_bytes = 2u * 64u * (uint32_t)G * (uint32_t)m.block * 2u;
+            const uint32_t q_bytes = 2u * 64u * (uint32_t)G * (uint32_t)(m.block * m.pack) * 2u;
             uint8_t* qdst = smem + kOffQ + L * kTileBytes;
             uint8_t* kdst = smem + kOffK + L * kTileBytes;
             uint8_t* vdst = smem + kOffV + L * kTileBytes;
@@ -502,7 +507,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const TileRef& t = pick ? t1 : t0;
                 const float* sp = stat + (pick * 2 + (int)(k & 1)) * 256;
                 const float m_l = sp[r], l = sp[128 + r];
-                const float inv = 1.f / l;
+                const float inv = l > 0.f ? 1.f / l : 0.f;  // a row that sees no key: O = 0, LSE = -inf
                 float* op = o_part + t.id * (int64_t)R * 128;
                 const uint32_t to = tmem + kColO + 128u * pick + lane_off;
 #pragma unroll 1
@@ -525,7 +530,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         }
                     }
                 }
-                if (r < R) lse_part[t.id * R + r] = (m_l + lg2_approx(l)) * 0.6931471805599453f;
+                if (r < R) lse_part[t.id * R + r] = l > 0.f ? (m_l + lg2_approx(l)) * 0.6931471805599453f : -INFINITY;
                 if (pick) {
                     ++k1;
                     has1 = lane_next(m, anchors, item_id, queue_items, w1, 1, t1, status);
@@ -556,6 +561,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             TileRef t;
             while (ok && lane_next(m, anchors, item_id, queue_items, w, L, t, status)) {
                 float m_l = -INFINITY, l = 0.f;  // reference max and row sum (relative to m_l)
+                // Keys of the chunk this row sees: its own block's prefix (a row of no block of the tile,
+                // or of a self item beyond the block's own rows, sees none). A row's keys lie in the
+                // item's first tiles, so a row that sees nothing in tile 0 sees nothing at all.
+                int32_t row_nvis = 0;
+                {
+                    const int32_t x = r / m.rows;
+                    if (t.self_item) row_nvis = x == 0 ? m.block : 0;
+                    else if (x < t.nbt) row_nvis = visible_in_chunk(m, t.s, t.c, __ldg(anchors + t.j + x));
+                }
                 for (int32_t tt = 0; tt < t.ntiles; ++tt, ++n) {
                     // The whole warp leaves together on a timeout: the TMEM accesses below are collective.
                     if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_full[L], n & 1u, abort_flag, kTimeoutNs))) {
@@ -563,7 +577,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         break;
                     }
                     tc_fence_after();
-                    const int valid = t.nvis - tt * kKeysPerTile;  // keys of the tile the block sees (>= 1)
+                    const int valid = row_nvis - tt * kKeysPerTile;  // keys of the tile this row sees
                     // Pass 1: row max over the visible keys, 64 columns per TMEM wait. tcgen05.ld/st are
                     // warp-collective, so the rescale below is decided by a warp vote (rows that do not
                     // move scale by 1).
@@ -595,7 +609,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                         ok = false;
                         break;
                     }
-                    const uint64_t negm2 = f2_pack(-m_l, -m_l);
+                    const float m_use = m_l == -INFINITY ? 0.f : m_l;  // fully masked row: P = 2^-inf = 0
+                    const uint64_t negm2 = f2_pack(-m_use, -m_use);
                     uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll 1
                     for (int h = 0; h < 2; ++h) {
@@ -684,7 +699,7 @@ bool make_bf16_map(CUtensorMap* map, const void* base, int64_t rows, int heads, 
 
 
 bool fwd_tc_supported(const Meta& m) {
-    return m.dtype == SPLITKV_BF16 && m.d == 128 && m.rows <= 128 && m.block <= 256 && m.group <= 256 &&
+    return m.dtype == SPLITKV_BF16 && m.d == 128 && m.rows_item <= 128 && m.block <= 256 && m.group <= 256 &&
            m.total_keys < INT32_MAX && m.n_queries < INT32_MAX;
 }
 
@@ -694,7 +709,7 @@ cudaError_t launch_fwd_tc(const Meta& m, const void* q, const void* k, const voi
                           int32_t* status, cudaStream_t st) {
     CUtensorMap tq, tk, tv, tkb, tvb;
     if (m.n_queries == 0 || m.total_keys == 0) return cudaSuccess;
-    if (!make_bf16_map(&tq, q, m.n_queries, m.hq, m.d, m.group, m.block) ||
+    if (!make_bf16_map(&tq, q, m.n_queries, m.hq, m.d, m.group, m.block * m.pack) ||
         !make_bf16_map(&tk, k, m.total_keys, m.hkv, m.d, 1, kKeysPerTile) ||
         !make_bf16_map(&tv, v, m.total_keys, m.hkv, m.d, 1, kKeysPerTile) ||
         !make_bf16_map(&tkb, kb, m.n_queries, m.hkv, m.d, 1, kKeysPerTile) ||

@@ -2,9 +2,10 @@
 // Parallelism for Training Diffusion Drafters, Abstract: exact attention assembled from
 // chunk-local, query-sized partial results).
 //
-// Block j, kv head g has the self partial (its own keys, slot n_items + j*Hkv + g) and one chunk
-// partial per visible chunk c < ceil(a/C) (item base_s + (c*Hkv + g)*nb_s + b). For each of its
-// block*G query rows r:
+// Block j (block b of sample s), kv head g has the self partial (its own keys, slot
+// n_items + j*Hkv + g, rows 0 ..) and one chunk partial per visible chunk c < ceil(a/C): item
+// base_s + (c*Hkv + g)*nt_s + b/P of the query tiles of P blocks, rows (b % P)*block*G ... For each
+// of its block*G query rows r:
 //   L = log( sum_p exp(LSE_p) ),     O = sum_p exp(LSE_p - L) O_p
 // over those partials p, accumulated online (running maximum, rescaled sum) so that the partial
 // tiles are read exactly once, in one pass.
@@ -43,11 +44,12 @@ __device__ __forceinline__ void online_add(Online& st, float lse_p, const float4
     }
 }
 
-__device__ __forceinline__ void load_cols(const float4* __restrict__ tile, int R, int r, int d40, int D4,
+// Row `r` of a partial tile of `RT` rows, float4 columns d40 .. d40 + kCols - 1.
+__device__ __forceinline__ void load_cols(const float4* __restrict__ tile, int RT, int r, int d40, int D4,
                                           float4 (&x)[kCols]) {
 #pragma unroll
     for (int u = 0; u < kCols; ++u)
-        x[u] = (d40 + u < D4) ? __ldcs(tile + (int64_t)(d40 + u) * R + r) : make_float4(0.f, 0.f, 0.f, 0.f);
+        x[u] = (d40 + u < D4) ? __ldcs(tile + (int64_t)(d40 + u) * RT + r) : make_float4(0.f, 0.f, 0.f, 0.f);
 }
 
 template <typename T>
@@ -72,9 +74,12 @@ __global__ void __launch_bounds__(kThreads) merge_kernel(Meta m, int32_t ctas_pe
     int32_t nv = (int32_t)(((int64_t)a + m.chunk - 1) / m.chunk);
     if (nv < 0) nv = 0;
     if (nv > m.n_chunk_s[s]) nv = m.n_chunk_s[s];
-    const int64_t item0 = m.item_base[s] + (int64_t)g * nb + b;  // chunk 0; chunk c adds c*Hkv*nb
-    const int64_t cstride = (int64_t)m.hkv * nb;
-    const int64_t tile4 = (int64_t)R * D4;  // float4s per partial tile
+    const int32_t nt = (nb + m.pack - 1) / m.pack;  // query tiles of the sample
+    const int64_t item0 = m.item_base[s] + (int64_t)g * nt + b / m.pack;  // chunk 0; chunk c adds c*Hkv*nt
+    const int64_t cstride = (int64_t)m.hkv * nt;
+    const int RT = m.rows_item;                 // rows of a partial tile
+    const int rc = (b % m.pack) * R + r;        // this row within its chunk partials
+    const int64_t tile4 = (int64_t)RT * D4;     // float4s per partial tile
     const float4* op = reinterpret_cast<const float4*>(o_part);
 
     Online st;
@@ -85,8 +90,8 @@ __global__ void __launch_bounds__(kThreads) merge_kernel(Meta m, int32_t ctas_pe
     {
         const int64_t self = m.n_items + jg;
         float4 x[kCols];
-        load_cols(op + self * tile4, R, r, d40, D4, x);
-        online_add(st, __ldcs(lse_part + self * R + r), x);
+        load_cols(op + self * tile4, RT, r, d40, D4, x);
+        online_add(st, __ldcs(lse_part + self * RT + r), x);
     }
     int32_t c = 0;
     for (; c + kUnroll <= nv; c += kUnroll) {
@@ -95,8 +100,8 @@ __global__ void __launch_bounds__(kThreads) merge_kernel(Meta m, int32_t ctas_pe
 #pragma unroll
         for (int k = 0; k < kUnroll; ++k) {
             const int64_t item = item0 + (int64_t)(c + k) * cstride;
-            lp[k] = __ldcs(lse_part + item * R + r);
-            load_cols(op + item * tile4, R, r, d40, D4, x[k]);
+            lp[k] = __ldcs(lse_part + item * RT + rc);
+            load_cols(op + item * tile4, RT, rc, d40, D4, x[k]);
         }
 #pragma unroll
         for (int k = 0; k < kUnroll; ++k) online_add(st, lp[k], x[k]);
@@ -104,8 +109,8 @@ __global__ void __launch_bounds__(kThreads) merge_kernel(Meta m, int32_t ctas_pe
     for (; c < nv; ++c) {
         const int64_t item = item0 + (int64_t)c * cstride;
         float4 x[kCols];
-        load_cols(op + item * tile4, R, r, d40, D4, x);
-        online_add(st, __ldcs(lse_part + item * R + r), x);
+        load_cols(op + item * tile4, RT, rc, d40, D4, x);
+        online_add(st, __ldcs(lse_part + item * RT + rc), x);
     }
 
     const float inv = 1.f / st.l;

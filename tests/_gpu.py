@@ -27,7 +27,7 @@ def run_forward(inp, n_workers=None, flags=0, device="cuda"):
     w = inp.workload
     nw = n_workers if n_workers is not None else w.n_workers
     skv = SplitKV(w.seq_lens, counts_of(inp), w.n_q_heads, w.n_kv_heads, w.head_dim, w.block, w.chunk, w.key_tile,
-                  w.scale, w.torch_dtype, n_workers=nw, device=device)
+                  w.scale, w.torch_dtype, n_workers=nw, device=device, blocks_per_item=w.blocks_per_item)
     dev = {k: getattr(inp, k).to(device) for k in ("q", "k", "v", "kb", "vb")}
     anchors = inp.anchors.to(device)
     o, lse = skv.forward(dev["q"], dev["k"], dev["v"], dev["kb"], dev["vb"], anchors, flags=flags)
@@ -54,7 +54,7 @@ def check_cost_and_plan(skv, inp):
     """Costs, compacted item list, chunk costs and the LPT plan must equal the oracle bit for bit."""
     w = inp.workload
     ids, costs, chunk_costs = OS.costs_closed_form(anchors_per_sample(inp), w.seq_lens, w.chunk, w.key_tile,
-                                                   w.n_kv_heads)
+                                                   w.n_kv_heads, pack=w.blocks_per_item)
     n = int(skv.n_items.item())
     assert n == len(ids)
     assert skv.item_id[:n].cpu().numpy().tolist() == ids.tolist()
@@ -77,29 +77,33 @@ def check_partials(skv, inp, ids):
     O_part, L_part = skv.o_part_view()
     O_part = O_part.cpu().numpy()
     L_part = L_part.cpu().numpy()
-    G, R = w.group, w.block * w.group
+    G, R, P = w.group, w.block * w.group, w.blocks_per_item
+    RT = int(skv.sizes.rows_per_item)  # rows of a partial tile: P blocks of R rows
     nb = counts_of(inp)
-    base, bases = 0, []
-    for s, S in enumerate(w.seq_lens):
-        bases.append(base)
-        base += (-(-S // w.chunk)) * w.n_kv_heads * nb[s]
+    layout, _ = OS.item_layout(nb, w.seq_lens, w.chunk, w.n_kv_heads, P)
+    bases = [x[0] for x in layout]
     got_O, ref_O, got_L, ref_L = [], [], [], []
     off = inp.anchor_off.tolist()
+    anchors = inp.anchors.tolist()
     for item in ids.tolist():
         s = max(i for i in range(len(bases)) if bases[i] <= item)
+        nt = layout[s][2]
         local = item - bases[s]
-        b = local % nb[s]
-        c = (local // nb[s]) // w.n_kv_heads
-        g = (local // nb[s]) % w.n_kv_heads
-        j = off[s] + b
-        o_tile = O_part[item].transpose(1, 0, 2).reshape(R, -1)  # [rows, d]
-        for hl in range(G):
-            ref_o, ref_l = parts[(s, c, j, g * G + hl)]
-            rows = [i * G + hl for i in range(w.block)]
-            got_O.append(o_tile[rows])
-            ref_O.append(ref_o)
-            got_L.append(L_part[item][rows])
-            ref_L.append(ref_l)
+        t = local % nt
+        c = (local // nt) // w.n_kv_heads
+        g = (local // nt) % w.n_kv_heads
+        o_tile = O_part[item].transpose(1, 0, 2).reshape(RT, -1)  # [rows, d]
+        for x in range(min(P, nb[s] - t * P)):
+            j = off[s] + t * P + x
+            if anchors[j] <= c * w.chunk:
+                continue  # this block of the tile sees no key of the chunk (its rows hold O = 0, LSE = -inf)
+            for hl in range(G):
+                ref_o, ref_l = parts[(s, c, j, g * G + hl)]
+                rows = [x * R + i * G + hl for i in range(w.block)]
+                got_O.append(o_tile[rows])
+                ref_O.append(ref_o)
+                got_L.append(L_part[item][rows])
+                ref_L.append(ref_l)
     assert_close("O_part", np.stack(got_O), np.stack(ref_O), w.dtype)
     assert_close("LSE_part", np.stack(got_L), np.stack(ref_L), w.dtype)
     n_max = int(skv.sizes.n_items_max)
@@ -108,7 +112,7 @@ def check_partials(skv, inp, ids):
         for j in range(off[s], off[s + 1]):
             for g in range(w.n_kv_heads):
                 slot = n_max + j * w.n_kv_heads + g
-                o_tile = O_part[slot].transpose(1, 0, 2).reshape(R, -1)
+                o_tile = O_part[slot].transpose(1, 0, 2).reshape(RT, -1)
                 for hl in range(G):
                     ref_o, ref_l = parts[(s, -1, j, g * G + hl)]
                     rows = [i * G + hl for i in range(w.block)]

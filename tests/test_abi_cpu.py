@@ -54,6 +54,11 @@ def test_query_sizes():
     # partial slots: every item, then one self partial per (block, kv head)
     assert s.o_part_elems == (s.n_items_max + 5 * 2) * 64 * 64 and s.lse_part_elems == (s.n_items_max + 5 * 2) * 64
     assert B.splitkv_workspace_size(prob(), 4) > 0
+    # two blocks per query tile: sample 0 has 3 blocks (2 tiles), sample 1 has 2 (1 tile)
+    s2 = B.splitkv_query(prob(seq_lens=[1000, 300], anchor_off=[0, 3, 5], n_q_heads=8, n_kv_heads=2, chunk=256,
+                              blocks_per_item=2))
+    assert s2.n_items_max == 4 * 2 * 2 + 2 * 2 * 1 and s2.rows_per_item == 2 * 16 * 4
+    assert s2.o_part_elems == (s2.n_items_max + 5 * 2) * 128 * 64
 
 
 @pytest.mark.parametrize("kw,code", [

@@ -59,11 +59,22 @@ def test_score_jumps_inside_items(flags):
     full_check(inp, n_workers=7, flags=flags)
 
 
+@pytest.mark.parametrize("full_tiles", [False, True])
 @pytest.mark.parametrize("hq,hkv", [(32, 8), (8, 4), (4, 4)])
-def test_other_group_sizes(hq, hkv):
-    # G = 4, 2, 1: 64-, 32- and 16-row query tiles in the 128-row MMA.
-    inp = small("groups", "skewed_s256k", [4096], [9], chunk=2048, n_q_heads=hq, n_kv_heads=hkv)
+def test_other_group_sizes(hq, hkv, full_tiles):
+    # G = 4, 2, 1: 64-, 32- and 16-row blocks, alone in the 128-row MMA tile or 128/(16G) of them
+    # sharing it (9 blocks: the sample's last tile is partly empty).
+    P = 128 // (16 * (hq // hkv)) if full_tiles else 1
+    inp = small("groups", "skewed_s256k", [4096], [9], chunk=2048, n_q_heads=hq, n_kv_heads=hkv, blocks_per_item=P)
     full_check(inp, n_workers=5)
+
+
+@pytest.mark.parametrize("flags", [0, SIMT])
+def test_multi_block_tiles_batch(flags):
+    # Two blocks per query tile across three samples with 3, 1 and 4 blocks (odd counts leave half-empty
+    # tiles at sample ends, where the next sample's rows follow in memory) and ragged chunks.
+    inp = small("packs", "skewed_s256k", [3000, 700, 5000], [3, 1, 4], chunk=1024, blocks_per_item=2)
+    full_check(inp, n_workers=6, flags=flags)
 
 
 def test_anchor_edges():
@@ -103,10 +114,14 @@ def test_backward_bf16_batch():
     backward_check(small("bwd", "train_4x64k", [3000, 2048, 4096], [2, 3, 4], chunk=1024))
 
 
+@pytest.mark.parametrize("full_tiles", [False, True])
 @pytest.mark.parametrize("hq,hkv", [(32, 8), (8, 4), (4, 4)])
-def test_backward_other_group_sizes(hq, hkv):
-    # G = 4, 2, 1: 64-, 32- and 16-row query tiles; ragged key tiles at both sample ends.
-    inp = small("bwd_groups", "train_4x64k", [2500, 1300], [3, 2], chunk=1024, n_q_heads=hq, n_kv_heads=hkv)
+def test_backward_other_group_sizes(hq, hkv, full_tiles):
+    # G = 4, 2, 1: 64-, 32- and 16-row blocks, one per query tile or sharing it; ragged key tiles at
+    # both sample ends.
+    P = 128 // (16 * (hq // hkv)) if full_tiles else 1
+    inp = small("bwd_groups", "train_4x64k", [2500, 1300], [3, 2], chunk=1024, n_q_heads=hq, n_kv_heads=hkv,
+                blocks_per_item=P)
     backward_check(inp, n_workers=5)
 
 

@@ -44,6 +44,7 @@ class Workload:
     key_tile: int = 128              # Tk, the key tile of the cost model
     backward: bool = False
     n_workers: Optional[int] = None  # None: one queue per SM of the device
+    blocks_per_item: int = 1         # consecutive blocks sharing one 128-row query tile (G < 8)
 
     @property
     def group(self) -> int:
@@ -69,7 +70,9 @@ WORKLOADS = {
         # Long context: S=131072, 128 anchors, chunk 2048.
         Workload("long_s128k", 32, 4, 128, [131072], [128], 2048, "bf16", 2),
         # Skewed anchors: 32 q / 8 kv heads, S=262144, 256 draws of floor(S*Beta(5,1)), chunk 2048.
-        Workload("skewed_s256k", 32, 8, 128, [262144], [256], 2048, "bf16", 3, sampler="beta51"),
+        # G = 4: a block has 64 query rows, so two blocks share one 128-row query tile.
+        Workload("skewed_s256k", 32, 8, 128, [262144], [256], 2048, "bf16", 3, sampler="beta51",
+                 blocks_per_item=2),
         # Training step: 4 samples of S=65536 with 32/64/96/128 anchors, chunk 1024, fwd+bwd.
         Workload("train_4x64k", 32, 4, 128, [65536] * 4, [32, 64, 96, 128], 1024, "bf16", 4,
                  backward=True),
