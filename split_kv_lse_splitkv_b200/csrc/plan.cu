@@ -112,11 +112,12 @@ __global__ void __launch_bounds__(kThreads) plan_runs_kernel(const int32_t* __re
 
     if (status_bad(status)) return;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int nwarps = (int)(blockDim.x >> 5);
     const int32_t n = *n_items_d;
-    const int32_t nblk = (n + kThreads - 1) / kThreads;
+    const int32_t nblk = (n + kThreads - 1) / kThreads;  // CTAs of plan_hist_kernel
 
     // Bucket totals, per-CTA offsets within each bucket, bucket starts (cost descending).
-    for (int w = tid; w <= W; w += kThreads) {
+    for (int w = tid; w <= W; w += blockDim.x) {
         int32_t acc = 0;
         for (int32_t b = 0; b < nblk; ++b) {
             int32_t c = ws.hist[(size_t)b * (W + 1) + w];
@@ -133,7 +134,7 @@ __global__ void __launch_bounds__(kThreads) plan_runs_kernel(const int32_t* __re
         start[0] = s;
     }
     __syncthreads();
-    for (int w = tid; w <= W; w += kThreads)
+    for (int w = tid; w <= W; w += blockDim.x)
         for (int32_t b = 0; b < nblk; ++b) ws.hist[(size_t)b * (W + 1) + w] += start[w];
 
     if (tid < m) { L[tid] = 0; qcount[tid] = 0; }
@@ -148,11 +149,11 @@ __global__ void __launch_bounds__(kThreads) plan_runs_kernel(const int32_t* __re
         const int64_t li = tid < m ? L[tid] : INT64_MAX;
         int64_t v = warp_reduce_min(li);
         if (lane == 0) red64[warp] = v;
-        for (int i = tid; i < 32 * (kMaxCost + 1); i += kThreads) (&cnt_w[0][0])[i] = 0;
-        for (int i = tid; i <= W + 1; i += kThreads) cnt_r[i] = 0;
+        for (int i = tid; i < 32 * (kMaxCost + 1); i += blockDim.x) (&cnt_w[0][0])[i] = 0;
+        for (int i = tid; i <= W + 1; i += blockDim.x) cnt_r[i] = 0;
         __syncthreads();
         if (tid < 32) {
-            int64_t x = red64[tid];
+            int64_t x = tid < nwarps ? red64[tid] : INT64_MAX;  // one entry per warp of the block
             x = warp_reduce_min(x);
             if (tid == 0) red64[0] = x;
         }
@@ -181,7 +182,7 @@ __global__ void __launch_bounds__(kThreads) plan_runs_kernel(const int32_t* __re
         }
         if (tid == 32) {
             int32_t x = 0;
-            for (int y = 0; y < 32; ++y) x = red32[y] > x ? red32[y] : x;
+            for (int y = 0; y < nwarps; ++y) x = red32[y] > x ? red32[y] : x;
             red32[32] = x;
         }
         __syncthreads();
@@ -341,7 +342,11 @@ cudaError_t launch_plan(const int32_t* item_cost, const int32_t* n_items, int32_
     int32_t nblk = (max_items + kThreads - 1) / kThreads;
     if (nblk < 1) nblk = 1;
     plan_hist_kernel<<<nblk, kThreads, 0, st>>>(item_cost, n_items, max_items, max_cost, w, status);
-    plan_runs_kernel<<<1, kThreads, 0, st>>>(n_items, max_items, max_cost, n_workers, w, queue_off, load, status);
+    // One CTA with a thread per worker (at least 4 warps: offsets up to max_cost <= 64 get a thread
+    // each): the run loop is bound by its barriers, which cost less with fewer warps.
+    int32_t runs_threads = ((n_workers + 31) / 32) * 32;
+    if (runs_threads < 128) runs_threads = 128;
+    plan_runs_kernel<<<1, runs_threads, 0, st>>>(n_items, max_items, max_cost, n_workers, w, queue_off, load, status);
     plan_assign_kernel<<<nblk, kThreads, 0, st>>>(item_cost, n_items, max_cost, n_workers, w, queue_off,
                                                   item_worker, queue_items, status);
     return cudaGetLastError();
