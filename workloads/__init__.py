@@ -76,6 +76,9 @@ WORKLOADS = {
         # Training step: 4 samples of S=65536 with 32/64/96/128 anchors, chunk 1024, fwd+bwd.
         Workload("train_4x64k", 32, 4, 128, [65536] * 4, [32, 64, 96, 128], 1024, "bf16", 4,
                  backward=True),
+        # The training shape at a quarter of the context and anchors (4 x 16384 keys, 8/16/24/32
+        # anchors): small enough for counter captures that replay each kernel many times.
+        Workload("train_4x16k", 32, 4, 128, [16384] * 4, [8, 16, 24, 32], 1024, "bf16", 5, backward=True),
     ]
 }
 
