@@ -176,13 +176,18 @@ int splitkv_plan_lpt_noalloc(const int32_t *item_cost_d, const int32_t *n_items_
  *   lse_part[slot][block*G]          float32: LSE_p = log sum exp(s), natural log
  * Entries of items that are not visible are not written.
  * item_id_d, queue_off_d and queue_items_d come from splitkv_cost and splitkv_plan_lpt.
+ * On the tensor-core path each worker runs its queue, then claims self items from a shared counter
+ * as it runs out of work (which SM computes a self partial varies from run to run; its value does
+ * not). workspace_d: splitkv_workspace_size() bytes, 16-byte aligned (the claim counter, reset by
+ * this call); the CUDA-core path, which deals self items round-robin, ignores it (may be NULL).
  * q, k, v, kb, vb and o_part must be 16-byte aligned. flags: SPLITKV_FWD_DEFAULT or
  * SPLITKV_FWD_SIMT.
  */
 int splitkv_attn_fwd(const splitkv_problem *problem, const void *q, const void *k, const void *v,
                      const void *kb, const void *vb, const int32_t *anchors_d, const int32_t *item_id_d,
                      const int32_t *queue_off_d, const int32_t *queue_items_d, int32_t n_workers,
-                     float *o_part, float *lse_part, int32_t *status_d, int32_t flags, void *stream);
+                     float *o_part, float *lse_part, int32_t *status_d, int32_t flags, void *workspace_d,
+                     size_t workspace_bytes, void *stream);
 
 /*
  * Exact log-sum-exp merge (Split-KV paper, Abstract: exactness with query-sized exchange). For each

@@ -63,7 +63,8 @@ _SIGS = {
     "splitkv_cost": (_i32, [_PP, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "splitkv_plan_lpt": (_i32, [_vp, _vp, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "splitkv_plan_lpt_noalloc": (_i32, [_vp, _vp, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _vp]),
-    "splitkv_attn_fwd": (_i32, [_PP, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _vp, _i32, _vp]),
+    "splitkv_attn_fwd": (_i32, [_PP, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _vp, _i32, _vp,
+                                _sz, _vp]),
     "splitkv_lse_merge": (_i32, [_PP, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
     "splitkv_attn_bwd": (_i32, [_PP] + [_vp] * 12 + [_i32] + [_vp] * 6 + [_vp, _sz, _vp]),
 }
@@ -165,10 +166,11 @@ def splitkv_plan_lpt_noalloc(item_cost, n_items, max_items, max_cost, n_workers,
 
 
 def splitkv_attn_fwd(problem, q, k, v, kb, vb, anchors, item_id, queue_off, queue_items, n_workers, o_part,
-                     lse_part, status, flags=FWD_DEFAULT, stream=None):
+                     lse_part, status, flags=FWD_DEFAULT, workspace=None, stream=None):
+    nbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(_lib.splitkv_attn_fwd(problem.ptr, _p(q), _p(k), _p(v), _p(kb), _p(vb), _p(anchors), _p(item_id),
                                  _p(queue_off), _p(queue_items), int(n_workers), _p(o_part), _p(lse_part), _p(status),
-                                 int(flags), _stream(stream)), "splitkv_attn_fwd")
+                                 int(flags), _p(workspace), nbytes, _stream(stream)), "splitkv_attn_fwd")
 
 
 def splitkv_lse_merge(problem, o_part, lse_part, anchors, o, lse, status, stream=None):
@@ -244,7 +246,7 @@ class SplitKV:
 
     def attn_fwd(self, q, k, v, kb, vb, anchors, flags=FWD_DEFAULT, stream=None):
         splitkv_attn_fwd(self.problem, q, k, v, kb, vb, anchors, self.item_id, self.queue_off, self.queue_items,
-                         self.n_workers, self.o_part, self.lse_part, self.status, flags, stream)
+                         self.n_workers, self.o_part, self.lse_part, self.status, flags, self.workspace, stream)
 
     def lse_merge(self, anchors, o=None, lse=None, stream=None):
         Nq, Hq, d = int(self.sizes.n_queries), self.n_q_heads, self.head_dim

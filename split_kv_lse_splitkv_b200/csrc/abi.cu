@@ -117,6 +117,7 @@ SPLITKV_API size_t splitkv_workspace_size(const splitkv_problem* problem, int32_
     size_t a = cost_workspace(m);
     size_t b = plan_workspace((int32_t)m.n_items, m.chunk / m.key_tile, n_workers);
     size_t c = bwd_workspace(m);
+    if (kFwdWorkspaceBytes > c) c = kFwdWorkspaceBytes;
     if (bwd_tc_workspace(m) > c) c = bwd_tc_workspace(m);
     size_t r = a > b ? a : b;
     return r > c ? r : c;
@@ -189,7 +190,8 @@ SPLITKV_API int splitkv_attn_fwd(const splitkv_problem* problem, const void* q, 
                                  const void* kb, const void* vb, const int32_t* anchors_d, const int32_t* item_id_d,
                                  const int32_t* queue_off_d,
                                  const int32_t* queue_items_d, int32_t n_workers, float* o_part, float* lse_part,
-                                 int32_t* status_d, int32_t flags, void* stream) {
+                                 int32_t* status_d, int32_t flags, void* workspace_d, size_t workspace_bytes,
+                                 void* stream) {
     clear_error();
     Meta m;
     int rc = build_meta(problem, &m);
@@ -202,9 +204,12 @@ SPLITKV_API int splitkv_attn_fwd(const splitkv_problem* problem, const void* q, 
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(kb) || !aligned16(vb) || !aligned16(o_part))
         return SPLITKV_EINVAL;
     cudaStream_t st = (cudaStream_t)stream;
-    if (!(flags & SPLITKV_FWD_SIMT) && fwd_tc_supported(m))
+    if (!(flags & SPLITKV_FWD_SIMT) && fwd_tc_supported(m)) {
+        if (!workspace_d || workspace_bytes < kFwdWorkspaceBytes) return SPLITKV_ENOSPACE;
+        if (!aligned16(workspace_d)) return SPLITKV_EINVAL;
         return cuda_status(launch_fwd_tc(m, q, k, v, kb, vb, anchors_d, item_id_d, queue_off_d, queue_items_d,
-                                         n_workers, o_part, lse_part, status_d, st));
+                                         n_workers, o_part, lse_part, status_d, workspace_d, st));
+    }
     return cuda_status(launch_fwd_simt(m, q, k, v, kb, vb, anchors_d, item_id_d, queue_off_d, queue_items_d,
                                        n_workers, o_part, lse_part, status_d, st));
 }

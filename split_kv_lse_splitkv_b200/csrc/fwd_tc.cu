@@ -55,9 +55,9 @@ constexpr int kLoadWarp0 = 12;  // TMA producer of lane 0 (lane 1: warp 15)
 constexpr int kLoadWarp1 = 15;
 constexpr int kMmaWarp0 = 13;  // issuer of lane 0, TMEM owner (lane 1: warp 14)
 constexpr int kMmaWarp1 = 14;
-constexpr int kSoftmaxRegs = 152;  // per SM sub-partition: 152 + 152 + 88 + 120 = 512 = 4 x 128 launched
+constexpr int kSoftmaxRegs = 160;  // per SM sub-partition: 160 + 160 + 88 + 104 = 512 = 4 x 128 launched
 constexpr int kEpilogueRegs = 88;
-constexpr int kControlRegs = 120;
+constexpr int kControlRegs = 104;
 constexpr int kTileBytes = 32768;  // 128 x 128 bf16, as two 128-byte-wide halves
 constexpr int kHalfBytes = 16384;
 constexpr int kKeysPerTile = 128;
@@ -66,6 +66,10 @@ constexpr float kRescaleLog2 = 8.0f;
 constexpr int kWgThreads = 128;
 
 constexpr uint32_t kColS = 0, kColO = 256;  // S_L at 128 L, O_L at 256 + 128 L
+
+constexpr int kRing = 128;           // entries of the item ring
+constexpr int kReaders = 20;         // producers 2, issuers 2, softmax warps 8, epilogue warps 4 x 2 lanes
+constexpr int32_t kRingEnd = -1;
 
 constexpr int kOffQ = 0;                  // Q[lane]
 constexpr int kOffK = 2 * kTileBytes;     // K[lane]
@@ -85,6 +89,15 @@ struct Bars {
     uint64_t stat_full[2][2];        // [lane][k % 2]: (m, l) of item k written
     uint64_t drain[2];               // all MMAs of issuer L complete
     int32_t exp_slot[4];             // per SM sub-partition: 1 while a softmax warp is in its exponential pass
+    // The CTA's item sequence, written by one claiming thread, read by every role (see ring_next).
+    int32_t ring_id[kRing];          // item id (n_items + j*Hkv + g: self item; kRingEnd: no more)
+    int32_t ring_lane[kRing];        // lane the item is dealt to
+    int32_t ring_nvis[kRing];        // keys of the chunk its last block sees
+    int32_t ring_j[kRing];           // first block of its query tile
+    int32_t ring_c[kRing];           // chunk
+    int32_t ring_sgn[kRing];         // sample | blocks in the tile << 8 | kv head << 16
+    int32_t ring_w;                  // entries written
+    int32_t ring_r[kReaders];        // entries read, per reader
     uint32_t tmem_base;
     int32_t abort_flag;
     int32_t status0;
@@ -271,29 +284,143 @@ __device__ __forceinline__ void rescale_o(uint32_t to, float alpha) {
     }
 }
 
-// Items dealt to lane L: every role walks the CTA's items in order and gives each to the lane with
-// fewer key tiles so far (ties to lane 0), keeping those of lane L.
-struct LaneWalk {
-    ItemStream st;
-    int32_t tiles0, tiles1;
-};
+// ---------------------------------------------------------------- item ring
+// The CTA's work is its LPT queue, in queue order, then self items (one key tile each, outside the
+// plan) claimed one at a time through a global counter once its own work runs low, so that SMs that
+// finish their queue early take more of them. (Also putting the smallest quarter of every queue into
+// that pool was measured slower: 310 vs 295 us on the 32k-context drafter shape.) One thread, the
+// claimer, turns this into the CTA's item sequence: it deals each item to the lane with fewer key
+// tiles so far and writes the decoded item into a ring in shared memory that every role reads.
 
-__device__ __forceinline__ void lane_init(const Meta& m, const int32_t* anchors, const int32_t* item_id,
-                                          const int32_t* queue_items, int32_t first, int32_t end, LaneWalk& w) {
-    stream_init(m, anchors, item_id, queue_items, first, end, w.st);
-    w.tiles0 = w.tiles1 = 0;
+// Next ring entry for lane L, or for either lane if L < 0. blocking: wait for the entry; otherwise
+// return 0 at once if none has been written. Returns 1 (entry in t, its lane in *lane_out), or -1 at
+// the end of the sequence or on abort/timeout. `slot` is this reader's progress word; a warp-wide
+// reader (all 32 lanes in step) publishes after __syncwarp.
+__device__ __forceinline__ int ring_next(const Meta& m, Bars* bars, int32_t& idx, int slot, int L, bool blocking,
+                                         bool warp_wide, TileRef& t, int* lane_out, volatile int* abort_flag) {
+    volatile int32_t* rw = &bars->ring_w;
+    uint64_t t0 = 0;
+    for (uint32_t spin = 0;; ++spin) {
+        if (idx < *rw) {
+            const int e = idx % kRing;
+            const int32_t id = ((volatile int32_t*)bars->ring_id)[e];
+            const int lane = ((volatile int32_t*)bars->ring_lane)[e];
+            const int32_t nvis = ((volatile int32_t*)bars->ring_nvis)[e];
+            const int32_t jj = ((volatile int32_t*)bars->ring_j)[e];
+            const int32_t cc = ((volatile int32_t*)bars->ring_c)[e];
+            const int32_t sgn = ((volatile int32_t*)bars->ring_sgn)[e];
+            if (id == kRingEnd) return -1;  // the end entry stays: every later call sees it again
+            ++idx;
+            if (warp_wide) __syncwarp();
+            if (!warp_wide || (threadIdx.x & 31) == 0) ((volatile int32_t*)bars->ring_r)[slot] = idx;
+            if (L >= 0 && lane != L) continue;
+            *lane_out = lane;
+            t.nvis = nvis;
+            t.ntiles = (nvis + kKeysPerTile - 1) / kKeysPerTile;
+            t.id = id;
+            t.self_item = id >= m.n_items ? 1 : 0;
+            t.j = jj;
+            t.c = cc;
+            t.s = sgn & 0xff;
+            t.nbt = (sgn >> 8) & 0xff;
+            t.g = sgn >> 16;
+            return 1;
+        }
+        if (!blocking) return 0;
+        if ((spin & 63u) == 63u) {
+            if (*abort_flag) return -1;
+            if (t0 == 0) t0 = globaltimer();
+            else if (globaltimer() - t0 > kTimeoutNs) {
+                *abort_flag = 1;
+                return -1;
+            }
+        }
+        __nanosleep(32);
+    }
 }
 
-__device__ __forceinline__ bool lane_next(const Meta& m, const int32_t* anchors, const int32_t* item_id,
-                                          const int32_t* queue_items, LaneWalk& w, int L, TileRef& t,
-                                          int32_t* status) {
-    while (next_item(m, anchors, item_id, queue_items, w.st, t, status)) {
-        const int lane = w.tiles0 <= w.tiles1 ? 0 : 1;
-        if (lane == 0) w.tiles0 += t.ntiles;
-        else w.tiles1 += t.ntiles;
-        if (lane == L) return true;
+// The claimer: the CTA's queue, then self items while a producer runs low, then the end entry.
+// One thread.
+__device__ void claim_items(const Meta& m, Bars* bars, const int32_t* __restrict__ anchors,
+                            const int32_t* __restrict__ item_id, const int32_t* __restrict__ queue_off,
+                            const int32_t* __restrict__ queue_items, int32_t* pool,
+                            int32_t* status, volatile int* abort_flag) {
+    const int32_t q0 = queue_off[blockIdx.x], q1 = queue_off[blockIdx.x + 1];
+    volatile int32_t* rr = bars->ring_r;
+    int32_t tiles[2] = {0, 0};
+    int32_t w = 0;
+    bool ok = true;
+    // Wait until slot w is free (every reader is past entry w - kRing) and, if ahead > 0, until one of
+    // the producers has fewer than `ahead` entries left to read (pool items are claimed when needed).
+    auto wait_room = [&](int ahead) -> bool {
+        const uint64_t t0 = globaltimer();
+        for (uint32_t spin = 0;; ++spin) {
+            int32_t lo = rr[0];
+            for (int x = 1; x < kReaders; ++x) lo = min(lo, rr[x]);
+            const bool room = lo > w - kRing;
+            const bool low = ahead <= 0 || max(rr[0], rr[1]) > w - ahead;  // a producer is running low
+            if (room && low) return true;
+            if ((spin & 63u) == 63u && (*abort_flag || globaltimer() - t0 > kTimeoutNs)) {
+                *abort_flag = 1;
+                return false;
+            }
+            __nanosleep(64);
+        }
+    };
+    auto put = [&](int32_t id, int lane, int32_t nvis) {
+        const int e = w % kRing;
+        int32_t j = 0, c = 0, sgn = 0;
+        if (id >= m.n_items) {  // self item n_items + j*Hkv + g
+            const int32_t sid = id - (int32_t)m.n_items;
+            j = sid / m.hkv;
+            sgn = sample_of_block(m, j) | (1 << 8) | ((sid % m.hkv) << 16);
+        } else if (id >= 0) {
+            const Item it = decode_item(m, id);
+            j = it.j;
+            c = it.c;
+            sgn = it.s | (it.nbt << 8) | (it.g << 16);
+        }
+        ((volatile int32_t*)bars->ring_id)[e] = id;
+        ((volatile int32_t*)bars->ring_lane)[e] = lane;
+        ((volatile int32_t*)bars->ring_nvis)[e] = nvis;
+        ((volatile int32_t*)bars->ring_j)[e] = j;
+        ((volatile int32_t*)bars->ring_c)[e] = c;
+        ((volatile int32_t*)bars->ring_sgn)[e] = sgn;
+        __threadfence_block();
+        ++w;
+        ((volatile int32_t*)&bars->ring_w)[0] = w;
+    };
+    // Emits queue entry `pos` (if the item is visible) or a self item; ahead as in wait_room.
+    auto emit = [&](int32_t id, int32_t nvis, int ahead) -> bool {
+        if (nvis <= 0) return true;
+        if (!wait_room(ahead)) return false;
+        const int lane = tiles[0] <= tiles[1] ? 0 : 1;
+        tiles[lane] += (nvis + kKeysPerTile - 1) / kKeysPerTile;
+        put(id, lane, nvis);
+        return true;
+    };
+    auto queue_entry = [&](int32_t pos, int ahead) -> bool {
+        const int32_t id = __ldg(item_id + __ldg(queue_items + pos));
+        if (id < 0 || id >= m.n_items) {
+            raise_status(status, SPLITKV_DEV_BAD_PLAN);
+            return true;
+        }
+        const Item it = decode_item(m, id);
+        return emit(id, visible_in_chunk(m, it.s, it.c, __ldg(anchors + it.j + it.nbt - 1)), ahead);
+    };
+    for (int32_t pos = q0; ok && pos < q1; ++pos) ok = queue_entry(pos, 0);
+    const int64_t n_self = m.n_blocks * m.hkv;
+    while (ok) {
+        // Claim when a producer has fewer than 2 entries left to read.
+        if (!wait_room(2)) {
+            ok = false;
+            break;
+        }
+        const int64_t p = atomicAdd(pool, 1);
+        if (p >= n_self) break;
+        ok = emit((int32_t)(m.n_items + p), m.block, 0);
     }
-    return false;
+    if (ok && wait_room(0)) put(kRingEnd, 0, 0);
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -302,7 +429,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                   const __grid_constant__ CUtensorMap tmKb, const __grid_constant__ CUtensorMap tmVb,
                   const int32_t* __restrict__ anchors, const int32_t* __restrict__ item_id,
                   const int32_t* __restrict__ queue_off, const int32_t* __restrict__ queue_items,
-                  float* __restrict__ o_part, float* __restrict__ lse_part, int32_t* __restrict__ status) {
+                  float* __restrict__ o_part, float* __restrict__ lse_part, int32_t* __restrict__ pool,
+                  int32_t* __restrict__ status) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     float* stat = reinterpret_cast<float*>(smem + kOffStat);
@@ -310,7 +438,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     volatile int* abort_flag = &bars->abort_flag;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int32_t q0 = queue_off[blockIdx.x], q1 = queue_off[blockIdx.x + 1];
 
     if (threadIdx.x == 0) {
         for (int b = 0; b < 2; ++b) {
@@ -330,6 +457,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&bars->drain[b], 1);
         }
         for (int q = 0; q < 4; ++q) bars->exp_slot[q] = 0;
+        bars->ring_w = 0;
+        for (int x = 0; x < kReaders; ++x) bars->ring_r[x] = 0;
         bars->abort_flag = 0;
         bars->status0 = status_bad(status) ? 1 : 0;
         fence_barrier_init();
@@ -346,7 +475,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = bars->tmem_base;
-    const bool skip = bars->status0 != 0 || (q0 >= q1 && (int64_t)blockIdx.x >= m.n_blocks * m.hkv);
+    const bool skip = bars->status0 != 0;  // every CTA may take pool items
     const int G = m.group, R = m.rows_item;
 
     if (warp >= kLoadWarp0) {
@@ -361,13 +490,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint8_t* qdst = smem + kOffQ + L * kTileBytes;
             uint8_t* kdst = smem + kOffK + L * kTileBytes;
             uint8_t* vdst = smem + kOffV + L * kTileBytes;
-            LaneWalk w;
-            lane_init(m, anchors, item_id, queue_items, q0, q1, w);
+            int32_t ridx = 0;
+            int rlane;
             TileRef t;
             uint32_t k = 0, n = 0;
             uint32_t inflight = 0;  // 1: Q(k-1), 2: K(n-1), 4: V(n-1) may still be landing
             bool ok = true;
-            while (ok && lane_next(m, anchors, item_id, queue_items, w, L, t, status)) {
+            while (ok && ring_next(m, bars, ridx, L, L, true, false, t, &rlane, abort_flag) == 1) {
                 if (k >= 1 && !mbar_wait(&bars->q_empty[L], (k - 1) & 1u, abort_flag, kTimeoutNs)) {
                     ok = false;
                     break;
@@ -409,6 +538,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (k > 0) mbar_wait(&bars->q_full[L], (k - 1) & 1u, &never, kTimeoutNs);
             if (n > 0 && (inflight & 2)) mbar_wait(&bars->k_full[L], (n - 1) & 1u, &never, kTimeoutNs);
             if (n > 0 && (inflight & 4)) mbar_wait(&bars->v_full[L], (n - 1) & 1u, &never, kTimeoutNs);
+        } else if (!skip && warp == kLoadWarp0 && lane == 1) {
+            claim_items(m, bars, anchors, item_id, queue_off, queue_items, pool, status, abort_flag);
         } else if (!skip && (warp == kMmaWarp0 || warp == kMmaWarp1) && lane == 0) {
             // Issuer L: QK(n) -> wait P(n) -> PV(n) -> QK(n+1) -> ...
             const int L = warp == kMmaWarp0 ? 0 : 1;
@@ -419,12 +550,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint64_t dk = umma_desc_sw128(smem_u32(smem + kOffK + L * kTileBytes), 16, 1024);
             const uint64_t dv = umma_desc_sw128(smem_u32(smem + kOffV + L * kTileBytes), kHalfBytes, 1024);
             const uint32_t ts = tmem + kColS + 128u * L, to = tmem + kColO + 128u * L;
-            LaneWalk w;
-            lane_init(m, anchors, item_id, queue_items, q0, q1, w);
+            int32_t ridx = 0;
+            int rlane;
             TileRef t;
             uint32_t k = 0, n = 0;
             bool ok = true;
-            while (ok && lane_next(m, anchors, item_id, queue_items, w, L, t, status)) {
+            while (ok && ring_next(m, bars, ridx, 2 + L, L, true, false, t, &rlane, abort_flag) == 1) {
                 if (!mbar_wait(&bars->q_full[L], k & 1u, abort_flag, kTimeoutNs)) {
                     ok = false;
                     break;
@@ -474,21 +605,31 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int quad = warp & 3;
             const int r = quad * 32 + lane;
             const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
-            LaneWalk w0, w1;
-            lane_init(m, anchors, item_id, queue_items, q0, q1, w0);
-            lane_init(m, anchors, item_id, queue_items, q0, q1, w1);
+            // Per lane: 1 = holding its next item, 0 = none read yet, -1 = its sequence ended.
+            int32_t idx0 = 0, idx1 = 0;
+            int rlane;
             TileRef t0, t1;
-            bool has0 = lane_next(m, anchors, item_id, queue_items, w0, 0, t0, status);
-            bool has1 = lane_next(m, anchors, item_id, queue_items, w1, 1, t1, status);
+            int has0 = 0, has1 = 0;
             uint32_t k0 = 0, k1 = 0;
             uint64_t deadline = globaltimer() + kTimeoutNs;
             bool ok = true;
-            while (has0 || has1) {
+            const int slot0 = 12 + 2 * quad;
+            while (has0 >= 0 || has1 >= 0) {
+                if (has0 == 0)
+                    has0 = __shfl_sync(0xffffffffu,
+                                       ring_next(m, bars, idx0, slot0, 0, false, true, t0, &rlane, abort_flag), 0);
+                if (has1 == 0)
+                    has1 = __shfl_sync(0xffffffffu,
+                                       ring_next(m, bars, idx1, slot0 + 1, 1, false, true, t1, &rlane, abort_flag), 0);
+                if (*abort_flag) {
+                    ok = false;
+                    break;
+                }
                 int pick = -1;
-                if (has0 && mbar_try_wait(&bars->stat_full[0][k0 & 1], (k0 >> 1) & 1u) &&
+                if (has0 == 1 && mbar_try_wait(&bars->stat_full[0][k0 & 1], (k0 >> 1) & 1u) &&
                     mbar_try_wait(&bars->o_ready[0], k0 & 1u))
                     pick = 0;
-                else if (has1 && mbar_try_wait(&bars->stat_full[1][k1 & 1], (k1 >> 1) & 1u) &&
+                else if (has1 == 1 && mbar_try_wait(&bars->stat_full[1][k1 & 1], (k1 >> 1) & 1u) &&
                          mbar_try_wait(&bars->o_ready[1], k1 & 1u))
                     pick = 1;
                 pick = __shfl_sync(0xffffffffu, pick, 0);
@@ -533,10 +674,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (r < R) lse_part[t.id * R + r] = l > 0.f ? (m_l + lg2_approx(l)) * 0.6931471805599453f : -INFINITY;
                 if (pick) {
                     ++k1;
-                    has1 = lane_next(m, anchors, item_id, queue_items, w1, 1, t1, status);
+                    has1 = 0;
                 } else {
                     ++k0;
-                    has0 = lane_next(m, anchors, item_id, queue_items, w0, 0, t0, status);
+                    has0 = 0;
                 }
                 deadline = globaltimer() + kTimeoutNs;
             }
@@ -556,10 +697,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint64_t c2 = f2_pack(c, c);
             uint32_t k = 0, n = 0;
             bool ok = true;
-            LaneWalk w;
-            lane_init(m, anchors, item_id, queue_items, q0, q1, w);
+            int32_t ridx = 0;
+            int rlane;
             TileRef t;
-            while (ok && lane_next(m, anchors, item_id, queue_items, w, L, t, status)) {
+            while (ok && ring_next(m, bars, ridx, 4 + warp, L, true, true, t, &rlane, abort_flag) == 1) {
                 float m_l = -INFINITY, l = 0.f;  // reference max and row sum (relative to m_l)
                 // Keys of the chunk this row sees: its own block's prefix (a row of no block of the tile,
                 // or of a self item beyond the block's own rows, sees none). A row's keys lie in the
@@ -706,7 +847,7 @@ bool fwd_tc_supported(const Meta& m) {
 cudaError_t launch_fwd_tc(const Meta& m, const void* q, const void* k, const void* v, const void* kb, const void* vb,
                           const int32_t* anchors, const int32_t* item_id, const int32_t* queue_off,
                           const int32_t* queue_items, int32_t n_workers, float* o_part, float* lse_part,
-                          int32_t* status, cudaStream_t st) {
+                          int32_t* status, void* ws, cudaStream_t st) {
     CUtensorMap tq, tk, tv, tkb, tvb;
     if (m.n_queries == 0 || m.total_keys == 0) return cudaSuccess;
     if (!make_bf16_map(&tq, q, m.n_queries, m.hq, m.d, m.group, m.block * m.pack) ||
@@ -717,8 +858,11 @@ cudaError_t launch_fwd_tc(const Meta& m, const void* q, const void* k, const voi
         return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return note_error(e, "cudaFuncSetAttribute(fwd_tc_kernel, smem)");
+    int32_t* pool = reinterpret_cast<int32_t*>(ws);  // the shared pool's claim counter
+    e = cudaMemsetAsync(pool, 0, sizeof(int32_t), st);
+    if (e != cudaSuccess) return note_error(e, "cudaMemsetAsync(pool counter)");
     fwd_tc_kernel<<<n_workers, kThreads, kSmemBytes, st>>>(m, tq, tk, tv, tkb, tvb, anchors, item_id, queue_off,
-                                                           queue_items, o_part, lse_part, status);
+                                                           queue_items, o_part, lse_part, pool, status);
     e = cudaGetLastError();
     if (e != cudaSuccess) {
         cudaFuncAttributes fa;

@@ -121,6 +121,9 @@ def test_null_pointers_and_small_workspace_rejected_before_launch():
     with pytest.raises(B.SplitKVError) as e:  # misaligned vb
         B.splitkv_attn_fwd(p, fake, fake, fake, fake, fake[1:], fake, fake, fake, fake, 4, fake, fake, fake, stream=0)
     assert e.value.code == B.EINVAL
+    with pytest.raises(B.SplitKVError) as e:  # the tensor-core forward needs its workspace (pool counter)
+        B.splitkv_attn_fwd(prob(head_dim=128, dtype=torch.bfloat16), *([fake] * 9), 4, fake, fake, fake, stream=0)
+    assert e.value.code == B.ENOSPACE
     with pytest.raises(B.SplitKVError) as e:
         B.splitkv_lse_merge(p, fake, fake, fake, None, fake, fake, stream=0)
     assert e.value.code == B.EINVAL
