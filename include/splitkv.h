@@ -167,13 +167,15 @@ int splitkv_plan_lpt_noalloc(const int32_t *item_cost_d, const int32_t *n_items_
 /*
  * Partial forward (Split-KV paper, Abstract: the method is exact and exchanges only tensors the
  * size of the query set). One persistent CTA per worker walks its queue; for each item
- * (s, c, g, b) it computes, over the keys of chunk c that block b sees, the chunk-local softmax of
- * s = scale * q.k for the block*G query rows (r = i*G + hl: query i of the block, query head
- * g*G + hl). After the queues the same CTAs compute the self partials: for global block j and kv
- * head g, the softmax over the block's own `block` keys, kb/vb rows block*j .. block*j + block - 1
- * ([Nq, Hkv, d], problem dtype), stored at slot n_items_max + j*Hkv + g. Both kinds write
- *   o_part  [slot][d/4][block*G][4]  float32: O_p = sum softmax * v, normalised
- *   lse_part[slot][block*G]          float32: LSE_p = log sum exp(s), natural log
+ * (s, c, g, t) it computes, over the keys of chunk c that each row's block sees, the chunk-local
+ * softmax of s = scale * q.k for the tile's rows (row x*block*G + i*G + hl: query i of its x-th
+ * block, query head g*G + hl). Then the self partials: for global block j and kv head g, the
+ * softmax over the block's own `block` keys, kb/vb rows block*j .. block*j + block - 1
+ * ([Nq, Hkv, d], problem dtype), stored at slot n_items_max + j*Hkv + g (rows 0 .. block*G - 1).
+ * Both kinds write, with rows = sizes.rows_per_item and E = 16 / sizeof(problem dtype) elements
+ * per 16-byte group (4 for float32, 8 for bf16):
+ *   o_part  [slot][d/E][rows][E]  problem dtype: O_p = sum softmax * v, normalised
+ *   lse_part[slot][rows]          float32: LSE_p = log sum exp(s), natural log (-inf: no key)
  * Entries of items that are not visible are not written.
  * item_id_d, queue_off_d and queue_items_d come from splitkv_cost and splitkv_plan_lpt.
  * On the tensor-core path each worker runs its queue, then claims self items from a shared counter
@@ -186,7 +188,7 @@ int splitkv_plan_lpt_noalloc(const int32_t *item_cost_d, const int32_t *n_items_
 int splitkv_attn_fwd(const splitkv_problem *problem, const void *q, const void *k, const void *v,
                      const void *kb, const void *vb, const int32_t *anchors_d, const int32_t *item_id_d,
                      const int32_t *queue_off_d, const int32_t *queue_items_d, int32_t n_workers,
-                     float *o_part, float *lse_part, int32_t *status_d, int32_t flags, void *workspace_d,
+                     void *o_part, float *lse_part, int32_t *status_d, int32_t flags, void *workspace_d,
                      size_t workspace_bytes, void *stream);
 
 /*
@@ -197,7 +199,7 @@ int splitkv_attn_fwd(const splitkv_problem *problem, const void *q, const void *
  * and writes o [Nq, Hq, d] (problem dtype) and lse [Nq, Hq] (float32, natural log). o_part,
  * lse_part and o must be 16-byte aligned. Reads only what splitkv_attn_fwd wrote.
  */
-int splitkv_lse_merge(const splitkv_problem *problem, const float *o_part, const float *lse_part,
+int splitkv_lse_merge(const splitkv_problem *problem, const void *o_part, const float *lse_part,
                       const int32_t *anchors_d, void *o, float *lse, int32_t *status_d, void *stream);
 
 /*

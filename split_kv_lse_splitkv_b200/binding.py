@@ -227,7 +227,7 @@ class SplitKV:
         if ws == 0:
             raise SplitKVError(EINVAL, "splitkv_workspace_size")
         self.workspace = torch.empty(ws, dtype=torch.uint8, device=dev)
-        self.o_part = torch.empty(max(4, int(s.o_part_elems)), dtype=torch.float32, device=dev)
+        self.o_part = torch.empty(max(8, int(s.o_part_elems)), dtype=dtype, device=dev)  # problem dtype
         self.lse_part = torch.empty(max(1, int(s.lse_part_elems)), dtype=torch.float32, device=dev)
 
     # -- steps
@@ -285,8 +285,10 @@ class SplitKV:
             raise RuntimeError(f"device status word 0x{st:x}")
 
     def o_part_view(self):
-        """Partials as [slots, d/4, rows, 4] and their LSEs as [slots, rows]: chunk items first
-        (n_items_max slots), then the self partials, slot n_items_max + j*Hkv + g."""
+        """Partials as [slots, d/E, rows, E] (problem dtype, E = 16 bytes / element size) and their LSEs
+        as [slots, rows]: chunk items first (n_items_max slots), then the self partials, slot
+        n_items_max + j*Hkv + g."""
         R, d = int(self.sizes.rows_per_item), self.head_dim
+        E = 16 // self.o_part.element_size()
         n = int(self.sizes.lse_part_elems) // R
-        return self.o_part[: n * R * d].view(n, d // 4, R, 4), self.lse_part[: n * R].view(n, R)
+        return self.o_part[: n * R * d].view(n, d // E, R, E), self.lse_part[: n * R].view(n, R)

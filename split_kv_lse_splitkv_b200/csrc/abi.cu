@@ -189,7 +189,7 @@ SPLITKV_API int splitkv_plan_lpt_noalloc(const int32_t* item_cost_d, const int32
 SPLITKV_API int splitkv_attn_fwd(const splitkv_problem* problem, const void* q, const void* k, const void* v,
                                  const void* kb, const void* vb, const int32_t* anchors_d, const int32_t* item_id_d,
                                  const int32_t* queue_off_d,
-                                 const int32_t* queue_items_d, int32_t n_workers, float* o_part, float* lse_part,
+                                 const int32_t* queue_items_d, int32_t n_workers, void* o_part, float* lse_part,
                                  int32_t* status_d, int32_t flags, void* workspace_d, size_t workspace_bytes,
                                  void* stream) {
     clear_error();
@@ -214,7 +214,7 @@ SPLITKV_API int splitkv_attn_fwd(const splitkv_problem* problem, const void* q, 
                                        n_workers, o_part, lse_part, status_d, st));
 }
 
-SPLITKV_API int splitkv_lse_merge(const splitkv_problem* problem, const float* o_part, const float* lse_part,
+SPLITKV_API int splitkv_lse_merge(const splitkv_problem* problem, const void* o_part, const float* lse_part,
                                   const int32_t* anchors_d, void* o, float* lse, int32_t* status_d, void* stream) {
     clear_error();
     Meta m;

@@ -109,17 +109,17 @@ cudaError_t static_plan_scratch(void** out);
 
 cudaError_t launch_fwd_simt(const Meta& m, const void* q, const void* k, const void* v, const void* kb,
                             const void* vb, const int32_t* anchors, const int32_t* item_id, const int32_t* queue_off,
-                            const int32_t* queue_items, int32_t n_workers, float* o_part, float* lse_part,
+                            const int32_t* queue_items, int32_t n_workers, void* o_part, float* lse_part,
                             int32_t* status, cudaStream_t st);
 
 cudaError_t launch_fwd_tc(const Meta& m, const void* q, const void* k, const void* v, const void* kb, const void* vb,
                           const int32_t* anchors, const int32_t* item_id, const int32_t* queue_off,
-                          const int32_t* queue_items, int32_t n_workers, float* o_part, float* lse_part,
+                          const int32_t* queue_items, int32_t n_workers, void* o_part, float* lse_part,
                           int32_t* status, void* ws, cudaStream_t st);
 bool fwd_tc_supported(const Meta& m);
 constexpr size_t kFwdWorkspaceBytes = 256;  // the tensor-core forward's pool counter
 
-cudaError_t launch_merge(const Meta& m, const float* o_part, const float* lse_part, const int32_t* anchors, void* o,
+cudaError_t launch_merge(const Meta& m, const void* o_part, const float* lse_part, const int32_t* anchors, void* o,
                          float* lse, int32_t* status, cudaStream_t st);
 
 bool bwd_tc_supported(const Meta& m);

@@ -24,7 +24,7 @@ __global__ void __launch_bounds__(kThreads) fwd_simt_kernel(Meta m, const T* __r
                                                             const int32_t* __restrict__ item_id,
                                                             const int32_t* __restrict__ queue_off,
                                                             const int32_t* __restrict__ queue_items,
-                                                            float* __restrict__ o_part, float* __restrict__ lse_part,
+                                                            T* __restrict__ o_part, float* __restrict__ lse_part,
                                                             int32_t* __restrict__ status) {
     extern __shared__ float smem[];
     if (status_bad(status)) return;
@@ -139,12 +139,15 @@ __global__ void __launch_bounds__(kThreads) fwd_simt_kernel(Meta m, const T* __r
             }
             __syncthreads();
         }
-        // Normalise and store in the [d/4][R][4] tile layout, plus the natural-log LSE.
-        float* op = o_part + id * (int64_t)R * d;
+        // Normalise and store in the [d/E][R][E] tile layout (E = 16 / sizeof(T) elements per 16-byte
+        // group), plus the natural-log LSE.
+        constexpr int E = 16 / (int)sizeof(T);
+        T* op = o_part + id * (int64_t)R * d;
         for (int e = tid; e < R * d; e += kThreads) {
-            int d4 = e / (R * 4), rem = e % (R * 4);
-            int r = rem / 4, c4 = rem % 4;
-            op[e] = lS[r] > 0.f ? Os[r * d + d4 * 4 + c4] / lS[r] : 0.f;  // a row that sees no key: O = 0
+            int grp = e / (R * E), rem = e % (R * E);
+            int r = rem / E, ce = rem % E;
+            // a row that sees no key: O = 0
+            op[e] = from_f32<T>(lS[r] > 0.f ? Os[r * d + grp * E + ce] / lS[r] : 0.f);
         }
         for (int r = tid; r < R; r += kThreads) lse_part[id * R + r] = lS[r] > 0.f ? mS[r] + logf(lS[r]) : -INFINITY;
         __syncthreads();
@@ -154,7 +157,7 @@ __global__ void __launch_bounds__(kThreads) fwd_simt_kernel(Meta m, const T* __r
 template <typename T>
 cudaError_t launch_t(const Meta& m, const void* q, const void* k, const void* v, const void* kb, const void* vb,
                      const int32_t* anchors, const int32_t* item_id, const int32_t* queue_off,
-                     const int32_t* queue_items, int32_t n_workers, float* o_part, float* lse_part, int32_t* status,
+                     const int32_t* queue_items, int32_t n_workers, void* o_part, float* lse_part, int32_t* status,
                      cudaStream_t st) {
     const int R = m.rows_item, d = m.d;
     size_t smem = sizeof(float) * ((size_t)2 * R * d + kBK * (d + 1) + kBK * d + R * kBK + 4 * R);
@@ -162,7 +165,7 @@ cudaError_t launch_t(const Meta& m, const void* q, const void* k, const void* v,
     if (e != cudaSuccess) return e;
     fwd_simt_kernel<T><<<n_workers, kThreads, smem, st>>>(m, (const T*)q, (const T*)k, (const T*)v, (const T*)kb,
                                                           (const T*)vb, anchors, item_id, queue_off, queue_items,
-                                                          o_part, lse_part, status);
+                                                          (T*)o_part, lse_part, status);
     return cudaGetLastError();
 }
 
@@ -170,7 +173,7 @@ cudaError_t launch_t(const Meta& m, const void* q, const void* k, const void* v,
 
 cudaError_t launch_fwd_simt(const Meta& m, const void* q, const void* k, const void* v, const void* kb,
                             const void* vb, const int32_t* anchors, const int32_t* item_id, const int32_t* queue_off,
-                            const int32_t* queue_items, int32_t n_workers, float* o_part, float* lse_part,
+                            const int32_t* queue_items, int32_t n_workers, void* o_part, float* lse_part,
                             int32_t* status, cudaStream_t st) {
     if (m.dtype == SPLITKV_F32)
         return launch_t<float>(m, q, k, v, kb, vb, anchors, item_id, queue_off, queue_items, n_workers, o_part,

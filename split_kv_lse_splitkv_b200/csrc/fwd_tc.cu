@@ -429,7 +429,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                   const __grid_constant__ CUtensorMap tmKb, const __grid_constant__ CUtensorMap tmVb,
                   const int32_t* __restrict__ anchors, const int32_t* __restrict__ item_id,
                   const int32_t* __restrict__ queue_off, const int32_t* __restrict__ queue_items,
-                  float* __restrict__ o_part, float* __restrict__ lse_part, int32_t* __restrict__ pool,
+                  __nv_bfloat16* __restrict__ o_part, float* __restrict__ lse_part, int32_t* __restrict__ pool,
                   int32_t* __restrict__ status) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -649,7 +649,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const float* sp = stat + (pick * 2 + (int)(k & 1)) * 256;
                 const float m_l = sp[r], l = sp[128 + r];
                 const float inv = l > 0.f ? 1.f / l : 0.f;  // a row that sees no key: O = 0, LSE = -inf
-                float* op = o_part + t.id * (int64_t)R * 128;
+                __nv_bfloat16* op = o_part + t.id * (int64_t)R * 128;  // [d/8][R][8] bf16
                 const uint32_t to = tmem + kColO + 128u * pick + lane_off;
 #pragma unroll 1
                 for (int cc = 0; cc < 8; ++cc) {
@@ -660,14 +660,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                         tc_fence_before();
                         mbar_arrive(&bars->o_free[pick][k & 1]);
                     }
-                    if (r < R) {
+                    if (r < R) {  // 16 columns: two groups of 8 bf16, 16 bytes each
 #pragma unroll
-                        for (int u = 0; u < 4; ++u) {
-                            const float4 x = make_float4(__uint_as_float(ov[4 * u]) * inv,
-                                                         __uint_as_float(ov[4 * u + 1]) * inv,
-                                                         __uint_as_float(ov[4 * u + 2]) * inv,
-                                                         __uint_as_float(ov[4 * u + 3]) * inv);
-                            *reinterpret_cast<float4*>(op + ((int64_t)(cc * 4 + u) * R + r) * 4) = x;
+                        for (int u = 0; u < 2; ++u) {
+                            uint32_t pk[4];
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(ov[8 * u + 2 * e]) * inv,
+                                                                         __uint_as_float(ov[8 * u + 2 * e + 1]) * inv);
+                                pk[e] = *reinterpret_cast<uint32_t*>(&h);
+                            }
+                            *reinterpret_cast<uint4*>(op + ((int64_t)(cc * 2 + u) * R + r) * 8) =
+                                make_uint4(pk[0], pk[1], pk[2], pk[3]);
                         }
                     }
                 }
@@ -846,7 +850,7 @@ bool fwd_tc_supported(const Meta& m) {
 
 cudaError_t launch_fwd_tc(const Meta& m, const void* q, const void* k, const void* v, const void* kb, const void* vb,
                           const int32_t* anchors, const int32_t* item_id, const int32_t* queue_off,
-                          const int32_t* queue_items, int32_t n_workers, float* o_part, float* lse_part,
+                          const int32_t* queue_items, int32_t n_workers, void* o_part, float* lse_part,
                           int32_t* status, void* ws, cudaStream_t st) {
     CUtensorMap tq, tk, tv, tkb, tvb;
     if (m.n_queries == 0 || m.total_keys == 0) return cudaSuccess;
@@ -862,7 +866,7 @@ cudaError_t launch_fwd_tc(const Meta& m, const void* q, const void* k, const voi
     e = cudaMemsetAsync(pool, 0, sizeof(int32_t), st);
     if (e != cudaSuccess) return note_error(e, "cudaMemsetAsync(pool counter)");
     fwd_tc_kernel<<<n_workers, kThreads, kSmemBytes, st>>>(m, tq, tk, tv, tkb, tvb, anchors, item_id, queue_off,
-                                                           queue_items, o_part, lse_part, pool, status);
+                                                           queue_items, (__nv_bfloat16*)o_part, lse_part, pool, status);
     e = cudaGetLastError();
     if (e != cudaSuccess) {
         cudaFuncAttributes fa;

@@ -35,7 +35,10 @@ def run_forward(inp, n_workers=None, flags=0, device="cuda"):
     return skv, dev, anchors, o, lse
 
 
-def assert_close(name, got, ref, dtype):
+def assert_close(name, got, ref, dtype, magnitude_scaled=False):
+    """Max error within the bound of `dtype`. magnitude_scaled: inputs deliberately far from the
+    workloads' N(0,1) scale (e.g. keys with 12x the norm); the bf16 absolute bound is then taken
+    relative to max(1, max|ref|), since bf16 roundings of O scale with |O|."""
     got = np.asarray(got, np.float64)
     ref = np.asarray(ref, np.float64)
     assert got.shape == ref.shape, (name, got.shape, ref.shape)
@@ -45,7 +48,8 @@ def assert_close(name, got, ref, dtype):
     if dtype == "f32":
         assert err <= F32_REL * scale + 1e-30, f"{name}: max err {err:.3e} > {F32_REL} x {scale:.3e}"
     else:
-        assert err <= BF16_ABS, f"{name}: max abs err {err:.3e} > {BF16_ABS}"
+        bound = BF16_ABS * (max(1.0, scale) if magnitude_scaled else 1.0)
+        assert err <= bound, f"{name}: max abs err {err:.3e} > {bound:.3e}"
         assert err <= BF16_REL * scale + 1e-30, f"{name}: max err {err:.3e} > {BF16_REL} x max|ref| {scale:.3e}"
     return err, scale
 
@@ -68,14 +72,14 @@ def check_cost_and_plan(skv, inp):
     return ids, costs
 
 
-def check_partials(skv, inp, ids):
+def check_partials(skv, inp, ids, magnitude_scaled=False):
     """Every visible item's partial (O_c, LSE_c), and every block's self partial over its own keys,
     against the oracle's chunk-local softmax."""
     w = inp.workload
     p = oracle_problem(inp)
     parts = OA.chunk_partials(p, w.chunk)
     O_part, L_part = skv.o_part_view()
-    O_part = O_part.cpu().numpy()
+    O_part = O_part.float().cpu().numpy()
     L_part = L_part.cpu().numpy()
     G, R, P = w.group, w.block * w.group, w.blocks_per_item
     RT = int(skv.sizes.rows_per_item)  # rows of a partial tile: P blocks of R rows
@@ -104,8 +108,8 @@ def check_partials(skv, inp, ids):
                 ref_O.append(ref_o)
                 got_L.append(L_part[item][rows])
                 ref_L.append(ref_l)
-    assert_close("O_part", np.stack(got_O), np.stack(ref_O), w.dtype)
-    assert_close("LSE_part", np.stack(got_L), np.stack(ref_L), w.dtype)
+    assert_close("O_part", np.stack(got_O), np.stack(ref_O), w.dtype, magnitude_scaled)
+    assert_close("LSE_part", np.stack(got_L), np.stack(ref_L), w.dtype, magnitude_scaled)
     n_max = int(skv.sizes.n_items_max)
     got_O, ref_O, got_L, ref_L = [], [], [], []
     for s in range(len(w.seq_lens)):
@@ -121,5 +125,5 @@ def check_partials(skv, inp, ids):
                     got_L.append(L_part[slot][rows])
                     ref_L.append(ref_l)
     if got_O:
-        assert_close("O_self", np.stack(got_O), np.stack(ref_O), w.dtype)
-        assert_close("LSE_self", np.stack(got_L), np.stack(ref_L), w.dtype)
+        assert_close("O_self", np.stack(got_O), np.stack(ref_O), w.dtype, magnitude_scaled)
+        assert_close("LSE_self", np.stack(got_L), np.stack(ref_L), w.dtype, magnitude_scaled)
