@@ -286,8 +286,25 @@ def run_ours(args):
         e1.record(stream)
         phases[name].append((e0, e1))
 
+    naive_load = None
+    if args.plan == "naive":
+        # Cost-blind equal-count split of the item list (index order) into contiguous queues, for the
+        # comparison with LPT; built once (the anchors do not change), so each step runs the cost
+        # pass and then the same kernels with these queues.
+        skv.cost(dev["anchors"], stream)
+        torch.cuda.synchronize(device)
+        n, mq = int(skv.n_items.item()), skv.n_workers
+        bounds = torch.tensor([(x * n) // mq for x in range(mq + 1)], dtype=torch.int64)
+        skv.queue_off = bounds.to(torch.int32).to(device)
+        skv.queue_items = torch.arange(max(1, n), dtype=torch.int32, device=device)
+        csum = torch.cat([torch.zeros(1, dtype=torch.int64), skv.item_cost[:n].cpu().to(torch.int64).cumsum(0)])
+        naive_load = (csum[bounds[1:]] - csum[bounds[:-1]]).double()
+
     def step(d, time_phases=False):
-        timed("plan", lambda: skv.plan(d["anchors"], stream), time_phases)
+        if args.plan == "naive":
+            timed("plan", lambda: skv.cost(d["anchors"], stream), time_phases)
+        else:
+            timed("plan", lambda: skv.plan(d["anchors"], stream), time_phases)
         timed("fwd", lambda: skv.attn_fwd(d["q"], d["k"], d["v"], d["kb"], d["vb"], d["anchors"], stream=stream),
               time_phases)
         timed("merge", lambda: skv.lse_merge(d["anchors"], o, lse, stream=stream), time_phases)
@@ -372,7 +389,7 @@ def run_ours(args):
                 "peak_source": "derived fp32 FFMA peak at max SM clock"}
     achieved = fwd_kernel_flops / (fwd_ms * 1e-3) / 1e12
     peak = roof["peak"]
-    load = skv.load.cpu().double()
+    load = naive_load if naive_load is not None else skv.load.cpu().double()
     predicted_imb = float(load.max() / load.mean() - 1.0) if load.sum() > 0 else 0.0
     csum = clocks.summary()
 
@@ -389,12 +406,12 @@ def run_ours(args):
             "config": {"workload": w.name, "seq_lens": list(w.seq_lens), "anchors": counts,
                        "heads": f"{w.n_q_heads}q/{w.n_kv_heads}kv", "head_dim": w.head_dim, "chunk": w.chunk,
                        "queues": skv.n_workers, "l2": "flushed (256 MB write) before every timed step",
-                       "parallelism": f"replicas x{world}"},
+                       "parallelism": f"replicas x{world}", "plan": args.plan},
             "roofline": dict(roof, achieved=achieved, unit="TFLOP/s", frac=achieved / peak,
                              traffic=profiled_traffic("fwd_tc_kernel", w.name) if w.dtype == "bf16" else None,
                              kernel_ms=fwd_ms, algorithmic_flop=fwd_kernel_flops),
             "phase_ms": phase_ms,
-            "imbalance": {"predicted_lpt": predicted_imb},
+            "imbalance": {f"predicted_{args.plan}": predicted_imb},
             **({"backward_roofline": {"kernels": "rows_kernel + bwd_kv_kernel + bwd_q_kernel",
                                       "algorithmic_flop": flops - fwd_kernel_flops,
                                       "achieved": (flops - fwd_kernel_flops) / (phase_ms["bwd"] * 1e-3) / 1e12,
@@ -424,6 +441,8 @@ def main():
     ap.add_argument("--ref-budget", type=float, default=0.0,
                     help="seconds of CPU work per oracle sample (default: ~150 s spread over all reference steps)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--plan", default="lpt", choices=["lpt", "naive"],
+                    help="naive: the cost-blind equal-count split instead of the LPT plan (for comparison)")
     args = ap.parse_args()
     try:
         if args.impl == "reference":
