@@ -443,7 +443,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
     QBars* bars = reinterpret_cast<QBars*>(smem + kQOffBar);
     volatile int* abort_flag = &bars->abort_flag;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int G = m.group, R = m.rows_item, RB = m.rows;  // rows of a query tile / of one block
+    const int G = m.group, RB = m.rows;  // rows of one block
     const int32_t q0 = queue_off[blockIdx.x], q1 = queue_off[blockIdx.x + 1];
 
     if (threadIdx.x == 0) {
