@@ -273,7 +273,10 @@ def run_ours(args):
         grads = (torch.empty(inp.q.shape, **f), torch.empty(inp.k.shape, **f), torch.empty(inp.v.shape, **f),
                  torch.empty(inp.kb.shape, **f), torch.empty(inp.vb.shape, **f))
     flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=device)
-    stream = torch.cuda.current_stream(device)
+    # One non-default stream for every launch and copy (a CUDA graph is captured on a non-default stream).
+    torch.cuda.synchronize(device)
+    stream = torch.cuda.Stream(device)
+    torch.cuda.set_stream(stream)
     phases = {"plan": [], "fwd": [], "merge": [], "bwd": []}
 
     def timed(name, fn, on):
@@ -318,23 +321,48 @@ def run_ours(args):
     torch.cuda.synchronize(device)
     skv.check_status()
 
+    # The step's launches (cost, plan, forward, merge[, backward]) captured once as a CUDA graph and
+    # replayed: the same kernels on the same buffers, without the host launch gaps between them.
+    graph = None
+    if not args.no_graph:
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream, capture_error_mode="thread_local"):
+            step(dev)
+        torch.cuda.synchronize(device)
+        for _ in range(2):
+            graph.replay()
+        torch.cuda.synchronize(device)
+        skv.check_status()
+
+    def timed_steps(n, run, time_phases):
+        evs = []
+        for _ in range(n):
+            flush.fill_(1.0)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            run(time_phases)
+            e1.record(stream)
+            evs.append((e0, e1))
+        return evs
+
     # ---- device-timed region
-    evs = []
     barrier(world)
     torch.cuda.synchronize(device)
     wall0 = time.perf_counter()
     with ClockSampler(local) as clocks:
-        for _ in range(args.steps):
-            flush.fill_(1.0)
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-            step(dev, time_phases=True)
-            e1.record(stream)
-            evs.append((e0, e1))
+        if graph is not None:
+            evs = timed_steps(args.steps, lambda _: graph.replay(), False)
+        else:
+            evs = timed_steps(args.steps, lambda tp: step(dev, time_phases=tp), True)
         torch.cuda.synchronize(device)
     barrier(world)
     wall = time.perf_counter() - wall0
     ms = sum(a.elapsed_time(b) for a, b in evs) / len(evs)
+    if graph is not None:
+        # Per-phase times (for the roofline of the forward kernel) from as many eager steps, timed
+        # the same way, after the graph-timed region.
+        timed_steps(args.steps, lambda tp: step(dev, time_phases=tp), True)
+        torch.cuda.synchronize(device)
     phase_ms = {k: (sum(a.elapsed_time(b) for a, b in v) / len(v)) for k, v in phases.items() if v}
     fwd_ms = phase_ms["fwd"]
     ms_max = max_over_ranks(ms, world, device)
@@ -406,7 +434,8 @@ def run_ours(args):
             "config": {"workload": w.name, "seq_lens": list(w.seq_lens), "anchors": counts,
                        "heads": f"{w.n_q_heads}q/{w.n_kv_heads}kv", "head_dim": w.head_dim, "chunk": w.chunk,
                        "queues": skv.n_workers, "l2": "flushed (256 MB write) before every timed step",
-                       "parallelism": f"replicas x{world}", "plan": args.plan},
+                       "parallelism": f"replicas x{world}", "plan": args.plan,
+                       "launch": "eager" if graph is None else "cuda graph of the step"},
             "roofline": dict(roof, achieved=achieved, unit="TFLOP/s", frac=achieved / peak,
                              traffic=profiled_traffic("fwd_tc_kernel", w.name) if w.dtype == "bf16" else None,
                              kernel_ms=fwd_ms, algorithmic_flop=fwd_kernel_flops),
@@ -441,6 +470,8 @@ def main():
     ap.add_argument("--ref-budget", type=float, default=0.0,
                     help="seconds of CPU work per oracle sample (default: ~150 s spread over all reference steps)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-graph", action="store_true",
+                    help="time eagerly launched steps instead of replaying one captured CUDA graph of the step")
     ap.add_argument("--plan", default="lpt", choices=["lpt", "naive"],
                     help="naive: the cost-blind equal-count split instead of the LPT plan (for comparison)")
     args = ap.parse_args()
