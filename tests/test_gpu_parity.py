@@ -221,3 +221,58 @@ def test_full_size_training_step():
             want_v = sum(don[r, h].sum(0) for h in range(g * w.group, (g + 1) * w.group))
             got_v_ = dvn[ko[s]:ko[s + 1], g].sum(0) + dvbn[r, g].sum(0)
             assert np.allclose(got_v_, want_v, rtol=1e-3, atol=1e-2)
+
+
+# ------------------------------------------------------------------ CUDA graph of the step
+@pytest.mark.parametrize("backward", [False, True])
+def test_cuda_graph_replay_matches_eager(backward):
+    """The step (cost, plan, forward, merge[, backward]) captured once as a CUDA graph and replayed
+    on new inputs gives what eager launches give on those inputs (the same bits, dQ to rounding):
+    every launch is stream ordered and takes its sizes from the problem, not from device data read
+    on the host."""
+    from split_kv_lse_splitkv_b200 import SplitKV
+    base = "train_4x16k" if backward else "drafter_s32k"
+    inp = small("graph", base, [4096, 3072], [6, 4], chunk=1024, seed=21)
+    w = inp.workload
+    skv = SplitKV(w.seq_lens, counts_of(inp), w.n_q_heads, w.n_kv_heads, w.head_dim, w.block, w.chunk, w.key_tile,
+                  w.scale, w.torch_dtype, n_workers=148, device="cuda", blocks_per_item=w.blocks_per_item)
+    names = ("q", "k", "v", "kb", "vb") + (("do",) if backward else ())
+    dev = {k: getattr(inp, k).cuda() for k in names}
+    anchors = inp.anchors.cuda()
+    o = torch.empty(inp.q.shape, dtype=w.torch_dtype, device="cuda")
+    lse = torch.empty(inp.q.shape[:2], dtype=torch.float32, device="cuda")
+    f = dict(dtype=torch.float32, device="cuda")
+    grads = (torch.empty(inp.q.shape, **f), torch.empty(inp.k.shape, **f), torch.empty(inp.v.shape, **f),
+             torch.empty(inp.kb.shape, **f), torch.empty(inp.vb.shape, **f))
+    stream = torch.cuda.Stream()
+
+    def step():
+        skv.forward(dev["q"], dev["k"], dev["v"], dev["kb"], dev["vb"], anchors, o=o, lse=lse, stream=stream)
+        if backward:
+            skv.backward(dev["q"], dev["k"], dev["v"], dev["kb"], dev["vb"], o, lse, dev["do"], anchors, grads,
+                         stream=stream)
+
+    with torch.cuda.stream(stream):
+        step()
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream, capture_error_mode="thread_local"):
+        step()
+    torch.cuda.synchronize()
+    # New values in the same buffers: the replay must compute from them, not repeat the capture's.
+    gen = torch.Generator().manual_seed(5)
+    for k in names:
+        dev[k].copy_(torch.randn(dev[k].shape, generator=gen).to(dev[k].dtype))
+    graph.replay()
+    torch.cuda.synchronize()
+    skv.check_status()
+    got = [o.clone(), lse.clone()] + ([g.clone() for g in grads] if backward else [])
+    with torch.cuda.stream(stream):
+        step()
+    torch.cuda.synchronize()
+    ref = [o, lse] + (list(grads) if backward else [])
+    for i, (a, b) in enumerate(zip(got, ref)):
+        if i == 2:  # dQ: summed over items with float atomics, so the order of the additions varies
+            assert torch.allclose(a, b, rtol=1e-5, atol=1e-6 * float(b.abs().max())), "dQ"
+        else:
+            assert torch.equal(a, b), i
