@@ -16,13 +16,16 @@
 //   the MUFU unit has two warps to interleave) form P^T and dS^T in bf16 over the first 32 columns
 //   of their half of each (two rows per column); dV += P^T dO_b and dK += dS^T Q_b with P^T / dS^T
 //   as the TMEM operand and Q_b / dO_b read MN-major from shared memory, each query half as soon as
-//   it is written. The issuer's MMAs execute in issue order, so the next pair's S^T and dP^T
-//   overwrite P^T and dS^T only after dV and dK have read them. (Measured: 1085 -> 1042 us for the
-//   backward of train_4x16k against one thread per key.)
-// Query-stationary kernel (bwd_q_kernel), per item key tile: S = Q K^T and dP = dO V^T into TMEM;
-//   two threads per query row (keys 0-63 / 64-127, two warps per SM sub-partition) form dS in bf16
-//   over the first 32 columns of their half of S; dQ += dS K, each key half as soon as it is
-//   written. (Measured: the backward of train_4x64k 14.10 -> 13.62 ms against one thread per row.)
+//   it is written. Two issuing threads, one per accumulator pair (S^T then dV, dP^T then dK): one
+//   thread gets one tcgen05.mma per ~120 cycles, two interleave; each issuer's MMAs execute in its
+//   issue order, so the next pair's S^T (dP^T) overwrites P^T (dS^T) only after dV (dK) has read it.
+//   (Measured on the backward of train_4x16k: 1085 -> 1042 us for two threads per key, and on
+//   train_4x64k 13.65 -> 12.98 ms for two issuers here and in the dQ kernel.)
+// Query-stationary kernel (bwd_q_kernel), per item key tile: S = Q K^T and dP = dO V^T into TMEM,
+//   from two issuing threads; two threads per query row (keys 0-63 / 64-127, two warps per SM
+//   sub-partition) form dS in bf16 over the first 32 columns of their half of S; dQ += dS K, each key
+//   half as soon as it is written. (Measured: the backward of train_4x64k 14.10 -> 13.62 ms against
+//   one thread per row.)
 //
 // Every wait is bounded (2 s); on expiry the CTA raises SPLITKV_DEV_TIMEOUT, drains its copies and
 // MMAs in flight, frees TMEM and returns.
@@ -71,8 +74,9 @@ __global__ void __launch_bounds__(256) rows_kernel(Meta m, const T* __restrict__
 }
 
 // ------------------------------------------------------------------ key-stationary: dK, dV
-constexpr int kKvThreads = 320;  // warps 0-7: elementwise (key row x query half); warp 8: TMA producer; warp 9: MMA issuer
-constexpr int kKvLoadWarp = 8, kKvMmaWarp = 9;
+constexpr int kKvThreads = 352;  // warps 0-7: elementwise (key row x query half); warp 8: TMA producer;
+                                 // warps 9, 10: MMA issuers (S^T then dV; dP^T then dK)
+constexpr int kKvLoadWarp = 8, kKvMmaWarp = 9, kKvMma2Warp = 10;
 constexpr int kKvOffK = 0;
 constexpr int kKvOffV = kTileBytes;
 constexpr int kKvOffQ = 2 * kTileBytes;     // Q_b[2]
@@ -83,10 +87,10 @@ constexpr int kKvOffBar = kKvOffRows + 2 * 2 * 128 * 4;
 struct KvBars {
     uint64_t kv_full;
     uint64_t qd_full[2], qd_empty[2];  // Q_b, dO_b, rows of pair p in slot p % 2
-    uint64_t s_full;                   // S^T, dP^T of the current pair complete
+    uint64_t s_full;                   // S^T, dP^T of the current pair complete (one commit per issuer)
     uint64_t p_half[2];                // P^T, dS^T of query rows 64h .. 64h+63 written
     uint64_t acc_done;                 // every MMA complete: dV, dK final
-    uint64_t drain;
+    uint64_t drain[2];
     uint32_t tmem_base;
     int32_t abort_flag;
     int32_t status0;
@@ -151,13 +155,14 @@ __global__ void __launch_bounds__(kKvThreads, 1)
         mbar_init(&bars->kv_full, 1);
         for (int b = 0; b < 2; ++b) {
             mbar_init(&bars->qd_full[b], 1);
-            mbar_init(&bars->qd_empty[b], 1);
+            mbar_init(&bars->qd_empty[b], 2);
         }
-        mbar_init(&bars->s_full, 1);
+        mbar_init(&bars->s_full, 2);
         mbar_init(&bars->p_half[0], 128);
         mbar_init(&bars->p_half[1], 128);
-        mbar_init(&bars->acc_done, 1);
-        mbar_init(&bars->drain, 1);
+        mbar_init(&bars->acc_done, 2);
+        mbar_init(&bars->drain[0], 1);
+        mbar_init(&bars->drain[1], 1);
         bars->abort_flag = 0;
         bars->status0 = status_bad(status) ? 1 : 0;
         fence_barrier_init();
@@ -212,33 +217,34 @@ __global__ void __launch_bounds__(kKvThreads, 1)
             for (int32_t p = (issued > 2 ? issued - 2 : 0); p < issued; ++p)
                 mbar_wait(&bars->qd_full[p & 1], (p >> 1) & 1u, &never, kTimeoutNs);
         }
-    } else if (warp == kKvMmaWarp) {
+    } else if (warp == kKvMmaWarp || warp == kKvMma2Warp) {
+        // Two issuers, each with its own pair of accumulators, so that the tensor core interleaves two
+        // instruction streams (one thread issues one tcgen05.mma per ~120 cycles): A: S^T = K Q_b^T, then
+        // dV += P^T dO_b reading P^T from S^T's columns; B: dP^T = V dO_b^T, then dK += dS^T Q_b. Each
+        // issuer's MMAs execute in its issue order, so the next pair's S^T (dP^T) overwrites P^T (dS^T)
+        // only after dV (dK) has read it.
+        const bool isA = warp == kKvMmaWarp;
         if (!skip && lane == 0 && np > 0) {
             bool ok = mbar_wait(&bars->kv_full, 0, abort_flag, kTimeoutNs);
             tc_fence_after();
-            const uint64_t dK = umma_desc_sw128(smem_u32(smem + kKvOffK), 16, 1024);
-            const uint64_t dV = umma_desc_sw128(smem_u32(smem + kKvOffV), 16, 1024);
+            const uint64_t dA1 = umma_desc_sw128(smem_u32(smem + (isA ? kKvOffK : kKvOffV)), 16, 1024);
+            const uint32_t t1 = isA ? tS : tdP, t2 = isA ? tdV : tdK;
             for (int32_t p = 0; ok && p < np; ++p) {
                 const int slot = p & 1;
                 const uint32_t aq = smem_u32(smem + kKvOffQ + slot * kTileBytes);
                 const uint32_t ado = smem_u32(smem + kKvOffDo + slot * kTileBytes);
-                const uint64_t dq = umma_desc_sw128(aq, 16, 1024), ddo = umma_desc_sw128(ado, 16, 1024);
-                const uint64_t dq_mn = umma_desc_sw128(aq, kHalfBytes, 1024);
-                const uint64_t ddo_mn = umma_desc_sw128(ado, kHalfBytes, 1024);
+                // First GEMM: B = Q_b (A) or dO_b (B), K-major; second: B = dO_b (A) or Q_b (B), MN-major.
+                const uint64_t dB1 = umma_desc_sw128(isA ? aq : ado, 16, 1024);
+                const uint64_t dB2 = umma_desc_sw128(isA ? ado : aq, kHalfBytes, 1024);
                 if (!mbar_wait(&bars->qd_full[slot], (p >> 1) & 1u, abort_flag, kTimeoutNs)) { ok = false; break; }
                 tc_fence_after();
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {  // S^T = K Q_b^T
+                for (int kk = 0; kk < 8; ++kk) {  // S^T = K Q_b^T  /  dP^T = V dO_b^T
                     const uint64_t off = (uint64_t)(((kk >> 2) * kHalfBytes + (kk & 3) * 32) / 16);
-                    mma_ss(tS, dK + off, dq + off, kIdescSS, kk > 0 ? 1u : 0u);
-                }
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {  // dP^T = V dO_b^T
-                    const uint64_t off = (uint64_t)(((kk >> 2) * kHalfBytes + (kk & 3) * 32) / 16);
-                    mma_ss(tdP, dV + off, ddo + off, kIdescSS, kk > 0 ? 1u : 0u);
+                    mma_ss(t1, dA1 + off, dB1 + off, kIdescSS, kk > 0 ? 1u : 0u);
                 }
                 mma_commit(&bars->s_full);
-                // dV += P^T dO_b and dK += dS^T Q_b, 16 query rows per step, each query half as soon as its
+                // dV += P^T dO_b  /  dK += dS^T Q_b, 16 query rows per step, each query half as soon as its
                 // P^T, dS^T are written (half h: columns 64h .. 64h+31 of S^T / dP^T).
                 for (int h = 0; ok && h < 2; ++h) {
                     if (!mbar_wait(&bars->p_half[h], p & 1u, abort_flag, kTimeoutNs)) { ok = false; break; }
@@ -246,13 +252,7 @@ __global__ void __launch_bounds__(kKvThreads, 1)
 #pragma unroll
                     for (int kq = 0; kq < 4; ++kq) {
                         const int kk = 4 * h + kq;
-                        mma_ts(tdV, tS + (uint32_t)(64 * h + kq * 8), ddo_mn + (uint64_t)(kk * 2048 / 16), kIdescTS,
-                               (p > 0 || kk > 0) ? 1u : 0u);
-                    }
-#pragma unroll
-                    for (int kq = 0; kq < 4; ++kq) {
-                        const int kk = 4 * h + kq;
-                        mma_ts(tdK, tdP + (uint32_t)(64 * h + kq * 8), dq_mn + (uint64_t)(kk * 2048 / 16), kIdescTS,
+                        mma_ts(t2, t1 + (uint32_t)(64 * h + kq * 8), dB2 + (uint64_t)(kk * 2048 / 16), kIdescTS,
                                (p > 0 || kk > 0) ? 1u : 0u);
                     }
                 }
@@ -261,9 +261,10 @@ __global__ void __launch_bounds__(kKvThreads, 1)
             }
             if (ok) mma_commit(&bars->acc_done);
             else *abort_flag = 1;
-            mma_commit(&bars->drain);
+            uint64_t* dr = &bars->drain[isA ? 0 : 1];
+            mma_commit(dr);
             volatile int never = 0;
-            mbar_wait(&bars->drain, 0, &never, kTimeoutNs);
+            mbar_wait(dr, 0, &never, kTimeoutNs);
         }
     } else if (!skip) {
         // ------------------------------------------------ one thread per (key kr, query half)
@@ -362,8 +363,9 @@ __global__ void __launch_bounds__(kKvThreads, 1)
 }
 
 // ------------------------------------------------------------------ query-stationary: dQ
-constexpr int kQThreads = 320;  // warps 0-7: elementwise (query row x key half); warp 8: TMA producer; warp 9: MMA issuer
-constexpr int kQLoadWarp = 8, kQMmaWarp = 9;
+constexpr int kQThreads = 352;  // warps 0-7: elementwise (query row x key half); warp 8: TMA producer;
+                                // warps 9, 10: MMA issuers (S then dQ; dP)
+constexpr int kQLoadWarp = 8, kQMmaWarp = 9, kQMma2Warp = 10;
 constexpr int kQOffQ = 0;                   // Q of the current item
 constexpr int kQOffDo = kTileBytes;         // dO of the current item
 constexpr int kQOffK = 2 * kTileBytes;      // K[2], by key tile parity
@@ -376,7 +378,7 @@ struct QBars {
     uint64_t s_full;                 // S, dP of the current tile complete
     uint64_t p_half[2];              // dS of keys 64h .. 64h+63 written
     uint64_t dq_ready, dq_free;      // last dQ MMA of item i complete / dQ read by the epilogue
-    uint64_t drain;
+    uint64_t drain[2];
     uint32_t tmem_base;
     int32_t abort_flag;
     int32_t status0;
@@ -451,17 +453,18 @@ __global__ void __launch_bounds__(kQThreads, 1)
 
     if (threadIdx.x == 0) {
         mbar_init(&bars->qd_full, 1);
-        mbar_init(&bars->qd_empty, 1);
+        mbar_init(&bars->qd_empty, 2);
         for (int b = 0; b < 2; ++b) {
             mbar_init(&bars->kv_full[b], 1);
-            mbar_init(&bars->kv_empty[b], 1);
+            mbar_init(&bars->kv_empty[b], 2);
         }
-        mbar_init(&bars->s_full, 1);
+        mbar_init(&bars->s_full, 2);
         mbar_init(&bars->p_half[0], 128);
         mbar_init(&bars->p_half[1], 128);
         mbar_init(&bars->dq_ready, 1);
         mbar_init(&bars->dq_free, 256);
-        mbar_init(&bars->drain, 1);
+        mbar_init(&bars->drain[0], 1);
+        mbar_init(&bars->drain[1], 1);
         bars->abort_flag = 0;
         bars->status0 = status_bad(status) ? 1 : 0;
         fence_barrier_init();
@@ -527,10 +530,13 @@ __global__ void __launch_bounds__(kQThreads, 1)
                 for (uint32_t x = (n > 2 ? n - 2 : 0); x < n; ++x)
                     mbar_wait(&bars->kv_full[x & 1], (x >> 1) & 1u, &never, kTimeoutNs);
         }
-    } else if (warp == kQMmaWarp) {
+    } else if (warp == kQMmaWarp || warp == kQMma2Warp) {
+        // Two issuers, so that the tensor core interleaves two instruction streams: A: S = Q K^T, then
+        // dQ += dS K reading dS from S's columns (its own order keeps the next S after that read);
+        // B: dP = dO V^T, the next one only once the elementwise pass has read this one.
+        const bool isA = warp == kQMmaWarp;
         if (!skip && lane == 0) {
-            const uint64_t dQd = umma_desc_sw128(smem_u32(smem + kQOffQ), 16, 1024);
-            const uint64_t dDo = umma_desc_sw128(smem_u32(smem + kQOffDo), 16, 1024);
+            const uint64_t dA1 = umma_desc_sw128(smem_u32(smem + (isA ? kQOffQ : kQOffDo)), 16, 1024);
             int32_t pos = q0;
             int64_t self_pos = blockIdx.x;
             QItem t;
@@ -541,50 +547,55 @@ __global__ void __launch_bounds__(kQThreads, 1)
                 for (int32_t tt = 0; tt < t.ntiles; ++tt, ++n) {
                     const int b = n & 1;
                     const uint32_t ak = smem_u32(smem + kQOffK + b * kTileBytes);
-                    const uint64_t dKd = umma_desc_sw128(ak, 16, 1024);
-                    const uint64_t dKmn = umma_desc_sw128(ak, kHalfBytes, 1024);
-                    const uint64_t dVd = umma_desc_sw128(smem_u32(smem + kQOffV + b * kTileBytes), 16, 1024);
+                    const uint64_t dB1 = umma_desc_sw128(isA ? ak : smem_u32(smem + kQOffV + b * kTileBytes), 16, 1024);
                     if (!mbar_wait(&bars->kv_full[b], (n >> 1) & 1u, abort_flag, kTimeoutNs)) { ok = false; break; }
-                    tc_fence_after();
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk) {  // S = Q K^T
-                        const uint64_t off = (uint64_t)(((kk >> 2) * kHalfBytes + (kk & 3) * 32) / 16);
-                        mma_ss(tS, dQd + off, dKd + off, kIdescSS, kk > 0 ? 1u : 0u);
-                    }
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk) {  // dP = dO V^T
-                        const uint64_t off = (uint64_t)(((kk >> 2) * kHalfBytes + (kk & 3) * 32) / 16);
-                        mma_ss(tdP, dDo + off, dVd + off, kIdescSS, kk > 0 ? 1u : 0u);
-                    }
-                    mma_commit(&bars->s_full);
-                    if (tt == t.ntiles - 1) mma_commit(&bars->qd_empty);  // Q, dO free once these complete
-                    // The first dQ MMA of item i overwrites dQ once the epilogue has read item i-1.
-                    if (tt == 0 && i >= 1 && !mbar_wait(&bars->dq_free, (i - 1) & 1u, abort_flag, kTimeoutNs)) {
+                    // B: dP(n) overwrites dP(n-1) once both halves of the elementwise pass have read it.
+                    if (!isA && n >= 1 &&
+                        !(mbar_wait(&bars->p_half[0], (n - 1) & 1u, abort_flag, kTimeoutNs) &&
+                          mbar_wait(&bars->p_half[1], (n - 1) & 1u, abort_flag, kTimeoutNs))) {
                         ok = false;
                         break;
                     }
-                    // dQ += dS K, 16 keys per step, each key half as soon as its dS is written (half h:
-                    // columns 64h .. 64h+31 of S).
-                    for (int h = 0; ok && h < 2; ++h) {
-                        if (!mbar_wait(&bars->p_half[h], n & 1u, abort_flag, kTimeoutNs)) { ok = false; break; }
-                        tc_fence_after();
+                    tc_fence_after();
+                    const uint32_t t1 = isA ? tS : tdP;
 #pragma unroll
-                        for (int kq = 0; kq < 4; ++kq) {
-                            const int kk = 4 * h + kq;
-                            mma_ts(tdQ, tS + (uint32_t)(64 * h + kq * 8), dKmn + (uint64_t)(kk * 2048 / 16), kIdescTS,
-                                   (tt > 0 || kk > 0) ? 1u : 0u);
-                        }
+                    for (int kk = 0; kk < 8; ++kk) {  // S = Q K^T  /  dP = dO V^T
+                        const uint64_t off = (uint64_t)(((kk >> 2) * kHalfBytes + (kk & 3) * 32) / 16);
+                        mma_ss(t1, dA1 + off, dB1 + off, kIdescSS, kk > 0 ? 1u : 0u);
                     }
-                    if (!ok) break;
+                    mma_commit(&bars->s_full);
+                    if (tt == t.ntiles - 1) mma_commit(&bars->qd_empty);  // Q, dO free once these complete
+                    if (isA) {
+                        const uint64_t dKmn = umma_desc_sw128(ak, kHalfBytes, 1024);
+                        // The first dQ MMA of item i overwrites dQ once the epilogue has read item i-1.
+                        if (tt == 0 && i >= 1 && !mbar_wait(&bars->dq_free, (i - 1) & 1u, abort_flag, kTimeoutNs)) {
+                            ok = false;
+                            break;
+                        }
+                        // dQ += dS K, 16 keys per step, each key half as soon as its dS is written (half h:
+                        // columns 64h .. 64h+31 of S).
+                        for (int h = 0; ok && h < 2; ++h) {
+                            if (!mbar_wait(&bars->p_half[h], n & 1u, abort_flag, kTimeoutNs)) { ok = false; break; }
+                            tc_fence_after();
+#pragma unroll
+                            for (int kq = 0; kq < 4; ++kq) {
+                                const int kk = 4 * h + kq;
+                                mma_ts(tdQ, tS + (uint32_t)(64 * h + kq * 8), dKmn + (uint64_t)(kk * 2048 / 16), kIdescTS,
+                                       (tt > 0 || kk > 0) ? 1u : 0u);
+                            }
+                        }
+                        if (!ok) break;
+                    }
                     mma_commit(&bars->kv_empty[b]);
-                    if (tt == t.ntiles - 1) mma_commit(&bars->dq_ready);
+                    if (isA && tt == t.ntiles - 1) mma_commit(&bars->dq_ready);
                 }
                 ++i;
             }
             if (!ok) *abort_flag = 1;
-            mma_commit(&bars->drain);
+            uint64_t* dr = &bars->drain[isA ? 0 : 1];
+            mma_commit(dr);
             volatile int never = 0;
-            mbar_wait(&bars->drain, 0, &never, kTimeoutNs);
+            mbar_wait(dr, 0, &never, kTimeoutNs);
         }
     } else if (!skip) {
         // ------------------------------------------------ one thread per (query row r, key half)
