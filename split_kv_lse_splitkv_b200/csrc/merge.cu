@@ -13,8 +13,8 @@
 // Memory-bound. The partial tiles are stored [d/E][rows][E] in the problem dtype (E elements per
 // 16-byte group: 4 float32 or 8 bf16). A thread owns one row r and 16 consecutive columns (4 or 2
 // groups); a CTA owns kThreads consecutive (row, column block) units of one (j, g), so a warp's 32
-// consecutive rows read 512 contiguous bytes per group, and each thread keeps four partials' loads
-// in flight. The output row receives 16 contiguous values.
+// consecutive rows read 512 contiguous bytes per group, and each thread keeps two (bf16) or four
+// (float32) partials' loads in flight. The output row receives 16 contiguous values.
 #include "common.cuh"
 
 namespace splitkv {
@@ -23,7 +23,17 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kVals = 16;   // columns per thread
-constexpr int kUnroll = 4;  // partials loaded ahead
+// Partials loaded ahead, and CTAs per SM the registers are sized for: bf16 tiles take two partials
+// ahead at four CTAs per SM (64 registers), float32 tiles four at the default. (On drafter_s32k the
+// bf16 merge measured 65.5 -> 62.5 us against four ahead at three CTAs per SM.)
+template <typename T>
+struct MergeShape {
+    static constexpr int kUnroll = 4, kMinBlocks = 1;
+};
+template <>
+struct MergeShape<__nv_bfloat16> {
+    static constexpr int kUnroll = 2, kMinBlocks = 4;
+};
 
 struct Online {
     float m, l;
@@ -69,11 +79,12 @@ __device__ __forceinline__ void load_row(const uint4* __restrict__ tile, int RT,
 }
 
 template <typename T>
-__global__ void __launch_bounds__(kThreads) merge_kernel(Meta m, int32_t ctas_per_head, const T* __restrict__ o_part,
+__global__ void __launch_bounds__(kThreads, MergeShape<T>::kMinBlocks) merge_kernel(Meta m, int32_t ctas_per_head, const T* __restrict__ o_part,
                                                          const float* __restrict__ lse_part,
                                                          const int32_t* __restrict__ anchors, T* __restrict__ o,
                                                          float* __restrict__ lse, const int32_t* __restrict__ status) {
     constexpr int E = 16 / (int)sizeof(T);
+    constexpr int kUnroll = MergeShape<T>::kUnroll;
     if (status_bad(status)) return;
     const int R = m.rows, d = m.d, G = m.group, BL = m.block, ngroups = d / E;
     const int64_t jg = blockIdx.x / ctas_per_head;
