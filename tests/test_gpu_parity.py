@@ -151,6 +151,32 @@ def test_planner_rejects_out_of_range_costs():
     assert skv.status_value() & DEV_BAD_COST
 
 
+@pytest.mark.parametrize("n_workers", [1, 31, 33, 148, 256, 257, 300])
+def test_planner_random_costs(n_workers):
+    # The run walk has a one-warp kernel for up to 256 workers and a one-CTA kernel above; both
+    # must give the oracle's LPT plan bit for bit. Costs cover every bucket 1..64, skewed towards
+    # small ones like the workloads', with a few thousand items so most runs are non-trivial.
+    from oracle import schedule as OS
+    from split_kv_lse_splitkv_b200 import SplitKV
+    skv = SplitKV([262144], [512], 32, 4, 128, chunk=8192, n_workers=n_workers)
+    W_ = int(skv.sizes.max_cost)
+    n = min(int(skv.sizes.n_items_max), 3000)
+    rng = np.random.default_rng(17 + n_workers)
+    costs = np.minimum(W_, rng.geometric(0.08, size=n)).astype(np.int32)
+    costs[:W_] = np.arange(1, W_ + 1)
+    rng.shuffle(costs)
+    skv.item_cost[:n] = torch.from_numpy(costs).cuda()
+    skv.n_items.fill_(n)
+    skv.plan_lpt()
+    torch.cuda.synchronize()
+    skv.check_status()
+    iw, qo, qi, load = OS.lpt(costs.tolist(), n_workers)
+    assert skv.item_worker[:n].cpu().numpy().tolist() == iw.tolist()
+    assert skv.queue_off.cpu().numpy().tolist() == qo.tolist()
+    assert skv.queue_items[:n].cpu().numpy().tolist() == qi.tolist()
+    assert skv.load.cpu().numpy().tolist() == load.tolist()
+
+
 # ------------------------------------------------------------------ full-size workloads
 def sampled_blocks(inp, k=4):
     n = int(inp.anchor_off[-1])
