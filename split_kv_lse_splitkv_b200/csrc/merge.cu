@@ -14,7 +14,12 @@
 // 16-byte group: 4 float32 or 8 bf16). A thread owns one row r and 16 consecutive columns (4 or 2
 // groups); a CTA owns kThreads consecutive (row, column block) units of one (j, g), so a warp's 32
 // consecutive rows read 512 contiguous bytes per group, and each thread keeps two (bf16) or four
-// (float32) partials' loads in flight. The output row receives 16 contiguous values.
+// (float32) partials' loads in flight. The output row receives 16 contiguous values, written as
+// 16-byte stores: with one element per store, each warp store touched 32 rows' sectors for 64 bytes
+// and the stores took as much of the load/store path as the partial loads (drafter_s32k: 62.5 us
+// with scalar stores, 36.8 us with 16-byte ones). CTAs start at the last query block: within a sample
+// blocks are numbered by anchor, so the last ones merge the most chunks and, launched last, would
+// form the tail (36.8 -> 31.7 us).
 #include "common.cuh"
 
 namespace splitkv {
@@ -24,8 +29,7 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int kVals = 16;   // columns per thread
 // Partials loaded ahead, and CTAs per SM the registers are sized for: bf16 tiles take two partials
-// ahead at four CTAs per SM (64 registers), float32 tiles four at the default. (On drafter_s32k the
-// bf16 merge measured 65.5 -> 62.5 us against four ahead at three CTAs per SM.)
+// ahead at four CTAs per SM (64 registers), float32 tiles four at the default.
 template <typename T>
 struct MergeShape {
     static constexpr int kUnroll = 4, kMinBlocks = 1;
@@ -65,6 +69,24 @@ __device__ __forceinline__ void unpack16(const uint4& v, float* x, __nv_bfloat16
     }
 }
 
+// 16 values x inv to 16-byte aligned `dst`: four float32 or two bf16 16-byte stores.
+__device__ __forceinline__ void store_vals(float* dst, const float (&x)[kVals], float inv) {
+#pragma unroll
+    for (int u = 0; u < kVals; u += 4)
+        *reinterpret_cast<float4*>(dst + u) = make_float4(x[u] * inv, x[u + 1] * inv, x[u + 2] * inv, x[u + 3] * inv);
+}
+__device__ __forceinline__ void store_vals(__nv_bfloat16* dst, const float (&x)[kVals], float inv) {
+    uint32_t w[kVals / 2];
+#pragma unroll
+    for (int e = 0; e < kVals / 2; ++e) {
+        const __nv_bfloat162 h = __floats2bfloat162_rn(x[2 * e] * inv, x[2 * e + 1] * inv);  // low half first
+        w[e] = *reinterpret_cast<const uint32_t*>(&h);
+    }
+#pragma unroll
+    for (int u = 0; u < kVals / 8; ++u)
+        *reinterpret_cast<uint4*>(dst + 8 * u) = make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
+}
+
 // Row `r` of a partial tile of `RT` rows: 16 columns from 16-byte group g0 on, zero past d.
 template <typename T>
 __device__ __forceinline__ void load_row(const uint4* __restrict__ tile, int RT, int r, int g0, int ngroups,
@@ -87,7 +109,7 @@ __global__ void __launch_bounds__(kThreads, MergeShape<T>::kMinBlocks) merge_ker
     constexpr int kUnroll = MergeShape<T>::kUnroll;
     if (status_bad(status)) return;
     const int R = m.rows, d = m.d, G = m.group, BL = m.block, ngroups = d / E;
-    const int64_t jg = blockIdx.x / ctas_per_head;
+    const int64_t jg = (int64_t)m.n_blocks * m.hkv - 1 - blockIdx.x / ctas_per_head;  // last blocks (most chunks) first
     const int32_t j = (int32_t)(jg / m.hkv), g = (int32_t)(jg % m.hkv);
     const int unit = (blockIdx.x % ctas_per_head) * kThreads + threadIdx.x;
     const int blocks = (d + kVals - 1) / kVals;  // 16-column blocks per row
@@ -144,9 +166,14 @@ __global__ void __launch_bounds__(kThreads, MergeShape<T>::kMinBlocks) merge_ker
     const int i = r / G, hl = r % G;
     const int64_t orow = ((int64_t)BL * j + i) * m.hq + (int64_t)g * G + hl;
     T* dst = o + orow * d + c0;
+    if (d % E == 0 && c0 + kVals <= d) {
+        // A whole 16-column block: 16-byte stores (rows of d elements keep 16-byte alignment).
+        store_vals(dst, st.acc, inv);
+    } else {
 #pragma unroll
-    for (int u = 0; u < kVals; ++u)
-        if (c0 + u < d) dst[u] = from_f32<T>(st.acc[u] * inv);
+        for (int u = 0; u < kVals; ++u)
+            if (c0 + u < d) dst[u] = from_f32<T>(st.acc[u] * inv);
+    }
     if (c0 == 0) lse[orow] = st.m + logf(st.l);
 }
 
