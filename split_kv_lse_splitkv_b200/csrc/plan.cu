@@ -90,7 +90,8 @@ __global__ void __launch_bounds__(kThreads) plan_hist_kernel(const int32_t* __re
     for (int i = threadIdx.x; i <= W; i += kThreads) ws.hist[(size_t)blockIdx.x * (W + 1) + i] = h[i];
 }
 
-__global__ void __launch_bounds__(kThreads) plan_runs_kernel(const int32_t* __restrict__ n_items_d,
+// (The explicit one-block minimum keeps ptxas from holding this kernel to 32 registers with spills.)
+__global__ void __launch_bounds__(kThreads, 1) plan_runs_kernel(const int32_t* __restrict__ n_items_d,
                                                              int32_t max_items, int32_t W, int32_t m, PlanWs ws,
                                                              int32_t* __restrict__ queue_off,
                                                              int64_t* __restrict__ load_out,
@@ -161,9 +162,17 @@ __global__ void __launch_bounds__(kThreads) plan_runs_kernel(const int32_t* __re
         const int64_t V0 = red64[0];
         int32_t ri = 0, oi = w;  // threads without a worker sort into an unused bucket
         if (tid < m) {
-            const int64_t dlt = li - V0;
-            ri = (int32_t)(dlt / w);
-            oi = (int32_t)(dlt % w);
+            // Window and offset in 32 bits (a 64-bit division is a long dependent sequence on this
+            // latency-bound path): a valid plan keeps loads within (W + 1) w of the minimum, and a
+            // difference that does not fit in 32 bits is a window past W all the same.
+            const uint64_t dlt = (uint64_t)(li - V0);
+            if (dlt > 0xffffffffull) {
+                ri = W + 1;
+                oi = 0;
+            } else {
+                ri = (int32_t)((uint32_t)dlt / (uint32_t)w);
+                oi = (int32_t)((uint32_t)dlt % (uint32_t)w);
+            }
             rr[tid] = ri;
             if (ri > W) atomicOr(&bad, 1);
             else atomicAdd(&cnt_r[ri], 1);
@@ -175,20 +184,21 @@ __global__ void __launch_bounds__(kThreads) plan_runs_kernel(const int32_t* __re
         int32_t rmax = warp_reduce_max(tid < m ? ri : 0);
         if (lane == 0) red32[warp] = rmax;
         __syncthreads();
-        if (tid <= W) {  // per-offset totals (offsets < w <= W)
-            int32_t c = 0;
-            for (int x = 0; x < 32; ++x) c += cnt_w[x][tid];
-            start_o[tid] = c;
+        if (warp == 0) {  // per-offset totals and their exclusive prefix (offsets < w <= 64: two per lane)
+            int32_t c0 = 0, c1 = 0;
+            for (int x = 0; x < nwarps; ++x) {
+                if (lane < w) c0 += cnt_w[x][lane];
+                if (lane + 32 < w) c1 += cnt_w[x][lane + 32];
+            }
+            const int32_t i0 = warp_inclusive_scan(c0);
+            const int32_t i1 = warp_inclusive_scan(c1) + __shfl_sync(0xffffffffu, i0, 31);
+            if (lane < w) start_o[lane] = i0 - c0;
+            if (lane + 32 < w) start_o[lane + 32] = i1 - c1;
         }
         if (tid == 32) {
             int32_t x = 0;
             for (int y = 0; y < nwarps; ++y) x = red32[y] > x ? red32[y] : x;
             red32[32] = x;
-        }
-        __syncthreads();
-        if (tid == 0) {
-            int32_t acc = 0;
-            for (int o = 0; o < w; ++o) { const int32_t c = start_o[o]; start_o[o] = acc; acc += c; }
         }
         __syncthreads();
         if (bad) break;
@@ -217,17 +227,31 @@ __global__ void __launch_bounds__(kThreads) plan_runs_kernel(const int32_t* __re
             ws.run_r[(size_t)w * m + tid] = ri;
         }
         // Catch-up windows r < R: participants (r_i <= r) in q order get ranks P[r] + position.
-        // Thread x handles the worker at q position x.
+        // Thread x handles the worker at q position x. A participant's position is the participants
+        // before it in its warp (a ballot) plus those of the earlier warps: per-warp counts for every
+        // window (cnt_w[warp][r]: the offset counts are consumed), then their prefix over warps.
         const int32_t wx = tid < m ? by_q[tid] : -1;
         const int32_t rx = wx >= 0 ? rr[wx] : 0;
+        const unsigned below = (1u << lane) - 1u;
         int32_t picks_x = 0;
         for (int r = 0; r < R; ++r) {
-            const int32_t part = (wx >= 0 && rx <= r) ? 1 : 0;
-            const int32_t pos = block_exclusive_scan<int32_t>(part, scan_sh, nullptr);
-            const int32_t rank = P[r] + pos;
-            if (part && rank < nw) {
-                ws.run_catch[(size_t)w * m * W + rank] = make_int2(wx, r - rx);
-                ++picks_x;
+            const unsigned b = __ballot_sync(0xffffffffu, wx >= 0 && rx <= r);
+            if (lane == 0) cnt_w[warp][r] = __popc(b);
+        }
+        __syncthreads();
+        if (tid < R) {
+            int32_t acc = 0;
+            for (int y = 0; y < nwarps; ++y) { const int32_t c = cnt_w[y][tid]; cnt_w[y][tid] = acc; acc += c; }
+        }
+        __syncthreads();
+        for (int r = 0; r < R; ++r) {
+            const unsigned b = __ballot_sync(0xffffffffu, wx >= 0 && rx <= r);
+            if (wx >= 0 && rx <= r) {
+                const int32_t rank = P[r] + cnt_w[warp][r] + __popc(b & below);
+                if (rank < nw) {
+                    ws.run_catch[(size_t)w * m * W + rank] = make_int2(wx, r - rx);
+                    ++picks_x;
+                }
             }
         }
         __syncthreads();
