@@ -61,6 +61,18 @@ def test_query_sizes():
     assert s2.o_part_elems == (s2.n_items_max + 5 * 2) * 128 * 64
 
 
+def test_query_sizes_with_samples_without_anchors():
+    # A sample without anchors has no block and no item; its keys still count (they sit between the
+    # other samples' keys in K and V). A problem without any anchor is valid and empty.
+    s = B.splitkv_query(prob(seq_lens=[1000, 700, 300], anchor_off=[0, 3, 3, 5], n_q_heads=8, n_kv_heads=2,
+                             chunk=256))
+    assert s.n_items_max == 4 * 2 * 3 + 0 + 2 * 2 * 2
+    assert s.n_chunks == 4 + 3 + 2 and s.total_keys == 2000 and s.n_blocks == 5 and s.n_queries == 80
+    e = B.splitkv_query(prob(seq_lens=[1000], anchor_off=[0, 0]))
+    assert e.n_items_max == 0 and e.n_blocks == 0 and e.n_queries == 0 and e.o_part_elems == 0
+    assert B.splitkv_workspace_size(prob(seq_lens=[1000], anchor_off=[0, 0]), 4) > 0
+
+
 @pytest.mark.parametrize("kw,code", [
     (dict(n_kv_heads=3, n_q_heads=4), B.EINVAL),          # Hkv does not divide Hq
     (dict(chunk=100), B.EUNSUPPORTED),                    # chunk not a multiple of key_tile
