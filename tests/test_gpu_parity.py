@@ -110,14 +110,6 @@ def backward_check(inp, n_workers=4):
         assert_close(name, to_np(g), r, inp.workload.dtype)
 
 
-def test_batch_with_an_empty_sample():
-    # The middle sample has no anchor: no block, item or self partial of its own, while its keys sit
-    # between the other samples' in K and V (their gradients must come out zero).
-    inp = small("empty_mid", "train_4x64k", [3000, 2048, 2500], [4, 0, 3], chunk=1024, seed=21)
-    full_check(inp, n_workers=5)
-    backward_check(inp, n_workers=5)
-
-
 def test_backward_bf16_batch():
     backward_check(small("bwd", "train_4x64k", [3000, 2048, 4096], [2, 3, 4], chunk=1024))
 
@@ -310,3 +302,11 @@ def test_cuda_graph_replay_matches_eager(backward):
             assert torch.allclose(a, b, rtol=1e-5, atol=1e-6 * float(b.abs().max())), "dQ"
         else:
             assert torch.equal(a, b), i
+
+
+def test_batch_with_an_empty_sample():
+    # The middle sample has no anchor: no block, item or self partial of its own, while its keys sit
+    # between the other samples' in K and V (their gradients must come out zero).
+    inp = small("empty_mid", "train_4x64k", [3000, 2048, 2500], [4, 0, 3], chunk=1024, seed=21)
+    full_check(inp, n_workers=5)
+    backward_check(inp, n_workers=5)
