@@ -1,0 +1,59 @@
+"""Host-side logic of bench.py on CPU: the roofline's DRAM traffic comes from a committed ncu summary
+only while every source file that summary hashes is unchanged; otherwise it is reported as null."""
+import os
+import shutil
+import sys
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+import bench  # noqa: E402
+
+SUMMARY = "fwd_tc_kernel.drafter_s32k.txt"
+
+
+def _copy_summary_and_sources(dst):
+    src_summary = os.path.join(ROOT, "profiles", SUMMARY)
+    lines = open(src_summary).read().splitlines()
+    rels = [ln[len("source_sha256 "):].split(": ")[0] for ln in lines if ln.startswith("source_sha256 ")]
+    assert rels, "the summary names the sources it was captured from"
+    os.makedirs(os.path.join(dst, "profiles"))
+    shutil.copy(src_summary, os.path.join(dst, "profiles", SUMMARY))
+    for rel in rels:
+        os.makedirs(os.path.dirname(os.path.join(dst, rel)), exist_ok=True)
+        shutil.copy(os.path.join(ROOT, rel), os.path.join(dst, rel))
+    traffic = int([ln for ln in lines if ln.startswith("traffic_bytes_per_launch:")][0].split(":")[1])
+    return rels, traffic
+
+
+def _write_hashes_of_current_sources(root, rels):
+    # Make the copied summary describe the copied sources exactly as they are.
+    import hashlib
+    path = os.path.join(root, "profiles", SUMMARY)
+    out = []
+    for ln in open(path).read().splitlines():
+        if ln.startswith("source_sha256 "):
+            rel = ln[len("source_sha256 "):].split(": ")[0]
+            ln = f"source_sha256 {rel}: " + hashlib.sha256(open(os.path.join(root, rel), "rb").read()).hexdigest()
+        out.append(ln)
+    open(path, "w").write("\n".join(out) + "\n")
+
+
+def test_traffic_reported_while_sources_match(tmp_path, monkeypatch):
+    rels, traffic = _copy_summary_and_sources(str(tmp_path))
+    _write_hashes_of_current_sources(str(tmp_path), rels)
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.profiled_traffic("fwd_tc_kernel", "drafter_s32k") == traffic > 0
+
+
+def test_traffic_null_once_a_source_changed(tmp_path, monkeypatch):
+    rels, _ = _copy_summary_and_sources(str(tmp_path))
+    _write_hashes_of_current_sources(str(tmp_path), rels)
+    with open(os.path.join(str(tmp_path), rels[-1]), "a") as f:
+        f.write("\n// edited after the capture\n")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.profiled_traffic("fwd_tc_kernel", "drafter_s32k") is None
+
+
+def test_traffic_null_without_a_summary(tmp_path, monkeypatch):
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.profiled_traffic("fwd_tc_kernel", "drafter_s32k") is None
