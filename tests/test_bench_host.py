@@ -57,3 +57,22 @@ def test_traffic_null_once_a_source_changed(tmp_path, monkeypatch):
 def test_traffic_null_without_a_summary(tmp_path, monkeypatch):
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
     assert bench.profiled_traffic("fwd_tc_kernel", "drafter_s32k") is None
+
+
+def test_useful_flops_count_the_pairs_the_oracle_sees():
+    # 4 d FLOP per (query row, visible key, query head) forward (QK^T and PV), 10 d backward, with the
+    # visible keys taken from the oracle's own visibility rule, block by block.
+    import workloads as W
+    from tests._util import oracle_problem
+    for w in (W.get("tiny_f32"), W.scaled(W.get("train_4x64k"), "flops", [3000, 2048], [3, 2], chunk=1024)):
+        inp = W.make_inputs(w)
+        p = oracle_problem(inp)
+        pairs = 0
+        for s, j, a in p.blocks():
+            for h in range(p.Hq):
+                keys, _ = p.visible(s, j, a, h // p.G)
+                pairs += p.block * keys.shape[0]
+        total, fwd = bench.useful_flops(inp, backward=True)
+        assert fwd == 4 * p.d * pairs
+        assert total == 14 * p.d * pairs
+        assert bench.useful_flops(inp, backward=False) == (fwd, fwd)
