@@ -83,7 +83,8 @@ def peaks():
 
 class ClockSampler:
     """SM clock and clock-event (throttle) reasons sampled through NVML every millisecond while the
-    timed region runs, plus one sample as it ends; falls back to nvidia-smi when NVML is missing."""
+    timed region runs, plus one sample as it ends. Without NVML (or without a GPU) it records nothing
+    and the summary says so ("source": "none")."""
 
     REASONS = (("hw_slowdown", 0x8), ("hw_thermal_slowdown", 0x40), ("sw_thermal_slowdown", 0x20),
                ("sw_power_cap", 0x4))

@@ -76,3 +76,20 @@ def test_useful_flops_count_the_pairs_the_oracle_sees():
         assert fwd == 4 * p.d * pairs
         assert total == 14 * p.d * pairs
         assert bench.useful_flops(inp, backward=False) == (fwd, fwd)
+
+
+def test_clock_reason_bits_are_nvmls():
+    pynvml = __import__("pynvml")
+    names = {"hw_slowdown": "HwSlowdown", "hw_thermal_slowdown": "HwThermalSlowdown",
+             "sw_thermal_slowdown": "SwThermalSlowdown", "sw_power_cap": "SwPowerCap"}
+    for name, bit in bench.ClockSampler.REASONS:
+        assert bit == getattr(pynvml, "nvmlClocksEventReason" + names[name]), name
+
+
+def test_clock_summary_of_samples():
+    c = bench.ClockSampler(0)
+    assert c.summary()["source"] == "none" and c.summary()["samples"] == 0
+    c.samples = [(1965.0, 1965.0, 0x0), (1800.0, 1965.0, 0x4), (1700.0, 1965.0, 0x4 | 0x40)]
+    s = c.summary()
+    assert s["sm_mhz"] == 1800.0 and s["sm_max_mhz"] == 1965.0 and s["samples"] == 3
+    assert s["reasons"] == ["hw_thermal_slowdown", "sw_power_cap"]
