@@ -207,10 +207,9 @@ def cpu_oracle_sample(inp, budget_s, backward):
     done = []
     for j in order:
         a = int(inp.anchors[j])
-        OA.forward(p, blocks=[j])
+        O, L = OA.forward(p, blocks=[j])
         flops += 4 * w.head_dim * w.n_q_heads * w.block * (a + w.block)
-        if backward:
-            O, L = OA.forward(p, blocks=[j])
+        if backward:  # from this forward's O and LSE, as a training step would
             OA.backward(p, f64(inp.do), O=O, LSE=L, blocks=[j])
             flops += 10 * w.head_dim * w.n_q_heads * w.block * (a + w.block)
         done.append(int(j))
