@@ -25,6 +25,9 @@
  *       kb, vb, dkb, dvb    [Nq, Hkv, d]     each block's own keys / values
  *       lse                 [Nq, Hq]         float32, natural log
  *     Query head h reads kv head h / (Hq/Hkv).
+ *     A problem without any anchor (Nq = 0) has nothing to compute: its query-side tensors (q, o,
+ *     dout, kb, vb, lse, dq, dkb, dvb) and anchors_d are empty and may be NULL; the calls then
+ *     write only what has keys (chunk_cost = 0, n_items = 0, an empty plan, dK = dV = 0).
  *   - Return value: SPLITKV_OK, or a negative code detected on the host BEFORE anything is
  *     enqueued (nothing was launched), or SPLITKV_ECUDA if a launch failed. Errors that only the
  *     device can see (bad anchors, costs out of range, an in-kernel wait that ran out) are ORed into

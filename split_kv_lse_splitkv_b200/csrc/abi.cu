@@ -197,8 +197,10 @@ SPLITKV_API int splitkv_attn_fwd(const splitkv_problem* problem, const void* q, 
     int rc = build_meta(problem, &m);
     if (rc) return rc;
     if (n_workers < 1 || n_workers > 65535 || (flags & ~SPLITKV_FWD_SIMT)) return SPLITKV_EINVAL;
-    if (!q || !k || !v || !kb || !vb || !item_id_d || !queue_off_d || !queue_items_d || !o_part || !lse_part ||
-        !status_d)
+    // Query-side buffers are empty (possibly NULL) when the problem has no anchor at all.
+    const bool queries = m.n_queries > 0;
+    if ((queries && (!q || !kb || !vb)) || !k || !v || !item_id_d || !queue_off_d || !queue_items_d || !o_part ||
+        !lse_part || !status_d)
         return SPLITKV_EINVAL;
     if (m.n_blocks && !anchors_d) return SPLITKV_EINVAL;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(kb) || !aligned16(vb) || !aligned16(o_part))
@@ -220,7 +222,7 @@ SPLITKV_API int splitkv_lse_merge(const splitkv_problem* problem, const void* o_
     Meta m;
     int rc = build_meta(problem, &m);
     if (rc) return rc;
-    if (!o_part || !lse_part || !o || !lse || !status_d) return SPLITKV_EINVAL;
+    if (!o_part || !lse_part || (m.n_queries > 0 && (!o || !lse)) || !status_d) return SPLITKV_EINVAL;
     if (m.n_blocks && !anchors_d) return SPLITKV_EINVAL;
     if (!aligned16(o_part) || !aligned16(lse_part) || !aligned16(o)) return SPLITKV_EINVAL;
     return cuda_status(launch_merge(m, o_part, lse_part, anchors_d, o, lse, status_d, (cudaStream_t)stream));
@@ -236,7 +238,9 @@ SPLITKV_API int splitkv_attn_bwd(const splitkv_problem* problem, const void* q, 
     Meta m;
     int rc = build_meta(problem, &m);
     if (rc) return rc;
-    if (!q || !k || !v || !kb || !vb || !o || !lse || !dout || !dq || !dk || !dv || !dkb || !dvb || !status_d)
+    const bool queries = m.n_queries > 0;  // without any anchor the query-side buffers are empty
+    if ((queries && (!q || !kb || !vb || !o || !lse || !dout || !dq || !dkb || !dvb)) || !k || !v || !dk || !dv ||
+        !status_d)
         return SPLITKV_EINVAL;
     if (m.n_blocks && !anchors_d) return SPLITKV_EINVAL;
     cudaStream_t st = (cudaStream_t)stream;

@@ -241,9 +241,9 @@ cudaError_t launch_t(const Meta& m, const void* q, const void* k, const void* v,
                      const void* o, const float* lse, const void* dout, const int32_t* anchors, float* dq, float* dk,
                      float* dv, float* dkb, float* dvb, int32_t* status, void* ws, cudaStream_t st) {
     float* dvec = (float*)ws;
-    cudaError_t e = cudaMemsetAsync(dq, 0, sizeof(float) * (size_t)m.n_queries * m.hq * m.d, st);
-    if (e != cudaSuccess) return e;
     const int64_t rows = m.n_queries * m.hq;
+    cudaError_t e = rows > 0 ? cudaMemsetAsync(dq, 0, sizeof(float) * (size_t)rows * m.d, st) : cudaSuccess;
+    if (e != cudaSuccess) return e;
     if (rows > 0) {
         dvec_kernel<T><<<(unsigned)((rows * 32 + kThreads - 1) / kThreads), kThreads, 0, st>>>(
             m, (const T*)o, (const T*)dout, dvec);

@@ -708,14 +708,15 @@ cudaError_t launch_bwd_tc(const Meta& m, const void* q, const void* k, const voi
                           int32_t n_workers, float* dq, float* dk, float* dv, float* dkb, float* dvb,
                           int32_t* status, void* ws, cudaStream_t st) {
     const size_t nrows = (size_t)m.n_queries * m.hq;
-    cudaError_t e = cudaMemsetAsync(dq, 0, sizeof(float) * nrows * m.d, st);
-    if (e != cudaSuccess) return note_error(e, "cudaMemsetAsync(dq)");
+    cudaError_t e;
     if (m.n_queries == 0) {
-        // No query: every key gradient is zero.
+        // No query (the query-side buffers are empty): every key gradient is zero.
         e = cudaMemsetAsync(dk, 0, sizeof(float) * (size_t)m.total_keys * m.hkv * m.d, st);
         if (e == cudaSuccess) e = cudaMemsetAsync(dv, 0, sizeof(float) * (size_t)m.total_keys * m.hkv * m.d, st);
         return note_error(e, "cudaMemsetAsync(dk, dv)");
     }
+    e = cudaMemsetAsync(dq, 0, sizeof(float) * nrows * m.d, st);
+    if (e != cudaSuccess) return note_error(e, "cudaMemsetAsync(dq)");
     float* l2 = reinterpret_cast<float*>((reinterpret_cast<uintptr_t>(ws) + 255) & ~uintptr_t(255));
     float* dvec = l2 + nrows;
     rows_kernel<__nv_bfloat16><<<(unsigned)((nrows * 32 + 255) / 256), 256, 0, st>>>(

@@ -159,6 +159,7 @@ cudaError_t launch_t(const Meta& m, const void* q, const void* k, const void* v,
                      const int32_t* anchors, const int32_t* item_id, const int32_t* queue_off,
                      const int32_t* queue_items, int32_t n_workers, void* o_part, float* lse_part, int32_t* status,
                      cudaStream_t st) {
+    if (m.n_queries == 0) return cudaSuccess;  // no anchor: no partial to compute
     const int R = m.rows_item, d = m.d;
     size_t smem = sizeof(float) * ((size_t)2 * R * d + kBK * (d + 1) + kBK * d + R * kBK + 4 * R);
     cudaError_t e = cudaFuncSetAttribute(fwd_simt_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

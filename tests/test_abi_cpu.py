@@ -163,3 +163,25 @@ def test_strerror():
     assert B.splitkv_strerror(0) == "ok"
     assert "workspace" in B.splitkv_strerror(B.ENOSPACE)
     assert B.splitkv_strerror(12345) == "unknown status"
+
+
+@pytest.mark.parametrize("dtype,d", [(torch.bfloat16, 128), (torch.float32, 64)])
+def test_problem_without_anchors_needs_no_query_buffers(dtype, d):
+    # No anchor at all: nothing to compute. The forward (tensor-core or CUDA-core path) and the merge
+    # accept empty (NULL) query-side buffers and return before any CUDA call, so this runs anywhere.
+    p = prob(seq_lens=[1000], anchor_off=[0, 0], n_q_heads=8, n_kv_heads=2, head_dim=d, chunk=256, dtype=dtype)
+    host = torch.empty(64, dtype=torch.int32)  # never dereferenced: the calls return before any access
+    ws = torch.empty(B.splitkv_workspace_size(p, 4), dtype=torch.uint8)
+    h = B._p(host)
+    rc = B._lib.splitkv_attn_fwd(p.ptr, None, h, h, None, None, None, h, h, h, 4, h, h, h, B.FWD_DEFAULT, B._p(ws),
+                                 ws.numel(), None)
+    assert rc == B.OK, B.splitkv_strerror(rc)
+    rc = B._lib.splitkv_lse_merge(p.ptr, h, h, None, None, None, h, None)
+    assert rc == B.OK, B.splitkv_strerror(rc)
+    # With anchors, the same NULL query buffers are refused.
+    p1 = prob(seq_lens=[1000], anchor_off=[0, 2], n_q_heads=8, n_kv_heads=2, head_dim=d, chunk=256, dtype=dtype)
+    rc = B._lib.splitkv_attn_fwd(p1.ptr, None, h, h, None, None, h, h, h, h, 4, h, h, h, B.FWD_DEFAULT, B._p(ws),
+                                 ws.numel(), None)
+    assert rc == B.EINVAL
+    rc = B._lib.splitkv_lse_merge(p1.ptr, h, h, h, None, None, h, None)
+    assert rc == B.EINVAL

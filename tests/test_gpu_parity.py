@@ -310,3 +310,11 @@ def test_batch_with_an_empty_sample():
     inp = small("empty_mid", "train_4x64k", [3000, 2048, 2500], [4, 0, 3], chunk=1024, seed=21)
     full_check(inp, n_workers=5)
     backward_check(inp, n_workers=5)
+
+
+def test_problem_without_anchors():
+    # No anchor at all: empty query tensors (NULL device pointers), no item, an empty plan, zero
+    # chunk costs and zero key gradients.
+    inp = small("empty_all", "train_4x64k", [2048], [0], chunk=1024, seed=22)
+    full_check(inp, n_workers=3)
+    backward_check(inp, n_workers=3)
