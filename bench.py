@@ -188,6 +188,33 @@ def barrier(world):
         dist.barrier()
 
 
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for ln in f:
+                if ln.startswith("model name"):
+                    return ln.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
+
+
+def cpu_oracle_plan(inp, n_workers):
+    """The oracle's cost pass and LPT plan (pure Python, one thread) over the whole workload, timed once."""
+    from oracle import schedule as OS
+    w = inp.workload
+    per_sample = [inp.anchors_of(s) for s in range(len(w.seq_lens))]
+    t0 = time.perf_counter()
+    _, costs, _ = OS.costs_closed_form(per_sample, w.seq_lens, w.chunk, w.key_tile, w.n_kv_heads,
+                                       pack=w.blocks_per_item)
+    t1 = time.perf_counter()
+    OS.lpt(costs.tolist(), n_workers)
+    t2 = time.perf_counter()
+    return {"cost_ms": (t1 - t0) * 1e3, "lpt_ms": (t2 - t1) * 1e3, "items": int(len(costs)),
+            "workers": int(n_workers), "threads": 1}
+
+
 def cpu_oracle_sample(inp, budget_s, backward):
     """Time the float64 oracle on whole blocks of the workload until ~budget_s of CPU work."""
     import numpy as np
@@ -221,8 +248,10 @@ def cpu_oracle_sample(inp, budget_s, backward):
         cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
     except Exception:
         cores = os.cpu_count()
-    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": int(cores), "kind": "oracle",
-            "sample": f"{len(done)} of {n} draft blocks (all {w.n_q_heads} heads{', fwd+bwd' if backward else ', fwd'}), "
+    what = "fwd+bwd" if backward else "fwd"
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": int(cores), "cpu_model": cpu_model(),
+            "kind": "oracle",
+            "sample": f"{len(done)} of {n} draft blocks (all {w.n_q_heads} heads, {what}), "
                       f"{dt:.1f} s float64 NumPy on the host"}
 
 
@@ -240,6 +269,9 @@ def run_reference(args):
             vals.append(r["value"])
     value = statistics.mean(vals)
     r["value"] = value
+    workers = w.n_workers or (torch.cuda.get_device_properties(0).multi_processor_count
+                              if torch.cuda.is_available() else 148)
+    r["plan"] = cpu_oracle_plan(inp, workers)
     line = {"impl": "reference", "metric": "useful block-sparse attention TFLOP/s (fwd+bwd)" if w.backward else
             "useful block-sparse attention TFLOP/s (fwd)", "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
@@ -277,7 +309,7 @@ def run_ours(args):
     torch.cuda.synchronize(device)
     stream = torch.cuda.Stream(device)
     torch.cuda.set_stream(stream)
-    phases = {"plan": [], "fwd": [], "merge": [], "bwd": []}
+    phases = {"cost": [], "plan": [], "fwd": [], "merge": [], "bwd": []}
 
     def timed(name, fn, on):
         if not on:
@@ -304,10 +336,9 @@ def run_ours(args):
         naive_load = (csum[bounds[1:]] - csum[bounds[:-1]]).double()
 
     def step(d, time_phases=False):
-        if args.plan == "naive":
-            timed("plan", lambda: skv.cost(d["anchors"], stream), time_phases)
-        else:
-            timed("plan", lambda: skv.plan(d["anchors"], stream), time_phases)
+        timed("cost", lambda: skv.cost(d["anchors"], stream), time_phases)
+        if args.plan != "naive":  # the naive split's queues were built once, above
+            timed("plan", lambda: skv.plan_lpt(stream), time_phases)
         timed("fwd", lambda: skv.attn_fwd(d["q"], d["k"], d["v"], d["kb"], d["vb"], d["anchors"], stream=stream),
               time_phases)
         timed("merge", lambda: skv.lse_merge(d["anchors"], o, lse, stream=stream), time_phases)
@@ -315,7 +346,8 @@ def run_ours(args):
             timed("bwd", lambda: skv.backward(d["q"], d["k"], d["v"], d["kb"], d["vb"], o, lse, d["do"], d["anchors"],
                                               grads, stream=stream), time_phases)
 
-    launches_per_step = 3 + 3 + 1 + 1 + (3 if w.backward else 0)  # cost, plan, fwd, merge; bwd: rows, kv, q
+    # cost 3, LPT plan 3 (not with the naive split), fwd 1, merge 1; bwd: rows, kv, q
+    launches_per_step = 3 + (0 if args.plan == "naive" else 3) + 1 + 1 + (3 if w.backward else 0)
     for _ in range(args.warmup):
         step(dev)
     torch.cuda.synchronize(device)
@@ -425,6 +457,7 @@ def run_ours(args):
         cpu = None
         if world == 1 and not args.no_cpu_baseline:
             cpu = cpu_oracle_sample(inp, args.ref_budget or 10.0, w.backward)
+            cpu["plan"] = cpu_oracle_plan(inp, skv.n_workers)
         line = {
             "metric": "useful block-sparse attention TFLOP/s (fwd+bwd)" if w.backward else
                       "useful block-sparse attention TFLOP/s (fwd)",

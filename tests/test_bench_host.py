@@ -93,3 +93,12 @@ def test_clock_summary_of_samples():
     s = c.summary()
     assert s["sm_mhz"] == 1800.0 and s["sm_max_mhz"] == 1965.0 and s["samples"] == 3
     assert s["reasons"] == ["hw_thermal_slowdown", "sw_power_cap"]
+
+
+def test_oracle_planning_time_and_cpu_model():
+    import workloads as W
+    inp = W.make_inputs(W.get("tiny_f32"))
+    r = bench.cpu_oracle_plan(inp, 4)
+    assert r["items"] == 19 and r["workers"] == 4 and r["threads"] == 1
+    assert r["cost_ms"] >= 0 and r["lpt_ms"] >= 0
+    assert isinstance(bench.cpu_model(), str) and bench.cpu_model()
