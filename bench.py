@@ -255,6 +255,16 @@ def cpu_oracle_sample(inp, budget_s, backward):
                       f"{dt:.1f} s float64 NumPy on the host"}
 
 
+def workload_config(w, counts, n_workers, world, plan):
+    """The `config` object of the JSON line: the same dict for both arms (how the steps are launched
+    is reported beside it, under "launch")."""
+    return {"workload": w.name, "seq_lens": list(w.seq_lens), "anchors": counts,
+            "heads": f"{w.n_q_heads}q/{w.n_kv_heads}kv", "head_dim": w.head_dim, "chunk": w.chunk,
+            "blocks_per_item": w.blocks_per_item, "queues": n_workers,
+            "l2": "flushed (256 MB write) before every timed step",
+            "parallelism": f"replicas x{world}", "plan": plan}
+
+
 def run_reference(args):
     world, rank, _ = dist_setup(args)
     if rank != 0:
@@ -276,7 +286,9 @@ def run_reference(args):
             "useful block-sparse attention TFLOP/s (fwd)", "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": w.name}, "cpu_baseline": r,
+            "config": workload_config(w, [int(inp.anchor_off[i + 1] - inp.anchor_off[i])
+                                          for i in range(len(w.seq_lens))], workers, args.gpus, args.plan),
+            "launch": "host: float64 NumPy oracle", "cpu_baseline": r,
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line))
 
@@ -397,6 +409,7 @@ def run_ours(args):
         torch.cuda.synchronize(device)
     phase_ms = {k: (sum(a.elapsed_time(b) for a, b in v) / len(v)) for k, v in phases.items() if v}
     fwd_ms = phase_ms["fwd"]
+    merge_ms = phase_ms["merge"]
     ms_max = max_over_ranks(ms, world, device)
     skv.check_status()
 
@@ -464,14 +477,14 @@ def run_ours(args):
             "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": ms_max, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16" if w.dtype == "bf16" else "f32", "data": "synthetic",
-            "config": {"workload": w.name, "seq_lens": list(w.seq_lens), "anchors": counts,
-                       "heads": f"{w.n_q_heads}q/{w.n_kv_heads}kv", "head_dim": w.head_dim, "chunk": w.chunk,
-                       "queues": skv.n_workers, "l2": "flushed (256 MB write) before every timed step",
-                       "parallelism": f"replicas x{world}", "plan": args.plan,
-                       "launch": "eager" if graph is None else "cuda graph of the step"},
+            "config": workload_config(w, counts, skv.n_workers, world, args.plan),
+            "launch": "eager" if graph is None else "cuda graph of the step",
             "roofline": dict(roof, achieved=achieved, unit="TFLOP/s", frac=achieved / peak,
                              traffic=profiled_traffic("fwd_tc_kernel", w.name) if w.dtype == "bf16" else None,
-                             kernel_ms=fwd_ms, algorithmic_flop=fwd_kernel_flops),
+                             kernel_ms=fwd_ms, algorithmic_flop=fwd_kernel_flops,
+                             # useful TFLOP/s over the forward plus the merge, against the same peak
+                             frac_fwd_merge=fwd_kernel_flops / ((fwd_ms + merge_ms) * 1e-3) / 1e12 / peak,
+                             fwd_merge_ms=fwd_ms + merge_ms),
             "phase_ms": phase_ms,
             "imbalance": {f"predicted_{args.plan}": predicted_imb},
             **({"backward_roofline": {"kernels": "rows_kernel + bwd_kv_kernel + bwd_q_kernel",
@@ -498,7 +511,8 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="drafter_s32k", choices=sorted(W.WORKLOADS))
+    ap.add_argument("--workload", default="skewed_s256k", choices=sorted(W.WORKLOADS),
+                    help="default: the largest single-GPU forward workload (S = 262144, ~4080 queries)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--ref-budget", type=float, default=0.0,
                     help="seconds of CPU work per oracle sample (default: ~150 s spread over all reference steps)")

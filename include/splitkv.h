@@ -94,7 +94,8 @@ typedef struct {
     int64_t n_queries;      /* Nq                                                                     */
     int64_t total_keys;     /* sum_s S_s                                                              */
     int64_t n_blocks;       /* total anchors                                                          */
-    int64_t o_part_elems;   /* float32 elements of o_part: (n_items_max + n_blocks*Hkv) * rows * d   */
+    int64_t o_part_elems;   /* elements of o_part, in the problem dtype (bf16 or float32):
+                               (n_items_max + n_blocks*Hkv) * rows * d                               */
     int64_t lse_part_elems; /* float32 elements of lse_part: (n_items_max + n_blocks*Hkv) * rows       */
     int32_t max_cost;       /* chunk / key_tile: the largest item cost                                */
     int32_t rows_per_item;  /* rows = P * block * G: query rows of one item (its query tile)          */
@@ -156,8 +157,13 @@ int splitkv_plan_lpt(const int32_t *item_cost_d, const int32_t *n_items_d, int32
  *   - The first call on a device looks up the array's device address (cudaGetSymbolAddress) with
  *     that device current and caches it; make that first call before any stream capture.
  *   - Returns SPLITKV_ENOSPACE (with splitkv_last_error() stating both sizes) when the plan would
- *     need more scratch than the array holds, i.e. splitkv_workspace_size() grows with max_items,
- *     max_cost and n_workers.
+ *     need more scratch than the array holds. The scratch grows with max_items (16 bytes per 1024
+ *     items and cost bucket), max_cost and n_workers; every max_cost <= 64 with n_workers <= 1024
+ *     fits, and the item count sets the limit: at max_cost 64, up to 14.7 million items on 148
+ *     workers and 4.3 million on 1024; at max_cost 16, 61 million on 148.
+ *   - The cached address belongs to the device's current CUDA context. cudaDeviceReset destroys that
+ *     context (the array is re-created, possibly elsewhere, in the next one), so do not call this
+ *     entry point after a cudaDeviceReset in the same process.
  *   - It allocates nothing and frees nothing. Every call shares the one array and leaves its
  *     contents behind (the planner rewrites all it reads before reading it), so calls whose GPU
  *     work overlaps — on two streams, or from two host threads — race and corrupt each other's

@@ -45,8 +45,14 @@ struct PlanWs {
     int32_t* run_qinv;   // [W+1][m]: worker at q position
     int32_t* run_r;      // [W+1][m]: first window of each worker
     int32_t* run_qbase;  // [W+1][m]: items the worker got in earlier runs
-    int2* run_catch;     // [W+1][m*W]: (worker, k) of each catch-up rank
+    int32_t* run_cbase;  // [W+1]: start of run w's catch-up list in run_catch
+    int2* run_catch;     // run w: m * floor(W / w) entries (worker, k), one per catch-up rank
 };
+
+// Catch-up entries run w can produce. Every load stays within W (the largest cost) of the smallest
+// (each item goes to a least-loaded worker), so a worker's first window is r_i <= floor(W / w) and the
+// catch-up windows r < R = max r_i hold at most m * floor(W / w) elements.
+__host__ __device__ inline int64_t catch_cap(int32_t W, int32_t m, int32_t w) { return (int64_t)m * (W / w); }
 
 __host__ __device__ inline PlanWs carve(void* ws, int32_t max_items, int32_t W, int32_t m, size_t* bytes) {
     char* p = (char*)ws;
@@ -62,7 +68,10 @@ __host__ __device__ inline PlanWs carve(void* ws, int32_t max_items, int32_t W, 
     w.run_qinv = (int32_t*)take(sizeof(int32_t) * (size_t)(W + 1) * m);
     w.run_r = (int32_t*)take(sizeof(int32_t) * (size_t)(W + 1) * m);
     w.run_qbase = (int32_t*)take(sizeof(int32_t) * (size_t)(W + 1) * m);
-    w.run_catch = (int2*)take(sizeof(int2) * (size_t)(W + 1) * m * W);
+    w.run_cbase = (int32_t*)take(sizeof(int32_t) * (W + 1));
+    int64_t ncatch = 0;
+    for (int32_t v = 1; v <= W; ++v) ncatch += catch_cap(W, m, v);
+    w.run_catch = (int2*)take(sizeof(int2) * (size_t)(ncatch > 0 ? ncatch : 1));
     if (bytes) *bytes = off;
     return w;
 }
@@ -106,6 +115,7 @@ __global__ void __launch_bounds__(kThreads, 1) plan_runs_kernel(const int32_t* _
     __shared__ int32_t start[kMaxCost + 1];
     __shared__ int32_t cnt_r[kMaxCost + 2];
     __shared__ int32_t P[kMaxCost + 2];
+    __shared__ int32_t cbase[kMaxCost + 1];
     __shared__ int64_t red64[32];
     __shared__ int32_t red32[33];
     __shared__ int32_t scan_sh[33];
@@ -133,6 +143,8 @@ __global__ void __launch_bounds__(kThreads, 1) plan_runs_kernel(const int32_t* _
         int32_t s = 0;
         for (int w = W; w >= 1; --w) { start[w] = s; s += total[w]; }
         start[0] = s;
+        int32_t cb = 0;
+        for (int w = 1; w <= W; ++w) { cbase[w] = cb; ws.run_cbase[w] = cb; cb += (int32_t)catch_cap(W, m, w); }
     }
     __syncthreads();
     for (int w = tid; w <= W; w += blockDim.x)
@@ -163,8 +175,8 @@ __global__ void __launch_bounds__(kThreads, 1) plan_runs_kernel(const int32_t* _
         int32_t ri = 0, oi = w;  // threads without a worker sort into an unused bucket
         if (tid < m) {
             // Window and offset in 32 bits (a 64-bit division is a long dependent sequence on this
-            // latency-bound path): a valid plan keeps loads within (W + 1) w of the minimum, and a
-            // difference that does not fit in 32 bits is a window past W all the same.
+            // latency-bound path): a valid plan keeps loads within W of the minimum (r_i <= W / w),
+            // and a difference that does not fit in 32 bits is a window past that all the same.
             const uint64_t dlt = (uint64_t)(li - V0);
             if (dlt > 0xffffffffull) {
                 ri = W + 1;
@@ -174,7 +186,7 @@ __global__ void __launch_bounds__(kThreads, 1) plan_runs_kernel(const int32_t* _
                 oi = (int32_t)((uint32_t)dlt % (uint32_t)w);
             }
             rr[tid] = ri;
-            if (ri > W) atomicOr(&bad, 1);
+            if (ri > W / w) atomicOr(&bad, 1);
             else atomicAdd(&cnt_r[ri], 1);
         }
         // q_i: stable position of worker i in (offset, worker) order, by counting sort.
@@ -202,7 +214,7 @@ __global__ void __launch_bounds__(kThreads, 1) plan_runs_kernel(const int32_t* _
         }
         __syncthreads();
         if (bad) break;
-        const int32_t R = red32[32];  // <= W
+        const int32_t R = red32[32];  // <= W / w
         int32_t qi = 0;
         if (tid < m) {
             qi = start_o[oi] + rank_warp;
@@ -249,7 +261,7 @@ __global__ void __launch_bounds__(kThreads, 1) plan_runs_kernel(const int32_t* _
             if (wx >= 0 && rx <= r) {
                 const int32_t rank = P[r] + cnt_w[warp][r] + __popc(b & below);
                 if (rank < nw) {
-                    ws.run_catch[(size_t)w * m * W + rank] = make_int2(wx, r - rx);
+                    ws.run_catch[cbase[w] + rank] = make_int2(wx, r - rx);
                     ++picks_x;
                 }
             }
@@ -313,7 +325,7 @@ __global__ void __launch_bounds__(kThreads) plan_assign_kernel(const int32_t* __
     int32_t worker, kk;
     const int32_t ncatch = ws.run_ncatch[w];
     if (j < ncatch) {
-        int2 e = ws.run_catch[(size_t)w * m * W + j];
+        int2 e = ws.run_catch[ws.run_cbase[w] + j];
         worker = e.x;
         kk = e.y;
     } else {

@@ -36,9 +36,15 @@ def run_forward(inp, n_workers=None, flags=0, device="cuda"):
 
 
 def assert_close(name, got, ref, dtype, magnitude_scaled=False):
-    """Max error within the bound of `dtype`. magnitude_scaled: inputs deliberately far from the
-    workloads' N(0,1) scale (e.g. keys with 12x the norm); the bf16 absolute bound is then taken
-    relative to max(1, max|ref|), since bf16 roundings of O scale with |O|."""
+    """Max error within the bound of `dtype`; prints the measured error, the bound and max|ref| so the
+    headroom shows in the test log.
+
+    magnitude_scaled (O tensors only): inputs deliberately far from the workloads' N(0,1) scale, e.g.
+    rows dominated by one key of 12x the norm, where |O| reaches the size of a single V row. The bf16
+    absolute bound is then 2e-2 x max(1, max|ref|): the path rounds to bf16 three times (P before the
+    PV product, the stored partial O_c, the output O), each within 2^-9 of the value rounded, so the
+    rounding error alone grows with |O| (at most 3 x 2^-9 x max|V|, before any accumulation error).
+    LSE is float32 from float32 row sums and is never scaled."""
     got = np.asarray(got, np.float64)
     ref = np.asarray(ref, np.float64)
     assert got.shape == ref.shape, (name, got.shape, ref.shape)
@@ -46,9 +52,15 @@ def assert_close(name, got, ref, dtype, magnitude_scaled=False):
     err = float(np.max(np.abs(got - ref))) if got.size else 0.0
     scale = float(np.max(np.abs(ref))) if ref.size else 0.0
     if dtype == "f32":
-        assert err <= F32_REL * scale + 1e-30, f"{name}: max err {err:.3e} > {F32_REL} x {scale:.3e}"
+        bound = F32_REL * scale + 1e-30
+        print(f"[parity] {name}: max err {err:.3e}, bound {bound:.3e} (f32 rel), max|ref| {scale:.3e}")
+        assert err <= bound, f"{name}: max err {err:.3e} > {F32_REL} x {scale:.3e}"
     else:
+        if magnitude_scaled:
+            assert not name.startswith("LSE"), "LSE keeps the plain absolute bound"
         bound = BF16_ABS * (max(1.0, scale) if magnitude_scaled else 1.0)
+        print(f"[parity] {name}: max abs err {err:.3e}, bound {bound:.3e} (bf16 abs), "
+              f"rel bound {BF16_REL * scale:.3e}, max|ref| {scale:.3e}")
         assert err <= bound, f"{name}: max abs err {err:.3e} > {bound:.3e}"
         assert err <= BF16_REL * scale + 1e-30, f"{name}: max err {err:.3e} > {BF16_REL} x max|ref| {scale:.3e}"
     return err, scale
@@ -111,7 +123,7 @@ def check_partials(skv, inp, ids, magnitude_scaled=False):
     assert bool(got_O) == (len(ids) > 0), "every problem with items has visible chunk partials to compare"
     if got_O:
         assert_close("O_part", np.stack(got_O), np.stack(ref_O), w.dtype, magnitude_scaled)
-        assert_close("LSE_part", np.stack(got_L), np.stack(ref_L), w.dtype, magnitude_scaled)
+        assert_close("LSE_part", np.stack(got_L), np.stack(ref_L), w.dtype)
     n_max = int(skv.sizes.n_items_max)
     got_O, ref_O, got_L, ref_L = [], [], [], []
     for s in range(len(w.seq_lens)):
@@ -128,4 +140,4 @@ def check_partials(skv, inp, ids, magnitude_scaled=False):
                     ref_L.append(ref_l)
     if got_O:
         assert_close("O_self", np.stack(got_O), np.stack(ref_O), w.dtype, magnitude_scaled)
-        assert_close("LSE_self", np.stack(got_L), np.stack(ref_L), w.dtype, magnitude_scaled)
+        assert_close("LSE_self", np.stack(got_L), np.stack(ref_L), w.dtype)

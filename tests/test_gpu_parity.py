@@ -31,7 +31,7 @@ def full_check(inp, n_workers, flags=0, partials=True, magnitude_scaled=False):
     O, L = OA.forward(oracle_problem(inp))
     dt = inp.workload.dtype
     assert_close("O", to_np(o), O, dt, magnitude_scaled)
-    assert_close("LSE", to_np(lse), L, dt, magnitude_scaled)
+    assert_close("LSE", to_np(lse), L, dt)
     return skv, dev, anchors, o, lse
 
 
@@ -153,8 +153,8 @@ def test_planner_rejects_out_of_range_costs():
 
 @pytest.mark.parametrize("n_workers", [1, 31, 33, 148, 256, 257, 300])
 def test_planner_random_costs(n_workers):
-    # The run walk has a one-warp kernel for up to 256 workers and a one-CTA kernel above; both
-    # must give the oracle's LPT plan bit for bit. Costs cover every bucket 1..64, skewed towards
+    # The run walk (one CTA, a thread per worker) must give the oracle's LPT plan bit for bit for
+    # worker counts below, at and above one warp and the SM count. Costs cover every bucket 1..64, skewed towards
     # small ones like the workloads', with a few thousand items so most runs are non-trivial.
     from oracle import schedule as OS
     from split_kv_lse_splitkv_b200 import SplitKV

@@ -7,6 +7,8 @@ that it returns exactly the plan of the workspace-taking splitkv_plan_lpt on two
 array keeps the previous call's contents), and that it refuses a problem too large for the array.
 This file is collected last on purpose: it runs after every other test, and also passes on its own.
 """
+import re
+
 import pytest
 import torch
 
@@ -21,7 +23,24 @@ def test_noalloc_refuses_problems_beyond_its_static_scratch():
     with pytest.raises(B.SplitKVError) as e:
         B.splitkv_plan_lpt_noalloc(fake, fake, 40_000_000, 64, 1024, fake, fake, fake, i64, fake, stream=0)
     assert e.value.code == B.ENOSPACE
-    assert "static array" in str(e.value)
+    msg = str(e.value)
+    assert "static array" in msg
+    nums = [int(x) for x in re.findall(r"\d+", msg)]
+    assert 4 << 20 in nums and any(x > 4 << 20 for x in nums), msg  # both sizes, the need above the array
+
+
+def test_noalloc_accepts_the_largest_cost_on_every_sm():
+    # max_cost 64 (chunk = 64 key tiles) on 148 queues with 200k items fits the static array: the call
+    # passes the size check and, on a host without a GPU, fails only at the device lookup (ECUDA).
+    # With a GPU these host tensors would reach a launch, so the case runs on GPU-less hosts only; the
+    # GPU test below plans a max_cost 64 problem on 148 queues through this entry point.
+    if torch.cuda.is_available():
+        pytest.skip("host-only check of the size limit")
+    fake = torch.empty(64, dtype=torch.int32)
+    i64 = torch.empty(64, dtype=torch.int64)
+    with pytest.raises(B.SplitKVError) as e:
+        B.splitkv_plan_lpt_noalloc(fake, fake, 200_000, 64, 148, fake, fake, fake, i64, fake, stream=0)
+    assert e.value.code == B.ECUDA, str(e.value)
 
 
 def _plans(name, base, seq_lens, counts, chunk):
@@ -51,6 +70,7 @@ def _plans(name, base, seq_lens, counts, chunk):
     ("small", "drafter_s32k", [5000], [7], 1024),
     ("skewed", "skewed_s256k", [262144], [256], 2048),
     ("batch", "train_4x64k", [65536] * 4, [32, 64, 96, 128], 1024),
+    ("wide_chunks", "drafter_s32k", [131072], [256], 8192),  # max_cost 64 on 148 queues
 ])
 def test_noalloc_plan_equals_workspace_plan(case):
     ref, outs, n = _plans(*case)
