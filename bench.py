@@ -95,6 +95,7 @@ class ClockSampler:
         self.stop = threading.Event()
         self.nvml = None
         self.handle = None
+        self.max_mhz = None
 
     def _open(self):
         import pynvml
@@ -116,14 +117,17 @@ class ClockSampler:
         self.handle = pynvml.nvmlDeviceGetHandleByIndex(self.device_index)
 
     def _sample(self):
+        # Two NVML queries per sample (the maximum clock is read once): each query takes a few
+        # milliseconds, so fewer queries give more samples of a short timed region.
         n = self.nvml
+        if self.max_mhz is None:
+            self.max_mhz = float(n.nvmlDeviceGetMaxClockInfo(self.handle, n.NVML_CLOCK_SM))
         sm = n.nvmlDeviceGetClockInfo(self.handle, n.NVML_CLOCK_SM)
-        mx = n.nvmlDeviceGetMaxClockInfo(self.handle, n.NVML_CLOCK_SM)
         try:
             bits = n.nvmlDeviceGetCurrentClocksEventReasons(self.handle)
         except AttributeError:
             bits = n.nvmlDeviceGetCurrentClocksThrottleReasons(self.handle)
-        self.samples.append((float(sm), float(mx), int(bits)))
+        self.samples.append((float(sm), self.max_mhz, int(bits)))
 
     def _loop(self):
         while not self.stop.wait(0.001):

@@ -68,6 +68,12 @@ extern "C" {
 /* Flags of splitkv_attn_fwd. */
 #define SPLITKV_FWD_DEFAULT 0 /* bf16 with head_dim 128: tcgen05/TMEM/TMA kernel; else SIMT fp32 */
 #define SPLITKV_FWD_SIMT 1    /* force the CUDA-core kernel (any dtype): an independent GPU cross-check */
+/* Test of the in-kernel wait limit (tensor-core path only; EUNSUPPORTED elsewhere): the first CTA
+ * (cluster) is given no item and its waits a 20 us limit instead of 2 s, so it gives up before issuing
+ * any copy or MMA and the call ends with SPLITKV_DEV_TIMEOUT in status_d; the other CTAs run their
+ * queues. The partials of the first queue are not written. The next call on the same device, with
+ * status_d cleared, computes normally. */
+#define SPLITKV_FWD_TEST_STARVE 0x100
 
 /* Problem description (host memory). */
 typedef struct {

@@ -17,7 +17,7 @@ _lib = ctypes.CDLL(LIB_PATH)
 OK, EINVAL, EUNSUPPORTED, ECUDA, ENOSPACE = 0, -1, -2, -3, -4
 DEV_ANCHOR_ORDER, DEV_ANCHOR_RANGE, DEV_BAD_COST, DEV_BAD_PLAN, DEV_TIMEOUT = 0x1, 0x2, 0x4, 0x8, 0x10
 F32, BF16 = 0, 1
-FWD_DEFAULT, FWD_SIMT = 0, 1
+FWD_DEFAULT, FWD_SIMT, FWD_TEST_STARVE = 0, 1, 0x100
 MAX_BATCH = 64
 
 _i32, _i64, _f32, _vp, _sz = ctypes.c_int32, ctypes.c_int64, ctypes.c_float, ctypes.c_void_p, ctypes.c_size_t

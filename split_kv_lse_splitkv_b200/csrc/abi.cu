@@ -196,7 +196,8 @@ SPLITKV_API int splitkv_attn_fwd(const splitkv_problem* problem, const void* q, 
     Meta m;
     int rc = build_meta(problem, &m);
     if (rc) return rc;
-    if (n_workers < 1 || n_workers > 65535 || (flags & ~SPLITKV_FWD_SIMT)) return SPLITKV_EINVAL;
+    if (n_workers < 1 || n_workers > 65535 || (flags & ~(SPLITKV_FWD_SIMT | SPLITKV_FWD_TEST_STARVE)))
+        return SPLITKV_EINVAL;
     // Query-side buffers are empty (possibly NULL) when the problem has no anchor at all.
     const bool queries = m.n_queries > 0;
     if ((queries && (!q || !kb || !vb)) || !k || !v || !item_id_d || !queue_off_d || !queue_items_d || !o_part ||
@@ -210,8 +211,9 @@ SPLITKV_API int splitkv_attn_fwd(const splitkv_problem* problem, const void* q, 
         if (!workspace_d || workspace_bytes < kFwdWorkspaceBytes) return SPLITKV_ENOSPACE;
         if (!aligned16(workspace_d)) return SPLITKV_EINVAL;
         return cuda_status(launch_fwd_tc(m, q, k, v, kb, vb, anchors_d, item_id_d, queue_off_d, queue_items_d,
-                                         n_workers, o_part, lse_part, status_d, workspace_d, st));
+                                         n_workers, o_part, lse_part, status_d, workspace_d, flags, st));
     }
+    if (flags & SPLITKV_FWD_TEST_STARVE) return SPLITKV_EUNSUPPORTED;  // a tensor-core path test
     return cuda_status(launch_fwd_simt(m, q, k, v, kb, vb, anchors_d, item_id_d, queue_off_d, queue_items_d,
                                        n_workers, o_part, lse_part, status_d, st));
 }

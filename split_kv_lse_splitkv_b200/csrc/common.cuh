@@ -115,7 +115,7 @@ cudaError_t launch_fwd_simt(const Meta& m, const void* q, const void* k, const v
 cudaError_t launch_fwd_tc(const Meta& m, const void* q, const void* k, const void* v, const void* kb, const void* vb,
                           const int32_t* anchors, const int32_t* item_id, const int32_t* queue_off,
                           const int32_t* queue_items, int32_t n_workers, void* o_part, float* lse_part,
-                          int32_t* status, void* ws, cudaStream_t st);
+                          int32_t* status, void* ws, int32_t flags, cudaStream_t st);
 bool fwd_tc_supported(const Meta& m);
 constexpr size_t kFwdWorkspaceBytes = 256;  // the tensor-core forward's pool counter
 

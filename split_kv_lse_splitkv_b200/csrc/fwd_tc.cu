@@ -59,6 +59,7 @@ constexpr int kTileBytes = 32768;  // 128 x 128 bf16, as two 128-byte-wide halve
 constexpr int kHalfBytes = 16384;
 constexpr int kKeysPerTile = 128;
 constexpr uint64_t kTimeoutNs = 2000000000ull;
+constexpr uint64_t kTestLimitNs = 20000ull;  // the starved CTA's limit in test mode (20 us)
 constexpr float kRescaleLog2 = 8.0f;
 constexpr int kSoftmaxThreads = 256;
 
@@ -162,7 +163,7 @@ __device__ __forceinline__ void exp_half(const uint32_t (&ra)[32], const uint32_
 // Returns 1 (entry in t), or -1 at the end of the sequence or on abort/timeout. `slot` is this
 // reader's progress word; a warp-wide reader (all 32 lanes in step) publishes after __syncwarp.
 __device__ __forceinline__ int ring_next(const Meta& m, Bars* bars, int32_t& idx, int slot, bool blocking,
-                                         bool warp_wide, TileRef& t, volatile int* abort_flag) {
+                                         bool warp_wide, TileRef& t, volatile int* abort_flag, uint64_t lim) {
     volatile int32_t* rw = &bars->ring_w;
     uint64_t t0 = 0;
     for (uint32_t spin = 0;; ++spin) {
@@ -192,7 +193,7 @@ __device__ __forceinline__ int ring_next(const Meta& m, Bars* bars, int32_t& idx
         if ((spin & 63u) == 63u) {
             if (*abort_flag) return -1;
             if (t0 == 0) t0 = globaltimer();
-            else if (globaltimer() - t0 > kTimeoutNs) {
+            else if (globaltimer() - t0 > lim) {
                 *abort_flag = 1;
                 return -1;
             }
@@ -206,7 +207,7 @@ __device__ __forceinline__ int ring_next(const Meta& m, Bars* bars, int32_t& idx
 __device__ void claim_items(const Meta& m, Bars* bars, const int32_t* __restrict__ anchors,
                             const int32_t* __restrict__ item_id, const int32_t* __restrict__ queue_off,
                             const int32_t* __restrict__ queue_items, int32_t* pool, int32_t* status,
-                            volatile int* abort_flag) {
+                            volatile int* abort_flag, uint64_t lim) {
     const int32_t q0 = queue_off[blockIdx.x], q1 = queue_off[blockIdx.x + 1];
     volatile int32_t* rr = bars->ring_r;
     int32_t w = 0;
@@ -219,7 +220,7 @@ __device__ void claim_items(const Meta& m, Bars* bars, const int32_t* __restrict
             int32_t lo = rr[0];
             for (int x = 1; x < kReaders; ++x) lo = min(lo, rr[x]);
             if (lo > w - kRing && (ahead <= 0 || rr[0] > w - ahead)) return true;
-            if ((spin & 63u) == 63u && (*abort_flag || globaltimer() - t0 > kTimeoutNs)) {
+            if ((spin & 63u) == 63u && (*abort_flag || globaltimer() - t0 > lim)) {
                 *abort_flag = 1;
                 return false;
             }
@@ -304,7 +305,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                   const int32_t* __restrict__ anchors, const int32_t* __restrict__ item_id,
                   const int32_t* __restrict__ queue_off, const int32_t* __restrict__ queue_items,
                   __nv_bfloat16* __restrict__ o_part, float* __restrict__ lse_part, int32_t* __restrict__ pool,
-                  int32_t* __restrict__ status) {
+                  int32_t* __restrict__ status, int32_t test_starve) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     float* stat = reinterpret_cast<float*>(smem + kOffStat);
@@ -312,6 +313,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     Bars* bars = reinterpret_cast<Bars*>(smem + kOffBar);
     volatile int* abort_flag = &bars->abort_flag;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    // Limit of every wait that can run out while work is expected (drains keep the full limit).
+    const uint64_t lim = (test_starve && blockIdx.x == 0) ? kTestLimitNs : kTimeoutNs;
 
     if (threadIdx.x == 0) {
         for (int b = 0; b < 2; ++b) {
@@ -364,9 +367,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             TileRef t;
             uint32_t k = 0, nk = 0, nv = 0;  // copies issued: Q, K, V
             bool ok = true;
-            while (ok && ring_next(m, bars, ridx, 0, true, false, t, abort_flag) == 1) {
+            while (ok && ring_next(m, bars, ridx, 0, true, false, t, abort_flag, lim) == 1) {
                 const int qb = k & 1;
-                if (k >= 2 && !mbar_wait(&bars->q_empty[qb], ((k >> 1) - 1) & 1u, abort_flag, kTimeoutNs)) {
+                if (k >= 2 && !mbar_wait(&bars->q_empty[qb], ((k >> 1) - 1) & 1u, abort_flag, lim)) {
                     ok = false;
                     break;
                 }
@@ -384,7 +387,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const int32_t row = t.self_item ? m.block * t.j
                                                     : (int32_t)(m.key_off[t.s] + (int64_t)t.c * m.chunk +
                                                                 (int64_t)tt * kKeysPerTile);
-                    if (!mbar_wait(&bars->s_full[b], ph, abort_flag, kTimeoutNs)) {  // QK(n-2) done
+                    if (!mbar_wait(&bars->s_full[b], ph, abort_flag, lim)) {  // QK(n-2) done
                         ok = false;
                         break;
                     }
@@ -393,7 +396,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tma_load_3d(kdst, mk, &bars->k_full[b], 0, t.g, row);
                     tma_load_3d(kdst + kHalfBytes, mk, &bars->k_full[b], 64, t.g, row);
                     ++nk;
-                    if (!mbar_wait(&bars->pv_done[b], ph, abort_flag, kTimeoutNs)) {  // PV(n-2) done
+                    if (!mbar_wait(&bars->pv_done[b], ph, abort_flag, lim)) {  // PV(n-2) done
                         ok = false;
                         break;
                     }
@@ -414,7 +417,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (uint32_t x = (nv > 2 ? nv - 2 : 0); x < nv; ++x)
                 mbar_wait(&bars->v_full[x & 1], (x >> 1) & 1u, &never, kTimeoutNs);
         } else if (!skip && warp == kLoadWarp && lane == 1) {
-            claim_items(m, bars, anchors, item_id, queue_off, queue_items, pool, status, abort_flag);
+            // Test mode (SPLITKV_FWD_TEST_STARVE): the first CTA's claimer publishes nothing, so every
+            // role of that CTA waits for its first item with no copy or MMA issued, and gives up.
+            if (!(test_starve && blockIdx.x == 0))
+                claim_items(m, bars, anchors, item_id, queue_off, queue_items, pool, status, abort_flag, lim);
         } else if (!skip && (warp == kMmaWarp || warp == kPvWarp) && lane == 0) {
             // Two issuers on one tensor core. QK issuer: S[n % 2] = Q K(n)^T once K(n) has landed and
             // PV(n-2) has read P(n-2) out of S[n % 2]. PV issuer: O[k % 2] += P(n) V(n) once P(n) is
@@ -433,17 +439,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             TileRef t;
             uint32_t k = 0, n = 0;
             bool ok = true;
-            while (ok && ring_next(m, bars, ridx, is_qk ? 1 : 2, true, false, t, abort_flag) == 1) {
+            while (ok && ring_next(m, bars, ridx, is_qk ? 1 : 2, true, false, t, abort_flag, lim) == 1) {
                 const int ib = k & 1;
                 if (is_qk) {
-                    if (!mbar_wait(&bars->q_full[ib], (k >> 1) & 1u, abort_flag, kTimeoutNs)) {
+                    if (!mbar_wait(&bars->q_full[ib], (k >> 1) & 1u, abort_flag, lim)) {
                         ok = false;
                         break;
                     }
                     for (int32_t tt = 0; tt < t.ntiles; ++tt, ++n) {
                         const int b = n & 1;
-                        if (!mbar_wait(&bars->k_full[b], (n >> 1) & 1u, abort_flag, kTimeoutNs) ||
-                            !mbar_wait(&bars->pv_done[b], ((n >> 1) & 1u) ^ 1u, abort_flag, kTimeoutNs)) {
+                        if (!mbar_wait(&bars->k_full[b], (n >> 1) & 1u, abort_flag, lim) ||
+                            !mbar_wait(&bars->pv_done[b], ((n >> 1) & 1u) ^ 1u, abort_flag, lim)) {
                             ok = false;
                             break;
                         }
@@ -461,10 +467,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint32_t tO = tmem + kColO + 128u * ib;
                     for (int32_t tt = 0; tt < t.ntiles; ++tt, ++n) {
                         const int b = n & 1;
-                        if (!mbar_wait(&bars->p_full[b], (n >> 1) & 1u, abort_flag, kTimeoutNs) ||
+                        if (!mbar_wait(&bars->p_full[b], (n >> 1) & 1u, abort_flag, lim) ||
                             (tt == 0 && k >= 2 &&
-                             !mbar_wait(&bars->o_free[ib], ((k >> 1) & 1u) ^ 1u, abort_flag, kTimeoutNs)) ||
-                            !mbar_wait(&bars->v_full[b], (n >> 1) & 1u, abort_flag, kTimeoutNs)) {
+                             !mbar_wait(&bars->o_free[ib], ((k >> 1) & 1u) ^ 1u, abort_flag, lim)) ||
+                            !mbar_wait(&bars->v_full[b], (n >> 1) & 1u, abort_flag, lim)) {
                             ok = false;
                             break;
                         }
@@ -499,10 +505,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             TileRef t;
             uint32_t k = 0;
             bool ok = true;
-            while (ok && ring_next(m, bars, ridx, 11 + quad, true, true, t, abort_flag) == 1) {
+            while (ok && ring_next(m, bars, ridx, 11 + quad, true, true, t, abort_flag, lim) == 1) {
                 const int ob = k & 1;
-                ok = __all_sync(0xffffffffu, mbar_wait(&bars->stat_full[ob], (k >> 1) & 1u, abort_flag, kTimeoutNs) &&
-                                                 mbar_wait(&bars->o_ready[ob], (k >> 1) & 1u, abort_flag, kTimeoutNs));
+                ok = __all_sync(0xffffffffu, mbar_wait(&bars->stat_full[ob], (k >> 1) & 1u, abort_flag, lim) &&
+                                                 mbar_wait(&bars->o_ready[ob], (k >> 1) & 1u, abort_flag, lim));
                 if (!ok) break;
                 tc_fence_after();
                 const float* sp = stat + ob * 384;
@@ -557,12 +563,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             bool ok = true;
             int32_t ridx = 0;
             TileRef t;
-            while (ok && ring_next(m, bars, ridx, 3 + warp, true, true, t, abort_flag) == 1) {
+            while (ok && ring_next(m, bars, ridx, 3 + warp, true, true, t, abort_flag, lim) == 1) {
                 const int32_t row_nvis = row_keys(m, anchors, t, r);
                 float m_l = -INFINITY, l = 0.f;  // reference max and this half's row sum (relative to m_l)
                 for (int32_t tt = 0; tt < t.ntiles; ++tt, ++n) {
                     // The whole warp leaves together on a timeout: the TMEM accesses below are collective.
-                    if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_full[n & 1], (n >> 1) & 1u, abort_flag, kTimeoutNs))) {
+                    if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_full[n & 1], (n >> 1) & 1u, abort_flag, lim))) {
                         ok = false;
                         break;
                     }
@@ -583,7 +589,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     {
                         const uint64_t t0 = globaltimer();
                         for (uint32_t spin = 0; *other_flag < (int32_t)(n + 1); ++spin) {
-                            if ((spin & 63u) == 63u && (*abort_flag || globaltimer() - t0 > kTimeoutNs)) {
+                            if ((spin & 63u) == 63u && (*abort_flag || globaltimer() - t0 > lim)) {
                                 got = false;
                                 break;
                             }
@@ -603,7 +609,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         if (__any_sync(0xffffffffu, move)) {
                             // The max moved: rescale my columns of O once PV(n-1) is complete, and my sum.
                             if (!__all_sync(0xffffffffu, mbar_wait(&bars->pv_done[(n - 1) & 1], ((n - 1) >> 1) & 1u,
-                                                                   abort_flag, kTimeoutNs))) {
+                                                                   abort_flag, lim))) {
                                 ok = false;
                                 break;
                             }
@@ -637,7 +643,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!ok) break;
                 // Hand (m, l) of item k to the epilogue; stat[k % 2] was last read for item k-2.
                 const int ob = k & 1;
-                if (k >= 2 && !mbar_wait(&bars->o_free[ob], ((k >> 1) - 1) & 1u, abort_flag, kTimeoutNs)) {
+                if (k >= 2 && !mbar_wait(&bars->o_free[ob], ((k >> 1) - 1) & 1u, abort_flag, lim)) {
                     ok = false;
                     break;
                 }
@@ -710,7 +716,7 @@ bool fwd_tc_supported(const Meta& m) {
 cudaError_t launch_fwd_tc(const Meta& m, const void* q, const void* k, const void* v, const void* kb, const void* vb,
                           const int32_t* anchors, const int32_t* item_id, const int32_t* queue_off,
                           const int32_t* queue_items, int32_t n_workers, void* o_part, float* lse_part,
-                          int32_t* status, void* ws, cudaStream_t st) {
+                          int32_t* status, void* ws, int32_t flags, cudaStream_t st) {
     CUtensorMap tq, tk, tv, tkb, tvb;
     if (m.n_queries == 0 || m.total_keys == 0) return cudaSuccess;
     if (!make_bf16_map(&tq, q, m.n_queries, m.hq, m.d, m.group, m.block * m.pack) ||
@@ -725,7 +731,8 @@ cudaError_t launch_fwd_tc(const Meta& m, const void* q, const void* k, const voi
     e = cudaMemsetAsync(pool, 0, sizeof(int32_t), st);
     if (e != cudaSuccess) return note_error(e, "cudaMemsetAsync(pool counter)");
     fwd_tc_kernel<<<n_workers, kThreads, kSmemBytes, st>>>(m, tq, tk, tv, tkb, tvb, anchors, item_id, queue_off,
-                                                           queue_items, (__nv_bfloat16*)o_part, lse_part, pool, status);
+                                                           queue_items, (__nv_bfloat16*)o_part, lse_part, pool, status,
+                                                           (flags & SPLITKV_FWD_TEST_STARVE) ? 1 : 0);
     e = cudaGetLastError();
     if (e != cudaSuccess) {
         cudaFuncAttributes fa;

@@ -141,6 +141,26 @@ def test_bad_anchors_raise_device_status():
         assert skv.status_value() & bit
 
 
+def test_in_kernel_wait_limit_returns_a_status():
+    """The forward's waits are bounded. In test mode the first CTA gets no item and a 20 us limit, so
+    every role of it waits, with no copy or MMA issued, until the limit runs out: the kernel must end,
+    raise SPLITKV_DEV_TIMEOUT and leave the context usable, so that the next call (status cleared)
+    gives exactly what a call without the test mode gives."""
+    from split_kv_lse_splitkv_b200 import DEV_TIMEOUT, FWD_TEST_STARVE
+    inp = small("starve", "drafter_s32k", [5000], [7], chunk=1024)
+    skv, dev, anchors, o_ref, lse_ref = run_forward(inp, n_workers=4)
+    skv.check_status()
+    skv.plan(anchors)
+    skv.attn_fwd(dev["q"], dev["k"], dev["v"], dev["kb"], dev["vb"], anchors, flags=FWD_TEST_STARVE)
+    torch.cuda.synchronize()
+    assert skv.status_value() & DEV_TIMEOUT, skv.status_value()
+    skv.status.zero_()
+    o, lse = skv.forward(dev["q"], dev["k"], dev["v"], dev["kb"], dev["vb"], anchors)
+    torch.cuda.synchronize()
+    skv.check_status()
+    assert torch.equal(o, o_ref) and torch.equal(lse, lse_ref)
+
+
 def test_planner_rejects_out_of_range_costs():
     from split_kv_lse_splitkv_b200 import DEV_BAD_COST, SplitKV
     skv = SplitKV([4096], [4], 32, 4, 128, chunk=1024, n_workers=8)
