@@ -211,7 +211,7 @@ def cpu_oracle_plan(inp, n_workers):
     per_sample = [inp.anchors_of(s) for s in range(len(w.seq_lens))]
     t0 = time.perf_counter()
     _, costs, _ = OS.costs_closed_form(per_sample, w.seq_lens, w.chunk, w.key_tile, w.n_kv_heads,
-                                       pack=w.blocks_per_item)
+                                       pack=w.blocks_per_item, runs=w.chunks_per_item)
     t1 = time.perf_counter()
     OS.lpt(costs.tolist(), n_workers)
     t2 = time.perf_counter()
@@ -259,12 +259,23 @@ def cpu_oracle_sample(inp, budget_s, backward):
                       f"{dt:.1f} s float64 NumPy on the host"}
 
 
+def workload_of(args):
+    """The chosen workload, with --blocks-per-item overriding its query-tile packing when given."""
+    import dataclasses
+    w = W.get(args.workload)
+    if args.blocks_per_item:
+        w = dataclasses.replace(w, blocks_per_item=args.blocks_per_item)
+    if args.chunks_per_item:
+        w = dataclasses.replace(w, chunks_per_item=args.chunks_per_item)
+    return w
+
+
 def workload_config(w, counts, n_workers, world, plan):
     """The `config` object of the JSON line: the same dict for both arms (how the steps are launched
     is reported beside it, under "launch")."""
     return {"workload": w.name, "seq_lens": list(w.seq_lens), "anchors": counts,
             "heads": f"{w.n_q_heads}q/{w.n_kv_heads}kv", "head_dim": w.head_dim, "chunk": w.chunk,
-            "blocks_per_item": w.blocks_per_item, "queues": n_workers,
+            "blocks_per_item": w.blocks_per_item, "chunks_per_item": w.chunks_per_item, "queues": n_workers,
             "l2": "flushed (256 MB write) before every timed step",
             "parallelism": f"replicas x{world}", "plan": plan}
 
@@ -273,7 +284,7 @@ def run_reference(args):
     world, rank, _ = dist_setup(args)
     if rank != 0:
         return
-    w = W.get(args.workload)
+    w = workload_of(args)
     inp = W.make_inputs(w)
     vals = []
     budget = args.ref_budget if args.ref_budget else max(1.0, 150.0 / (args.warmup + args.steps))
@@ -303,11 +314,12 @@ def run_ours(args):
     world, rank, local = dist_setup(args)
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
-    w = W.get(args.workload)
+    w = workload_of(args)
     inp = W.make_inputs(w)
     counts = [int(inp.anchor_off[i + 1] - inp.anchor_off[i]) for i in range(len(w.seq_lens))]
     skv = SplitKV(w.seq_lens, counts, w.n_q_heads, w.n_kv_heads, w.head_dim, w.block, w.chunk, w.key_tile, w.scale,
-                  w.torch_dtype, n_workers=w.n_workers, device=device, blocks_per_item=w.blocks_per_item)
+                  w.torch_dtype, n_workers=w.n_workers, device=device, blocks_per_item=w.blocks_per_item,
+                  chunks_per_item=w.chunks_per_item)
     host = {k: getattr(inp, k) for k in ("q", "k", "v", "kb", "vb", "anchors")}
     if w.backward:
         host["do"] = inp.do
@@ -457,15 +469,21 @@ def run_ours(args):
     flops, fwd_kernel_flops = useful_flops(inp, w.backward)
     value = world * flops / (ms_max * 1e-3) / 1e12
     pk, src = peaks()
+    fwd_kernel = "fwd_tc2_kernel" if int(skv.sizes.ctas_per_worker) == 2 else "fwd_tc_kernel"
     if w.dtype == "bf16":
-        roof = {"bound": "tensor", "kernel": "fwd_tc_kernel", "peak": float(pk["bf16_tflops"]),
-                "peak_source": f"{src} bf16 dense (burst)"}
+        roof = {"bound": "tensor", "kernel": fwd_kernel, "peak": float(pk["bf16_tflops"]),
+                "peak_source": f"{src} bf16 dense (burst)",
+                "frac_of_sustained_peak": None}
     else:
         # fp32 CUDA-core kernel: 148 SMs x 128 FMA lanes x 2 FLOP x 1.965 GHz.
         roof = {"bound": "alu", "kernel": "fwd_simt_kernel<float>", "peak": 148 * 128 * 2 * 1.965e9 / 1e12,
                 "peak_source": "derived fp32 FFMA peak at max SM clock"}
     achieved = fwd_kernel_flops / (fwd_ms * 1e-3) / 1e12
     peak = roof["peak"]
+    if w.dtype == "bf16":
+        # The same kernel against the measured sustained GEMM figure (clocks under the power cap), for
+        # launches long enough to run in that regime.
+        roof["frac_of_sustained_peak"] = achieved / float(pk.get("bf16_tflops_sustained", peak))
     load = naive_load if naive_load is not None else skv.load.cpu().double()
     predicted_imb = float(load.max() / load.mean() - 1.0) if load.sum() > 0 else 0.0
     csum = clocks.summary()
@@ -484,7 +502,7 @@ def run_ours(args):
             "config": workload_config(w, counts, skv.n_workers, world, args.plan),
             "launch": "eager" if graph is None else "cuda graph of the step",
             "roofline": dict(roof, achieved=achieved, unit="TFLOP/s", frac=achieved / peak,
-                             traffic=profiled_traffic("fwd_tc_kernel", w.name) if w.dtype == "bf16" else None,
+                             traffic=profiled_traffic(fwd_kernel, w.name) if w.dtype == "bf16" else None,
                              kernel_ms=fwd_ms, algorithmic_flop=fwd_kernel_flops,
                              # useful TFLOP/s over the forward plus the merge, against the same peak
                              frac_fwd_merge=fwd_kernel_flops / ((fwd_ms + merge_ms) * 1e-3) / 1e12 / peak,
@@ -523,6 +541,11 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", action="store_true",
                     help="time eagerly launched steps instead of replaying one captured CUDA graph of the step")
+    ap.add_argument("--blocks-per-item", type=int, default=0,
+                    help="query-tile packing P (blocks per item) instead of the workload's: 256-row items "
+                         "(P * 16 * G = 256) run on pairs of SMs, smaller ones on one SM")
+    ap.add_argument("--chunks-per-item", type=int, default=0,
+                    help="runs of L chunks per item (one partial per run) instead of the workload's L")
     ap.add_argument("--plan", default="lpt", choices=["lpt", "naive"],
                     help="naive: the cost-blind equal-count split instead of the LPT plan (for comparison)")
     args = ap.parse_args()

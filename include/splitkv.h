@@ -84,18 +84,25 @@ typedef struct {
     int32_t n_kv_heads;         /* Hkv, divides Hq                                                  */
     int32_t head_dim;           /* d: 128 for bf16; 8..128 (multiple of 4) for f32                  */
     int32_t block;              /* queries per draft block (16)                                     */
-    int32_t chunk;              /* context chunk C, a multiple of key_tile, chunk/key_tile <= 64    */
+    int32_t chunk;              /* context chunk C, a multiple of key_tile                          */
     int32_t key_tile;           /* Tk, the key tile of the cost model (128 in every workload)       */
     float scale;                /* score scale, normally 1/sqrt(d)                                  */
     int32_t dtype;              /* SPLITKV_F32 or SPLITKV_BF16                                      */
     int32_t blocks_per_item;    /* P: consecutive blocks of a sample sharing one query tile (0 = 1);
-                                   an item is then (sample, chunk, kv head, tile of P blocks) and
-                                   P * block * G <= 128 on the tensor-core path                     */
+                                   an item is then (sample, chunk, kv head, tile of P blocks). The
+                                   tensor-core forward runs P * block * G <= 128 on one SM per
+                                   worker and P * block * G = 256 (P even, P * block <= 128) on a
+                                   pair of SMs per worker                                            */
+    int32_t chunks_per_item;    /* L: consecutive chunks one item covers (0 = 1). An item is then
+                                   (sample, run of L chunks, kv head, query tile): its worker carries
+                                   the softmax across the run and leaves one partial per run (L times
+                                   fewer partials to write and merge). chunk_cost_d stays per chunk.
+                                   L * chunk / key_tile <= 64                                         */
 } splitkv_problem;
 
 /* Derived sizes of a problem. */
 typedef struct {
-    int64_t n_items_max;    /* every (sample, chunk, kv head, query tile) item, visible or not      */
+    int64_t n_items_max;    /* every (sample, run of chunks, kv head, query tile) item, visible or not */
     int64_t n_chunks;       /* sum_s ceil(S_s / chunk): length of chunk_cost_d                       */
     int64_t n_queries;      /* Nq                                                                     */
     int64_t total_keys;     /* sum_s S_s                                                              */
@@ -103,8 +110,11 @@ typedef struct {
     int64_t o_part_elems;   /* elements of o_part, in the problem dtype (bf16 or float32):
                                (n_items_max + n_blocks*Hkv) * rows * d                               */
     int64_t lse_part_elems; /* float32 elements of lse_part: (n_items_max + n_blocks*Hkv) * rows       */
-    int32_t max_cost;       /* chunk / key_tile: the largest item cost                                */
+    int32_t max_cost;       /* L * chunk / key_tile: the largest item cost                            */
     int32_t rows_per_item;  /* rows = P * block * G: query rows of one item (its query tile)          */
+    int32_t ctas_per_worker;/* SMs that run one worker's queue in splitkv_attn_fwd's default path: 2
+                               for 256-row items (a pair of SMs), else 1. Plan onto (SM count) /
+                               ctas_per_worker workers for one queue per SM or pair.               */
 } splitkv_sizes;
 
 /* Fill `out` for `problem`. Returns SPLITKV_EINVAL / SPLITKV_EUNSUPPORTED for a bad problem. */
@@ -113,6 +123,13 @@ int splitkv_query(const splitkv_problem *problem, splitkv_sizes *out);
 /* Bytes of scratch that splitkv_cost, splitkv_plan_lpt and splitkv_attn_bwd need for this problem
  * with `n_workers` queues (0 on a bad problem). One buffer of this size serves every call. */
 size_t splitkv_workspace_size(const splitkv_problem *problem, int32_t n_workers);
+
+/* Largest worker count whose queues all run at once on the current device in splitkv_attn_fwd's
+ * default path: the SM count for one-SM workers, the number of two-CTA clusters the device holds at
+ * once for pair workers (sizes.ctas_per_worker = 2; a GPC with an odd number of usable SMs leaves
+ * one SM unpaired). The plan should use at most this many workers: more queues than fit run in a
+ * second wave. Returns SPLITKV_ECUDA without a usable device. */
+int splitkv_max_workers(const splitkv_problem *problem, int32_t *n_workers);
 
 /* Human-readable text of a host return code (static storage). */
 const char *splitkv_strerror(int code);
@@ -195,7 +212,11 @@ int splitkv_plan_lpt_noalloc(const int32_t *item_cost_d, const int32_t *n_items_
  * item_id_d, queue_off_d and queue_items_d come from splitkv_cost and splitkv_plan_lpt.
  * On the tensor-core path each worker runs its queue, then claims self items from a shared counter
  * as it runs out of work (which SM computes a self partial varies from run to run; its value does
- * not). workspace_d: splitkv_workspace_size() bytes, 16-byte aligned (the claim counter, reset by
+ * not). With 256-row items (sizes.ctas_per_worker = 2) each worker is a pair of SMs, a two-CTA
+ * cluster that issues M = 256 tensor-core instructions over both SMs (2 * n_workers CTAs, n_workers
+ * <= 32767); its self items are (query tile of P blocks, kv head), whose rows of block x see key
+ * columns block*x .. block*x + block - 1 of one key tile of kb/vb, and each block's self partial
+ * still goes to slot n_items_max + j*Hkv + g. workspace_d: splitkv_workspace_size() bytes, 16-byte aligned (the claim counter, reset by
  * this call); the CUDA-core path, which deals self items round-robin, ignores it (may be NULL).
  * q, k, v, kb, vb and o_part must be 16-byte aligned. flags: SPLITKV_FWD_DEFAULT or
  * SPLITKV_FWD_SIMT.

@@ -21,6 +21,13 @@ Readings (the pages give neither the cost unit nor the LPT details):
   of sample s (their rows stacked, each row masked by its own block's anchor), and
   its cost counts the key tiles that any of those rows sees. P = 1 is the item of
   the lines above. Index: ``base_s + (c * Hkv + g) * ceil(n_blocks_s / P) + t``.
+* Runs of chunks (``runs`` = L >= 1, default 1). With L > 1 an item covers the L
+  consecutive chunks ``rL .. rL+L-1`` of its sample (run r: keys ``[rLC, min((r+1)LC, S))``),
+  so one worker carries the softmax of a query tile across them and leaves one partial
+  per run. Its cost counts the key tiles of the run that any of its rows sees; the chunk
+  cost stays per chunk of C keys (the sum over items of their tiles inside that chunk),
+  so it does not depend on L. Index: ``base_s + (r * Hkv + g) * n_tiles_s + t`` with
+  ``ceil(ceil(S/C) / L)`` runs. L = 1 is the item of the lines above.
 * LPT: order items by (cost descending, item index ascending); give each in turn
   to the worker with the least (load, worker index); loads start at 0; a
   worker's queue lists its items in assignment order.
@@ -36,12 +43,13 @@ import numpy as np
 
 
 def item_layout(anchor_counts: Sequence[int], seq_lens: Sequence[int], chunk: int, n_kv_heads: int,
-                pack: int = 1):
-    """Per-sample (base item index, n_chunks, n_query_tiles) and the total item count."""
+                pack: int = 1, runs: int = 1):
+    """Per-sample (base item index, n_item_chunks, n_query_tiles) and the total item count; an item
+    chunk is a run of ``runs`` chunks (the last one of a sample may be shorter)."""
     out = []
     base = 0
     for nb, S in zip(anchor_counts, seq_lens):
-        nc = -(-int(S) // chunk)
+        nc = -(-(-(-int(S) // chunk)) // runs)
         nt = -(-int(nb) // pack)
         out.append((base, nc, nt))
         base += nc * n_kv_heads * nt
@@ -49,22 +57,23 @@ def item_layout(anchor_counts: Sequence[int], seq_lens: Sequence[int], chunk: in
 
 
 def costs_bruteforce(anchors_per_sample: Sequence[Sequence[int]], seq_lens: Sequence[int], chunk: int,
-                     key_tile: int, n_kv_heads: int, group: int, block: int = 16, pack: int = 1):
+                     key_tile: int, n_kv_heads: int, group: int, block: int = 16, pack: int = 1, runs: int = 1):
     """Item costs by enumerating the boolean mask of every (query tile, key tile).
 
     Returns ``(item_ids, item_costs, chunk_costs)``: visible items in ascending
-    index order, their costs, and per-(sample, chunk) costs (flattened, sample-major).
-    For small inputs only.
+    index order, their costs, and per-(sample, chunk) costs (flattened, sample-major;
+    a chunk is ``chunk`` keys whatever ``runs`` is). For small inputs only.
     """
-    layout, _ = item_layout([len(a) for a in anchors_per_sample], seq_lens, chunk, n_kv_heads, pack)
+    layout, _ = item_layout([len(a) for a in anchors_per_sample], seq_lens, chunk, n_kv_heads, pack, runs)
+    span = chunk * runs  # keys of an item chunk (a run of chunks)
     ids, costs, chunk_costs = [], [], []
     for s, anchors in enumerate(anchors_per_sample):
-        base, nc, nt = layout[s]
+        base, nr, nt = layout[s]
         S = int(seq_lens[s])
-        for c in range(nc):
-            lo, hi = c * chunk, min((c + 1) * chunk, S)
+        per_chunk = np.zeros(-(-S // chunk), np.int64)
+        for r in range(nr):
+            lo, hi = r * span, min((r + 1) * span, S)
             keys = np.arange(lo, hi)
-            total = 0
             for g in range(n_kv_heads):
                 for t in range(nt):
                     # rows of every block of the tile; a row sees context key k iff k < its block's anchor
@@ -75,36 +84,38 @@ def costs_bruteforce(anchors_per_sample: Sequence[Sequence[int]], seq_lens: Sequ
                     for kt in range(n_tiles):
                         if mask[:, kt * key_tile:(kt + 1) * key_tile].any():
                             cost += 1
+                            per_chunk[(lo + kt * key_tile) // chunk] += 1  # the chunk holding this key tile
                     if cost:
-                        ids.append(base + (c * n_kv_heads + g) * nt + t)
+                        ids.append(base + (r * n_kv_heads + g) * nt + t)
                         costs.append(cost)
-                        total += cost
-            chunk_costs.append(total)
+        chunk_costs.extend(per_chunk.tolist())
     return np.array(ids, np.int64), np.array(costs, np.int64), np.array(chunk_costs, np.int64)
 
 
-def costs_closed_form(anchors_per_sample, seq_lens, chunk, key_tile, n_kv_heads, pack: int = 1):
-    """Same result in closed form: ``cost = ceil(clamp(a - c*C, 0, min(C, S - c*C)) / Tk)`` with ``a``
-    the largest anchor of the item's blocks (the last one: anchors ascend)."""
-    layout, _ = item_layout([len(a) for a in anchors_per_sample], seq_lens, chunk, n_kv_heads, pack)
+def costs_closed_form(anchors_per_sample, seq_lens, chunk, key_tile, n_kv_heads, pack: int = 1, runs: int = 1):
+    """Same result in closed form: ``cost = ceil(clamp(a - r*LC, 0, min(LC, S - r*LC)) / Tk)`` over the
+    item's run of L = ``runs`` chunks, with ``a`` the largest anchor of the item's blocks (the last
+    one: anchors ascend); chunk c's cost sums ``ceil(clamp(a - c*C, 0, min(C, S - c*C)) / Tk)`` over
+    the tiles and kv heads (key tiles never straddle a chunk: C is a multiple of Tk)."""
+    layout, _ = item_layout([len(a) for a in anchors_per_sample], seq_lens, chunk, n_kv_heads, pack, runs)
+    span = chunk * runs
     ids, costs, chunk_costs = [], [], []
     for s, anchors in enumerate(anchors_per_sample):
-        base, nc, nt = layout[s]
+        base, nr, nt = layout[s]
         S = int(seq_lens[s])
         a = np.asarray(anchors, np.int64)
         a_last = np.array([a[min((t + 1) * pack, len(a)) - 1] for t in range(nt)], np.int64)
-        for c in range(nc):
-            width = min(chunk, S - c * chunk)
-            nvis = np.clip(a_last - c * chunk, 0, width)
-            cost = -(-nvis // key_tile)
-            total = 0
+        for r in range(nr):
+            width = min(span, S - r * span)
+            cost = -(-np.clip(a_last - r * span, 0, width) // key_tile)
             for g in range(n_kv_heads):
                 for t in range(nt):
                     if cost[t]:
-                        ids.append(base + (c * n_kv_heads + g) * nt + t)
+                        ids.append(base + (r * n_kv_heads + g) * nt + t)
                         costs.append(int(cost[t]))
-                        total += int(cost[t])
-            chunk_costs.append(total)
+        for c in range(-(-S // chunk)):
+            width = min(chunk, S - c * chunk)
+            chunk_costs.append(int(n_kv_heads * np.sum(-(-np.clip(a_last - c * chunk, 0, width) // key_tile))))
     return np.array(ids, np.int64), np.array(costs, np.int64), np.array(chunk_costs, np.int64)
 
 

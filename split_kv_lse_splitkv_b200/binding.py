@@ -37,6 +37,7 @@ class Problem(ctypes.Structure):
         ("scale", _f32),
         ("dtype", _i32),
         ("blocks_per_item", _i32),
+        ("chunks_per_item", _i32),
     ]
 
 
@@ -51,6 +52,7 @@ class Sizes(ctypes.Structure):
         ("lse_part_elems", _i64),
         ("max_cost", _i32),
         ("rows_per_item", _i32),
+        ("ctas_per_worker", _i32),
     ]
 
 
@@ -58,6 +60,7 @@ _PP = ctypes.POINTER(Problem)
 _SIGS = {
     "splitkv_query": (_i32, [_PP, ctypes.POINTER(Sizes)]),
     "splitkv_workspace_size": (_sz, [_PP, _i32]),
+    "splitkv_max_workers": (_i32, [_PP, ctypes.POINTER(_i32)]),
     "splitkv_strerror": (ctypes.c_char_p, [_i32]),
     "splitkv_last_error": (ctypes.c_char_p, []),
     "splitkv_cost": (_i32, [_PP, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
@@ -100,11 +103,11 @@ class ProblemHolder:
 
     def __init__(self, seq_lens: Sequence[int], anchor_off: Sequence[int], n_q_heads: int, n_kv_heads: int,
                  head_dim: int, block: int, chunk: int, key_tile: int, scale: float, dtype: int,
-                 blocks_per_item: int = 1):
+                 blocks_per_item: int = 1, chunks_per_item: int = 1):
         self.seq_arr = (_i64 * len(seq_lens))(*[int(x) for x in seq_lens])
         self.off_arr = (_i32 * len(anchor_off))(*[int(x) for x in anchor_off])
         self.struct = Problem(len(seq_lens), self.seq_arr, self.off_arr, n_q_heads, n_kv_heads, head_dim, block,
-                              chunk, key_tile, float(scale), dtype, int(blocks_per_item))
+                              chunk, key_tile, float(scale), dtype, int(blocks_per_item), int(chunks_per_item))
 
     @property
     def ptr(self):
@@ -112,13 +115,13 @@ class ProblemHolder:
 
 
 def make_problem(seq_lens, anchor_off, n_q_heads, n_kv_heads, head_dim, block=16, chunk=1024, key_tile=128,
-                 scale=None, dtype=torch.bfloat16, blocks_per_item=1) -> ProblemHolder:
+                 scale=None, dtype=torch.bfloat16, blocks_per_item=1, chunks_per_item=1) -> ProblemHolder:
     code = F32 if dtype == torch.float32 else BF16 if dtype == torch.bfloat16 else None
     if code is None:
         raise SplitKVError(EUNSUPPORTED, f"dtype {dtype}")
     scale = 1.0 / math.sqrt(head_dim) if scale is None else scale
     return ProblemHolder(seq_lens, anchor_off, n_q_heads, n_kv_heads, head_dim, block, chunk, key_tile, scale, code,
-                         blocks_per_item)
+                         blocks_per_item, chunks_per_item)
 
 
 def _p(t: Optional[torch.Tensor]):
@@ -136,6 +139,13 @@ def splitkv_query(problem: ProblemHolder) -> Sizes:
     out = Sizes()
     _check(_lib.splitkv_query(problem.ptr, ctypes.byref(out)), "splitkv_query")
     return out
+
+
+def splitkv_max_workers(problem: ProblemHolder) -> int:
+    """Workers whose queues all run at once on the current device (SMs, or co-resident SM pairs)."""
+    out = _i32(0)
+    _check(_lib.splitkv_max_workers(problem.ptr, ctypes.byref(out)), "splitkv_max_workers")
+    return int(out.value)
 
 
 def splitkv_workspace_size(problem: ProblemHolder, n_workers: int) -> int:
@@ -196,7 +206,8 @@ class SplitKV:
     """
 
     def __init__(self, seq_lens, anchor_counts, n_q_heads, n_kv_heads, head_dim, block=16, chunk=1024,
-                 key_tile=128, scale=None, dtype=torch.bfloat16, n_workers=None, device="cuda", blocks_per_item=1):
+                 key_tile=128, scale=None, dtype=torch.bfloat16, n_workers=None, device="cuda", blocks_per_item=1,
+                 chunks_per_item=1):
         off = [0]
         for c in anchor_counts:
             off.append(off[-1] + int(c))
@@ -204,11 +215,13 @@ class SplitKV:
         self.dtype = dtype
         self.n_q_heads, self.n_kv_heads, self.head_dim = int(n_q_heads), int(n_kv_heads), int(head_dim)
         self.problem = make_problem(seq_lens, off, n_q_heads, n_kv_heads, head_dim, block, chunk, key_tile, scale,
-                                    dtype, blocks_per_item)
+                                    dtype, blocks_per_item, chunks_per_item)
         self.blocks_per_item = int(blocks_per_item) or 1
+        self.chunks_per_item = int(chunks_per_item) or 1
         self.sizes = splitkv_query(self.problem)
-        if n_workers is None:
-            n_workers = torch.cuda.get_device_properties(self.device).multi_processor_count
+        if n_workers is None:  # one queue per SM, or per co-resident pair of SMs for 256-row items
+            with torch.cuda.device(self.device):
+                n_workers = splitkv_max_workers(self.problem)
         self.n_workers = int(n_workers)
         s = self.sizes
         dev = self.device

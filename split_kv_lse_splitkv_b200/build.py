@@ -20,7 +20,7 @@ CSRC = os.path.join(HERE, "csrc")
 BUILD = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libsplitkv.so")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
-SOURCES = ["abi.cu", "cost.cu", "plan.cu", "fwd_simt.cu", "fwd_tc.cu", "merge.cu", "bwd.cu", "bwd_tc.cu"]
+SOURCES = ["abi.cu", "cost.cu", "plan.cu", "fwd_simt.cu", "fwd_tc.cu", "fwd_tc2.cu", "merge.cu", "bwd.cu", "bwd_tc.cu"]
 
 
 def nvcc() -> str:

@@ -31,7 +31,9 @@ int build_meta(const splitkv_problem* p, Meta* m) {
     if (p->batch < 1 || p->batch > kMaxBatch || !p->seq_len || !p->anchor_off) return SPLITKV_EINVAL;
     if (p->n_q_heads < 1 || p->n_kv_heads < 1 || p->n_q_heads % p->n_kv_heads) return SPLITKV_EINVAL;
     if (p->block < 1 || p->chunk < 1 || p->key_tile < 1 || p->head_dim < 1) return SPLITKV_EINVAL;
-    if (p->chunk % p->key_tile || p->chunk / p->key_tile > kMaxCost) return SPLITKV_EUNSUPPORTED;
+    const int32_t runs = p->chunks_per_item == 0 ? 1 : p->chunks_per_item;
+    if (runs < 1) return SPLITKV_EINVAL;
+    if (p->chunk % p->key_tile || (int64_t)p->chunk * runs / p->key_tile > kMaxCost) return SPLITKV_EUNSUPPORTED;
     if (!(p->scale > 0.f) || p->scale != p->scale) return SPLITKV_EINVAL;
     if (p->dtype != SPLITKV_F32 && p->dtype != SPLITKV_BF16) return SPLITKV_EUNSUPPORTED;
     if (p->head_dim % 4 || p->head_dim > 128 || p->head_dim < 8) return SPLITKV_EUNSUPPORTED;
@@ -43,7 +45,9 @@ int build_meta(const splitkv_problem* p, Meta* m) {
     m->group = p->n_q_heads / p->n_kv_heads;
     m->d = p->head_dim;
     m->block = p->block;
-    m->chunk = p->chunk;
+    m->chunk = p->chunk * runs;  // an item's key range: a run of `runs` chunks
+    m->cost_chunk = p->chunk;
+    m->runs = runs;
     m->key_tile = p->key_tile;
     m->rows = p->block * m->group;
     m->pack = p->blocks_per_item == 0 ? 1 : p->blocks_per_item;
@@ -58,7 +62,8 @@ int build_meta(const splitkv_problem* p, Meta* m) {
         int64_t S = p->seq_len[s];
         int32_t nb = p->anchor_off[s + 1] - p->anchor_off[s];
         if (S < 1 || nb < 0) return SPLITKV_EINVAL;
-        int64_t nc = (S + p->chunk - 1) / p->chunk;
+        int64_t nc = (S + m->chunk - 1) / m->chunk;        // item chunks
+        int64_t ncc = (S + p->chunk - 1) / p->chunk;       // cost chunks
         m->seq_len[s] = S;
         m->key_off[s] = keys;
         m->item_base[s] = items;
@@ -67,7 +72,7 @@ int build_meta(const splitkv_problem* p, Meta* m) {
         m->n_chunk_s[s] = (int32_t)nc;
         if (nc > INT32_MAX) return SPLITKV_EUNSUPPORTED;
         keys += S;
-        chunks += nc;
+        chunks += ncc;
         items += nc * m->hkv * ((nb + m->pack - 1) / m->pack);
     }
     m->key_off[p->batch] = keys;
@@ -108,6 +113,7 @@ SPLITKV_API int splitkv_query(const splitkv_problem* problem, splitkv_sizes* out
     out->lse_part_elems = (m.n_items + m.n_blocks * m.hkv) * m.rows_item;
     out->max_cost = m.chunk / m.key_tile;
     out->rows_per_item = m.rows_item;
+    out->ctas_per_worker = fwd_tc2_supported(m) ? 2 : 1;
     return SPLITKV_OK;
 }
 
@@ -121,6 +127,21 @@ SPLITKV_API size_t splitkv_workspace_size(const splitkv_problem* problem, int32_
     if (bwd_tc_workspace(m) > c) c = bwd_tc_workspace(m);
     size_t r = a > b ? a : b;
     return r > c ? r : c;
+}
+
+SPLITKV_API int splitkv_max_workers(const splitkv_problem* problem, int32_t* n_workers) {
+    clear_error();
+    Meta m;
+    int rc = build_meta(problem, &m);
+    if (rc) return rc;
+    if (!n_workers) return SPLITKV_EINVAL;
+    if (fwd_tc2_supported(m)) return cuda_status(fwd_tc2_max_workers(n_workers));
+    int dev = 0, sms = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return cuda_status(note_error(e, "cudaDeviceGetAttribute(multiprocessor count)"));
+    *n_workers = sms;
+    return SPLITKV_OK;
 }
 
 SPLITKV_API const char* splitkv_last_error(void) { return g_last_error; }
@@ -207,6 +228,13 @@ SPLITKV_API int splitkv_attn_fwd(const splitkv_problem* problem, const void* q, 
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(kb) || !aligned16(vb) || !aligned16(o_part))
         return SPLITKV_EINVAL;
     cudaStream_t st = (cudaStream_t)stream;
+    if (!(flags & SPLITKV_FWD_SIMT) && fwd_tc2_supported(m)) {
+        if (!workspace_d || workspace_bytes < kFwdWorkspaceBytes) return SPLITKV_ENOSPACE;
+        if (!aligned16(workspace_d)) return SPLITKV_EINVAL;
+        if (n_workers > 32767) return SPLITKV_EINVAL;  // two CTAs per worker
+        return cuda_status(launch_fwd_tc2(m, q, k, v, kb, vb, anchors_d, item_id_d, queue_off_d, queue_items_d,
+                                          n_workers, o_part, lse_part, status_d, workspace_d, flags, st));
+    }
     if (!(flags & SPLITKV_FWD_SIMT) && fwd_tc_supported(m)) {
         if (!workspace_d || workspace_bytes < kFwdWorkspaceBytes) return SPLITKV_ENOSPACE;
         if (!aligned16(workspace_d)) return SPLITKV_EINVAL;

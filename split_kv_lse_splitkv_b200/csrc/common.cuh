@@ -18,6 +18,10 @@ constexpr int kMaxCost = 64;  // chunk / key_tile upper bound (planner bucket co
 struct Meta {
     int32_t batch;
     int32_t hq, hkv, group, d, block, chunk, key_tile, rows;  // rows = block * group (one block)
+    // chunk is the key range of one item: a run of `runs` chunks of cost_chunk keys (runs = 1: the
+    // chunk itself). Items, partials, the forward, merge and backward work in units of `chunk`;
+    // only the per-chunk costs of the cost pass count in cost_chunk.
+    int32_t cost_chunk, runs;
     int32_t pack, rows_item;              // blocks per query tile; rows_item = pack * rows
     float scale;
     int32_t dtype;
@@ -29,9 +33,9 @@ struct Meta {
     int64_t seq_len[kMaxBatch];
     int64_t key_off[kMaxBatch + 1];       // first context row of each sample
     int64_t item_base[kMaxBatch + 1];     // first item index of each sample
-    int64_t chunk_base[kMaxBatch + 1];    // first chunk index (sample-major) of each sample
+    int64_t chunk_base[kMaxBatch + 1];    // first cost chunk (cost_chunk keys; sample-major) of each sample
     int32_t anchor_off[kMaxBatch + 1];    // first global block of each sample
-    int32_t n_chunk_s[kMaxBatch];         // ceil(S_s / chunk)
+    int32_t n_chunk_s[kMaxBatch];         // ceil(S_s / chunk): item chunks of each sample
 };
 
 // Decoded work item: query tile t of sample s (blocks b .. b + nbt - 1 of the sample) against chunk c
@@ -70,7 +74,7 @@ __host__ __device__ inline int sample_of_block(const Meta& m, int32_t j) {
     return s;
 }
 
-// Keys of chunk c that a block with anchor a sees (context keys [0, a)).
+// Keys of item chunk c (chunk keys from c * chunk) that a block with anchor a sees (context keys [0, a)).
 __host__ __device__ inline int32_t visible_in_chunk(const Meta& m, int s, int c, int32_t a) {
     int64_t lo = (int64_t)c * m.chunk;
     int64_t width = m.seq_len[s] - lo;
@@ -117,6 +121,13 @@ cudaError_t launch_fwd_tc(const Meta& m, const void* q, const void* k, const voi
                           const int32_t* queue_items, int32_t n_workers, void* o_part, float* lse_part,
                           int32_t* status, void* ws, int32_t flags, cudaStream_t st);
 bool fwd_tc_supported(const Meta& m);
+// Pairs of SMs (two-CTA clusters, cta_group::2 MMAs) for 256-row items: n_workers queues, 2 CTAs each.
+cudaError_t launch_fwd_tc2(const Meta& m, const void* q, const void* k, const void* v, const void* kb,
+                           const void* vb, const int32_t* anchors, const int32_t* item_id, const int32_t* queue_off,
+                           const int32_t* queue_items, int32_t n_workers, void* o_part, float* lse_part,
+                           int32_t* status, void* ws, int32_t flags, cudaStream_t st);
+bool fwd_tc2_supported(const Meta& m);
+cudaError_t fwd_tc2_max_workers(int32_t* out);
 constexpr size_t kFwdWorkspaceBytes = 256;  // the tensor-core forward's pool counter
 
 cudaError_t launch_merge(const Meta& m, const void* o_part, const float* lse_part, const int32_t* anchors, void* o,

@@ -2,9 +2,12 @@
 // Abstract: chunks are weighted by the attention work they actually incur).
 //
 // One thread per item (s, c, g, t) of the chunk-major index space: query tile t holds blocks
-// tP .. tP+P-1 of sample s (P = 1: one block). The cost of an item is the number of key tiles of
-// chunk c holding a key one of its rows sees; with a the tile's largest (last) anchor:
-//     nvis = clamp(a - c*C, 0, min(C, S - c*C)),  cost = ceil(nvis / Tk).
+// tP .. tP+P-1 of sample s (P = 1: one block), and c is a run of L consecutive chunks (L = 1: one
+// chunk; the item's key range is C' = L*C keys). The cost of an item is the number of key tiles of
+// its range holding a key one of its rows sees; with a the tile's largest (last) anchor:
+//     nvis = clamp(a - c*C', 0, min(C', S - c*C')),  cost = ceil(nvis / Tk).
+// Each chunk of C keys gets the item's key tiles that lie inside it (the chunk costs of the cost
+// model do not depend on L).
 // Three launches: count visible items per CTA (and validate anchors, add chunk costs), scan the
 // CTA counts, then write the compacted (item id, cost) list in ascending id order.
 #include "common.cuh"
@@ -44,7 +47,19 @@ __global__ void __launch_bounds__(kThreads) cost_count_kernel(Meta m, const int3
         }
         if (cost > 0) {
             vis = 1;
-            atomicAdd((unsigned long long*)&chunk_cost[m.chunk_base[it.s] + it.c], (unsigned long long)cost);
+            // The item's key tiles, added to the cost chunk (cost_chunk keys) that holds each of them.
+            const int32_t a = anchors[it.j + it.nbt - 1];
+            for (int32_t x = 0; x < m.runs; ++x) {
+                const int64_t cc = (int64_t)it.c * m.runs + x;  // cost chunk of the sample
+                const int64_t lo = cc * m.cost_chunk;
+                if (lo >= m.seq_len[it.s]) break;
+                int64_t n = (int64_t)a - lo, width = m.seq_len[it.s] - lo;
+                if (width > m.cost_chunk) width = m.cost_chunk;
+                n = n < 0 ? 0 : (n > width ? width : n);
+                const int64_t tiles = (n + m.key_tile - 1) / m.key_tile;
+                if (tiles > 0)
+                    atomicAdd((unsigned long long*)&chunk_cost[m.chunk_base[it.s] + cc], (unsigned long long)tiles);
+            }
         }
     }
     int32_t total;

@@ -28,7 +28,9 @@ __global__ void __launch_bounds__(kThreads) fwd_simt_kernel(Meta m, const T* __r
                                                             int32_t* __restrict__ status) {
     extern __shared__ float smem[];
     if (status_bad(status)) return;
-    const int R = m.rows_item, d = m.d, G = m.group;
+    // Rows of an item's tile, and the rows of one pass over its keys (a tile of more than 128 rows, a
+    // 256-row item, takes two passes so that its rows fit in shared memory).
+    const int RT = m.rows_item, R = RT > 128 ? 128 : RT, d = m.d, G = m.group;
     const int dp = d + 1;
     float* Qs = smem;                 // [R][d]
     float* Os = Qs + R * d;           // [R][d]
@@ -69,9 +71,10 @@ __global__ void __launch_bounds__(kThreads) fwd_simt_kernel(Meta m, const T* __r
             vp = vb;
         }
 
+        for (int r0 = 0; r0 < RT; r0 += R) {  // this pass: tile rows r0 .. r0 + R - 1
         for (int e = tid; e < R * d; e += kThreads) {
             int r = e / d, dd = e % d;
-            int i = r / G, hl = r % G;
+            int i = (r0 + r) / G, hl = (r0 + r) % G;
             int64_t row = (int64_t)m.block * it.j + i;  // rows past the tile's blocks are masked below
             Qs[e] = row < m.n_queries ? to_f32(q[(row * m.hq + (int64_t)it.g * G + hl) * d + dd]) : 0.f;
             Os[e] = 0.f;
@@ -79,7 +82,7 @@ __global__ void __launch_bounds__(kThreads) fwd_simt_kernel(Meta m, const T* __r
         for (int r = tid; r < R; r += kThreads) {
             mS[r] = -INFINITY;
             lS[r] = 0.f;
-            const int x = r / m.rows;  // block of the tile this row belongs to
+            const int x = (r0 + r) / m.rows;  // block of the tile this row belongs to
             int v = 0;
             if (e_idx >= q1) v = x == 0 ? m.block : 0;  // self item: the block's own keys, its rows only
             else if (x < it.nbt) v = visible_in_chunk(m, it.s, it.c, anchors[it.j + x]);
@@ -142,15 +145,17 @@ __global__ void __launch_bounds__(kThreads) fwd_simt_kernel(Meta m, const T* __r
         // Normalise and store in the [d/E][R][E] tile layout (E = 16 / sizeof(T) elements per 16-byte
         // group), plus the natural-log LSE.
         constexpr int E = 16 / (int)sizeof(T);
-        T* op = o_part + id * (int64_t)R * d;
+        T* op = o_part + id * (int64_t)RT * d;
         for (int e = tid; e < R * d; e += kThreads) {
             int grp = e / (R * E), rem = e % (R * E);
             int r = rem / E, ce = rem % E;
             // a row that sees no key: O = 0
-            op[e] = from_f32<T>(lS[r] > 0.f ? Os[r * d + grp * E + ce] / lS[r] : 0.f);
+            op[((int64_t)grp * RT + r0 + r) * E + ce] = from_f32<T>(lS[r] > 0.f ? Os[r * d + grp * E + ce] / lS[r] : 0.f);
         }
-        for (int r = tid; r < R; r += kThreads) lse_part[id * R + r] = lS[r] > 0.f ? mS[r] + logf(lS[r]) : -INFINITY;
+        for (int r = tid; r < R; r += kThreads)
+            lse_part[id * RT + r0 + r] = lS[r] > 0.f ? mS[r] + logf(lS[r]) : -INFINITY;
         __syncthreads();
+        }  // pass
     }
 }
 
@@ -160,7 +165,7 @@ cudaError_t launch_t(const Meta& m, const void* q, const void* k, const void* v,
                      const int32_t* queue_items, int32_t n_workers, void* o_part, float* lse_part, int32_t* status,
                      cudaStream_t st) {
     if (m.n_queries == 0) return cudaSuccess;  // no anchor: no partial to compute
-    const int R = m.rows_item, d = m.d;
+    const int R = m.rows_item > 128 ? 128 : m.rows_item, d = m.d;  // rows of one pass
     size_t smem = sizeof(float) * ((size_t)2 * R * d + kBK * (d + 1) + kBK * d + R * kBK + 4 * R);
     cudaError_t e = cudaFuncSetAttribute(fwd_simt_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;

@@ -27,7 +27,8 @@ def run_forward(inp, n_workers=None, flags=0, device="cuda"):
     w = inp.workload
     nw = n_workers if n_workers is not None else w.n_workers
     skv = SplitKV(w.seq_lens, counts_of(inp), w.n_q_heads, w.n_kv_heads, w.head_dim, w.block, w.chunk, w.key_tile,
-                  w.scale, w.torch_dtype, n_workers=nw, device=device, blocks_per_item=w.blocks_per_item)
+                  w.scale, w.torch_dtype, n_workers=nw, device=device, blocks_per_item=w.blocks_per_item,
+                  chunks_per_item=w.chunks_per_item)
     dev = {k: getattr(inp, k).to(device) for k in ("q", "k", "v", "kb", "vb")}
     anchors = inp.anchors.to(device)
     o, lse = skv.forward(dev["q"], dev["k"], dev["v"], dev["kb"], dev["vb"], anchors, flags=flags)
@@ -70,7 +71,7 @@ def check_cost_and_plan(skv, inp):
     """Costs, compacted item list, chunk costs and the LPT plan must equal the oracle bit for bit."""
     w = inp.workload
     ids, costs, chunk_costs = OS.costs_closed_form(anchors_per_sample(inp), w.seq_lens, w.chunk, w.key_tile,
-                                                   w.n_kv_heads, pack=w.blocks_per_item)
+                                                   w.n_kv_heads, pack=w.blocks_per_item, runs=w.chunks_per_item)
     n = int(skv.n_items.item())
     assert n == len(ids)
     assert skv.item_id[:n].cpu().numpy().tolist() == ids.tolist()
@@ -89,14 +90,15 @@ def check_partials(skv, inp, ids, magnitude_scaled=False):
     against the oracle's chunk-local softmax."""
     w = inp.workload
     p = oracle_problem(inp)
-    parts = OA.chunk_partials(p, w.chunk)
+    # One partial per item: over a run of chunks_per_item chunks (the oracle's chunk partials at that size).
+    parts = OA.chunk_partials(p, w.chunk * w.chunks_per_item)
     O_part, L_part = skv.o_part_view()
     O_part = O_part.float().cpu().numpy()
     L_part = L_part.cpu().numpy()
     G, R, P = w.group, w.block * w.group, w.blocks_per_item
     RT = int(skv.sizes.rows_per_item)  # rows of a partial tile: P blocks of R rows
     nb = counts_of(inp)
-    layout, _ = OS.item_layout(nb, w.seq_lens, w.chunk, w.n_kv_heads, P)
+    layout, _ = OS.item_layout(nb, w.seq_lens, w.chunk, w.n_kv_heads, P, w.chunks_per_item)
     bases = [x[0] for x in layout]
     got_O, ref_O, got_L, ref_L = [], [], [], []
     off = inp.anchor_off.tolist()
@@ -111,7 +113,7 @@ def check_partials(skv, inp, ids, magnitude_scaled=False):
         o_tile = O_part[item].transpose(1, 0, 2).reshape(RT, -1)  # [rows, d]
         for x in range(min(P, nb[s] - t * P)):
             j = off[s] + t * P + x
-            if anchors[j] <= c * w.chunk:
+            if anchors[j] <= c * w.chunk * w.chunks_per_item:
                 continue  # this block of the tile sees no key of the chunk (its rows hold O = 0, LSE = -inf)
             for hl in range(G):
                 ref_o, ref_l = parts[(s, c, j, g * G + hl)]

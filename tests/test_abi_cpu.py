@@ -61,6 +61,22 @@ def test_query_sizes():
     assert s2.o_part_elems == (s2.n_items_max + 5 * 2) * 128 * 64
 
 
+def test_query_sizes_with_runs_of_chunks():
+    # Items over runs of 3 chunks: sample 0 has ceil(4/3) = 2 runs, sample 1 ceil(2/3) = 1; the chunk costs
+    # (n_chunks) stay per chunk, the largest item cost is 3 chunks' key tiles.
+    s = B.splitkv_query(prob(seq_lens=[1000, 300], anchor_off=[0, 3, 5], n_q_heads=8, n_kv_heads=2, chunk=256,
+                             chunks_per_item=3))
+    assert s.n_items_max == 2 * 2 * 3 + 1 * 2 * 2
+    assert s.n_chunks == 6 and s.max_cost == 6
+    assert s.o_part_elems == (s.n_items_max + 5 * 2) * 64 * 64
+    with pytest.raises(B.SplitKVError) as e:  # more than 64 key tiles per item
+        B.splitkv_query(prob(chunk=128 * 32, chunks_per_item=3))
+    assert e.value.code == B.EUNSUPPORTED
+    with pytest.raises(B.SplitKVError) as e:
+        B.splitkv_query(prob(chunks_per_item=-1))
+    assert e.value.code == B.EINVAL
+
+
 def test_query_sizes_with_samples_without_anchors():
     # A sample without anchors has no block and no item; its keys still count (they sit between the
     # other samples' keys in K and V). A problem without any anchor is valid and empty.

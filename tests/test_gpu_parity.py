@@ -77,6 +77,69 @@ def test_multi_block_tiles_batch(flags):
     full_check(inp, n_workers=6, flags=flags)
 
 
+# ------------------------------------------------------------------ pairs of SMs (256-row items)
+@pytest.mark.parametrize("flags", [0, SIMT])
+@pytest.mark.parametrize("n_workers", [3, None])
+def test_pair_kernel_drafter_shape(flags, n_workers):
+    # Two 128-row blocks (G = 8) per 256-row item, one per SM of a two-CTA cluster; 7 blocks leave the
+    # last tile with one block (the peer CTA's rows are empty). None: the co-resident pair count.
+    inp = small("drafter_pair", "drafter_s32k", [5000], [7], chunk=1024, blocks_per_item=2)
+    full_check(inp, n_workers, flags)
+
+
+@pytest.mark.parametrize("hq,hkv,P", [(32, 8, 4), (8, 4, 8)])
+def test_pair_kernel_other_group_sizes(hq, hkv, P):
+    # G = 4 (two 64-row blocks per SM) and G = 2 (four 32-row blocks per SM); 9 blocks: ragged last tile.
+    inp = small("pair_groups", "skewed_s256k", [4096], [9], chunk=2048, n_q_heads=hq, n_kv_heads=hkv,
+                blocks_per_item=P)
+    full_check(inp, n_workers=5)
+
+
+def test_pair_kernel_batch_edges_and_jumps():
+    # Three samples (3, 1 and 4 blocks, ragged chunks), anchors on tile and chunk boundaries, and keys of
+    # 12x the norm that move the running max inside items.
+    w = W.scaled(W.get("drafter_s32k"), "pair_batch", [3000, 700, 5000], [3, 1, 4], chunk=1024, seed=13,
+                 blocks_per_item=2)
+    inp = W.make_inputs(w)
+    inp.anchors = torch.tensor([127, 128, 2999, 16, 1023, 1024, 1025, 4999], dtype=torch.int32)
+    for pos in (5, 2 * 128 + 10, 3700 + 1024 + 5 * 128 + 70):
+        inp.k[pos] *= 12
+    full_check(inp, n_workers=4, magnitude_scaled=True)
+
+
+def test_pair_kernel_wait_limit_returns_a_status():
+    from split_kv_lse_splitkv_b200 import DEV_TIMEOUT, FWD_TEST_STARVE
+    inp = small("pair_starve", "drafter_s32k", [5000], [7], chunk=1024, blocks_per_item=2)
+    skv, dev, anchors, o_ref, lse_ref = run_forward(inp, n_workers=4)
+    skv.check_status()
+    skv.plan(anchors)
+    skv.attn_fwd(dev["q"], dev["k"], dev["v"], dev["kb"], dev["vb"], anchors, flags=FWD_TEST_STARVE)
+    torch.cuda.synchronize()
+    assert skv.status_value() & DEV_TIMEOUT, skv.status_value()
+    skv.status.zero_()
+    o, lse = skv.forward(dev["q"], dev["k"], dev["v"], dev["kb"], dev["vb"], anchors)
+    torch.cuda.synchronize()
+    skv.check_status()
+    assert torch.equal(o, o_ref) and torch.equal(lse, lse_ref)
+
+
+# ------------------------------------------------------------------ runs of chunks per item
+@pytest.mark.parametrize("flags", [0, SIMT])
+@pytest.mark.parametrize("runs,P", [(2, 1), (3, 1), (2, 2), (3, 2)])
+def test_runs_of_chunks(flags, runs, P):
+    # Items over runs of 2 or 3 chunks of 512 keys (ragged last run, S = 5000), one SM (P = 1) or a pair
+    # of SMs (P = 2) per worker: one partial per run, chunk costs per chunk, and O/LSE as always.
+    inp = small("runs", "drafter_s32k", [5000], [7], chunk=512, blocks_per_item=P, chunks_per_item=runs)
+    full_check(inp, n_workers=5, flags=flags)
+
+
+def test_runs_of_chunks_batch_and_groups():
+    # Three samples, G = 4 with two blocks per 128-row tile, runs of 2 chunks of 1024 keys.
+    inp = small("runs_batch", "skewed_s256k", [3000, 700, 5000], [3, 1, 4], chunk=1024, blocks_per_item=2,
+                chunks_per_item=2)
+    full_check(inp, n_workers=6)
+
+
 def test_anchor_edges():
     # Anchors on key-tile and chunk boundaries, the smallest and the largest allowed anchor.
     w = W.scaled(W.get("drafter_s32k"), "edges", [2048], [8], chunk=1024)
@@ -123,6 +186,11 @@ def test_backward_other_group_sizes(hq, hkv, full_tiles):
     inp = small("bwd_groups", "train_4x64k", [2500, 1300], [3, 2], chunk=1024, n_q_heads=hq, n_kv_heads=hkv,
                 blocks_per_item=P)
     backward_check(inp, n_workers=5)
+
+
+def test_backward_runs_of_chunks():
+    # The dQ kernel walks the forward's items, here runs of 2 chunks of 512 keys.
+    backward_check(small("bwd_runs", "train_4x64k", [3000, 2048, 4096], [2, 3, 4], chunk=512, chunks_per_item=2))
 
 
 def test_backward_f32_tiny():
@@ -281,7 +349,8 @@ def test_cuda_graph_replay_matches_eager(backward):
     inp = small("graph", base, [4096, 3072], [6, 4], chunk=1024, seed=21)
     w = inp.workload
     skv = SplitKV(w.seq_lens, counts_of(inp), w.n_q_heads, w.n_kv_heads, w.head_dim, w.block, w.chunk, w.key_tile,
-                  w.scale, w.torch_dtype, n_workers=148, device="cuda", blocks_per_item=w.blocks_per_item)
+                  w.scale, w.torch_dtype, n_workers=148, device="cuda", blocks_per_item=w.blocks_per_item,
+                  chunks_per_item=w.chunks_per_item)
     names = ("q", "k", "v", "kb", "vb") + (("do",) if backward else ())
     dev = {k: getattr(inp, k).cuda() for k in names}
     anchors = inp.anchors.cuda()

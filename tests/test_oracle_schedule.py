@@ -89,6 +89,60 @@ def test_multi_block_tile_costs(seed, pack):
     assert cf[2].tolist() != [] or not seq  # chunk costs present for every chunk
 
 
+def test_chunk_runs_worked_example():
+    # Runs of chunks, worked by hand: S = 640, C = Tk = 128 (five chunks), runs of L = 2 chunks (three
+    # runs: keys [0,256), [256,512), [512,640)), one kv head, one block with anchor 300.
+    #   run 0 sees keys [0,256): 2 tiles; run 1 sees [256,300): 1 tile; run 2 sees none (dropped);
+    #   chunks 0, 1, 2 each hold one visible tile ([0,128), [128,256), [256,300)); chunks 3, 4 none.
+    for fn, kw in ((Sch.costs_bruteforce, dict(group=1)), (Sch.costs_closed_form, {})):
+        ids, costs, chunk_costs = fn([[300]], [640], 128, 128, 1, runs=2, **kw)
+        assert ids.tolist() == [0, 1]
+        assert costs.tolist() == [2, 1]
+        assert chunk_costs.tolist() == [1, 1, 1, 0, 0]
+    layout, total = Sch.item_layout([1], [640], 128, 1, runs=2)
+    assert layout == [(0, 3, 1)] and total == 3
+
+
+@pytest.mark.parametrize("seed", range(10))
+@pytest.mark.parametrize("runs", [2, 3])
+@pytest.mark.parametrize("pack", [1, 2])
+def test_chunk_run_costs(seed, runs, pack):
+    # Runs of L chunks: brute-force mask enumeration equals the closed form; the chunk costs do not
+    # depend on L; every item tile lies in exactly one chunk (item costs and chunk costs add up to the
+    # same total); and a run's cost is the sum of its chunks' one-chunk item costs (a run's visible keys
+    # are the union of its chunks' visible keys, tile-aligned).
+    rng = np.random.default_rng(2000 + seed)
+    tk = int(rng.choice([8, 16, 32]))
+    chunk = tk * int(rng.integers(1, 4))
+    hkv = int(rng.integers(1, 3))
+    seq, anchors = [], []
+    for _ in range(int(rng.integers(1, 4))):
+        S = int(rng.integers(20, 300))
+        n = int(rng.integers(0, min(6, S - 16) + 1))
+        seq.append(S)
+        anchors.append(sorted(rng.choice(np.arange(16, S), size=n, replace=False).tolist()))
+    bf = Sch.costs_bruteforce(anchors, seq, chunk, tk, hkv, group=2, block=16, pack=pack, runs=runs)
+    cf = Sch.costs_closed_form(anchors, seq, chunk, tk, hkv, pack=pack, runs=runs)
+    for x, y in zip(bf, cf):
+        assert x.tolist() == y.tolist()
+    one = Sch.costs_closed_form(anchors, seq, chunk, tk, hkv, pack=pack)
+    assert cf[2].tolist() == one[2].tolist()
+    assert int(cf[1].sum()) == int(cf[2].sum())
+    one_cost = dict(zip(one[0].tolist(), one[1].tolist()))
+    lay1, _ = Sch.item_layout([len(a) for a in anchors], seq, chunk, hkv, pack)
+    layr, _ = Sch.item_layout([len(a) for a in anchors], seq, chunk, hkv, pack, runs)
+    got = dict(zip(cf[0].tolist(), cf[1].tolist()))
+    for s in range(len(seq)):
+        (b1, nc, nt), (br, nr, _) = lay1[s], layr[s]
+        assert nr == -(-nc // runs)
+        for r in range(nr):
+            for g in range(hkv):
+                for t in range(nt):
+                    want = sum(one_cost.get(b1 + (c * hkv + g) * nt + t, 0)
+                               for c in range(r * runs, min((r + 1) * runs, nc)))
+                    assert got.get(br + (r * hkv + g) * nt + t, 0) == want
+
+
 def test_lpt_worked_example():
     g = read_golden("lpt_worked_example.txt")
     iw, qo, qi, load = Sch.lpt(g["costs"], g["n_workers"])

@@ -48,7 +48,8 @@ def _plans(name, base, seq_lens, counts, chunk):
     inp = W.make_inputs(w)
     cnt = [int(inp.anchor_off[i + 1] - inp.anchor_off[i]) for i in range(len(w.seq_lens))]
     skv = B.SplitKV(w.seq_lens, cnt, w.n_q_heads, w.n_kv_heads, w.head_dim, w.block, w.chunk, w.key_tile, w.scale,
-                    w.torch_dtype, device="cuda", blocks_per_item=w.blocks_per_item)
+                    w.torch_dtype, device="cuda", blocks_per_item=w.blocks_per_item,
+                    chunks_per_item=w.chunks_per_item)
     skv.cost(inp.anchors.cuda())
     skv.plan_lpt()
     ref = [t.clone() for t in (skv.item_worker, skv.queue_off, skv.queue_items, skv.load)]

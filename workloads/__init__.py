@@ -44,7 +44,8 @@ class Workload:
     key_tile: int = 128              # Tk, the key tile of the cost model
     backward: bool = False
     n_workers: Optional[int] = None  # None: one queue per SM of the device
-    blocks_per_item: int = 1         # consecutive blocks sharing one 128-row query tile (G < 8)
+    blocks_per_item: int = 1         # consecutive blocks sharing one query tile (128 rows on one SM, 256 on two)
+    chunks_per_item: int = 1         # consecutive chunks one item covers (one partial per run of chunks)
 
     @property
     def group(self) -> int:
