@@ -216,8 +216,9 @@ int splitkv_plan_lpt_noalloc(const int32_t *item_cost_d, const int32_t *n_items_
  * cluster that issues M = 256 tensor-core instructions over both SMs (2 * n_workers CTAs, n_workers
  * <= 32767); its self items are (query tile of P blocks, kv head), whose rows of block x see key
  * columns block*x .. block*x + block - 1 of one key tile of kb/vb, and each block's self partial
- * still goes to slot n_items_max + j*Hkv + g. workspace_d: splitkv_workspace_size() bytes, 16-byte aligned (the claim counter, reset by
- * this call); the CUDA-core path, which deals self items round-robin, ignores it (may be NULL).
+ * still goes to slot n_items_max + j*Hkv + g. workspace_d: splitkv_workspace_size() bytes, 16-byte
+ * aligned (the claim counter, reset by this call); the CUDA-core path, which deals self items
+ * round-robin, ignores it (may be NULL).
  * q, k, v, kb, vb and o_part must be 16-byte aligned. flags: SPLITKV_FWD_DEFAULT or
  * SPLITKV_FWD_SIMT.
  */
@@ -256,6 +257,49 @@ int splitkv_attn_bwd(const splitkv_problem *problem, const void *q, const void *
                      const int32_t *queue_items_d, int32_t n_workers, float *dq, float *dk, float *dv,
                      float *dkb, float *dvb, int32_t *status_d, void *workspace_d, size_t workspace_bytes,
                      void *stream);
+
+/*
+ * Context parallelism across ranks (Split-KV paper, Abstract, and its table of context-parallel
+ * methods: every rank sees all draft queries, context chunks are placed on ranks by the cost-aware
+ * LPT on their realized cost, K/V stay on the rank that owns them, and only query-sized tensors are
+ * exchanged). One step on rank r of n ranks:
+ *   1. splitkv_cost (any rank; the same anchors give the same chunk costs everywhere), chunk costs
+ *      copied to the host, splitkv_cp_plan -> chunk_rank (identical on every rank, no exchange);
+ *   2. splitkv_cost_rank (this rank's items), splitkv_plan_lpt onto this GPU's SMs, splitkv_attn_fwd
+ *      (its chunks' partials; k/v need to hold only this rank's chunks, at their global rows);
+ *   3. splitkv_lse_merge_rank -> this rank's query-sized (O_r, LSE_r);
+ *   4. an all-gather of (O_r, LSE_r) over the ranks (NCCL, by the caller);
+ *   5. splitkv_lse_merge_ranks -> O, LSE: exactly the single-GPU result.
+ * Items must lie in one chunk (chunks_per_item = 1; EUNSUPPORTED otherwise).
+ */
+
+/* LPT of chunks onto ranks, on the host: chunks in order of (cost descending, index ascending), each to
+ * the rank with the least (load, rank index); loads start at 0. chunk_cost_h: host int64[n_chunks]
+ * (splitkv_cost's chunk_cost_d, sample-major), costs >= 0. Outputs (host): chunk_rank_h int32[n_chunks],
+ * rank_load_h int64[n_ranks]. SPLITKV_EINVAL on a negative cost or bad sizes. */
+int splitkv_cp_plan(const int64_t *chunk_cost_h, int64_t n_chunks, int32_t n_ranks, int32_t *chunk_rank_h,
+                    int64_t *rank_load_h);
+
+/* splitkv_cost for rank `rank` of n_ranks: items of the chunks with chunk_rank_d[c] == rank only
+ * (chunk_rank_d: device int32[n_chunks] from splitkv_cp_plan); chunk_cost_d still counts every chunk. */
+int splitkv_cost_rank(const splitkv_problem *problem, const int32_t *anchors_d, const int32_t *chunk_rank_d,
+                      int32_t rank, int32_t n_ranks, int32_t *item_id_d, int32_t *item_cost_d,
+                      int64_t *chunk_cost_d, int32_t *n_items_d, int32_t *status_d, void *workspace_d,
+                      size_t workspace_bytes, void *stream);
+
+/* splitkv_lse_merge for rank `rank`: merges the partials of this rank's visible chunks and, for the
+ * blocks j with j % n_ranks == rank, the self partial (every rank computes all self partials; each is
+ * merged on one rank). Writes o_r [Nq, Hq, d] (problem dtype) and lse_r [Nq, Hq] (float32); a row
+ * with nothing on this rank gets O = 0, LSE = -inf. */
+int splitkv_lse_merge_rank(const splitkv_problem *problem, const void *o_part, const float *lse_part,
+                           const int32_t *anchors_d, const int32_t *chunk_rank_d, int32_t rank, int32_t n_ranks,
+                           void *o_r, float *lse_r, int32_t *status_d, void *stream);
+
+/* Exact merge of the ranks' results: o_ranks [n_ranks][Nq, Hq, d] (problem dtype), lse_ranks
+ * [n_ranks][Nq, Hq] (float32, -inf: nothing) -> o [Nq, Hq, d], lse [Nq, Hq], with
+ * L = log sum_r exp(LSE_r), O = sum_r exp(LSE_r - L) O_r. */
+int splitkv_lse_merge_ranks(const splitkv_problem *problem, int32_t n_ranks, const void *o_ranks,
+                            const float *lse_ranks, void *o, float *lse, int32_t *status_d, void *stream);
 
 #ifdef __cplusplus
 }

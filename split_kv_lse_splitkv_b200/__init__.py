@@ -16,13 +16,17 @@ _EXPORTS = (
     "DEV_ANCHOR_ORDER", "DEV_ANCHOR_RANGE", "DEV_BAD_COST", "DEV_BAD_PLAN", "DEV_TIMEOUT", "FWD_DEFAULT", "FWD_SIMT",
     "FWD_TEST_STARVE",
     "LIB_PATH", "SplitKV", "SplitKVError", "make_problem", "splitkv_attn_bwd", "splitkv_attn_fwd", "splitkv_cost",
-    "splitkv_last_error", "splitkv_lse_merge", "splitkv_max_workers", "splitkv_plan_lpt", "splitkv_plan_lpt_noalloc", "splitkv_query", "splitkv_strerror",
+    "splitkv_last_error", "splitkv_lse_merge", "splitkv_max_workers", "splitkv_cp_plan", "splitkv_cost_rank",
+    "splitkv_lse_merge_rank", "splitkv_lse_merge_ranks", "ContextParallelSplitKV", "splitkv_plan_lpt", "splitkv_plan_lpt_noalloc", "splitkv_query", "splitkv_strerror",
     "splitkv_workspace_size",
 )
 __all__ = list(_EXPORTS)
 
 
 def __getattr__(name):
+    if name == "ContextParallelSplitKV":
+        from . import cp
+        return cp.ContextParallelSplitKV
     if name in _EXPORTS:
         from . import binding
         return getattr(binding, name)

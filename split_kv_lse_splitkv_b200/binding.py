@@ -70,6 +70,10 @@ _SIGS = {
                                 _sz, _vp]),
     "splitkv_lse_merge": (_i32, [_PP, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
     "splitkv_attn_bwd": (_i32, [_PP] + [_vp] * 12 + [_i32] + [_vp] * 6 + [_vp, _sz, _vp]),
+    "splitkv_cp_plan": (_i32, [_vp, _i64, _i32, _vp, _vp]),
+    "splitkv_cost_rank": (_i32, [_PP, _vp, _vp, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "splitkv_lse_merge_rank": (_i32, [_PP, _vp, _vp, _vp, _vp, _i32, _i32, _vp, _vp, _vp, _vp]),
+    "splitkv_lse_merge_ranks": (_i32, [_PP, _i32, _vp, _vp, _vp, _vp, _vp, _vp]),
 }
 EXPORTS = tuple(_SIGS)
 for _name, (_res, _args) in _SIGS.items():
@@ -194,6 +198,34 @@ def splitkv_attn_bwd(problem, q, k, v, kb, vb, o, lse, dout, anchors, item_id, q
                                  _p(anchors), _p(item_id), _p(queue_off), _p(queue_items), int(n_workers), _p(dq),
                                  _p(dk), _p(dv), _p(dkb), _p(dvb), _p(status), _p(workspace),
                                  workspace.numel() * workspace.element_size(), _stream(stream)), "splitkv_attn_bwd")
+
+
+def splitkv_cp_plan(chunk_cost, n_ranks):
+    """Host LPT of chunks onto ranks: (chunk_rank int32[n_chunks], rank_load int64[n_ranks]) as CPU tensors."""
+    cost = torch.as_tensor(chunk_cost, dtype=torch.int64).cpu().contiguous()
+    rank = torch.empty(cost.numel(), dtype=torch.int32)
+    load = torch.empty(int(n_ranks), dtype=torch.int64)
+    _check(_lib.splitkv_cp_plan(_p(cost), int(cost.numel()), int(n_ranks), _p(rank), _p(load)), "splitkv_cp_plan")
+    return rank, load
+
+
+def splitkv_cost_rank(problem, anchors, chunk_rank, rank, n_ranks, item_id, item_cost, chunk_cost, n_items, status,
+                      workspace, stream=None):
+    _check(_lib.splitkv_cost_rank(problem.ptr, _p(anchors), _p(chunk_rank), int(rank), int(n_ranks), _p(item_id),
+                                  _p(item_cost), _p(chunk_cost), _p(n_items), _p(status), _p(workspace),
+                                  workspace.numel() * workspace.element_size(), _stream(stream)), "splitkv_cost_rank")
+
+
+def splitkv_lse_merge_rank(problem, o_part, lse_part, anchors, chunk_rank, rank, n_ranks, o_r, lse_r, status,
+                           stream=None):
+    _check(_lib.splitkv_lse_merge_rank(problem.ptr, _p(o_part), _p(lse_part), _p(anchors), _p(chunk_rank), int(rank),
+                                       int(n_ranks), _p(o_r), _p(lse_r), _p(status), _stream(stream)),
+           "splitkv_lse_merge_rank")
+
+
+def splitkv_lse_merge_ranks(problem, n_ranks, o_ranks, lse_ranks, o, lse, status, stream=None):
+    _check(_lib.splitkv_lse_merge_ranks(problem.ptr, int(n_ranks), _p(o_ranks), _p(lse_ranks), _p(o), _p(lse),
+                                        _p(status), _stream(stream)), "splitkv_lse_merge_ranks")
 
 
 # ------------------------------------------------------------------ convenience: the whole path

@@ -1,7 +1,12 @@
 // C ABI entry points: host-side validation, problem decoding and kernel launches.
 // Every check here runs before anything is enqueued, so a rejected call launches nothing.
+#include <algorithm>
 #include <cstdio>
 #include <cstring>
+#include <functional>
+#include <queue>
+#include <utility>
+#include <vector>
 
 #include "common.cuh"
 
@@ -57,6 +62,9 @@ int build_meta(const splitkv_problem* p, Meta* m) {
     m->scale = p->scale;
     m->dtype = p->dtype;
     if (p->anchor_off[0] != 0) return SPLITKV_EINVAL;
+    m->chunk_rank = nullptr;
+    m->rank = -1;  // no context parallelism unless a rank entry point sets it
+    m->n_ranks = 1;
     int64_t items = 0, keys = 0, chunks = 0;
     for (int s = 0; s < p->batch; ++s) {
         int64_t S = p->seq_len[s];
@@ -169,6 +177,87 @@ SPLITKV_API int splitkv_cost(const splitkv_problem* problem, const int32_t* anch
     if (!workspace_d || workspace_bytes < cost_workspace(m)) return SPLITKV_ENOSPACE;
     return cuda_status(launch_cost(m, anchors_d, item_id_d, item_cost_d, chunk_cost_d, n_items_d, status_d,
                                    workspace_d, (cudaStream_t)stream));
+}
+
+// ---------------------------------------------------------------- context parallelism across ranks
+SPLITKV_API int splitkv_cp_plan(const int64_t* chunk_cost_h, int64_t n_chunks, int32_t n_ranks, int32_t* chunk_rank_h,
+                                int64_t* rank_load_h) {
+    clear_error();
+    if (n_chunks < 0 || n_ranks < 1 || (n_chunks > 0 && (!chunk_cost_h || !chunk_rank_h)) || !rank_load_h)
+        return SPLITKV_EINVAL;
+    for (int64_t c = 0; c < n_chunks; ++c)
+        if (chunk_cost_h[c] < 0) return SPLITKV_EINVAL;
+    // LPT: chunks by (cost descending, index ascending), each to the least (load, rank).
+    std::vector<int64_t> order((size_t)n_chunks);
+    for (int64_t c = 0; c < n_chunks; ++c) order[(size_t)c] = c;
+    std::stable_sort(order.begin(), order.end(),
+                     [&](int64_t a, int64_t b) { return chunk_cost_h[a] > chunk_cost_h[b]; });
+    using Entry = std::pair<int64_t, int32_t>;  // (load, rank): the smallest on top
+    std::priority_queue<Entry, std::vector<Entry>, std::greater<Entry>> heap;
+    for (int32_t r = 0; r < n_ranks; ++r) {
+        heap.push({0, r});
+        rank_load_h[r] = 0;
+    }
+    for (int64_t c : order) {
+        Entry e = heap.top();
+        heap.pop();
+        chunk_rank_h[c] = e.second;
+        e.first += chunk_cost_h[c];
+        rank_load_h[e.second] = e.first;
+        heap.push(e);
+    }
+    return SPLITKV_OK;
+}
+
+namespace {
+int rank_meta(const splitkv_problem* problem, const int32_t* chunk_rank_d, int32_t rank, int32_t n_ranks, Meta* m) {
+    int rc = build_meta(problem, m);
+    if (rc) return rc;
+    if (m->runs != 1) return SPLITKV_EUNSUPPORTED;  // ranks own chunks: an item must lie in one chunk
+    if (n_ranks < 1 || rank < 0 || rank >= n_ranks || (m->n_chunks > 0 && !chunk_rank_d)) return SPLITKV_EINVAL;
+    m->chunk_rank = chunk_rank_d;
+    m->rank = rank;
+    m->n_ranks = n_ranks;
+    return SPLITKV_OK;
+}
+}  // namespace
+
+SPLITKV_API int splitkv_cost_rank(const splitkv_problem* problem, const int32_t* anchors_d, const int32_t* chunk_rank_d,
+                                  int32_t rank, int32_t n_ranks, int32_t* item_id_d, int32_t* item_cost_d,
+                                  int64_t* chunk_cost_d, int32_t* n_items_d, int32_t* status_d, void* workspace_d,
+                                  size_t workspace_bytes, void* stream) {
+    clear_error();
+    Meta m;
+    int rc = rank_meta(problem, chunk_rank_d, rank, n_ranks, &m);
+    if (rc) return rc;
+    if ((m.n_blocks && !anchors_d) || !item_id_d || !item_cost_d || !chunk_cost_d || !n_items_d || !status_d)
+        return SPLITKV_EINVAL;
+    if (!workspace_d || workspace_bytes < cost_workspace(m)) return SPLITKV_ENOSPACE;
+    return cuda_status(launch_cost(m, anchors_d, item_id_d, item_cost_d, chunk_cost_d, n_items_d, status_d,
+                                   workspace_d, (cudaStream_t)stream));
+}
+
+SPLITKV_API int splitkv_lse_merge_rank(const splitkv_problem* problem, const void* o_part, const float* lse_part,
+                                       const int32_t* anchors_d, const int32_t* chunk_rank_d, int32_t rank,
+                                       int32_t n_ranks, void* o_r, float* lse_r, int32_t* status_d, void* stream) {
+    clear_error();
+    Meta m;
+    int rc = rank_meta(problem, chunk_rank_d, rank, n_ranks, &m);
+    if (rc) return rc;
+    if (!o_part || !lse_part || (m.n_queries > 0 && (!o_r || !lse_r)) || !status_d) return SPLITKV_EINVAL;
+    if (m.n_blocks && !anchors_d) return SPLITKV_EINVAL;
+    if (!aligned16(o_part) || !aligned16(lse_part) || !aligned16(o_r)) return SPLITKV_EINVAL;
+    return cuda_status(launch_merge(m, o_part, lse_part, anchors_d, o_r, lse_r, status_d, (cudaStream_t)stream));
+}
+
+SPLITKV_API int splitkv_lse_merge_ranks(const splitkv_problem* problem, int32_t n_ranks, const void* o_ranks,
+                                        const float* lse_ranks, void* o, float* lse, int32_t* status_d, void* stream) {
+    clear_error();
+    Meta m;
+    int rc = build_meta(problem, &m);
+    if (rc) return rc;
+    if (n_ranks < 1 || !status_d || (m.n_queries > 0 && (!o_ranks || !lse_ranks || !o || !lse))) return SPLITKV_EINVAL;
+    return cuda_status(launch_merge_ranks(m, n_ranks, o_ranks, lse_ranks, o, lse, status_d, (cudaStream_t)stream));
 }
 
 SPLITKV_API int splitkv_plan_lpt(const int32_t* item_cost_d, const int32_t* n_items_d, int32_t max_items,

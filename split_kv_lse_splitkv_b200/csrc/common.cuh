@@ -36,7 +36,18 @@ struct Meta {
     int64_t chunk_base[kMaxBatch + 1];    // first cost chunk (cost_chunk keys; sample-major) of each sample
     int32_t anchor_off[kMaxBatch + 1];    // first global block of each sample
     int32_t n_chunk_s[kMaxBatch];         // ceil(S_s / chunk): item chunks of each sample
+    // Context parallelism (rank >= 0): this rank keeps only the items of the chunks it owns
+    // (chunk_rank[chunk] == rank, device int32[n_chunks]) and the self partials of the blocks j with
+    // j % n_ranks == rank. rank < 0: everything (one GPU).
+    const int32_t* chunk_rank;
+    int32_t rank, n_ranks;
 };
+
+// This rank's share of the work (always true without context parallelism).
+__device__ __forceinline__ bool owns_chunk(const Meta& m, int s, int32_t c) {
+    return m.rank < 0 || __ldg(m.chunk_rank + m.chunk_base[s] + c) == m.rank;
+}
+__device__ __forceinline__ bool owns_self(const Meta& m, int64_t j) { return m.rank < 0 || j % m.n_ranks == m.rank; }
 
 // Decoded work item: query tile t of sample s (blocks b .. b + nbt - 1 of the sample) against chunk c
 // at kv head g.
@@ -132,6 +143,8 @@ constexpr size_t kFwdWorkspaceBytes = 256;  // the tensor-core forward's pool co
 
 cudaError_t launch_merge(const Meta& m, const void* o_part, const float* lse_part, const int32_t* anchors, void* o,
                          float* lse, int32_t* status, cudaStream_t st);
+cudaError_t launch_merge_ranks(const Meta& m, int32_t n_ranks, const void* o_ranks, const float* lse_ranks, void* o,
+                               float* lse, int32_t* status, cudaStream_t st);
 
 bool bwd_tc_supported(const Meta& m);
 size_t bwd_tc_workspace(const Meta& m);

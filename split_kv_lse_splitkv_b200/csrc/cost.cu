@@ -46,7 +46,7 @@ __global__ void __launch_bounds__(kThreads) cost_count_kernel(Meta m, const int3
             }
         }
         if (cost > 0) {
-            vis = 1;
+            vis = owns_chunk(m, it.s, it.c) ? 1 : 0;  // the chunk costs count every rank's items
             // The item's key tiles, added to the cost chunk (cost_chunk keys) that holds each of them.
             const int32_t a = anchors[it.j + it.nbt - 1];
             for (int32_t x = 0; x < m.runs; ++x) {
@@ -90,7 +90,11 @@ __global__ void __launch_bounds__(kThreads) cost_write_kernel(Meta m, const int3
     __shared__ int32_t sh[33];
     const int64_t id = (int64_t)blockIdx.x * kThreads + threadIdx.x;
     int32_t cost = 0;
-    if (id < m.n_items) cost = item_cost_of(m, anchors, id, nullptr);
+    if (id < m.n_items) {
+        Item it;
+        cost = item_cost_of(m, anchors, id, &it);
+        if (!owns_chunk(m, it.s, it.c)) cost = 0;  // another rank's item
+    }
     int32_t vis = cost > 0 ? 1 : 0;
     int32_t ex = block_exclusive_scan<int32_t>(vis, sh, nullptr);
     if (vis) {

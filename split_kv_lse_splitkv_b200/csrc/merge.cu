@@ -136,13 +136,22 @@ __global__ void __launch_bounds__(kThreads, MergeShape<T>::kMinBlocks) merge_ker
     st.l = 0.f;
 #pragma unroll
     for (int u = 0; u < kVals; ++u) st.acc[u] = 0.f;
-    {
+    if (owns_self(m, j)) {
         const int64_t self = m.n_items + jg;
         float x[kVals];
         load_row<T>(op + self * tile16, RT, r, g0, ngroups, x);
         online_add(st, __ldcs(lse_part + self * RT + r), x);
     }
     int32_t c = 0;
+    if (m.rank >= 0) {  // context parallelism: only the partials of this rank's chunks
+        for (; c < nv; ++c) {
+            if (!owns_chunk(m, s, c)) continue;
+            const int64_t item = item0 + (int64_t)c * cstride;
+            float x[kVals];
+            load_row<T>(op + item * tile16, RT, rc, g0, ngroups, x);
+            online_add(st, __ldcs(lse_part + item * RT + rc), x);
+        }
+    }
     for (; c + kUnroll <= nv; c += kUnroll) {
         float x[kUnroll][kVals];
         float lp[kUnroll];
@@ -162,7 +171,7 @@ __global__ void __launch_bounds__(kThreads, MergeShape<T>::kMinBlocks) merge_ker
         online_add(st, __ldcs(lse_part + item * RT + rc), x);
     }
 
-    const float inv = 1.f / st.l;
+    const float inv = st.l > 0.f ? 1.f / st.l : 0.f;  // nothing merged (a rank without this row's keys): O = 0
     const int i = r / G, hl = r % G;
     const int64_t orow = ((int64_t)BL * j + i) * m.hq + (int64_t)g * G + hl;
     T* dst = o + orow * d + c0;
@@ -174,7 +183,43 @@ __global__ void __launch_bounds__(kThreads, MergeShape<T>::kMinBlocks) merge_ker
         for (int u = 0; u < kVals; ++u)
             if (c0 + u < d) dst[u] = from_f32<T>(st.acc[u] * inv);
     }
-    if (c0 == 0) lse[orow] = st.m + logf(st.l);
+    if (c0 == 0) lse[orow] = st.l > 0.f ? st.m + logf(st.l) : -INFINITY;
+}
+
+// Merge across ranks: o_ranks [n_ranks][rows][d] (problem dtype), lse_ranks [n_ranks][rows] float32, rows =
+// Nq * Hq; a rank's -inf row holds nothing. One thread per (row, 16 columns).
+template <typename T>
+__global__ void __launch_bounds__(kThreads) merge_ranks_kernel(int64_t rows, int32_t d, int32_t n_ranks,
+                                                              const T* __restrict__ o_ranks,
+                                                              const float* __restrict__ lse_ranks,
+                                                              T* __restrict__ o, float* __restrict__ lse,
+                                                              const int32_t* __restrict__ status) {
+    if (status_bad(status)) return;
+    const int blocks = (d + kVals - 1) / kVals;
+    const int64_t unit = (int64_t)blockIdx.x * kThreads + threadIdx.x;
+    if (unit >= rows * blocks) return;
+    const int64_t row = unit / blocks;
+    const int c0 = (int)(unit % blocks) * kVals;
+    Online st;
+    st.m = -INFINITY;
+    st.l = 0.f;
+#pragma unroll
+    for (int u = 0; u < kVals; ++u) st.acc[u] = 0.f;
+    for (int32_t r = 0; r < n_ranks; ++r) {
+        const float lp = lse_ranks[(int64_t)r * rows + row];
+        if (lp == -INFINITY) continue;
+        const T* src = o_ranks + ((int64_t)r * rows + row) * d + c0;
+        float x[kVals];
+#pragma unroll
+        for (int u = 0; u < kVals; ++u) x[u] = c0 + u < d ? to_f32(src[u]) : 0.f;
+        online_add(st, lp, x);
+    }
+    const float inv = st.l > 0.f ? 1.f / st.l : 0.f;
+    T* dst = o + row * d + c0;
+#pragma unroll
+    for (int u = 0; u < kVals; ++u)
+        if (c0 + u < d) dst[u] = from_f32<T>(st.acc[u] * inv);
+    if (c0 == 0) lse[row] = st.l > 0.f ? st.m + logf(st.l) : -INFINITY;
 }
 
 template <typename T>
@@ -191,6 +236,22 @@ cudaError_t launch_t(const Meta& m, const void* o_part, const float* lse_part, c
 }
 
 }  // namespace
+
+cudaError_t launch_merge_ranks(const Meta& m, int32_t n_ranks, const void* o_ranks, const float* lse_ranks, void* o,
+                               float* lse, int32_t* status, cudaStream_t st) {
+    const int64_t rows = m.n_queries * m.hq;
+    const int64_t units = rows * ((m.d + kVals - 1) / kVals);
+    const int64_t grid = (units + kThreads - 1) / kThreads;
+    if (grid == 0) return cudaSuccess;
+    if (grid > 0x7fffffff) return note_error(cudaErrorInvalidConfiguration, "merge_ranks: grid too large");
+    if (m.dtype == SPLITKV_F32)
+        merge_ranks_kernel<float><<<(unsigned)grid, kThreads, 0, st>>>(rows, m.d, n_ranks, (const float*)o_ranks,
+                                                                        lse_ranks, (float*)o, lse, status);
+    else
+        merge_ranks_kernel<__nv_bfloat16><<<(unsigned)grid, kThreads, 0, st>>>(
+            rows, m.d, n_ranks, (const __nv_bfloat16*)o_ranks, lse_ranks, (__nv_bfloat16*)o, lse, status);
+    return note_error(cudaGetLastError(), "launch merge_ranks_kernel");
+}
 
 cudaError_t launch_merge(const Meta& m, const void* o_part, const float* lse_part, const int32_t* anchors, void* o,
                          float* lse, int32_t* status, cudaStream_t st) {

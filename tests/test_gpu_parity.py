@@ -19,6 +19,8 @@ SIMT = 1
 
 
 def small(name, base, seq_lens, counts, chunk=None, seed=11, **kw):
+    # Items over one chunk unless a test asks for runs (the full-size workloads use runs of chunks).
+    kw.setdefault("chunks_per_item", 1)
     return W.make_inputs(W.scaled(W.get(base), name, seq_lens, counts, chunk=chunk, seed=seed, **kw))
 
 
