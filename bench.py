@@ -211,7 +211,7 @@ def cpu_oracle_plan(inp, n_workers):
     per_sample = [inp.anchors_of(s) for s in range(len(w.seq_lens))]
     t0 = time.perf_counter()
     _, costs, _ = OS.costs_closed_form(per_sample, w.seq_lens, w.chunk, w.key_tile, w.n_kv_heads,
-                                       pack=w.blocks_per_item, runs=w.chunks_per_item)
+                                       pack=w.blocks_per_item, runs=w.chunks_per_item, overhead=w.item_overhead)
     t1 = time.perf_counter()
     OS.lpt(costs.tolist(), n_workers)
     t2 = time.perf_counter()
@@ -267,6 +267,8 @@ def workload_of(args):
         w = dataclasses.replace(w, blocks_per_item=args.blocks_per_item)
     if args.chunks_per_item:
         w = dataclasses.replace(w, chunks_per_item=args.chunks_per_item)
+    if args.item_overhead >= 0:
+        w = dataclasses.replace(w, item_overhead=args.item_overhead)
     return w
 
 
@@ -275,7 +277,8 @@ def workload_config(w, counts, n_workers, world, plan):
     is reported beside it, under "launch")."""
     return {"workload": w.name, "seq_lens": list(w.seq_lens), "anchors": counts,
             "heads": f"{w.n_q_heads}q/{w.n_kv_heads}kv", "head_dim": w.head_dim, "chunk": w.chunk,
-            "blocks_per_item": w.blocks_per_item, "chunks_per_item": w.chunks_per_item, "queues": n_workers,
+            "blocks_per_item": w.blocks_per_item, "chunks_per_item": w.chunks_per_item,
+            "item_overhead": w.item_overhead, "queues": n_workers,
             "l2": "flushed (256 MB write) before every timed step",
             "parallelism": f"replicas x{world}", "plan": plan}
 
@@ -319,7 +322,7 @@ def run_ours(args):
     counts = [int(inp.anchor_off[i + 1] - inp.anchor_off[i]) for i in range(len(w.seq_lens))]
     skv = SplitKV(w.seq_lens, counts, w.n_q_heads, w.n_kv_heads, w.head_dim, w.block, w.chunk, w.key_tile, w.scale,
                   w.torch_dtype, n_workers=w.n_workers, device=device, blocks_per_item=w.blocks_per_item,
-                  chunks_per_item=w.chunks_per_item)
+                  chunks_per_item=w.chunks_per_item, item_overhead=w.item_overhead)
     host = {k: getattr(inp, k) for k in ("q", "k", "v", "kb", "vb", "anchors")}
     if w.backward:
         host["do"] = inp.do
@@ -546,6 +549,8 @@ def main():
                          "(P * 16 * G = 256) run on pairs of SMs, smaller ones on one SM")
     ap.add_argument("--chunks-per-item", type=int, default=0,
                     help="runs of L chunks per item (one partial per run) instead of the workload's L")
+    ap.add_argument("--item-overhead", type=int, default=-1,
+                    help="per-item constant of the planner's cost in key tiles instead of the workload's")
     ap.add_argument("--plan", default="lpt", choices=["lpt", "naive"],
                     help="naive: the cost-blind equal-count split instead of the LPT plan (for comparison)")
     args = ap.parse_args()

@@ -97,7 +97,11 @@ typedef struct {
                                    (sample, run of L chunks, kv head, query tile): its worker carries
                                    the softmax across the run and leaves one partial per run (L times
                                    fewer partials to write and merge). chunk_cost_d stays per chunk.
-                                   L * chunk / key_tile <= 64                                         */
+                                   L * chunk / key_tile + item_overhead <= 64                         */
+    int32_t item_overhead;      /* kappa >= 0: per-item constant of the realized cost, in key tiles (0 by
+                                   default): a visible item costs tiles + kappa in the plan, for the work
+                                   every item carries (its query tile, its partial). Chunk costs count
+                                   key tiles only                                                    */
 } splitkv_problem;
 
 /* Derived sizes of a problem. */
@@ -110,7 +114,7 @@ typedef struct {
     int64_t o_part_elems;   /* elements of o_part, in the problem dtype (bf16 or float32):
                                (n_items_max + n_blocks*Hkv) * rows * d                               */
     int64_t lse_part_elems; /* float32 elements of lse_part: (n_items_max + n_blocks*Hkv) * rows       */
-    int32_t max_cost;       /* L * chunk / key_tile: the largest item cost                            */
+    int32_t max_cost;       /* L * chunk / key_tile + item_overhead: the largest item cost            */
     int32_t rows_per_item;  /* rows = P * block * G: query rows of one item (its query tile)          */
     int32_t ctas_per_worker;/* SMs that run one worker's queue in splitkv_attn_fwd's default path: 2
                                for 256-row items (a pair of SMs), else 1. Plan onto (SM count) /

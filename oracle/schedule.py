@@ -28,6 +28,10 @@ Readings (the pages give neither the cost unit nor the LPT details):
   cost stays per chunk of C keys (the sum over items of their tiles inside that chunk),
   so it does not depend on L. Index: ``base_s + (r * Hkv + g) * n_tiles_s + t`` with
   ``ceil(ceil(S/C) / L)`` runs. L = 1 is the item of the lines above.
+* Per-item constant (``overhead`` = kappa >= 0, default 0). The realized cost of a visible
+  item may add a fixed kappa (in key-tile units) for the work every item carries whatever
+  its length (loading its query tile, writing its partial): cost = tiles + kappa. Chunk
+  costs count key tiles only. kappa = 0 is the item cost of the lines above.
 * LPT: order items by (cost descending, item index ascending); give each in turn
   to the worker with the least (load, worker index); loads start at 0; a
   worker's queue lists its items in assignment order.
@@ -57,7 +61,8 @@ def item_layout(anchor_counts: Sequence[int], seq_lens: Sequence[int], chunk: in
 
 
 def costs_bruteforce(anchors_per_sample: Sequence[Sequence[int]], seq_lens: Sequence[int], chunk: int,
-                     key_tile: int, n_kv_heads: int, group: int, block: int = 16, pack: int = 1, runs: int = 1):
+                     key_tile: int, n_kv_heads: int, group: int, block: int = 16, pack: int = 1, runs: int = 1,
+                     overhead: int = 0):
     """Item costs by enumerating the boolean mask of every (query tile, key tile).
 
     Returns ``(item_ids, item_costs, chunk_costs)``: visible items in ascending
@@ -87,12 +92,13 @@ def costs_bruteforce(anchors_per_sample: Sequence[Sequence[int]], seq_lens: Sequ
                             per_chunk[(lo + kt * key_tile) // chunk] += 1  # the chunk holding this key tile
                     if cost:
                         ids.append(base + (r * n_kv_heads + g) * nt + t)
-                        costs.append(cost)
+                        costs.append(cost + overhead)
         chunk_costs.extend(per_chunk.tolist())
     return np.array(ids, np.int64), np.array(costs, np.int64), np.array(chunk_costs, np.int64)
 
 
-def costs_closed_form(anchors_per_sample, seq_lens, chunk, key_tile, n_kv_heads, pack: int = 1, runs: int = 1):
+def costs_closed_form(anchors_per_sample, seq_lens, chunk, key_tile, n_kv_heads, pack: int = 1, runs: int = 1,
+                      overhead: int = 0):
     """Same result in closed form: ``cost = ceil(clamp(a - r*LC, 0, min(LC, S - r*LC)) / Tk)`` over the
     item's run of L = ``runs`` chunks, with ``a`` the largest anchor of the item's blocks (the last
     one: anchors ascend); chunk c's cost sums ``ceil(clamp(a - c*C, 0, min(C, S - c*C)) / Tk)`` over
@@ -112,7 +118,7 @@ def costs_closed_form(anchors_per_sample, seq_lens, chunk, key_tile, n_kv_heads,
                 for t in range(nt):
                     if cost[t]:
                         ids.append(base + (r * n_kv_heads + g) * nt + t)
-                        costs.append(int(cost[t]))
+                        costs.append(int(cost[t]) + overhead)
         for c in range(-(-S // chunk)):
             width = min(chunk, S - c * chunk)
             chunk_costs.append(int(n_kv_heads * np.sum(-(-np.clip(a_last - c * chunk, 0, width) // key_tile))))

@@ -38,6 +38,7 @@ class Problem(ctypes.Structure):
         ("dtype", _i32),
         ("blocks_per_item", _i32),
         ("chunks_per_item", _i32),
+        ("item_overhead", _i32),
     ]
 
 
@@ -107,11 +108,12 @@ class ProblemHolder:
 
     def __init__(self, seq_lens: Sequence[int], anchor_off: Sequence[int], n_q_heads: int, n_kv_heads: int,
                  head_dim: int, block: int, chunk: int, key_tile: int, scale: float, dtype: int,
-                 blocks_per_item: int = 1, chunks_per_item: int = 1):
+                 blocks_per_item: int = 1, chunks_per_item: int = 1, item_overhead: int = 0):
         self.seq_arr = (_i64 * len(seq_lens))(*[int(x) for x in seq_lens])
         self.off_arr = (_i32 * len(anchor_off))(*[int(x) for x in anchor_off])
         self.struct = Problem(len(seq_lens), self.seq_arr, self.off_arr, n_q_heads, n_kv_heads, head_dim, block,
-                              chunk, key_tile, float(scale), dtype, int(blocks_per_item), int(chunks_per_item))
+                              chunk, key_tile, float(scale), dtype, int(blocks_per_item), int(chunks_per_item),
+                              int(item_overhead))
 
     @property
     def ptr(self):
@@ -119,13 +121,14 @@ class ProblemHolder:
 
 
 def make_problem(seq_lens, anchor_off, n_q_heads, n_kv_heads, head_dim, block=16, chunk=1024, key_tile=128,
-                 scale=None, dtype=torch.bfloat16, blocks_per_item=1, chunks_per_item=1) -> ProblemHolder:
+                 scale=None, dtype=torch.bfloat16, blocks_per_item=1, chunks_per_item=1,
+                 item_overhead=0) -> ProblemHolder:
     code = F32 if dtype == torch.float32 else BF16 if dtype == torch.bfloat16 else None
     if code is None:
         raise SplitKVError(EUNSUPPORTED, f"dtype {dtype}")
     scale = 1.0 / math.sqrt(head_dim) if scale is None else scale
     return ProblemHolder(seq_lens, anchor_off, n_q_heads, n_kv_heads, head_dim, block, chunk, key_tile, scale, code,
-                         blocks_per_item, chunks_per_item)
+                         blocks_per_item, chunks_per_item, item_overhead)
 
 
 def _p(t: Optional[torch.Tensor]):
@@ -239,7 +242,7 @@ class SplitKV:
 
     def __init__(self, seq_lens, anchor_counts, n_q_heads, n_kv_heads, head_dim, block=16, chunk=1024,
                  key_tile=128, scale=None, dtype=torch.bfloat16, n_workers=None, device="cuda", blocks_per_item=1,
-                 chunks_per_item=1):
+                 chunks_per_item=1, item_overhead=0):
         off = [0]
         for c in anchor_counts:
             off.append(off[-1] + int(c))
@@ -247,7 +250,7 @@ class SplitKV:
         self.dtype = dtype
         self.n_q_heads, self.n_kv_heads, self.head_dim = int(n_q_heads), int(n_kv_heads), int(head_dim)
         self.problem = make_problem(seq_lens, off, n_q_heads, n_kv_heads, head_dim, block, chunk, key_tile, scale,
-                                    dtype, blocks_per_item, chunks_per_item)
+                                    dtype, blocks_per_item, chunks_per_item, item_overhead)
         self.blocks_per_item = int(blocks_per_item) or 1
         self.chunks_per_item = int(chunks_per_item) or 1
         self.sizes = splitkv_query(self.problem)

@@ -37,8 +37,9 @@ int build_meta(const splitkv_problem* p, Meta* m) {
     if (p->n_q_heads < 1 || p->n_kv_heads < 1 || p->n_q_heads % p->n_kv_heads) return SPLITKV_EINVAL;
     if (p->block < 1 || p->chunk < 1 || p->key_tile < 1 || p->head_dim < 1) return SPLITKV_EINVAL;
     const int32_t runs = p->chunks_per_item == 0 ? 1 : p->chunks_per_item;
-    if (runs < 1) return SPLITKV_EINVAL;
-    if (p->chunk % p->key_tile || (int64_t)p->chunk * runs / p->key_tile > kMaxCost) return SPLITKV_EUNSUPPORTED;
+    if (runs < 1 || p->item_overhead < 0) return SPLITKV_EINVAL;
+    if (p->chunk % p->key_tile || (int64_t)p->chunk * runs / p->key_tile + p->item_overhead > kMaxCost)
+        return SPLITKV_EUNSUPPORTED;
     if (!(p->scale > 0.f) || p->scale != p->scale) return SPLITKV_EINVAL;
     if (p->dtype != SPLITKV_F32 && p->dtype != SPLITKV_BF16) return SPLITKV_EUNSUPPORTED;
     if (p->head_dim % 4 || p->head_dim > 128 || p->head_dim < 8) return SPLITKV_EUNSUPPORTED;
@@ -53,6 +54,7 @@ int build_meta(const splitkv_problem* p, Meta* m) {
     m->chunk = p->chunk * runs;  // an item's key range: a run of `runs` chunks
     m->cost_chunk = p->chunk;
     m->runs = runs;
+    m->item_overhead = p->item_overhead;
     m->key_tile = p->key_tile;
     m->rows = p->block * m->group;
     m->pack = p->blocks_per_item == 0 ? 1 : p->blocks_per_item;
@@ -119,7 +121,7 @@ SPLITKV_API int splitkv_query(const splitkv_problem* problem, splitkv_sizes* out
     out->n_blocks = m.n_blocks;
     out->o_part_elems = (m.n_items + m.n_blocks * m.hkv) * m.rows_item * m.d;
     out->lse_part_elems = (m.n_items + m.n_blocks * m.hkv) * m.rows_item;
-    out->max_cost = m.chunk / m.key_tile;
+    out->max_cost = m.chunk / m.key_tile + m.item_overhead;
     out->rows_per_item = m.rows_item;
     out->ctas_per_worker = fwd_tc2_supported(m) ? 2 : 1;
     return SPLITKV_OK;
@@ -129,7 +131,7 @@ SPLITKV_API size_t splitkv_workspace_size(const splitkv_problem* problem, int32_
     Meta m;
     if (build_meta(problem, &m) || n_workers < 1 || n_workers > 1024) return 0;
     size_t a = cost_workspace(m);
-    size_t b = plan_workspace((int32_t)m.n_items, m.chunk / m.key_tile, n_workers);
+    size_t b = plan_workspace((int32_t)m.n_items, m.chunk / m.key_tile + m.item_overhead, n_workers);
     size_t c = bwd_workspace(m);
     if (kFwdWorkspaceBytes > c) c = kFwdWorkspaceBytes;
     if (bwd_tc_workspace(m) > c) c = bwd_tc_workspace(m);

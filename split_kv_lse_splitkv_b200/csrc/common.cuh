@@ -22,6 +22,7 @@ struct Meta {
     // chunk itself). Items, partials, the forward, merge and backward work in units of `chunk`;
     // only the per-chunk costs of the cost pass count in cost_chunk.
     int32_t cost_chunk, runs;
+    int32_t item_overhead;  // per-item constant of the realized cost (key-tile units): cost = tiles + this
     int32_t pack, rows_item;              // blocks per query tile; rows_item = pack * rows
     float scale;
     int32_t dtype;

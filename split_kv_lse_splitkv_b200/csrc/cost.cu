@@ -95,6 +95,7 @@ __global__ void __launch_bounds__(kThreads) cost_write_kernel(Meta m, const int3
         cost = item_cost_of(m, anchors, id, &it);
         if (!owns_chunk(m, it.s, it.c)) cost = 0;  // another rank's item
     }
+    if (cost > 0) cost += m.item_overhead;  // the per-item constant of the realized cost
     int32_t vis = cost > 0 ? 1 : 0;
     int32_t ex = block_exclusive_scan<int32_t>(vis, sh, nullptr);
     if (vis) {

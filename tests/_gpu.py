@@ -28,7 +28,7 @@ def run_forward(inp, n_workers=None, flags=0, device="cuda"):
     nw = n_workers if n_workers is not None else w.n_workers
     skv = SplitKV(w.seq_lens, counts_of(inp), w.n_q_heads, w.n_kv_heads, w.head_dim, w.block, w.chunk, w.key_tile,
                   w.scale, w.torch_dtype, n_workers=nw, device=device, blocks_per_item=w.blocks_per_item,
-                  chunks_per_item=w.chunks_per_item)
+                  chunks_per_item=w.chunks_per_item, item_overhead=w.item_overhead)
     dev = {k: getattr(inp, k).to(device) for k in ("q", "k", "v", "kb", "vb")}
     anchors = inp.anchors.to(device)
     o, lse = skv.forward(dev["q"], dev["k"], dev["v"], dev["kb"], dev["vb"], anchors, flags=flags)
@@ -71,7 +71,8 @@ def check_cost_and_plan(skv, inp):
     """Costs, compacted item list, chunk costs and the LPT plan must equal the oracle bit for bit."""
     w = inp.workload
     ids, costs, chunk_costs = OS.costs_closed_form(anchors_per_sample(inp), w.seq_lens, w.chunk, w.key_tile,
-                                                   w.n_kv_heads, pack=w.blocks_per_item, runs=w.chunks_per_item)
+                                                   w.n_kv_heads, pack=w.blocks_per_item, runs=w.chunks_per_item,
+                                                   overhead=w.item_overhead)
     n = int(skv.n_items.item())
     assert n == len(ids)
     assert skv.item_id[:n].cpu().numpy().tolist() == ids.tolist()

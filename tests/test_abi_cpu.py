@@ -75,6 +75,14 @@ def test_query_sizes_with_runs_of_chunks():
     with pytest.raises(B.SplitKVError) as e:
         B.splitkv_query(prob(chunks_per_item=-1))
     assert e.value.code == B.EINVAL
+    # A per-item constant of the cost raises the largest cost by itself.
+    assert B.splitkv_query(prob(chunk=256, chunks_per_item=3, item_overhead=5)).max_cost == 6 + 5
+    with pytest.raises(B.SplitKVError) as e:
+        B.splitkv_query(prob(chunk=128 * 32, chunks_per_item=2, item_overhead=1))
+    assert e.value.code == B.EUNSUPPORTED
+    with pytest.raises(B.SplitKVError) as e:
+        B.splitkv_query(prob(item_overhead=-1))
+    assert e.value.code == B.EINVAL
 
 
 def test_query_sizes_with_samples_without_anchors():

@@ -135,6 +135,13 @@ def test_runs_of_chunks(flags, runs, P):
     full_check(inp, n_workers=5, flags=flags)
 
 
+def test_item_overhead_plan():
+    # The per-item constant of the cost: costs and the LPT plan equal the oracle's bit for bit, and the
+    # forward is unchanged by it.
+    inp = small("overhead", "drafter_s32k", [5000, 3000], [7, 4], chunk=512, chunks_per_item=2, item_overhead=3)
+    full_check(inp, n_workers=9)
+
+
 def test_runs_of_chunks_batch_and_groups():
     # Three samples, G = 4 with two blocks per 128-row tile, runs of 2 chunks of 1024 keys.
     inp = small("runs_batch", "skewed_s256k", [3000, 700, 5000], [3, 1, 4], chunk=1024, blocks_per_item=2,

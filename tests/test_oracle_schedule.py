@@ -143,6 +143,30 @@ def test_chunk_run_costs(seed, runs, pack):
                     assert got.get(br + (r * hkv + g) * nt + t, 0) == want
 
 
+@pytest.mark.parametrize("seed", range(6))
+@pytest.mark.parametrize("overhead", [1, 3])
+def test_item_overhead_costs(seed, overhead):
+    # The per-item constant: brute force equals the closed form; every visible item (and only those)
+    # costs exactly kappa more than without it; the chunk costs do not change.
+    rng = np.random.default_rng(3000 + seed)
+    tk = int(rng.choice([8, 16]))
+    chunk = tk * int(rng.integers(1, 4))
+    seq, anchors = [], []
+    for _ in range(int(rng.integers(1, 3))):
+        S = int(rng.integers(30, 250))
+        n = int(rng.integers(1, min(5, S - 16) + 1))
+        seq.append(S)
+        anchors.append(sorted(rng.choice(np.arange(16, S), size=n, replace=False).tolist()))
+    bf = Sch.costs_bruteforce(anchors, seq, chunk, tk, 2, group=2, block=16, pack=2, runs=2, overhead=overhead)
+    cf = Sch.costs_closed_form(anchors, seq, chunk, tk, 2, pack=2, runs=2, overhead=overhead)
+    base = Sch.costs_closed_form(anchors, seq, chunk, tk, 2, pack=2, runs=2)
+    for x, y in zip(bf, cf):
+        assert x.tolist() == y.tolist()
+    assert cf[0].tolist() == base[0].tolist()
+    assert (cf[1] - base[1]).tolist() == [overhead] * len(base[1])
+    assert cf[2].tolist() == base[2].tolist()
+
+
 def test_lpt_worked_example():
     g = read_golden("lpt_worked_example.txt")
     iw, qo, qi, load = Sch.lpt(g["costs"], g["n_workers"])

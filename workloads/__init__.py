@@ -46,6 +46,7 @@ class Workload:
     n_workers: Optional[int] = None  # None: one queue per SM of the device
     blocks_per_item: int = 1         # consecutive blocks sharing one query tile (128 rows on one SM, 256 on two)
     chunks_per_item: int = 1         # consecutive chunks one item covers (one partial per run of chunks)
+    item_overhead: int = 0           # per-item constant of the planner's cost, in key tiles
 
     @property
     def group(self) -> int:
