@@ -43,8 +43,9 @@ def test_noalloc_accepts_the_largest_cost_on_every_sm():
     assert e.value.code == B.ECUDA, str(e.value)
 
 
-def _plans(name, base, seq_lens, counts, chunk):
-    w = W.scaled(W.get(base), name, seq_lens, counts, chunk=chunk, seed=21)
+def _plans(name, base, seq_lens, counts, chunk, runs=None):
+    w = W.scaled(W.get(base), name, seq_lens, counts, chunk=chunk, seed=21,
+                 **({} if runs is None else {"chunks_per_item": runs}))
     inp = W.make_inputs(w)
     cnt = [int(inp.anchor_off[i + 1] - inp.anchor_off[i]) for i in range(len(w.seq_lens))]
     skv = B.SplitKV(w.seq_lens, cnt, w.n_q_heads, w.n_kv_heads, w.head_dim, w.block, w.chunk, w.key_tile, w.scale,
@@ -71,7 +72,7 @@ def _plans(name, base, seq_lens, counts, chunk):
     ("small", "drafter_s32k", [5000], [7], 1024),
     ("skewed", "skewed_s256k", [262144], [256], 2048),
     ("batch", "train_4x64k", [65536] * 4, [32, 64, 96, 128], 1024),
-    ("wide_chunks", "drafter_s32k", [131072], [256], 8192),  # max_cost 64 on 148 queues
+    ("wide_chunks", "drafter_s32k", [131072], [256], 8192, 1),  # max_cost 64 on 148 queues
 ])
 def test_noalloc_plan_equals_workspace_plan(case):
     ref, outs, n = _plans(*case)
