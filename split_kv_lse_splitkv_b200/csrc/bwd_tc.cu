@@ -47,7 +47,7 @@ constexpr int kHalfBytes = 16384;
 constexpr int kKeys = 128;
 constexpr uint64_t kTimeoutNs = 2000000000ull;
 constexpr float kLog2e = 1.4426950408889634f;
-constexpr uint32_t kIdescSS = umma_idesc_bf16_f32(128, 128, false, false);  // both operands K-major
+constexpr uint32_t kIdescSS64 = umma_idesc_bf16_f32(128, 64, false, false);  // N = 64 query rows (one step)
 constexpr uint32_t kIdescTS = umma_idesc_bf16_f32(128, 128, false, true);   // B MN-major
 
 // Per-row constants of one (block j, kv head g) query tile, rows r = i*G + hl contiguous:
@@ -87,8 +87,8 @@ constexpr int kKvOffBar = kKvOffRows + 2 * 2 * 128 * 4;
 struct KvBars {
     uint64_t kv_full;
     uint64_t qd_full[2], qd_empty[2];  // Q_b, dO_b, rows of pair p in slot p % 2
-    uint64_t s_full;                   // S^T, dP^T of the current pair complete (one commit per issuer)
-    uint64_t p_half[2];                // P^T, dS^T of query rows 64h .. 64h+63 written
+    uint64_t s_full[2];                // S^T, dP^T of step u (parity u % 2) complete (one commit per issuer)
+    uint64_t p_full[2];                // P^T, dS^T of step u written (8 elementwise warps)
     uint64_t acc_done;                 // every MMA complete: dV, dK final
     uint64_t drain[2];
     uint32_t tmem_base;
@@ -142,6 +142,10 @@ __global__ void __launch_bounds__(kKvThreads, 1)
         krow = (int64_t)m.block * j;
     }
     const int32_t np = hi - lo;
+    // Each pair runs as steps of 64 query rows (two for a block of more than 64 rows), so that S^T and
+    // dP^T are double-buffered in TMEM and the tensor core computes step u while the elementwise warps
+    // work on step u - 1.
+    const int32_t steps = m.rows > 64 ? 2 : 1;
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -157,9 +161,10 @@ __global__ void __launch_bounds__(kKvThreads, 1)
             mbar_init(&bars->qd_full[b], 1);
             mbar_init(&bars->qd_empty[b], 2);
         }
-        mbar_init(&bars->s_full, 2);
-        mbar_init(&bars->p_half[0], 128);
-        mbar_init(&bars->p_half[1], 128);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&bars->s_full[b], 2);
+            mbar_init(&bars->p_full[b], 8);
+        }
         mbar_init(&bars->acc_done, 2);
         mbar_init(&bars->drain[0], 1);
         mbar_init(&bars->drain[1], 1);
@@ -229,36 +234,48 @@ __global__ void __launch_bounds__(kKvThreads, 1)
             tc_fence_after();
             const uint64_t dA1 = umma_desc_sw128(smem_u32(smem + (isA ? kKvOffK : kKvOffV)), 16, 1024);
             const uint32_t t1 = isA ? tS : tdP, t2 = isA ? tdV : tdK;
-            for (int32_t p = 0; ok && p < np; ++p) {
+            // First GEMM of step u: S^T(u) = K Q_h^T  /  dP^T(u) = V dO_h^T into buffer u % 2 (64 columns),
+            // B = the step's 64 query rows of Q_b / dO_b (K-major, rows 64h .. of the slot's tile).
+            auto first = [&](int32_t u) -> bool {
+                const int32_t p = u / steps, h = u % steps;
                 const int slot = p & 1;
-                const uint32_t aq = smem_u32(smem + kKvOffQ + slot * kTileBytes);
-                const uint32_t ado = smem_u32(smem + kKvOffDo + slot * kTileBytes);
-                // First GEMM: B = Q_b (A) or dO_b (B), K-major; second: B = dO_b (A) or Q_b (B), MN-major.
-                const uint64_t dB1 = umma_desc_sw128(isA ? aq : ado, 16, 1024);
-                const uint64_t dB2 = umma_desc_sw128(isA ? ado : aq, kHalfBytes, 1024);
-                if (!mbar_wait(&bars->qd_full[slot], (p >> 1) & 1u, abort_flag, kTimeoutNs)) { ok = false; break; }
+                if (h == 0 && !mbar_wait(&bars->qd_full[slot], (p >> 1) & 1u, abort_flag, kTimeoutNs)) return false;
                 tc_fence_after();
+                const uint32_t src = smem_u32(smem + (isA ? kKvOffQ : kKvOffDo) + slot * kTileBytes) + 8192u * h;
+                const uint64_t dB1 = umma_desc_sw128(src, 16, 1024);
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {  // S^T = K Q_b^T  /  dP^T = V dO_b^T
+                for (int kk = 0; kk < 8; ++kk) {
                     const uint64_t off = (uint64_t)(((kk >> 2) * kHalfBytes + (kk & 3) * 32) / 16);
-                    mma_ss(t1, dA1 + off, dB1 + off, kIdescSS, kk > 0 ? 1u : 0u);
+                    mma_ss(t1 + 64u * (u & 1), dA1 + off, dB1 + off, kIdescSS64, kk > 0 ? 1u : 0u);
                 }
-                mma_commit(&bars->s_full);
-                // dV += P^T dO_b  /  dK += dS^T Q_b, 16 query rows per step, each query half as soon as its
-                // P^T, dS^T are written (half h: columns 64h .. 64h+31 of S^T / dP^T).
-                for (int h = 0; ok && h < 2; ++h) {
-                    if (!mbar_wait(&bars->p_half[h], p & 1u, abort_flag, kTimeoutNs)) { ok = false; break; }
-                    tc_fence_after();
+                mma_commit(&bars->s_full[u & 1]);
+                return true;
+            };
+            // Second GEMM of step u once its P^T / dS^T are written: dV += P^T(u) dO_h  /  dK += dS^T(u) Q_h,
+            // 16 query rows per MMA: rows 32w' + 16i of the step are bf16 pairs at columns 32w' + 8i of the
+            // buffer (each elementwise warp half w' writes its 32 rows into its own 32 columns).
+            auto second = [&](int32_t u) -> bool {
+                const int32_t p = u / steps, h = u % steps;
+                const int slot = p & 1;
+                if (!mbar_wait(&bars->p_full[u & 1], (u >> 1) & 1u, abort_flag, kTimeoutNs)) return false;
+                tc_fence_after();
+                const uint32_t src = smem_u32(smem + (isA ? kKvOffDo : kKvOffQ) + slot * kTileBytes);
+                const uint64_t dB2 = umma_desc_sw128(src, kHalfBytes, 1024);
 #pragma unroll
-                    for (int kq = 0; kq < 4; ++kq) {
-                        const int kk = 4 * h + kq;
-                        mma_ts(t2, t1 + (uint32_t)(64 * h + kq * 8), dB2 + (uint64_t)(kk * 2048 / 16), kIdescTS,
-                               (p > 0 || kk > 0) ? 1u : 0u);
-                    }
-                }
-                if (!ok) break;
-                mma_commit(&bars->qd_empty[slot]);
+                for (int kq = 0; kq < 4; ++kq)
+                    mma_ts(t2, t1 + 64u * (u & 1) + 32u * (kq >> 1) + 8u * (kq & 1),
+                           dB2 + (uint64_t)((4 * h + kq) * 2048 / 16), kIdescTS, (u > 0 || kq > 0) ? 1u : 0u);
+                if (h == steps - 1) mma_commit(&bars->qd_empty[slot]);  // pair p's Q_b / dO_b read for the last time
+                return true;
+            };
+            // S^T(u) / dP^T(u) run while the elementwise warps work on step u - 1: the buffer u % 2 they
+            // overwrite held step u - 2, whose second GEMM this thread issued before (its MMAs run in order).
+            const int32_t U = np * steps;
+            for (int32_t u = 0; ok && u < U; ++u) {
+                ok = first(u);
+                if (ok && u >= 1) ok = second(u - 1);
             }
+            if (ok) ok = second(U - 1);
             if (ok) mma_commit(&bars->acc_done);
             else *abort_flag = 1;
             uint64_t* dr = &bars->drain[isA ? 0 : 1];
@@ -267,20 +284,23 @@ __global__ void __launch_bounds__(kKvThreads, 1)
             mbar_wait(dr, 0, &never, kTimeoutNs);
         }
     } else if (!skip) {
-        // ------------------------------------------------ one thread per (key kr, query half)
-        // Warps w and w+4 share key rows 32 (w % 4) .. (their TMEM lane quadrant) and take query
-        // columns 0-63 / 64-127: two warps per SM sub-partition keep the MUFU unit busy.
+        // ------------------------------------------------ one thread per (key kr, 32 query rows of a step)
+        // Warps w and w+4 share key rows 32 (w % 4) .. (their TMEM lane quadrant) and take the step's query
+        // rows 0-31 / 32-63: two warps per SM sub-partition keep the MUFU unit busy.
         const int quad = warp & 3, half = warp >> 2;
         const int kr = quad * 32 + lane;
         const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
-        const int col0 = 64 * half;
         const float c = m.scale * kLog2e;
         bool ok = true;
-        for (int32_t p = 0; p < np; ++p) {
-            const int32_t b = lo + p;
-            const bool kvis = self ? kr < nk : key0 + kr < (int64_t)__ldg(anchors + b);
-            // S^T ready; the row constants of the slot landed with Q_b (waited here too, for visibility).
-            if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_full, p & 1u, abort_flag, kTimeoutNs) &&
+        bool kvis = false;
+        for (int32_t u = 0; u < np * steps; ++u) {
+            const int32_t p = u / steps, h = u % steps;
+            if (h == 0) {
+                const int32_t b = lo + p;
+                kvis = self ? kr < nk : key0 + kr < (int64_t)__ldg(anchors + b);
+            }
+            // S^T(u) ready; the row constants of the slot landed with Q_b (waited here too, for visibility).
+            if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_full[u & 1], (u >> 1) & 1u, abort_flag, kTimeoutNs) &&
                                              mbar_wait(&bars->qd_full[p & 1], (p >> 1) & 1u, abort_flag,
                                                        kTimeoutNs))) {
                 ok = false;
@@ -289,33 +309,32 @@ __global__ void __launch_bounds__(kKvThreads, 1)
             tc_fence_after();
             const float* L2s = rows + (p & 1) * 256;
             const float* Ds = L2s + 128;
-#pragma unroll 1
-            for (int cc = 0; cc < 2; ++cc) {
-                uint32_t sv[32], pv[32];
-                tmem_ld32(tS + lane_off + col0 + cc * 32, sv);
-                tmem_ld32(tdP + lane_off + col0 + cc * 32, pv);
-                tmem_wait_ld();
-                uint32_t pk[16], dk2[16];
+            const uint32_t col = 64u * (u & 1) + 32u * half;  // this warp's 32 query rows of the step
+            uint32_t sv[32], pv[32];
+            tmem_ld32(tS + lane_off + col, sv);
+            tmem_ld32(tdP + lane_off + col, pv);
+            tmem_wait_ld();
+            uint32_t pk[16], dk2[16];
 #pragma unroll
-                for (int x = 0; x < 16; ++x) {
-                    const int r0 = col0 + cc * 32 + 2 * x, r1 = r0 + 1;
-                    const bool v0 = kvis && r0 < R, v1 = kvis && r1 < R;
-                    const float p0 = v0 ? ex2_approx(fmaf(__uint_as_float(sv[2 * x]), c, -L2s[r0])) : 0.f;
-                    const float p1 = v1 ? ex2_approx(fmaf(__uint_as_float(sv[2 * x + 1]), c, -L2s[r1])) : 0.f;
-                    const float d0 = v0 ? p0 * (__uint_as_float(pv[2 * x]) - Ds[r0]) : 0.f;
-                    const float d1 = v1 ? p1 * (__uint_as_float(pv[2 * x + 1]) - Ds[r1]) : 0.f;
-                    __nv_bfloat162 hp = __floats2bfloat162_rn(p0, p1);  // .x (low half) = even row
-                    __nv_bfloat162 hd = __floats2bfloat162_rn(d0, d1);
-                    pk[x] = *reinterpret_cast<uint32_t*>(&hp);
-                    dk2[x] = *reinterpret_cast<uint32_t*>(&hd);
-                }
-                // Columns col0 + 16cc .. of S^T / dP^T were read by chunk cc / 2 <= cc: safe to overwrite.
-                tmem_st16(tS + lane_off + col0 + cc * 16, pk);
-                tmem_st16(tdP + lane_off + col0 + cc * 16, dk2);
+            for (int x = 0; x < 16; ++x) {
+                const int r0 = 64 * h + 32 * half + 2 * x, r1 = r0 + 1;
+                const bool v0 = kvis && r0 < R, v1 = kvis && r1 < R;
+                const float p0 = v0 ? ex2_approx(fmaf(__uint_as_float(sv[2 * x]), c, -L2s[r0])) : 0.f;
+                const float p1 = v1 ? ex2_approx(fmaf(__uint_as_float(sv[2 * x + 1]), c, -L2s[r1])) : 0.f;
+                const float d0 = v0 ? p0 * (__uint_as_float(pv[2 * x]) - Ds[r0]) : 0.f;
+                const float d1 = v1 ? p1 * (__uint_as_float(pv[2 * x + 1]) - Ds[r1]) : 0.f;
+                __nv_bfloat162 hp = __floats2bfloat162_rn(p0, p1);  // .x (low half) = even row
+                __nv_bfloat162 hd = __floats2bfloat162_rn(d0, d1);
+                pk[x] = *reinterpret_cast<uint32_t*>(&hp);
+                dk2[x] = *reinterpret_cast<uint32_t*>(&hd);
             }
+            // The first 16 of this warp's 32 columns: read above by this warp alone.
+            tmem_st16(tS + lane_off + col, pk);
+            tmem_st16(tdP + lane_off + col, dk2);
             tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(&bars->p_half[half]);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars->p_full[u & 1]);
         }
         // Epilogue: dV and scale * dK of this key, fp32, overwritten (zero if no block sees the tile).
         if (ok && np > 0 &&
@@ -375,8 +394,8 @@ constexpr int kQOffBar = 6 * kTileBytes;
 struct QBars {
     uint64_t qd_full, qd_empty;      // Q, dO of item i landed / every S, dP of item i complete
     uint64_t kv_full[2], kv_empty[2];
-    uint64_t s_full;                 // S, dP of the current tile complete
-    uint64_t p_half[2];              // dS of keys 64h .. 64h+63 written
+    uint64_t s_full[2];              // S, dP of step u (parity u % 2) complete (one commit per issuer)
+    uint64_t p_full[2];              // dS of step u written (8 elementwise warps)
     uint64_t dq_ready, dq_free;      // last dQ MMA of item i complete / dQ read by the epilogue
     uint64_t drain[2];
     uint32_t tmem_base;
@@ -458,9 +477,10 @@ __global__ void __launch_bounds__(kQThreads, 1)
             mbar_init(&bars->kv_full[b], 1);
             mbar_init(&bars->kv_empty[b], 2);
         }
-        mbar_init(&bars->s_full, 2);
-        mbar_init(&bars->p_half[0], 128);
-        mbar_init(&bars->p_half[1], 128);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&bars->s_full[b], 2);
+            mbar_init(&bars->p_full[b], 8);
+        }
         mbar_init(&bars->dq_ready, 1);
         mbar_init(&bars->dq_free, 256);
         mbar_init(&bars->drain[0], 1);
@@ -531,66 +551,79 @@ __global__ void __launch_bounds__(kQThreads, 1)
                     mbar_wait(&bars->kv_full[x & 1], (x >> 1) & 1u, &never, kTimeoutNs);
         }
     } else if (warp == kQMmaWarp || warp == kQMma2Warp) {
-        // Two issuers, so that the tensor core interleaves two instruction streams: A: S = Q K^T, then
-        // dQ += dS K reading dS from S's columns (its own order keeps the next S after that read);
-        // B: dP = dO V^T, the next one only once the elementwise pass has read this one.
+        // Two issuers, so that the tensor core interleaves two instruction streams. Each key tile runs as
+        // two steps of 64 keys (u = 2n + kh), with S and dP double-buffered by step parity (64 columns
+        // each): A: S(u) = Q K_kh^T, then dQ += dS(u-1) K_kh' of the previous step (reading dS from its S
+        // buffer; this thread's MMAs run in order, so S(u+1) overwrites it only after); B: dP(u) = dO V_kh^T
+        // once the elementwise pass has read dP(u-2) out of the same buffer.
         const bool isA = warp == kQMmaWarp;
         if (!skip && lane == 0) {
             const uint64_t dA1 = umma_desc_sw128(smem_u32(smem + (isA ? kQOffQ : kQOffDo)), 16, 1024);
             int32_t pos = q0;
             int64_t self_pos = blockIdx.x;
             QItem t;
-            uint32_t i = 0, n = 0;
+            uint32_t i = 0, n = 0, u = 0;
             bool ok = true;
+            // The previous step, whose dQ MMAs issuer A issues after the next step's S.
+            uint32_t pu = 0, pn = 0, pi = 0;
+            int pkh = 0;
+            bool have_prev = false, p_first = false, p_last = false;
+            auto dq_step = [&]() -> bool {
+                if (!mbar_wait(&bars->p_full[pu & 1], (pu >> 1) & 1u, abort_flag, kTimeoutNs)) return false;
+                // The first dQ MMA of item i overwrites dQ once the epilogue has read item i-1.
+                if (p_first && pi >= 1 && !mbar_wait(&bars->dq_free, (pi - 1) & 1u, abort_flag, kTimeoutNs))
+                    return false;
+                tc_fence_after();
+                const uint64_t dKmn = umma_desc_sw128(smem_u32(smem + kQOffK + (pn & 1) * kTileBytes), kHalfBytes, 1024);
+#pragma unroll
+                for (int kq = 0; kq < 4; ++kq)  // keys 32w' + 16i of the step: dS pairs at columns 32w' + 8i
+                    mma_ts(tdQ, tS + 64u * (pu & 1) + 32u * (kq >> 1) + 8u * (kq & 1),
+                           dKmn + (uint64_t)((4 * pkh + kq) * 2048 / 16), kIdescTS, (!p_first || kq > 0) ? 1u : 0u);
+                if (pkh == 1) mma_commit(&bars->kv_empty[pn & 1]);  // K(n) read for the last time
+                if (p_last) mma_commit(&bars->dq_ready);
+                return true;
+            };
             while (ok && q_next(m, anchors, item_id, queue_items, pos, q1, self_pos, t, status)) {
                 if (!mbar_wait(&bars->qd_full, i & 1u, abort_flag, kTimeoutNs)) { ok = false; break; }
-                for (int32_t tt = 0; tt < t.ntiles; ++tt, ++n) {
+                for (int32_t tt = 0; ok && tt < t.ntiles; ++tt, ++n) {
                     const int b = n & 1;
-                    const uint32_t ak = smem_u32(smem + kQOffK + b * kTileBytes);
-                    const uint64_t dB1 = umma_desc_sw128(isA ? ak : smem_u32(smem + kQOffV + b * kTileBytes), 16, 1024);
                     if (!mbar_wait(&bars->kv_full[b], (n >> 1) & 1u, abort_flag, kTimeoutNs)) { ok = false; break; }
-                    // B: dP(n) overwrites dP(n-1) once both halves of the elementwise pass have read it.
-                    if (!isA && n >= 1 &&
-                        !(mbar_wait(&bars->p_half[0], (n - 1) & 1u, abort_flag, kTimeoutNs) &&
-                          mbar_wait(&bars->p_half[1], (n - 1) & 1u, abort_flag, kTimeoutNs))) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    const uint32_t t1 = isA ? tS : tdP;
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk) {  // S = Q K^T  /  dP = dO V^T
-                        const uint64_t off = (uint64_t)(((kk >> 2) * kHalfBytes + (kk & 3) * 32) / 16);
-                        mma_ss(t1, dA1 + off, dB1 + off, kIdescSS, kk > 0 ? 1u : 0u);
-                    }
-                    mma_commit(&bars->s_full);
-                    if (tt == t.ntiles - 1) mma_commit(&bars->qd_empty);  // Q, dO free once these complete
-                    if (isA) {
-                        const uint64_t dKmn = umma_desc_sw128(ak, kHalfBytes, 1024);
-                        // The first dQ MMA of item i overwrites dQ once the epilogue has read item i-1.
-                        if (tt == 0 && i >= 1 && !mbar_wait(&bars->dq_free, (i - 1) & 1u, abort_flag, kTimeoutNs)) {
+                    for (int kh = 0; kh < 2; ++kh, ++u) {
+                        // B: dP(u) overwrites dP(u-2) once the elementwise pass has read it.
+                        if (!isA && u >= 2 &&
+                            !mbar_wait(&bars->p_full[u & 1], ((u >> 1) - 1) & 1u, abort_flag, kTimeoutNs)) {
                             ok = false;
                             break;
                         }
-                        // dQ += dS K, 16 keys per step, each key half as soon as its dS is written (half h:
-                        // columns 64h .. 64h+31 of S).
-                        for (int h = 0; ok && h < 2; ++h) {
-                            if (!mbar_wait(&bars->p_half[h], n & 1u, abort_flag, kTimeoutNs)) { ok = false; break; }
-                            tc_fence_after();
+                        tc_fence_after();
+                        const uint32_t src = smem_u32(smem + (isA ? kQOffK : kQOffV) + b * kTileBytes) + 8192u * kh;
+                        const uint64_t dB1 = umma_desc_sw128(src, 16, 1024);
+                        const uint32_t t1 = (isA ? tS : tdP) + 64u * (u & 1);
 #pragma unroll
-                            for (int kq = 0; kq < 4; ++kq) {
-                                const int kk = 4 * h + kq;
-                                mma_ts(tdQ, tS + (uint32_t)(64 * h + kq * 8), dKmn + (uint64_t)(kk * 2048 / 16), kIdescTS,
-                                       (tt > 0 || kk > 0) ? 1u : 0u);
-                            }
+                        for (int kk = 0; kk < 8; ++kk) {  // S = Q K_kh^T  /  dP = dO V_kh^T, 64 keys
+                            const uint64_t off = (uint64_t)(((kk >> 2) * kHalfBytes + (kk & 3) * 32) / 16);
+                            mma_ss(t1, dA1 + off, dB1 + off, kIdescSS64, kk > 0 ? 1u : 0u);
                         }
-                        if (!ok) break;
+                        mma_commit(&bars->s_full[u & 1]);
+                        const bool last_of_item = tt == t.ntiles - 1 && kh == 1;
+                        if (last_of_item) mma_commit(&bars->qd_empty);  // Q, dO free once these complete
+                        if (isA) {
+                            if (have_prev && !dq_step()) { ok = false; break; }
+                            pu = u;
+                            pn = n;
+                            pi = i;
+                            pkh = kh;
+                            p_first = tt == 0 && kh == 0;
+                            p_last = last_of_item;
+                            have_prev = true;
+                        } else if (kh == 1) {
+                            mma_commit(&bars->kv_empty[b]);  // V(n) read for the last time
+                        }
                     }
-                    mma_commit(&bars->kv_empty[b]);
-                    if (isA && tt == t.ntiles - 1) mma_commit(&bars->dq_ready);
                 }
                 ++i;
             }
+            if (ok && isA && have_prev && !dq_step()) ok = false;
             if (!ok) *abort_flag = 1;
             uint64_t* dr = &bars->drain[isA ? 0 : 1];
             mma_commit(dr);
@@ -604,12 +637,11 @@ __global__ void __launch_bounds__(kQThreads, 1)
         const int quad = warp & 3, half = warp >> 2;
         const int r = quad * 32 + lane;
         const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
-        const int col0 = 64 * half;
         const float c = m.scale * kLog2e;
         int32_t pos = q0;
         int64_t self_pos = blockIdx.x;
         QItem t;
-        uint32_t i = 0, n = 0;
+        uint32_t i = 0, u = 0;
         bool ok = true;
         while (ok && q_next(m, anchors, item_id, queue_items, pos, q1, self_pos, t, status)) {
             // Row r belongs to block t.j + x of the tile; it sees that block's prefix of the chunk (a
@@ -620,23 +652,23 @@ __global__ void __launch_bounds__(kQThreads, 1)
                 !live ? 0 : t.self_item ? m.block : visible_in_chunk(m, t.s, t.c, __ldg(anchors + t.j + x));
             const int64_t rb = ((int64_t)(t.j + x) * m.hkv + t.g) * RB + r % RB;
             const float L2 = live ? l2[rb] : 0.f, Dr = live ? dvec[rb] : 0.f;
-            for (int32_t tt = 0; tt < t.ntiles; ++tt, ++n) {
-                if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_full, n & 1u, abort_flag, kTimeoutNs))) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
-                const int valid = row_nvis - tt * kKeys;  // keys of the tile this row sees
-#pragma unroll 1
-                for (int cc = 0; cc < 2; ++cc) {
+            for (int32_t tt = 0; ok && tt < t.ntiles; ++tt) {
+                for (int kh = 0; kh < 2; ++kh, ++u) {
+                    if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_full[u & 1], (u >> 1) & 1u, abort_flag, kTimeoutNs))) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const int valid = row_nvis - tt * kKeys - 64 * kh - 32 * half;  // keys of my 32 this row sees
+                    const uint32_t col = 64u * (u & 1) + 32u * half;
                     uint32_t sv[32], pv[32];
-                    tmem_ld32(tS + lane_off + col0 + cc * 32, sv);
-                    tmem_ld32(tdP + lane_off + col0 + cc * 32, pv);
+                    tmem_ld32(tS + lane_off + col, sv);
+                    tmem_ld32(tdP + lane_off + col, pv);
                     tmem_wait_ld();
                     uint32_t dk2[16];
 #pragma unroll
                     for (int x = 0; x < 16; ++x) {
-                        const int k0 = col0 + cc * 32 + 2 * x;
+                        const int k0 = 2 * x;
                         const float p0 = k0 < valid ? ex2_approx(fmaf(__uint_as_float(sv[2 * x]), c, -L2)) : 0.f;
                         const float p1 =
                             k0 + 1 < valid ? ex2_approx(fmaf(__uint_as_float(sv[2 * x + 1]), c, -L2)) : 0.f;
@@ -645,12 +677,13 @@ __global__ void __launch_bounds__(kQThreads, 1)
                         __nv_bfloat162 hd = __floats2bfloat162_rn(d0, d1);  // .x (low half) = even key
                         dk2[x] = *reinterpret_cast<uint32_t*>(&hd);
                     }
-                    // Columns col0 + 16cc .. of S were read by chunk cc / 2 <= cc: safe to overwrite.
-                    tmem_st16(tS + lane_off + col0 + cc * 16, dk2);
+                    // The first 16 of this warp's 32 columns: read above by this warp alone.
+                    tmem_st16(tS + lane_off + col, dk2);
+                    tmem_wait_st();
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&bars->p_full[u & 1]);
                 }
-                tmem_wait_st();
-                tc_fence_before();
-                mbar_arrive(&bars->p_half[half]);
             }
             if (!ok) break;
             // Epilogue of item i: add scale * dQ into dq (zeroed before the launch).
