@@ -90,6 +90,7 @@ struct KvBars {
     uint64_t s_full[2];                // S^T, dP^T of step u (parity u % 2) complete (one commit per issuer)
     uint64_t p_full[2];                // P^T, dS^T of step u written (8 elementwise warps)
     uint64_t acc_done;                 // every MMA complete: dV, dK final
+    uint64_t epi_staged;               // all 8 elementwise warps staged their dV / dK rows
     uint64_t drain[2];
     uint32_t tmem_base;
     int32_t abort_flag;
@@ -166,6 +167,7 @@ __global__ void __launch_bounds__(kKvThreads, 1)
             mbar_init(&bars->p_full[b], 8);
         }
         mbar_init(&bars->acc_done, 2);
+        mbar_init(&bars->epi_staged, 8);
         mbar_init(&bars->drain[0], 1);
         mbar_init(&bars->drain[1], 1);
         bars->abort_flag = 0;
@@ -342,9 +344,12 @@ __global__ void __launch_bounds__(kKvThreads, 1)
             ok = false;
         if (ok) {
             tc_fence_after();
-            float* vrow = (self ? dvb : dv) + ((krow + kr) * m.hkv + g) * (int64_t)m.d;
-            float* krow_p = (self ? dkb : dk) + ((krow + kr) * m.hkv + g) * (int64_t)m.d;
-            const bool write = kr < nk;
+            // Stage the tile's dV and scale * dK rows in shared memory (the Q_b / dO_b slots, free now that
+            // every MMA is complete): 16-byte groups of key kr at group index g4 ^ (kr % 32), so that the 32
+            // rows a warp writes at once fall in different banks. Then every warp stores whole 512-byte rows:
+            // a thread per key writing its own row touched 32 rows' sectors per store instruction.
+            float4* stv = reinterpret_cast<float4*>(smem + kKvOffQ);  // [128 keys][32 groups] dV
+            float4* stk = stv + 128 * 32;                             // [128 keys][32 groups] scale * dK
 #pragma unroll 1
             for (int cc = 2 * half; cc < 2 * half + 2; ++cc) {
                 uint32_t xv[32], xk[32];
@@ -356,16 +361,29 @@ __global__ void __launch_bounds__(kKvThreads, 1)
 #pragma unroll
                     for (int e = 0; e < 32; ++e) xv[e] = xk[e] = 0u;
                 }
-                if (write) {
 #pragma unroll
-                    for (int e = 0; e < 32; e += 4) {
-                        *reinterpret_cast<float4*>(vrow + cc * 32 + e) =
-                            make_float4(__uint_as_float(xv[e]), __uint_as_float(xv[e + 1]),
-                                        __uint_as_float(xv[e + 2]), __uint_as_float(xv[e + 3]));
-                        *reinterpret_cast<float4*>(krow_p + cc * 32 + e) = make_float4(
-                            __uint_as_float(xk[e]) * m.scale, __uint_as_float(xk[e + 1]) * m.scale,
-                            __uint_as_float(xk[e + 2]) * m.scale, __uint_as_float(xk[e + 3]) * m.scale);
-                    }
+                for (int e = 0; e < 8; ++e) {
+                    const int at = kr * 32 + ((cc * 8 + e) ^ (kr & 31));
+                    stv[at] = make_float4(__uint_as_float(xv[4 * e]), __uint_as_float(xv[4 * e + 1]),
+                                          __uint_as_float(xv[4 * e + 2]), __uint_as_float(xv[4 * e + 3]));
+                    stk[at] = make_float4(__uint_as_float(xk[4 * e]) * m.scale, __uint_as_float(xk[4 * e + 1]) * m.scale,
+                                          __uint_as_float(xk[4 * e + 2]) * m.scale,
+                                          __uint_as_float(xk[4 * e + 3]) * m.scale);
+                }
+            }
+            // Every elementwise warp staged its rows (bounded wait; a warp that gave up earlier never arrives).
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars->epi_staged);
+            ok = __all_sync(0xffffffffu, mbar_wait(&bars->epi_staged, 0, abort_flag, kTimeoutNs));
+            if (ok) {
+                float* dv_t = (self ? dvb : dv) + (krow * m.hkv + g) * (int64_t)m.d;
+                float* dk_t = (self ? dkb : dk) + (krow * m.hkv + g) * (int64_t)m.d;
+                const int64_t rstride = (int64_t)m.hkv * m.d;
+#pragma unroll 2
+                for (int k = warp; k < nk; k += 8) {
+                    const int at = k * 32 + (lane ^ (k & 31));
+                    *reinterpret_cast<float4*>(dv_t + k * rstride + 4 * lane) = stv[at];
+                    *reinterpret_cast<float4*>(dk_t + k * rstride + 4 * lane) = stk[at];
                 }
             }
         }
