@@ -512,7 +512,7 @@ def run_ours(args):
                              fwd_merge_ms=fwd_ms + merge_ms),
             "phase_ms": phase_ms,
             "imbalance": {f"predicted_{args.plan}": predicted_imb},
-            **({"backward_roofline": {"kernels": "rows_kernel + bwd_kv_kernel + bwd_q_kernel",
+            **({"backward_roofline": {"kernels": "rows_kernel + bwd_tc_kernel",
                                       "algorithmic_flop": flops - fwd_kernel_flops,
                                       "achieved": (flops - fwd_kernel_flops) / (phase_ms["bwd"] * 1e-3) / 1e12,
                                       "peak": peak, "unit": "TFLOP/s",

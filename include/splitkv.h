@@ -57,6 +57,7 @@ extern "C" {
 #define SPLITKV_DEV_BAD_COST 0x4     /* planner input: a cost outside [1, max_cost] or too many items */
 #define SPLITKV_DEV_BAD_PLAN 0x8     /* a queue entry or item id out of range                      */
 #define SPLITKV_DEV_TIMEOUT 0x10     /* an in-kernel wait passed its time limit; the kernel returned */
+#define SPLITKV_DEV_SMEM_ALIGN 0x20  /* dynamic shared memory not 1024-byte aligned; the backward returned */
 
 /* Element types of q, k, v, kb, vb, o, dout. Accumulation is always float32. */
 #define SPLITKV_F32 0
@@ -249,18 +250,16 @@ int splitkv_lse_merge(const splitkv_problem *problem, const void *o_part, const 
  *   dV_j += P dO,  dS = P (dO.v_j - D),  dQ += scale dS k_j,  dK_j += scale dS q
  * for the context keys and the block's own keys. Outputs are float32 and are overwritten:
  *   dq [Nq, Hq, d], dk, dv [sum S, Hkv, d], dkb, dvb [Nq, Hkv, d].
- * bf16 with head_dim 128 runs on the tensor cores: dK/dV key tile by key tile, and dQ over the
- * forward's items along the plan (item_id_d, queue_off_d, queue_items_d, n_workers from
- * splitkv_cost and splitkv_plan_lpt); every other problem runs on CUDA cores and ignores the plan
- * (it may be NULL there). All tensor pointers must be 16-byte aligned on the tensor-core path.
- * Needs splitkv_workspace_size() bytes of workspace.
+ * bf16 with head_dim 128 runs on the tensor cores in one pass over 128-key tiles: dK/dV of a tile
+ * accumulate on its SM and dQ is added into dq with float32 reductions (the summation order of dq
+ * varies from run to run; dk, dv, dkb, dvb do not). Every other problem runs on CUDA cores. All tensor
+ * pointers must be 16-byte aligned on the tensor-core path. Needs no plan; needs
+ * splitkv_workspace_size() bytes of workspace.
  */
 int splitkv_attn_bwd(const splitkv_problem *problem, const void *q, const void *k, const void *v,
                      const void *kb, const void *vb, const void *o, const float *lse, const void *dout,
-                     const int32_t *anchors_d, const int32_t *item_id_d, const int32_t *queue_off_d,
-                     const int32_t *queue_items_d, int32_t n_workers, float *dq, float *dk, float *dv,
-                     float *dkb, float *dvb, int32_t *status_d, void *workspace_d, size_t workspace_bytes,
-                     void *stream);
+                     const int32_t *anchors_d, float *dq, float *dk, float *dv, float *dkb, float *dvb,
+                     int32_t *status_d, void *workspace_d, size_t workspace_bytes, void *stream);
 
 /*
  * Context parallelism across ranks (Split-KV paper, Abstract, and its table of context-parallel

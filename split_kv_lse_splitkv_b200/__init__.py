@@ -13,7 +13,7 @@ Entry points (same names as the C ABI): :func:`splitkv_query`,
 together with torch-allocated buffers.
 """
 _EXPORTS = (
-    "DEV_ANCHOR_ORDER", "DEV_ANCHOR_RANGE", "DEV_BAD_COST", "DEV_BAD_PLAN", "DEV_TIMEOUT", "FWD_DEFAULT", "FWD_SIMT",
+    "DEV_ANCHOR_ORDER", "DEV_ANCHOR_RANGE", "DEV_BAD_COST", "DEV_BAD_PLAN", "DEV_SMEM_ALIGN", "DEV_TIMEOUT", "FWD_DEFAULT", "FWD_SIMT",
     "FWD_TEST_STARVE",
     "LIB_PATH", "SplitKV", "SplitKVError", "make_problem", "splitkv_attn_bwd", "splitkv_attn_fwd", "splitkv_cost",
     "splitkv_last_error", "splitkv_lse_merge", "splitkv_max_workers", "splitkv_cp_plan", "splitkv_cost_rank",

@@ -16,6 +16,7 @@ _lib = ctypes.CDLL(LIB_PATH)
 # Constants mirrored from include/splitkv.h.
 OK, EINVAL, EUNSUPPORTED, ECUDA, ENOSPACE = 0, -1, -2, -3, -4
 DEV_ANCHOR_ORDER, DEV_ANCHOR_RANGE, DEV_BAD_COST, DEV_BAD_PLAN, DEV_TIMEOUT = 0x1, 0x2, 0x4, 0x8, 0x10
+DEV_SMEM_ALIGN = 0x20
 F32, BF16 = 0, 1
 FWD_DEFAULT, FWD_SIMT, FWD_TEST_STARVE = 0, 1, 0x100
 MAX_BATCH = 64
@@ -70,7 +71,7 @@ _SIGS = {
     "splitkv_attn_fwd": (_i32, [_PP, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _vp, _i32, _vp,
                                 _sz, _vp]),
     "splitkv_lse_merge": (_i32, [_PP, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
-    "splitkv_attn_bwd": (_i32, [_PP] + [_vp] * 12 + [_i32] + [_vp] * 6 + [_vp, _sz, _vp]),
+    "splitkv_attn_bwd": (_i32, [_PP] + [_vp] * 9 + [_vp] * 6 + [_vp, _sz, _vp]),
     "splitkv_cp_plan": (_i32, [_vp, _i64, _i32, _vp, _vp]),
     "splitkv_cost_rank": (_i32, [_PP, _vp, _vp, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "splitkv_lse_merge_rank": (_i32, [_PP, _vp, _vp, _vp, _vp, _i32, _i32, _vp, _vp, _vp, _vp]),
@@ -195,11 +196,10 @@ def splitkv_lse_merge(problem, o_part, lse_part, anchors, o, lse, status, stream
                                   _stream(stream)), "splitkv_lse_merge")
 
 
-def splitkv_attn_bwd(problem, q, k, v, kb, vb, o, lse, dout, anchors, item_id, queue_off, queue_items, n_workers,
-                     dq, dk, dv, dkb, dvb, status, workspace, stream=None):
+def splitkv_attn_bwd(problem, q, k, v, kb, vb, o, lse, dout, anchors, dq, dk, dv, dkb, dvb, status, workspace,
+                     stream=None):
     _check(_lib.splitkv_attn_bwd(problem.ptr, _p(q), _p(k), _p(v), _p(kb), _p(vb), _p(o), _p(lse), _p(dout),
-                                 _p(anchors), _p(item_id), _p(queue_off), _p(queue_items), int(n_workers), _p(dq),
-                                 _p(dk), _p(dv), _p(dkb), _p(dvb), _p(status), _p(workspace),
+                                 _p(anchors), _p(dq), _p(dk), _p(dv), _p(dkb), _p(dvb), _p(status), _p(workspace),
                                  workspace.numel() * workspace.element_size(), _stream(stream)), "splitkv_attn_bwd")
 
 
@@ -312,15 +312,14 @@ class SplitKV:
         return self.lse_merge(anchors, o, lse, stream)
 
     def backward(self, q, k, v, kb, vb, o, lse, dout, anchors, grads=None, stream=None):
-        """dQ, dK, dV, dKb, dVb (float32). The bf16 tensor-core path walks the items of the plan made by
-        the last :meth:`plan` call, which must be for these anchors (the forward's plan)."""
+        """dQ, dK, dV, dKb, dVb (float32), from the forward's o and lse (no plan needed)."""
         if grads is None:
             f = dict(dtype=torch.float32, device=self.device)
             grads = (torch.empty(q.shape, **f), torch.empty(k.shape, **f), torch.empty(v.shape, **f),
                      torch.empty(kb.shape, **f), torch.empty(vb.shape, **f))
         dq, dk, dv, dkb, dvb = grads
-        splitkv_attn_bwd(self.problem, q, k, v, kb, vb, o, lse, dout, anchors, self.item_id, self.queue_off,
-                         self.queue_items, self.n_workers, dq, dk, dv, dkb, dvb, self.status, self.workspace, stream)
+        splitkv_attn_bwd(self.problem, q, k, v, kb, vb, o, lse, dout, anchors, dq, dk, dv, dkb, dvb, self.status,
+                         self.workspace, stream)
         return grads
 
     # -- host-side reads (synchronizing; for tests and reports)

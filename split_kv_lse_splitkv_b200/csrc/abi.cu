@@ -351,10 +351,8 @@ SPLITKV_API int splitkv_lse_merge(const splitkv_problem* problem, const void* o_
 
 SPLITKV_API int splitkv_attn_bwd(const splitkv_problem* problem, const void* q, const void* k, const void* v,
                                  const void* kb, const void* vb, const void* o, const float* lse, const void* dout,
-                                 const int32_t* anchors_d, const int32_t* item_id_d, const int32_t* queue_off_d,
-                                 const int32_t* queue_items_d, int32_t n_workers, float* dq, float* dk, float* dv,
-                                 float* dkb, float* dvb, int32_t* status_d, void* workspace_d,
-                                 size_t workspace_bytes, void* stream) {
+                                 const int32_t* anchors_d, float* dq, float* dk, float* dv, float* dkb, float* dvb,
+                                 int32_t* status_d, void* workspace_d, size_t workspace_bytes, void* stream) {
     clear_error();
     Meta m;
     int rc = build_meta(problem, &m);
@@ -366,13 +364,12 @@ SPLITKV_API int splitkv_attn_bwd(const splitkv_problem* problem, const void* q, 
     if (m.n_blocks && !anchors_d) return SPLITKV_EINVAL;
     cudaStream_t st = (cudaStream_t)stream;
     if (bwd_tc_supported(m)) {
-        if (n_workers < 1 || n_workers > 65535 || !item_id_d || !queue_off_d || !queue_items_d) return SPLITKV_EINVAL;
         if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(kb) || !aligned16(vb) || !aligned16(dout) ||
             !aligned16(dq) || !aligned16(dk) || !aligned16(dv) || !aligned16(dkb) || !aligned16(dvb))
             return SPLITKV_EINVAL;
         if (!workspace_d || workspace_bytes < bwd_tc_workspace(m)) return SPLITKV_ENOSPACE;
-        return cuda_status(launch_bwd_tc(m, q, k, v, kb, vb, o, lse, dout, anchors_d, item_id_d, queue_off_d,
-                                         queue_items_d, n_workers, dq, dk, dv, dkb, dvb, status_d, workspace_d, st));
+        return cuda_status(
+            launch_bwd_tc(m, q, k, v, kb, vb, o, lse, dout, anchors_d, dq, dk, dv, dkb, dvb, status_d, workspace_d, st));
     }
     if (!workspace_d || workspace_bytes < bwd_workspace(m)) return SPLITKV_ENOSPACE;
     return cuda_status(launch_bwd(m, q, k, v, kb, vb, o, lse, dout, anchors_d, dq, dk, dv, dkb, dvb, status_d,

@@ -150,10 +150,8 @@ cudaError_t launch_merge_ranks(const Meta& m, int32_t n_ranks, const void* o_ran
 bool bwd_tc_supported(const Meta& m);
 size_t bwd_tc_workspace(const Meta& m);
 cudaError_t launch_bwd_tc(const Meta& m, const void* q, const void* k, const void* v, const void* kb, const void* vb,
-                          const void* o, const float* lse, const void* dout, const int32_t* anchors,
-                          const int32_t* item_id, const int32_t* queue_off, const int32_t* queue_items,
-                          int32_t n_workers, float* dq, float* dk, float* dv, float* dkb, float* dvb,
-                          int32_t* status, void* ws, cudaStream_t st);
+                          const void* o, const float* lse, const void* dout, const int32_t* anchors, float* dq,
+                          float* dk, float* dv, float* dkb, float* dvb, int32_t* status, void* ws, cudaStream_t st);
 
 cudaError_t launch_bwd(const Meta& m, const void* q, const void* k, const void* v, const void* kb, const void* vb,
                        const void* o, const float* lse, const void* dout, const int32_t* anchors, float* dq,

@@ -167,19 +167,19 @@ def test_null_pointers_and_small_workspace_rejected_before_launch():
         B.splitkv_lse_merge(p, fake, fake, fake, fake[1:], fake, fake, stream=0)
     assert e.value.code == B.EINVAL
     with pytest.raises(B.SplitKVError) as e:
-        B.splitkv_attn_bwd(p, *([fake] * 12), 4, *([fake] * 6), ws[:1], stream=0)
+        B.splitkv_attn_bwd(p, *([fake] * 9), *([fake] * 6), ws[:1], stream=0)
     assert e.value.code == B.ENOSPACE
-    # bf16, d = 128: the tensor-core backward needs the plan and 16-byte aligned tensors.
+    # bf16, d = 128: the tensor-core backward needs 16-byte aligned tensors.
     pb = prob(head_dim=128, dtype=torch.bfloat16)
     wsb = torch.empty(B.splitkv_workspace_size(pb, 4), dtype=torch.uint8)
-    with pytest.raises(B.SplitKVError) as e:  # no plan
-        B.splitkv_attn_bwd(pb, *([fake] * 9), None, None, None, 4, *([fake] * 6), wsb, stream=0)
+    with pytest.raises(B.SplitKVError) as e:  # no dq
+        B.splitkv_attn_bwd(pb, *([fake] * 9), None, *([fake] * 5), wsb, stream=0)
     assert e.value.code == B.EINVAL
     with pytest.raises(B.SplitKVError) as e:  # misaligned dk
-        B.splitkv_attn_bwd(pb, *([fake] * 12), 4, fake, fake[1:], *([fake] * 4), wsb, stream=0)
+        B.splitkv_attn_bwd(pb, *([fake] * 9), fake, fake[1:], *([fake] * 4), wsb, stream=0)
     assert e.value.code == B.EINVAL
     with pytest.raises(B.SplitKVError) as e:
-        B.splitkv_attn_bwd(pb, *([fake] * 12), 4, *([fake] * 6), wsb[:16], stream=0)
+        B.splitkv_attn_bwd(pb, *([fake] * 9), *([fake] * 6), wsb[:16], stream=0)
     assert e.value.code == B.ENOSPACE
 
 
