@@ -68,17 +68,17 @@ WORKLOADS = {
         # 1 q head / 1 kv head, d=64, S=1024, 4 uniform anchors, chunk 128, fp32, 4 workers.
         Workload("tiny_f32", 1, 1, 64, [1024], [4], 128, "f32", 0, n_workers=4),
         # Drafter shape A: 32 q / 4 kv heads, d=128, S=32768, 64 anchors, chunk 1024 (items over runs of
-        # 4 chunks: one partial per 4096 keys).
-        Workload("drafter_s32k", 32, 4, 128, [32768], [64], 1024, "bf16", 1, chunks_per_item=4),
-        # Long context: S=131072, 128 anchors, chunk 2048 (runs of 3 chunks).
-        Workload("long_s128k", 32, 4, 128, [131072], [128], 2048, "bf16", 2, chunks_per_item=3),
+        # 8 chunks: one partial per 8192 keys).
+        Workload("drafter_s32k", 32, 4, 128, [32768], [64], 1024, "bf16", 1, chunks_per_item=8),
+        # Long context: S=131072, 128 anchors, chunk 2048 (runs of 4 chunks).
+        Workload("long_s128k", 32, 4, 128, [131072], [128], 2048, "bf16", 2, chunks_per_item=4),
         # Skewed anchors: 32 q / 8 kv heads, S=262144, 256 draws of floor(S*Beta(5,1)), chunk 2048.
         # G = 4: a block has 64 query rows, so two blocks share one 128-row query tile (runs of 4 chunks).
         Workload("skewed_s256k", 32, 8, 128, [262144], [256], 2048, "bf16", 3, sampler="beta51",
                  blocks_per_item=2, chunks_per_item=4),
-        # Training step: 4 samples of S=65536 with 32/64/96/128 anchors, chunk 1024, fwd+bwd (runs of 4).
+        # Training step: 4 samples of S=65536 with 32/64/96/128 anchors, chunk 1024, fwd+bwd (runs of 8).
         Workload("train_4x64k", 32, 4, 128, [65536] * 4, [32, 64, 96, 128], 1024, "bf16", 4,
-                 backward=True, chunks_per_item=4),
+                 backward=True, chunks_per_item=8),
         # The training shape at a quarter of the context and anchors (4 x 16384 keys, 8/16/24/32
         # anchors): small enough for counter captures that replay each kernel many times.
         Workload("train_4x16k", 32, 4, 128, [16384] * 4, [8, 16, 24, 32], 1024, "bf16", 5, backward=True),
