@@ -20,6 +20,7 @@ from __future__ import annotations
 
 import argparse
 import json
+import math
 import os
 import statistics
 import sys
@@ -290,8 +291,9 @@ def run_reference(args):
     w = workload_of(args)
     inp = W.make_inputs(w)
     vals = []
-    budget = args.ref_budget if args.ref_budget else max(1.0, 150.0 / (args.warmup + args.steps))
-    for i in range(args.warmup + args.steps):
+    steps = args.steps if args.steps is not None else 20
+    budget = args.ref_budget if args.ref_budget else max(1.0, 150.0 / (args.warmup + steps))
+    for i in range(args.warmup + steps):
         r = cpu_oracle_sample(inp, budget, w.backward)
         if i >= args.warmup:
             vals.append(r["value"])
@@ -302,7 +304,7 @@ def run_reference(args):
     r["plan"] = cpu_oracle_plan(inp, workers)
     line = {"impl": "reference", "metric": "useful block-sparse attention TFLOP/s (fwd+bwd)" if w.backward else
             "useful block-sparse attention TFLOP/s (fwd)", "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
-            "steps": args.steps, "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
+            "steps": steps, "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": workload_config(w, [int(inp.anchor_off[i + 1] - inp.anchor_off[i])
                                           for i in range(len(w.seq_lens))], workers, args.gpus, args.plan),
@@ -377,8 +379,8 @@ def run_ours(args):
             timed("bwd", lambda: skv.backward(d["q"], d["k"], d["v"], d["kb"], d["vb"], o, lse, d["do"], d["anchors"],
                                               grads, stream=stream), time_phases)
 
-    # cost 3, LPT plan 3 (not with the naive split), fwd 1, merge 1; bwd: rows, kv, q
-    launches_per_step = 3 + (0 if args.plan == "naive" else 3) + 1 + 1 + (3 if w.backward else 0)
+    # cost 3, LPT plan 3 (not with the naive split), fwd 1, merge 1; bwd: rows, one-pass backward
+    launches_per_step = 3 + (0 if args.plan == "naive" else 3) + 1 + 1 + (2 if w.backward else 0)
     for _ in range(args.warmup):
         step(dev)
     torch.cuda.synchronize(device)
@@ -408,15 +410,24 @@ def run_ours(args):
             evs.append((e0, e1))
         return evs
 
+    replay = (lambda _: graph.replay()) if graph is not None else (lambda tp: step(dev, time_phases=tp))
+    if args.steps is not None:
+        steps = args.steps
+    else:
+        # Enough steps for at least 1 s of timed work (so that the clock record has hundreds of samples),
+        # at least 20; the same count on every rank.
+        probe = timed_steps(3, replay, False)
+        torch.cuda.synchronize(device)
+        t_step = max_over_ranks(sum(a.elapsed_time(b) for a, b in probe) / len(probe), world, device)
+        steps = max(20, int(math.ceil(1000.0 / max(t_step, 1e-3))))
+    aux_steps = min(steps, 50)  # per-phase and end-to-end timings
+
     # ---- device-timed region
     barrier(world)
     torch.cuda.synchronize(device)
     wall0 = time.perf_counter()
     with ClockSampler(local) as clocks:
-        if graph is not None:
-            evs = timed_steps(args.steps, lambda _: graph.replay(), False)
-        else:
-            evs = timed_steps(args.steps, lambda tp: step(dev, time_phases=tp), True)
+        evs = timed_steps(steps, replay, graph is None)
         torch.cuda.synchronize(device)
     barrier(world)
     wall = time.perf_counter() - wall0
@@ -424,7 +435,7 @@ def run_ours(args):
     if graph is not None:
         # Per-phase times (for the roofline of the forward kernel) from as many eager steps, timed
         # the same way, after the graph-timed region.
-        timed_steps(args.steps, lambda tp: step(dev, time_phases=tp), True)
+        timed_steps(aux_steps, lambda tp: step(dev, time_phases=tp), True)
         torch.cuda.synchronize(device)
     phase_ms = {k: (sum(a.elapsed_time(b) for a, b in v) / len(v)) for k, v in phases.items() if v}
     fwd_ms = phase_ms["fwd"]
@@ -459,7 +470,7 @@ def run_ours(args):
     torch.cuda.synchronize(device)
     barrier(world)
     e_evs = []
-    for _ in range(args.steps):
+    for _ in range(aux_steps):
         flush.fill_(1.0)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
@@ -499,7 +510,7 @@ def run_ours(args):
         line = {
             "metric": "useful block-sparse attention TFLOP/s (fwd+bwd)" if w.backward else
                       "useful block-sparse attention TFLOP/s (fwd)",
-            "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": steps, "warmup": args.warmup,
             "ms_per_step": ms_max, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16" if w.dtype == "bf16" else "f32", "data": "synthetic",
             "config": workload_config(w, counts, skv.n_workers, world, args.plan),
@@ -521,7 +532,7 @@ def run_ours(args):
             "clocks": csum,
             "e2e": {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-            "gpu_launches": launches_per_step * args.steps,
+            "gpu_launches": launches_per_step * steps,
             "wall_s": wall,
             "cpu_baseline": cpu,
         }
@@ -534,7 +545,8 @@ def run_ours(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=None,
+                    help="timed steps (default: enough for at least 1 s of timed work, at least 20)")
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="skewed_s256k", choices=sorted(W.WORKLOADS),
                     help="default: the largest single-GPU forward workload (S = 262144, ~4080 queries)")

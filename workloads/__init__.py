@@ -68,8 +68,8 @@ WORKLOADS = {
         # 1 q head / 1 kv head, d=64, S=1024, 4 uniform anchors, chunk 128, fp32, 4 workers.
         Workload("tiny_f32", 1, 1, 64, [1024], [4], 128, "f32", 0, n_workers=4),
         # Drafter shape A: 32 q / 4 kv heads, d=128, S=32768, 64 anchors, chunk 1024 (items over runs of
-        # 8 chunks: one partial per 8192 keys).
-        Workload("drafter_s32k", 32, 4, 128, [32768], [64], 1024, "bf16", 1, chunks_per_item=8),
+        # 6 chunks: one partial per 6144 keys).
+        Workload("drafter_s32k", 32, 4, 128, [32768], [64], 1024, "bf16", 1, chunks_per_item=6),
         # Long context: S=131072, 128 anchors, chunk 2048 (runs of 4 chunks).
         Workload("long_s128k", 32, 4, 128, [131072], [128], 2048, "bf16", 2, chunks_per_item=4),
         # Skewed anchors: 32 q / 8 kv heads, S=262144, 256 draws of floor(S*Beta(5,1)), chunk 2048.
