@@ -42,6 +42,14 @@ def test_tiny_f32_workload():
     full_check(W.make_inputs(W.get("tiny_f32")), n_workers=4)
 
 
+@pytest.mark.parametrize("hq,hkv,P", [(24, 8, 1), (24, 8, 2), (48, 8, 1)])
+def test_group_sizes_not_powers_of_two(hq, hkv, P):
+    # G = 3 (48-row blocks, alone or two to a tile) and G = 6 (96 rows): rows past the block's in the
+    # 128-row MMA tile stay masked.
+    inp = small("groups_odd", "skewed_s256k", [4096], [9], chunk=2048, n_q_heads=hq, n_kv_heads=hkv, blocks_per_item=P)
+    full_check(inp, n_workers=5)
+
+
 @pytest.mark.parametrize("flags", [0, SIMT])
 @pytest.mark.parametrize("n_workers", [3, 148])
 def test_drafter_shape_small(flags, n_workers):
@@ -197,8 +205,17 @@ def test_backward_other_group_sizes(hq, hkv, full_tiles):
     backward_check(inp, n_workers=5)
 
 
+@pytest.mark.parametrize("hq,hkv", [(24, 8), (48, 8)])
+def test_backward_group_sizes_not_powers_of_two(hq, hkv):
+    # G = 3 (48-row blocks, one step) and G = 6 (96 rows: a second step half inside the block): the dQ
+    # reductions walk query rows with a running (query, head) position instead of a compile-time group.
+    inp = small("bwd_groups_odd", "train_4x64k", [2500, 1300], [3, 2], chunk=1024, n_q_heads=hq, n_kv_heads=hkv)
+    backward_check(inp, n_workers=5)
+
+
 def test_backward_runs_of_chunks():
-    # The dQ kernel walks the forward's items, here runs of 2 chunks of 512 keys.
+    # The forward (whose O and LSE the backward starts from) runs items over 2 chunks of 512 keys; the
+    # backward is key-tile stationary whatever the items are.
     backward_check(small("bwd_runs", "train_4x64k", [3000, 2048, 4096], [2, 3, 4], chunk=512, chunks_per_item=2))
 
 
