@@ -217,7 +217,10 @@ int splitkv_plan_lpt_noalloc(const int32_t *item_cost_d, const int32_t *n_items_
  * item_id_d, queue_off_d and queue_items_d come from splitkv_cost and splitkv_plan_lpt.
  * On the tensor-core path each worker runs its queue, then claims self items from a shared counter
  * as it runs out of work (which SM computes a self partial varies from run to run; its value does
- * not). With 256-row items (sizes.ctas_per_worker = 2) each worker is a pair of SMs, a two-CTA
+ * not). When k and v together exceed the device's L2 cache, a one-SM worker runs the items of its
+ * queue in ascending item id rather than in queue order (the same items, so the same load; all
+ * workers then walk the context together and share its K/V in L2); queues of more than 512 items
+ * keep queue order. With 256-row items (sizes.ctas_per_worker = 2) each worker is a pair of SMs, a two-CTA
  * cluster that issues M = 256 tensor-core instructions over both SMs (2 * n_workers CTAs, n_workers
  * <= 32767); its self items are (query tile of P blocks, kv head), whose rows of block x see key
  * columns block*x .. block*x + block - 1 of one key tile of kb/vb, and each block's self partial
