@@ -276,6 +276,9 @@ int splitkv_attn_bwd(const splitkv_problem *problem, const void *q, const void *
  *   3. splitkv_lse_merge_rank -> this rank's query-sized (O_r, LSE_r);
  *   4. an all-gather of (O_r, LSE_r) over the ranks (NCCL, by the caller);
  *   5. splitkv_lse_merge_ranks -> O, LSE: exactly the single-GPU result.
+ * Backward on rank r: splitkv_attn_bwd_rank with the full O, LSE and dout, then a sum (all-reduce) of
+ * dq, dkb and dvb over the ranks; dk and dv of this rank's chunks are final as computed (K/V never
+ * leave their rank).
  * Items must lie in one chunk (chunks_per_item = 1; EUNSUPPORTED otherwise).
  */
 
@@ -306,6 +309,18 @@ int splitkv_lse_merge_rank(const splitkv_problem *problem, const void *o_part, c
  * L = log sum_r exp(LSE_r), O = sum_r exp(LSE_r - L) O_r. */
 int splitkv_lse_merge_ranks(const splitkv_problem *problem, int32_t n_ranks, const void *o_ranks,
                             const float *lse_ranks, void *o, float *lse, int32_t *status_d, void *stream);
+
+/* This rank's share of splitkv_attn_bwd (same arguments, plus the chunk placement of splitkv_cp_plan):
+ * the key tiles of the chunks with chunk_rank_d[c] == rank and the own keys of the blocks j with
+ * j % n_ranks == rank. Outputs are overwritten: dk, dv hold the gradients of this rank's chunks' key
+ * rows (zero on the other rows); dq is this rank's partial sum (over its keys); dkb, dvb hold its
+ * blocks' rows (zero on the others). Summed over the ranks, dq, dk, dv, dkb and dvb equal
+ * splitkv_attn_bwd's. o and lse are the merged forward outputs (splitkv_lse_merge_ranks). */
+int splitkv_attn_bwd_rank(const splitkv_problem *problem, const void *q, const void *k, const void *v,
+                          const void *kb, const void *vb, const void *o, const float *lse, const void *dout,
+                          const int32_t *anchors_d, const int32_t *chunk_rank_d, int32_t rank, int32_t n_ranks,
+                          float *dq, float *dk, float *dv, float *dkb, float *dvb, int32_t *status_d,
+                          void *workspace_d, size_t workspace_bytes, void *stream);
 
 #ifdef __cplusplus
 }

@@ -17,7 +17,7 @@ _EXPORTS = (
     "FWD_TEST_STARVE",
     "LIB_PATH", "SplitKV", "SplitKVError", "make_problem", "splitkv_attn_bwd", "splitkv_attn_fwd", "splitkv_cost",
     "splitkv_last_error", "splitkv_lse_merge", "splitkv_max_workers", "splitkv_cp_plan", "splitkv_cost_rank",
-    "splitkv_lse_merge_rank", "splitkv_lse_merge_ranks", "ContextParallelSplitKV", "splitkv_plan_lpt", "splitkv_plan_lpt_noalloc", "splitkv_query", "splitkv_strerror",
+    "splitkv_lse_merge_rank", "splitkv_lse_merge_ranks", "splitkv_attn_bwd_rank", "ContextParallelSplitKV", "splitkv_plan_lpt", "splitkv_plan_lpt_noalloc", "splitkv_query", "splitkv_strerror",
     "splitkv_workspace_size",
 )
 __all__ = list(_EXPORTS)

@@ -72,6 +72,7 @@ _SIGS = {
                                 _sz, _vp]),
     "splitkv_lse_merge": (_i32, [_PP, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
     "splitkv_attn_bwd": (_i32, [_PP] + [_vp] * 9 + [_vp] * 6 + [_vp, _sz, _vp]),
+    "splitkv_attn_bwd_rank": (_i32, [_PP] + [_vp] * 10 + [_i32, _i32] + [_vp] * 6 + [_vp, _sz, _vp]),
     "splitkv_cp_plan": (_i32, [_vp, _i64, _i32, _vp, _vp]),
     "splitkv_cost_rank": (_i32, [_PP, _vp, _vp, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "splitkv_lse_merge_rank": (_i32, [_PP, _vp, _vp, _vp, _vp, _i32, _i32, _vp, _vp, _vp, _vp]),
@@ -201,6 +202,15 @@ def splitkv_attn_bwd(problem, q, k, v, kb, vb, o, lse, dout, anchors, dq, dk, dv
     _check(_lib.splitkv_attn_bwd(problem.ptr, _p(q), _p(k), _p(v), _p(kb), _p(vb), _p(o), _p(lse), _p(dout),
                                  _p(anchors), _p(dq), _p(dk), _p(dv), _p(dkb), _p(dvb), _p(status), _p(workspace),
                                  workspace.numel() * workspace.element_size(), _stream(stream)), "splitkv_attn_bwd")
+
+
+def splitkv_attn_bwd_rank(problem, q, k, v, kb, vb, o, lse, dout, anchors, chunk_rank, rank, n_ranks, dq, dk, dv, dkb,
+                          dvb, status, workspace, stream=None):
+    _check(_lib.splitkv_attn_bwd_rank(problem.ptr, _p(q), _p(k), _p(v), _p(kb), _p(vb), _p(o), _p(lse), _p(dout),
+                                      _p(anchors), _p(chunk_rank), int(rank), int(n_ranks), _p(dq), _p(dk), _p(dv),
+                                      _p(dkb), _p(dvb), _p(status), _p(workspace),
+                                      workspace.numel() * workspace.element_size(), _stream(stream)),
+           "splitkv_attn_bwd_rank")
 
 
 def splitkv_cp_plan(chunk_cost, n_ranks):

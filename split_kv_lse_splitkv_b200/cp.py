@@ -19,6 +19,13 @@ the collective):
 4. ``combine``: the exact log-sum-exp merge over ranks (``splitkv_lse_merge_ranks``), equal to the
    single-GPU result.
 
+One backward on rank r, from the merged O and LSE (which every rank holds after ``combine``):
+
+5. ``local_backward``: this rank's share (``splitkv_attn_bwd_rank``): dK/dV of its chunks' keys, final as
+   they are (K/V never leave the rank), and partial dQ, dKb, dVb (its keys, its blocks' own keys);
+6. ``reduce_grads``: one all-reduce (sum) of dQ, dKb and dVb over the group: ``Nq * (Hq + 2 Hkv) * d``
+   values, again independent of the context length.
+
 K/V layout: each rank passes full-size ``k``/``v`` buffers ([sum S, Hkv, d]) of which only the rows of its
 own chunks are read (the others may hold anything); a compact per-rank layout would need a chunk-to-row
 map in the kernels and is not built. Items cover one chunk each (``chunks_per_item`` = 1).
@@ -30,6 +37,19 @@ from typing import Optional
 import torch
 
 from . import binding as B
+
+
+def reduce_rank_grads(dq, dkb, dvb, group=None):
+    """Sums this rank's partial dQ, dKb and dVb over ``group`` in place (one all-reduce of the three,
+    packed into one buffer): after it every rank holds the single-GPU gradients of the query side."""
+    import torch.distributed as dist
+    flat = torch.cat([dq.reshape(-1), dkb.reshape(-1), dvb.reshape(-1)])
+    dist.all_reduce(flat, op=dist.ReduceOp.SUM, group=group)
+    a, b = dq.numel(), dkb.numel()
+    dq.copy_(flat[:a].view_as(dq))
+    dkb.copy_(flat[a:a + b].view_as(dkb))
+    dvb.copy_(flat[a + b:].view_as(dvb))
+    return dq, dkb, dvb
 
 
 def cp_plan_chunks(chunk_cost, n_ranks: int):
@@ -103,3 +123,19 @@ class ContextParallelSplitKV:
         o_r, lse_r = self.local_forward(q, k, v, kb, vb, anchors, stream)
         o_all, lse_all = gather_rank_results(o_r, lse_r, self.group)
         return self.combine(o_all, lse_all, stream)
+
+    def local_backward(self, q, k, v, kb, vb, o, lse, dout, anchors, stream=None):
+        """This rank's share of the gradients (float32): dk, dv on its chunks' key rows (zero elsewhere),
+        partial dq, dkb, dvb. Needs the chunk placement of the last :meth:`plan`."""
+        skv = self.skv
+        f = dict(dtype=torch.float32, device=skv.device)
+        dq, dk, dv = torch.empty(q.shape, **f), torch.empty(k.shape, **f), torch.empty(v.shape, **f)
+        dkb, dvb = torch.empty(kb.shape, **f), torch.empty(vb.shape, **f)
+        B.splitkv_attn_bwd_rank(skv.problem, q, k, v, kb, vb, o, lse, dout, anchors, self.chunk_rank, self.rank,
+                                self.n_ranks, dq, dk, dv, dkb, dvb, skv.status, skv.workspace, stream)
+        return dq, dk, dv, dkb, dvb
+
+    def backward(self, q, k, v, kb, vb, o, lse, dout, anchors, stream=None):
+        dq, dk, dv, dkb, dvb = self.local_backward(q, k, v, kb, vb, o, lse, dout, anchors, stream)
+        reduce_rank_grads(dq, dkb, dvb, self.group)
+        return dq, dk, dv, dkb, dvb

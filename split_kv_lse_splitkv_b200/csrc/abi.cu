@@ -349,14 +349,10 @@ SPLITKV_API int splitkv_lse_merge(const splitkv_problem* problem, const void* o_
     return cuda_status(launch_merge(m, o_part, lse_part, anchors_d, o, lse, status_d, (cudaStream_t)stream));
 }
 
-SPLITKV_API int splitkv_attn_bwd(const splitkv_problem* problem, const void* q, const void* k, const void* v,
-                                 const void* kb, const void* vb, const void* o, const float* lse, const void* dout,
-                                 const int32_t* anchors_d, float* dq, float* dk, float* dv, float* dkb, float* dvb,
-                                 int32_t* status_d, void* workspace_d, size_t workspace_bytes, void* stream) {
-    clear_error();
-    Meta m;
-    int rc = build_meta(problem, &m);
-    if (rc) return rc;
+namespace {
+int attn_bwd(const Meta& m, const void* q, const void* k, const void* v, const void* kb, const void* vb, const void* o,
+             const float* lse, const void* dout, const int32_t* anchors_d, float* dq, float* dk, float* dv, float* dkb,
+             float* dvb, int32_t* status_d, void* workspace_d, size_t workspace_bytes, void* stream) {
     const bool queries = m.n_queries > 0;  // without any anchor the query-side buffers are empty
     if ((queries && (!q || !kb || !vb || !o || !lse || !dout || !dq || !dkb || !dvb)) || !k || !v || !dk || !dv ||
         !status_d)
@@ -374,4 +370,31 @@ SPLITKV_API int splitkv_attn_bwd(const splitkv_problem* problem, const void* q, 
     if (!workspace_d || workspace_bytes < bwd_workspace(m)) return SPLITKV_ENOSPACE;
     return cuda_status(launch_bwd(m, q, k, v, kb, vb, o, lse, dout, anchors_d, dq, dk, dv, dkb, dvb, status_d,
                                   workspace_d, st));
+}
+}  // namespace
+
+SPLITKV_API int splitkv_attn_bwd(const splitkv_problem* problem, const void* q, const void* k, const void* v,
+                                 const void* kb, const void* vb, const void* o, const float* lse, const void* dout,
+                                 const int32_t* anchors_d, float* dq, float* dk, float* dv, float* dkb, float* dvb,
+                                 int32_t* status_d, void* workspace_d, size_t workspace_bytes, void* stream) {
+    clear_error();
+    Meta m;
+    int rc = build_meta(problem, &m);
+    if (rc) return rc;
+    return attn_bwd(m, q, k, v, kb, vb, o, lse, dout, anchors_d, dq, dk, dv, dkb, dvb, status_d, workspace_d,
+                    workspace_bytes, stream);
+}
+
+SPLITKV_API int splitkv_attn_bwd_rank(const splitkv_problem* problem, const void* q, const void* k, const void* v,
+                                      const void* kb, const void* vb, const void* o, const float* lse,
+                                      const void* dout, const int32_t* anchors_d, const int32_t* chunk_rank_d,
+                                      int32_t rank, int32_t n_ranks, float* dq, float* dk, float* dv, float* dkb,
+                                      float* dvb, int32_t* status_d, void* workspace_d, size_t workspace_bytes,
+                                      void* stream) {
+    clear_error();
+    Meta m;
+    int rc = rank_meta(problem, chunk_rank_d, rank, n_ranks, &m);
+    if (rc) return rc;
+    return attn_bwd(m, q, k, v, kb, vb, o, lse, dout, anchors_d, dq, dk, dv, dkb, dvb, status_d, workspace_d,
+                    workspace_bytes, stream);
 }

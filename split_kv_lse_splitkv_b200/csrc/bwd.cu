@@ -166,7 +166,9 @@ __global__ void __launch_bounds__(kThreads) bwd_context_kernel(Meta m, TileMap t
         int32_t mid = (lo + hi) >> 1;
         if ((int64_t)anchors[mid] > k0) hi = mid; else lo = mid + 1;
     }
-    for (int32_t j = lo; j < b_hi; ++j) {
+    // Context parallelism: a rank computes only the key tiles of its own chunks (zeros elsewhere).
+    const int32_t j_end = owns_chunk(m, s, (int32_t)(k0 / m.chunk)) ? b_hi : lo;
+    for (int32_t j = lo; j < j_end; ++j) {
         const int64_t a = anchors[j];
         const int nvis = (int)min((int64_t)nk, a - k0);
         tile_rows<T>(m, j, g, nvis, Ks, Vs, q, dout, lse, dvec, dq, Qc, dOc, Ps, dSs, Lc, Dc, adk, adv);
@@ -221,7 +223,8 @@ __global__ void __launch_bounds__(kThreads) bwd_self_kernel(Meta m, const T* __r
 #pragma unroll
     for (int u = 0; u < kMaxAcc; ++u) adk[u] = adv[u] = 0.f;
     __syncthreads();
-    tile_rows<T>(m, j, g, BL, Ks, Vs, q, dout, lse, dvec, dq, Qc, dOc, Ps, dSs, Lc, Dc, adk, adv);
+    // Context parallelism: the block's own keys belong to rank j % n_ranks (zeros elsewhere).
+    if (owns_self(m, j)) tile_rows<T>(m, j, g, BL, Ks, Vs, q, dout, lse, dvec, dq, Qc, dOc, Ps, dSs, Lc, Dc, adk, adv);
 #pragma unroll
     for (int u = 0; u < kMaxAcc; ++u) {
         int e = tid + u * kThreads;

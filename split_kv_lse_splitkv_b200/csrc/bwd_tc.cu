@@ -168,12 +168,13 @@ __global__ void __launch_bounds__(kKvThreads, 1)
             else a = mid + 1;
         }
         lo = a;
+        if (!owns_chunk(m, s, (int32_t)(key0 / m.chunk))) hi = lo;  // another rank's chunk: zeros here
     } else {
         const int64_t sid = unit - n_ctx;
         const int32_t j = (int32_t)(sid / m.hkv);
         g = (int)(sid % m.hkv);
         lo = j;
-        hi = j + 1;
+        hi = owns_self(m, j) ? j + 1 : j;  // another rank's block: zeros here
         nk = m.block;
         krow = (int64_t)m.block * j;
     }

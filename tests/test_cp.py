@@ -8,7 +8,11 @@ Diffusion Drafters, Abstract and its table of context-parallel methods).
   fed with each rank's oracle partial over its own chunks, merges to the single-pass oracle result.
 * One GPU (``-m gpu``): the ranks' steps run one after another through the C ABI (cost of the rank,
   plan, forward, the rank's merge), then the merge over ranks; O and LSE match the oracle, for 1 to 4
-  ranks, and each rank reads K/V only from its own chunks (the other rows hold a large value).
+  ranks, and each rank reads K/V only from its own chunks (the other rows hold a large value). The
+  backward: each rank's share (``splitkv_attn_bwd_rank``) from the merged O and LSE, summed over the
+  ranks, matches the oracle's gradients (1 to 3 ranks, bf16 and fp32).
+* gloo, world size 2, on CPU: the gradient all-reduce (``reduce_rank_grads``) sums the ranks' parts.
+* The rank backward's argument checks, on CPU.
 """
 import os
 import socket
@@ -115,6 +119,50 @@ def _rank_main(rank, port, out_dir):
     dist.destroy_process_group()
 
 
+def _reduce_main(rank, port, out_dir):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), WORLD_SIZE="2", RANK=str(rank))
+    sys.path.insert(0, ROOT)
+    import datetime
+
+    import torch.distributed as dist
+
+    from split_kv_lse_splitkv_b200 import cp
+    dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=60))
+    g = torch.Generator().manual_seed(rank)
+    parts = [torch.randn(5, 4, 8, generator=g), torch.randn(5, 2, 8, generator=g), torch.randn(5, 2, 8, generator=g)]
+    mine = [x.clone() for x in parts]
+    cp.reduce_rank_grads(*mine)
+    torch.save({"parts": parts, "reduced": mine}, os.path.join(out_dir, f"grads{rank}.pt"))
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+def test_two_ranks_gloo_gradient_reduce(tmp_path):
+    mp.start_processes(_reduce_main, args=(_free_port(), str(tmp_path)), nprocs=2, join=True, start_method="spawn")
+    got = [torch.load(tmp_path / f"grads{r}.pt") for r in range(2)]
+    for i in range(3):
+        want = got[0]["parts"][i] + got[1]["parts"][i]
+        for r in range(2):
+            assert torch.equal(got[r]["reduced"][i], want)
+
+
+def test_rank_backward_argument_checks():
+    p = B.make_problem([1024], [0, 4], 1, 1, 64, 16, 128, 128, 0.125, torch.float32)
+    fake = torch.zeros(64, dtype=torch.uint8)
+    ws = torch.empty(B.splitkv_workspace_size(p, 4), dtype=torch.uint8)
+    for rank, n in ((-1, 2), (2, 2), (0, 0)):
+        with pytest.raises(B.SplitKVError) as e:
+            B.splitkv_attn_bwd_rank(p, *([fake] * 9), fake, rank, n, *([fake] * 6), ws, stream=0)
+        assert e.value.code == B.EINVAL
+    with pytest.raises(B.SplitKVError) as e:  # no chunk placement
+        B.splitkv_attn_bwd_rank(p, *([fake] * 9), None, 0, 2, *([fake] * 6), ws, stream=0)
+    assert e.value.code == B.EINVAL
+    runs = B.make_problem([1024], [0, 4], 1, 1, 64, 16, 128, 128, 0.125, torch.float32, chunks_per_item=2)
+    with pytest.raises(B.SplitKVError) as e:  # items must lie in one chunk
+        B.splitkv_attn_bwd_rank(runs, *([fake] * 9), fake, 0, 2, *([fake] * 6), ws, stream=0)
+    assert e.value.code == B.EUNSUPPORTED
+
+
 def test_two_ranks_gloo_plan_gather_and_merge(tmp_path):
     mp.start_processes(_rank_main, args=(_free_port(), str(tmp_path)), nprocs=2, join=True, start_method="spawn")
     for r in range(2):
@@ -160,3 +208,47 @@ def test_ranks_on_one_gpu_match_the_oracle(n_ranks):
     from tests._util import to_np
     assert_close("O (ranks)", to_np(o), O, w.dtype)
     assert_close("LSE (ranks)", to_np(lse), L, w.dtype)
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("n_ranks,base", [(1, "drafter_s32k"), (2, "drafter_s32k"), (3, "drafter_s32k"), (2, "tiny_f32")])
+def test_ranks_on_one_gpu_backward_matches_the_oracle(n_ranks, base):
+    # Forward on one GPU, then each rank's share of the backward (its chunks' key tiles, its blocks' own
+    # keys) with K/V rows of other ranks' chunks set to a large value; the sum of the shares is the
+    # single-GPU backward.
+    from split_kv_lse_splitkv_b200.cp import ContextParallelSplitKV
+    kw = dict(chunk=1024, seed=35) if base == "drafter_s32k" else dict(chunk=128, seed=36)
+    lens, cnts = ([5000, 3000], [5, 3]) if base == "drafter_s32k" else ([1024, 700], [4, 3])
+    inp = W.make_inputs(W.scaled(W.get(base), "cp_bwd", lens, cnts, backward=True, **kw))
+    w = inp.workload
+    counts = [int(inp.anchor_off[i + 1] - inp.anchor_off[i]) for i in range(len(w.seq_lens))]
+    dev = {k: getattr(inp, k).cuda() for k in ("q", "k", "v", "kb", "vb", "do")}
+    anchors = inp.anchors.cuda()
+    skv = B.SplitKV(w.seq_lens, counts, w.n_q_heads, w.n_kv_heads, w.head_dim, w.block, w.chunk, w.key_tile, w.scale,
+                    w.torch_dtype, n_workers=8)
+    o, lse = skv.forward(dev["q"], dev["k"], dev["v"], dev["kb"], dev["vb"], anchors)
+    total = None
+    for r in range(n_ranks):
+        cp = ContextParallelSplitKV(w.seq_lens, counts, w.n_q_heads, w.n_kv_heads, w.head_dim, w.block, w.chunk,
+                                    w.key_tile, w.scale, w.torch_dtype, n_workers=8, rank=r, n_ranks=n_ranks)
+        cp.plan(anchors)
+        cr, parts, base_c = cp.chunk_rank.cpu(), [], 0
+        for S in w.seq_lens:
+            nc = -(-int(S) // w.chunk)
+            parts.append(torch.repeat_interleave(cr[base_c:base_c + nc], w.chunk)[: int(S)])
+            base_c += nc
+        mine = (torch.cat(parts) == r).cuda()[:, None, None]
+        k_r = torch.where(mine, dev["k"], torch.full_like(dev["k"], 256.0))
+        v_r = torch.where(mine, dev["v"], torch.full_like(dev["v"], 256.0))
+        grads = cp.local_backward(dev["q"], k_r, v_r, dev["kb"], dev["vb"], o, lse, dev["do"], anchors)
+        torch.cuda.synchronize()
+        cp.skv.check_status()
+        other = ~mine[:, 0, 0]  # key rows of other ranks' chunks: their dK, dV stay zero here
+        if bool(other.any()):
+            assert float(grads[1][other].abs().max()) == 0.0 and float(grads[2][other].abs().max()) == 0.0
+        total = [g.clone() for g in grads] if total is None else [t + g for t, g in zip(total, grads)]
+    from tests._gpu import assert_close
+    from tests._util import to_np
+    ref = OA.backward(oracle_problem(inp), to_np(inp.do))
+    for name, g, rf in zip(("dQ", "dK", "dV", "dKb", "dVb"), total, ref):
+        assert_close(name + " (ranks)", to_np(g), rf, w.dtype)
