@@ -49,6 +49,12 @@ def useful_flops(inp, backward):
     return fwd + bwd, fwd
 
 
+def timed_step_count(step_ms: float, min_steps: int = 20, min_timed_ms: float = 1000.0) -> int:
+    """Steps to time when the caller gives none: enough for `min_timed_ms` of timed work at `step_ms` per
+    step, and at least `min_steps`."""
+    return max(min_steps, int(math.ceil(min_timed_ms / max(step_ms, 1e-3))))
+
+
 def profiled_traffic(kernel, workload):
     """DRAM bytes per launch from the committed ncu summary of `kernel` on `workload`, or None when
     the summary is missing or the kernel's sources changed since it was captured."""
@@ -419,7 +425,7 @@ def run_ours(args):
         probe = timed_steps(3, replay, False)
         torch.cuda.synchronize(device)
         t_step = max_over_ranks(sum(a.elapsed_time(b) for a, b in probe) / len(probe), world, device)
-        steps = max(20, int(math.ceil(1000.0 / max(t_step, 1e-3))))
+        steps = timed_step_count(t_step)
     aux_steps = min(steps, 50)  # per-phase and end-to-end timings
 
     # ---- device-timed region

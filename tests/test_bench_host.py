@@ -102,3 +102,13 @@ def test_oracle_planning_time_and_cpu_model():
     assert r["items"] == 19 and r["workers"] == 4 and r["threads"] == 1
     assert r["cost_ms"] >= 0 and r["lpt_ms"] >= 0
     assert isinstance(bench.cpu_model(), str) and bench.cpu_model()
+
+
+def test_timed_step_count_reaches_one_second():
+    # Without --steps the timed region holds at least 1 s of steps (and at least 20 steps).
+    assert bench.timed_step_count(15.0) == 67          # skewed_s256k-sized steps: 67 x 15 ms >= 1 s
+    assert bench.timed_step_count(0.35) == 2858        # drafter-sized steps
+    assert bench.timed_step_count(100.0) == 20         # long steps: the minimum count
+    for ms in (0.01, 0.2, 3.3, 12.4, 49.9):
+        n = bench.timed_step_count(ms)
+        assert n >= 20 and n * ms >= 1000.0 and (n == 20 or (n - 1) * ms < 1000.0)
