@@ -265,11 +265,12 @@ def test_planner_rejects_out_of_range_costs():
     assert skv.status_value() & DEV_BAD_COST
 
 
-@pytest.mark.parametrize("n_workers", [1, 31, 33, 148, 256, 257, 300])
+@pytest.mark.parametrize("n_workers", [1, 31, 33, 64, 65, 100, 148, 224, 256, 257, 300])
 def test_planner_random_costs(n_workers):
-    # The run walk (one CTA, a thread per worker) must give the oracle's LPT plan bit for bit for
-    # worker counts below, at and above one warp and the SM count. Costs cover every bucket 1..64, skewed towards
-    # small ones like the workloads', with a few thousand items so most runs are non-trivial.
+    # The run walk (one CTA, a thread per worker, at least four warps) must give the oracle's LPT plan bit
+    # for bit for worker counts below, at and above one, two and four warps' worth, the SM count and eight
+    # warps. Costs cover every bucket 1..64, skewed towards small ones like the workloads', with a few
+    # thousand items so most runs are non-trivial.
     from oracle import schedule as OS
     from split_kv_lse_splitkv_b200 import SplitKV
     skv = SplitKV([262144], [512], 32, 4, 128, chunk=8192, n_workers=n_workers)
