@@ -19,8 +19,10 @@ SIMT = 1
 
 
 def small(name, base, seq_lens, counts, chunk=None, seed=11, **kw):
-    # Items over one chunk unless a test asks for runs (the full-size workloads use runs of chunks).
+    # Items over one chunk, costs in 128-key tiles, unless a test asks otherwise (the full-size workloads
+    # use runs of chunks, skewed_s256k a coarser cost tile).
     kw.setdefault("chunks_per_item", 1)
+    kw.setdefault("key_tile", 128)
     return W.make_inputs(W.scaled(W.get(base), name, seq_lens, counts, chunk=chunk, seed=seed, **kw))
 
 
@@ -154,6 +156,14 @@ def test_runs_of_chunks_batch_and_groups():
     # Three samples, G = 4 with two blocks per 128-row tile, runs of 2 chunks of 1024 keys.
     inp = small("runs_batch", "skewed_s256k", [3000, 700, 5000], [3, 1, 4], chunk=1024, blocks_per_item=2,
                 chunks_per_item=2)
+    full_check(inp, n_workers=6)
+
+
+def test_long_runs_coarse_cost_tile():
+    # Runs of 16 chunks whose cost counts 512-key tiles (skewed_s256k's setting), two blocks per 128-row
+    # tile: items of up to 16384 keys in one pass of the online softmax, ragged last runs, two samples.
+    inp = small("long_runs", "skewed_s256k", [40000, 9000], [5, 2], chunk=1024, blocks_per_item=2,
+                chunks_per_item=16, key_tile=512)
     full_check(inp, n_workers=6)
 
 

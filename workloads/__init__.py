@@ -73,9 +73,10 @@ WORKLOADS = {
         # Long context: S=131072, 128 anchors, chunk 2048 (runs of 4 chunks).
         Workload("long_s128k", 32, 4, 128, [131072], [128], 2048, "bf16", 2, chunks_per_item=4),
         # Skewed anchors: 32 q / 8 kv heads, S=262144, 256 draws of floor(S*Beta(5,1)), chunk 2048.
-        # G = 4: a block has 64 query rows, so two blocks share one 128-row query tile (runs of 4 chunks).
+        # G = 4: a block has 64 query rows, so two blocks share one 128-row query tile. Runs of 8 chunks
+        # (one partial per 16384 keys), their cost counted in 256-key tiles (at most 64 per item).
         Workload("skewed_s256k", 32, 8, 128, [262144], [256], 2048, "bf16", 3, sampler="beta51",
-                 blocks_per_item=2, chunks_per_item=4),
+                 blocks_per_item=2, chunks_per_item=8, key_tile=256),
         # Training step: 4 samples of S=65536 with 32/64/96/128 anchors, chunk 1024, fwd+bwd (runs of 8).
         Workload("train_4x64k", 32, 4, 128, [65536] * 4, [32, 64, 96, 128], 1024, "bf16", 4,
                  backward=True, chunks_per_item=8),
