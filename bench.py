@@ -57,7 +57,8 @@ def timed_step_count(step_ms: float, min_steps: int = 20, min_timed_ms: float = 
 
 def profiled_traffic(kernel, workload):
     """DRAM bytes per launch from the committed ncu summary of `kernel` on `workload`, or None when
-    the summary is missing or the kernel's sources changed since it was captured."""
+    the summary is missing, the kernel's sources changed since it was captured, or the workload's
+    definition (its `workload:` line) is no longer the registered one."""
     import hashlib
     path = os.path.join(ROOT, "profiles", f"{kernel}.{workload}.txt")
     try:
@@ -76,7 +77,16 @@ def profiled_traffic(kernel, workload):
                 return None
             if cur != digest.strip():
                 return None
+        elif ln.startswith("workload: "):
+            if ln[len("workload: "):].strip() != repr(W.get(workload)):
+                return None
     return traffic
+
+
+def traffic_applies(w, plan):
+    """The committed ncu summaries hold the registered workloads under the LPT plan: another run length,
+    cost tile, packing or plan moves other bytes, so its line reports no traffic."""
+    return w.dtype == "bf16" and plan == "lpt" and w == W.get(w.name)
 
 
 def peaks():
@@ -267,13 +277,16 @@ def cpu_oracle_sample(inp, budget_s, backward):
 
 
 def workload_of(args):
-    """The chosen workload, with --blocks-per-item overriding its query-tile packing when given."""
+    """The chosen workload, with --blocks-per-item, --chunks-per-item, --key-tile and --item-overhead
+    overriding its query-tile packing, run length, cost tile and per-item cost constant when given."""
     import dataclasses
     w = W.get(args.workload)
     if args.blocks_per_item:
         w = dataclasses.replace(w, blocks_per_item=args.blocks_per_item)
     if args.chunks_per_item:
         w = dataclasses.replace(w, chunks_per_item=args.chunks_per_item)
+    if args.key_tile:
+        w = dataclasses.replace(w, key_tile=args.key_tile)
     if args.item_overhead >= 0:
         w = dataclasses.replace(w, item_overhead=args.item_overhead)
     return w
@@ -285,7 +298,7 @@ def workload_config(w, counts, n_workers, world, plan):
     return {"workload": w.name, "seq_lens": list(w.seq_lens), "anchors": counts,
             "heads": f"{w.n_q_heads}q/{w.n_kv_heads}kv", "head_dim": w.head_dim, "chunk": w.chunk,
             "blocks_per_item": w.blocks_per_item, "chunks_per_item": w.chunks_per_item,
-            "item_overhead": w.item_overhead, "queues": n_workers,
+            "key_tile": w.key_tile, "item_overhead": w.item_overhead, "queues": n_workers,
             "l2": "flushed (256 MB write) before every timed step",
             "parallelism": f"replicas x{world}", "plan": plan}
 
@@ -522,7 +535,7 @@ def run_ours(args):
             "config": workload_config(w, counts, skv.n_workers, world, args.plan),
             "launch": "eager" if graph is None else "cuda graph of the step",
             "roofline": dict(roof, achieved=achieved, unit="TFLOP/s", frac=achieved / peak,
-                             traffic=profiled_traffic(fwd_kernel, w.name) if w.dtype == "bf16" else None,
+                             traffic=profiled_traffic(fwd_kernel, w.name) if traffic_applies(w, args.plan) else None,
                              kernel_ms=fwd_ms, algorithmic_flop=fwd_kernel_flops,
                              # useful TFLOP/s over the forward plus the merge, against the same peak
                              frac_fwd_merge=fwd_kernel_flops / ((fwd_ms + merge_ms) * 1e-3) / 1e12 / peak,
@@ -567,6 +580,8 @@ def main():
                          "(P * 16 * G = 256) run on pairs of SMs, smaller ones on one SM")
     ap.add_argument("--chunks-per-item", type=int, default=0,
                     help="runs of L chunks per item (one partial per run) instead of the workload's L")
+    ap.add_argument("--key-tile", type=int, default=0,
+                    help="key tile of the planner's cost (Tk, a divisor of the chunk) instead of the workload's")
     ap.add_argument("--item-overhead", type=int, default=-1,
                     help="per-item constant of the planner's cost in key tiles instead of the workload's")
     ap.add_argument("--plan", default="lpt", choices=["lpt", "naive"],

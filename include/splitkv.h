@@ -86,7 +86,8 @@ typedef struct {
     int32_t head_dim;           /* d: 128 for bf16; 8..128 (multiple of 4) for f32                  */
     int32_t block;              /* queries per draft block (16)                                     */
     int32_t chunk;              /* context chunk C, a multiple of key_tile                          */
-    int32_t key_tile;           /* Tk, the key tile of the cost model (128 in every workload)       */
+    int32_t key_tile;           /* Tk, the key tile of the cost model (a divisor of chunk): it sets
+                                   the unit of the costs and the plan, not the kernels' tiling      */
     float scale;                /* score scale, normally 1/sqrt(d)                                  */
     int32_t dtype;              /* SPLITKV_F32 or SPLITKV_BF16                                      */
     int32_t blocks_per_item;    /* P: consecutive blocks of a sample sharing one query tile (0 = 1);

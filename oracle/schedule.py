@@ -11,7 +11,7 @@ Readings (the pages give neither the cost unit nor the LPT details):
 
 * Work item = (sample s, chunk c, kv head g, block b). Its query tile is the
   ``block * G`` rows of block b at the G query heads of kv head g; its key tiles
-  are the ``key_tile`` (Tk = 128) slices of chunk c. Item cost = number of key
+  are the ``key_tile`` (Tk, 128 unless a workload counts coarser tiles) slices of chunk c. Item cost = number of key
   tiles holding at least one key the block sees; items of cost 0 are dropped.
 * Item index (chunk-major): ``base_s + (c * Hkv + g) * n_blocks_s + b`` where
   ``base_s`` counts the items of earlier samples and ``n_chunks_s = ceil(S/C)``.

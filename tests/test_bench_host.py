@@ -7,6 +7,7 @@ import sys
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 sys.path.insert(0, ROOT)
 import bench  # noqa: E402
+import workloads as W  # noqa: E402
 
 SUMMARY = "fwd_tc_kernel.drafter_s32k.txt"
 
@@ -51,6 +52,22 @@ def test_traffic_null_once_a_source_changed(tmp_path, monkeypatch):
     with open(os.path.join(str(tmp_path), rels[-1]), "a") as f:
         f.write("\n// edited after the capture\n")
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.profiled_traffic("fwd_tc_kernel", "drafter_s32k") is None
+
+
+def test_traffic_follows_the_workload_definition(tmp_path, monkeypatch):
+    # A summary pins the workload it was captured on (its dataclass repr): another run length, cost tile
+    # or packing in the registry makes its traffic stale, whatever the source hashes say.
+    import dataclasses
+    rels, traffic = _copy_summary_and_sources(str(tmp_path))
+    _write_hashes_of_current_sources(str(tmp_path), rels)
+    path = os.path.join(str(tmp_path), "profiles", SUMMARY)
+    lines = [ln for ln in open(path).read().splitlines() if not ln.startswith("workload: ")]
+    open(path, "w").write("\n".join(lines + ["workload: " + repr(W.get("drafter_s32k"))]) + "\n")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.profiled_traffic("fwd_tc_kernel", "drafter_s32k") == traffic > 0
+    changed = dataclasses.replace(W.get("drafter_s32k"), chunks_per_item=W.get("drafter_s32k").chunks_per_item + 1)
+    monkeypatch.setitem(W.WORKLOADS, "drafter_s32k", changed)
     assert bench.profiled_traffic("fwd_tc_kernel", "drafter_s32k") is None
 
 
@@ -112,3 +129,18 @@ def test_timed_step_count_reaches_one_second():
     for ms in (0.01, 0.2, 3.3, 12.4, 49.9):
         n = bench.timed_step_count(ms)
         assert n >= 20 and n * ms >= 1000.0 and (n == 20 or (n - 1) * ms < 1000.0)
+
+
+def test_traffic_only_for_the_registered_workload_and_plan():
+    # An override of the run length, cost tile or packing, or the naive plan, moves other DRAM bytes than
+    # the committed ncu summary of the workload holds: no traffic in that line.
+    import argparse
+    args = argparse.Namespace(workload="long_s128k", blocks_per_item=0, chunks_per_item=0, key_tile=0,
+                              item_overhead=-1)
+    w = bench.workload_of(args)
+    assert w == W.get("long_s128k") and bench.traffic_applies(w, "lpt")
+    assert not bench.traffic_applies(w, "naive")
+    for k, v in (("chunks_per_item", w.chunks_per_item // 2), ("key_tile", w.key_tile // 2), ("blocks_per_item", 2)):
+        w2 = bench.workload_of(argparse.Namespace(**{**vars(args), k: v}))
+        assert getattr(w2, k) == v and not bench.traffic_applies(w2, "lpt")
+    assert not bench.traffic_applies(W.get("tiny_f32"), "lpt")

@@ -70,8 +70,9 @@ WORKLOADS = {
         # Drafter shape A: 32 q / 4 kv heads, d=128, S=32768, 64 anchors, chunk 1024 (items over runs of
         # 6 chunks: one partial per 6144 keys).
         Workload("drafter_s32k", 32, 4, 128, [32768], [64], 1024, "bf16", 1, chunks_per_item=6),
-        # Long context: S=131072, 128 anchors, chunk 2048 (runs of 4 chunks).
-        Workload("long_s128k", 32, 4, 128, [131072], [128], 2048, "bf16", 2, chunks_per_item=4),
+        # Long context: S=131072, 128 anchors, chunk 2048 (runs of 8 chunks, their cost counted in
+        # 256-key tiles).
+        Workload("long_s128k", 32, 4, 128, [131072], [128], 2048, "bf16", 2, chunks_per_item=8, key_tile=256),
         # Skewed anchors: 32 q / 8 kv heads, S=262144, 256 draws of floor(S*Beta(5,1)), chunk 2048.
         # G = 4: a block has 64 query rows, so two blocks share one 128-row query tile. Runs of 8 chunks
         # (one partial per 16384 keys), their cost counted in 256-key tiles (at most 64 per item).
