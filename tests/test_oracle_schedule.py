@@ -104,7 +104,7 @@ def test_chunk_runs_worked_example():
 
 
 @pytest.mark.parametrize("seed", range(10))
-@pytest.mark.parametrize("runs", [2, 3])
+@pytest.mark.parametrize("runs", [2, 3, 8])
 @pytest.mark.parametrize("pack", [1, 2])
 def test_chunk_run_costs(seed, runs, pack):
     # Runs of L chunks: brute-force mask enumeration equals the closed form; the chunk costs do not
@@ -113,11 +113,11 @@ def test_chunk_run_costs(seed, runs, pack):
     # are the union of its chunks' visible keys, tile-aligned).
     rng = np.random.default_rng(2000 + seed)
     tk = int(rng.choice([8, 16, 32]))
-    chunk = tk * int(rng.integers(1, 4))
+    chunk = tk * int(rng.integers(1, 9))  # up to 8 cost tiles per chunk (256-key tiles on 2048-key chunks)
     hkv = int(rng.integers(1, 3))
     seq, anchors = [], []
     for _ in range(int(rng.integers(1, 4))):
-        S = int(rng.integers(20, 300))
+        S = int(rng.integers(20, 40 * chunk // tk + 300))
         n = int(rng.integers(0, min(6, S - 16) + 1))
         seq.append(S)
         anchors.append(sorted(rng.choice(np.arange(16, S), size=n, replace=False).tolist()))
