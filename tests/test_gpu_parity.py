@@ -20,7 +20,7 @@ SIMT = 1
 
 def small(name, base, seq_lens, counts, chunk=None, seed=11, **kw):
     # Items over one chunk, costs in 128-key tiles, unless a test asks otherwise (the full-size workloads
-    # use runs of chunks, skewed_s256k a coarser cost tile).
+    # use runs of chunks, long_s128k and skewed_s256k a coarser cost tile).
     kw.setdefault("chunks_per_item", 1)
     kw.setdefault("key_tile", 128)
     return W.make_inputs(W.scaled(W.get(base), name, seq_lens, counts, chunk=chunk, seed=seed, **kw))
