@@ -321,9 +321,13 @@ def run_reference(args):
     workers = w.n_workers or (torch.cuda.get_device_properties(0).multi_processor_count
                               if torch.cuda.is_available() else 148)
     r["plan"] = cpu_oracle_plan(inp, workers)
+    flops, _ = useful_flops(inp, w.backward)
     line = {"impl": "reference", "metric": "useful block-sparse attention TFLOP/s (fwd+bwd)" if w.backward else
             "useful block-sparse attention TFLOP/s (fwd)", "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
-            "steps": steps, "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
+            "steps": steps, "warmup": args.warmup,
+            # each timed step is a bounded sample of the workload: the whole step at the sampled rate
+            "ms_per_step": flops / (value * 1e12) * 1e3, "ms_per_step_kind": "extrapolated from the sampled rate",
+            "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": workload_config(w, [int(inp.anchor_off[i + 1] - inp.anchor_off[i])
                                           for i in range(len(w.seq_lens))], workers, args.gpus, args.plan),
