@@ -144,6 +144,12 @@ const char *splitkv_strerror(int code);
  * if the last call succeeded. Valid until the next call from the same thread. */
 const char *splitkv_last_error(void);
 
+/* Build id: the sha256 (hex) of the sources the library was compiled from (every file under csrc/ and
+ * this header, by name and content), or "unknown" for a build that did not supply it. The Python binding
+ * compares it with the sources beside the library and warns when they differ (a stale build). Static
+ * storage; no failure. */
+const char *splitkv_build_id(void);
+
 /*
  * Realized cost pass (Split-KV paper, Abstract: chunks are weighted by the attention work they
  * actually incur). Validates the anchors (strictly ascending per sample, each in [block, S)) and, for every

@@ -4,6 +4,7 @@ from __future__ import annotations
 import ctypes
 import math
 import os
+import warnings
 from typing import Optional, Sequence
 
 import torch
@@ -65,6 +66,7 @@ _SIGS = {
     "splitkv_max_workers": (_i32, [_PP, ctypes.POINTER(_i32)]),
     "splitkv_strerror": (ctypes.c_char_p, [_i32]),
     "splitkv_last_error": (ctypes.c_char_p, []),
+    "splitkv_build_id": (ctypes.c_char_p, []),
     "splitkv_cost": (_i32, [_PP, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "splitkv_plan_lpt": (_i32, [_vp, _vp, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "splitkv_plan_lpt_noalloc": (_i32, [_vp, _vp, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _vp]),
@@ -80,9 +82,35 @@ _SIGS = {
 }
 EXPORTS = tuple(_SIGS)
 for _name, (_res, _args) in _SIGS.items():
-    _fn = getattr(_lib, _name)
+    try:
+        _fn = getattr(_lib, _name)
+    except AttributeError:
+        raise ImportError(f"{LIB_PATH} does not export {_name}: it was built from older sources; rebuild with "
+                          "`python -m split_kv_lse_splitkv_b200.build`") from None
     _fn.restype = _res
     _fn.argtypes = _args
+
+
+def library_build_id() -> str:
+    """sha256 of the sources the loaded library was compiled from ("unknown" if its build supplied none)."""
+    return _lib.splitkv_build_id().decode()
+
+
+def _warn_if_stale() -> None:
+    # A library built from other sources than those beside it runs other code than they say.
+    try:
+        from .build import source_digest
+        want = source_digest()
+    except (ImportError, OSError):  # no sources beside the library
+        return
+    got = library_build_id()
+    if got != want:
+        warnings.warn(f"{LIB_PATH} was built from other sources than those beside it (build id {got[:12]}, "
+                      f"sources {want[:12]}): rebuild with `python -m split_kv_lse_splitkv_b200.build`",
+                      RuntimeWarning, stacklevel=2)
+
+
+_warn_if_stale()
 
 
 class SplitKVError(RuntimeError):

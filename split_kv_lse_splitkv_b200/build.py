@@ -30,6 +30,19 @@ def nvcc() -> str:
     raise RuntimeError("nvcc not found")
 
 
+def source_digest() -> str:
+    """sha256 (hex) of the library's sources: every .cu/.cuh/.h under csrc/ and include/splitkv.h, by
+    relative name and content, in name order. Compiled into libsplitkv.so as its build id."""
+    import hashlib
+    h = hashlib.sha256()
+    files = [("csrc/" + f, os.path.join(CSRC, f)) for f in sorted(os.listdir(CSRC)) if f.endswith((".cu", ".cuh", ".h"))]
+    files.append(("include/splitkv.h", os.path.join(os.path.dirname(HERE), "include", "splitkv.h")))
+    for rel, path in files:
+        with open(path, "rb") as fh:
+            h.update(rel.encode() + b"\0" + fh.read() + b"\0")
+    return h.hexdigest()
+
+
 def _newer(target: str, deps) -> bool:
     if not os.path.exists(target):
         return False
@@ -46,13 +59,19 @@ def build(verbose_ptxas: bool = False, force: bool = False) -> str:
     if verbose_ptxas:
         flags += ["-Xptxas", "-v"]
     nv = nvcc()
+    # abi.cu carries the build id: it is recompiled whenever any source differs from the last build's.
+    digest = source_digest()
+    digest_file = os.path.join(BUILD, "source_digest.txt")
+    last = open(digest_file).read().strip() if os.path.exists(digest_file) else ""
 
     def compile_one(src):
         path = os.path.join(CSRC, src)
         obj = os.path.join(BUILD, src.replace(".cu", ".o"))
-        if not force and not verbose_ptxas and _newer(obj, [path] + headers):
+        stale_id = src == "abi.cu" and last != digest
+        if not force and not verbose_ptxas and not stale_id and _newer(obj, [path] + headers):
             return obj, ""
-        cmd = [nv, *flags, "-c", path, "-o", obj]
+        extra = [f'-DSPLITKV_SOURCE_SHA="{digest}"'] if src == "abi.cu" else []
+        cmd = [nv, *flags, *extra, "-c", path, "-o", obj]
         res = subprocess.run(cmd, capture_output=True, text=True)
         if res.returncode != 0:
             raise RuntimeError(f"nvcc failed on {src}:\n{res.stdout}\n{res.stderr}")
@@ -69,6 +88,8 @@ def build(verbose_ptxas: bool = False, force: bool = False) -> str:
         res = subprocess.run(cmd, capture_output=True, text=True)
         if res.returncode != 0:
             raise RuntimeError(f"link failed:\n{res.stdout}\n{res.stderr}")
+    with open(digest_file, "w") as fh:
+        fh.write(digest + "\n")
     return LIB
 
 

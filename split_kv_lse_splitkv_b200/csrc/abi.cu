@@ -156,6 +156,12 @@ SPLITKV_API int splitkv_max_workers(const splitkv_problem* problem, int32_t* n_w
 
 SPLITKV_API const char* splitkv_last_error(void) { return g_last_error; }
 
+// The build script passes the sha256 of the library's sources; other builds say "unknown".
+#ifndef SPLITKV_SOURCE_SHA
+#define SPLITKV_SOURCE_SHA "unknown"
+#endif
+SPLITKV_API const char* splitkv_build_id(void) { return SPLITKV_SOURCE_SHA; }
+
 SPLITKV_API const char* splitkv_strerror(int code) {
     switch (code) {
         case SPLITKV_OK: return "ok";

@@ -209,3 +209,10 @@ def test_problem_without_anchors_needs_no_query_buffers(dtype, d):
     assert rc == B.EINVAL
     rc = B._lib.splitkv_lse_merge(p1.ptr, h, h, h, None, None, h, None)
     assert rc == B.EINVAL
+
+
+def test_library_built_from_these_sources():
+    # The build id compiled into libsplitkv.so is the digest of the sources beside it: a library left over
+    # from other sources (edited, reverted or checked out after the build) fails here and warns on import.
+    from split_kv_lse_splitkv_b200 import build
+    assert B.library_build_id() == build.source_digest()
