@@ -83,6 +83,16 @@ def profiled_traffic(kernel, workload):
     return traffic
 
 
+def library_provenance():
+    """The loaded library's build id against the sources beside it: a stale build runs other code."""
+    try:
+        from split_kv_lse_splitkv_b200 import binding, build
+        got, want = binding.library_build_id(), build.source_digest()
+    except Exception as e:  # provenance is a report: it never ends the run
+        return {"build_id": None, "matches_sources": None, "error": repr(e)}
+    return {"build_id": got[:16], "matches_sources": got == want}
+
+
 def traffic_applies(w, plan):
     """The committed ncu summaries hold the registered workloads under the LPT plan: another run length,
     cost tile, packing or plan moves other bytes, so its line reports no traffic."""
@@ -558,6 +568,7 @@ def run_ours(args):
             "gpu_launches": launches_per_step * steps,
             "wall_s": wall,
             "cpu_baseline": cpu,
+            "library": library_provenance(),
         }
         print(json.dumps(line))
     if world > 1:

@@ -144,3 +144,8 @@ def test_traffic_only_for_the_registered_workload_and_plan():
         w2 = bench.workload_of(argparse.Namespace(**{**vars(args), k: v}))
         assert getattr(w2, k) == v and not bench.traffic_applies(w2, "lpt")
     assert not bench.traffic_applies(W.get("tiny_f32"), "lpt")
+
+
+def test_library_provenance_names_the_build():
+    prov = bench.library_provenance()
+    assert prov["matches_sources"] is True and len(prov["build_id"]) == 16
